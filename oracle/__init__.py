@@ -1,0 +1,157 @@
+"""CPU oracle for the dual-path sparse-quantized linear layer.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg are the only callers.  The product library never
+imports this package and this package never imports the product library.
+
+The arithmetic lives in ``sq_oracle.c`` (plain C, fp32 quantizer decisions,
+int64 integer path, fp64 16-bit branch and output).  This module compiles it
+with gcc on first use and wraps it with numpy arrays.  The method it follows
+is described in the C file's header: the OSC page (arXiv:2604.12782, abstract
+and technical framework: static outlier channels, compact gather, 4-bit GEMM
+plus 16-bit branch GEMM, fused sum) and the SQ-format write-up of
+arXiv:2512.05409 (section 9: symmetric quantization, column reordering by the
+static mask).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle_sq.so")
+_CFLAGS = ["-O2", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-std=c11"]
+_lock = threading.Lock()
+_lib = None
+
+QMAX = 7  # symmetric INT4 code range [-7, 7]
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (if missing or older than its source)."""
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", *_CFLAGS, _SRC, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = ctypes.CDLL(_LIB_PATH)
+            P = ctypes.c_void_p
+            I = ctypes.c_int64
+            lib.orc_validate_outliers.argtypes = [P, I, I]
+            lib.orc_quantize_rows.argtypes = [P, I, I, I, P, I, P, P, P]
+            lib.orc_pack_int4.argtypes = [P, I, I, I, P]
+            lib.orc_chan_table.argtypes = [P, I, I, P]
+            lib.orc_dual_linear_rows.argtypes = [P, P, P, I, P, P, P, I, I, I, P, P, P]
+            lib.orc_num_threads.argtypes = []
+            for f in (lib.orc_validate_outliers, lib.orc_quantize_rows, lib.orc_pack_int4,
+                      lib.orc_chan_table, lib.orc_dual_linear_rows, lib.orc_num_threads):
+                f.restype = ctypes.c_int
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _as_O(O) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(O, dtype=np.int32).reshape(-1))
+
+
+def num_threads() -> int:
+    """Host threads the oracle's row loops use (OMP_NUM_THREADS, else all cores)."""
+    return int(_load().orc_num_threads())
+
+
+def validate_outliers(O, K: int) -> bool:
+    O = _as_O(O)
+    return _load().orc_validate_outliers(_ptr(O), O.size, K) == 0
+
+
+def quantize_rows(src_bits: np.ndarray, K: int, O):
+    """Quantize-and-gather rows of a bf16 matrix given as uint16 bit patterns.
+
+    Returns (codes int8 [rows, K-nO], scale float32 [rows], outl uint16 [rows, nO]).
+    """
+    src = np.ascontiguousarray(src_bits, dtype=np.uint16)
+    if src.ndim != 2 or src.shape[1] < K:
+        raise ValueError("src must be [rows, ld>=K]")
+    O = _as_O(O)
+    rows, ld = src.shape
+    KN = K - O.size
+    codes = np.zeros((rows, KN), np.int8)
+    scale = np.zeros(rows, np.float32)
+    outl = np.zeros((rows, O.size), np.uint16)
+    rc = _load().orc_quantize_rows(_ptr(src), rows, K, ld, _ptr(O), O.size,
+                                   _ptr(codes), _ptr(scale), _ptr(outl))
+    if rc != 0:
+        raise ValueError("invalid outlier channel set")
+    return codes, scale, outl
+
+
+def pack_int4(codes: np.ndarray, row_bytes: int) -> np.ndarray:
+    """Packed storage of int4 codes: byte j = code 2j (low nibble) | code 2j+1 (high nibble)."""
+    codes = np.ascontiguousarray(codes, dtype=np.int8)
+    rows, KN = codes.shape
+    out = np.zeros((rows, row_bytes), np.uint8)
+    if _load().orc_pack_int4(_ptr(codes), rows, KN, row_bytes, _ptr(out)) != 0:
+        raise ValueError("row_bytes too small")
+    return out
+
+
+def chan_table(O, K: int) -> np.ndarray:
+    """Static channel table: word c = (#outliers below 8c) << 8 | outlier bits of 8c..8c+7."""
+    O = _as_O(O)
+    tab = np.zeros(K // 8, np.uint32)
+    if _load().orc_chan_table(_ptr(O), O.size, K, _ptr(tab)) != 0:
+        raise ValueError("invalid outlier channel set or K % 8 != 0")
+    return tab
+
+
+def dual_linear_rows(qx, sx, xo, qw, sw, wo):
+    """(acc_i int64, acc_o float64, y float64), each [rows of qx, rows of qw]."""
+    qx = np.ascontiguousarray(qx, np.int8)
+    qw = np.ascontiguousarray(qw, np.int8)
+    sx = np.ascontiguousarray(sx, np.float32)
+    sw = np.ascontiguousarray(sw, np.float32)
+    xo = np.ascontiguousarray(xo, np.uint16)
+    wo = np.ascontiguousarray(wo, np.uint16)
+    Mr, KN = qx.shape
+    N = qw.shape[0]
+    nO = xo.shape[1]
+    assert qw.shape[1] == KN and wo.shape == (N, nO) and xo.shape[0] == Mr
+    acc_i = np.zeros((Mr, N), np.int64)
+    acc_o = np.zeros((Mr, N), np.float64)
+    y = np.zeros((Mr, N), np.float64)
+    _load().orc_dual_linear_rows(_ptr(qx), _ptr(sx), _ptr(xo), Mr, _ptr(qw), _ptr(sw), _ptr(wo),
+                                 N, KN, nO, _ptr(acc_i), _ptr(acc_o), _ptr(y))
+    return acc_i, acc_o, y
+
+
+def linear(X_bits: np.ndarray, W_bits: np.ndarray, O, rows=None):
+    """Whole layer for the selected activation rows (all rows when None).
+
+    Returns a dict with the quantizer outputs of both operands and the
+    products: qx, sx, xo, qw, sw, wo, acc_i, acc_o, y.
+    """
+    K = W_bits.shape[1]
+    Xs = X_bits if rows is None else X_bits[np.asarray(rows)]
+    qx, sx, xo = quantize_rows(Xs, K, O)
+    qw, sw, wo = quantize_rows(W_bits, K, O)
+    acc_i, acc_o, y = dual_linear_rows(qx, sx, xo, qw, sw, wo)
+    return dict(qx=qx, sx=sx, xo=xo, qw=qw, sw=sw, wo=wo, acc_i=acc_i, acc_o=acc_o, y=y)

@@ -1,0 +1,216 @@
+/*
+ * CPU oracle for the dual-path sparse-quantized linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the package smoke check and the
+ * benchmark's CPU-baseline leg may load this file.  It shares no code, header,
+ * table or helper with the CUDA library and must never be linked into it.
+ *
+ * What it computes (a plain, slow, literal statement of the layer):
+ *
+ *   Y[m,n] = s_x[m] * s_w[n] * sum_{k not in O} q(X)[m,k] * q(W)[n,k]
+ *          +                   sum_{k in O}     X[m,k]   * W[n,k]
+ *
+ * Sources:
+ *   - OSC: Hardware Efficient W4A4 Quantization via Outlier Separation in
+ *     Channel Dimension (arXiv:2604.12782), abstract and "technical framework"
+ *     paragraph: a static set O of outlier input channels is chosen offline;
+ *     at inference the scattered outlier channels are coalesced into a compact
+ *     dense tensor and run through a 16-bit branch GEMM while every other
+ *     channel runs through a 4-bit GEMM; the two results are fused (summed).
+ *   - SQ-format write-up of arXiv:2512.05409, section 9 (technical details):
+ *     the low-precision part uses symmetric quantization, which leaves the
+ *     most negative two's-complement code unused (INT2 keeps {-1,0,1}); for
+ *     INT4 that is the range [-7, 7].  Section 9 also reorders weight columns
+ *     by the static mask; here the compact normal part keeps the channels in
+ *     ascending order and the compact outlier part keeps O in ascending order.
+ *   - Scale granularity (not fixed by the pages; the layer's formula above):
+ *     one scale per token row of X (computed online) and one per output
+ *     channel (row) of W (computed offline), each the absolute maximum over
+ *     the NON-outlier channels divided by 7.
+ *
+ * Readings taken where the pages are silent:
+ *   - s = a / 7 with a = max |x| over k not in O, both fp32 (bf16 widens to
+ *     fp32 exactly) with IEEE round-to-nearest division.
+ *   - code = clamp(rint(x / s), -7, 7) where x / s is the IEEE fp32 quotient
+ *     and rint rounds half to even (FE_TONEAREST).  The integer decision is
+ *     made in fp32, the same precision as the CUDA kernels.
+ *   - a == 0 (all normal channels zero, or no normal channels): s = 0 and
+ *     every code is 0.
+ *   - Integer products are summed exactly in int64; the 16-bit branch and the
+ *     final Y are computed in fp64 without any final rounding.
+ *
+ * The `omp parallel for` pragmas only distribute independent output rows over
+ * host threads; they do not change any arithmetic or its order.
+ *
+ * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_QMAX 7
+
+static float orc_bf16_to_f32(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* O must be strictly increasing inside [0, K).  Returns 0 when valid. */
+int orc_validate_outliers(const int32_t *O, int64_t nO, int64_t K)
+{
+    if (K <= 0 || nO < 0 || nO > K) return -1;
+    for (int64_t j = 0; j < nO; ++j) {
+        if (O[j] < 0 || O[j] >= K) return -1;
+        if (j > 0 && O[j] <= O[j - 1]) return -1;
+    }
+    return 0;
+}
+
+/*
+ * Quantize-and-gather of `rows` rows of a bf16 matrix (row stride `ld`
+ * elements).  Used for activations (rows = tokens, online) and for weights
+ * (rows = output channels, offline): the pages apply the same symmetric
+ * quantizer to both operands of the 4-bit path.
+ *
+ * Outputs (caller-allocated, dense):
+ *   codes [rows, K - nO]  int8 codes of the normal channels, ascending order
+ *   scale [rows]          fp32 scales
+ *   outl  [rows, nO]      bf16 bit copies of the outlier channels, O order
+ * Returns 0, or -1 when O is invalid.
+ */
+int orc_quantize_rows(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                      const int32_t *O, int64_t nO,
+                      int8_t *codes, float *scale, uint16_t *outl)
+{
+    if (orc_validate_outliers(O, nO, K) != 0 || ld < K) return -1;
+    char *is_outlier = (char *)calloc((size_t)K, 1);
+    if (!is_outlier) return -1;
+    for (int64_t j = 0; j < nO; ++j) is_outlier[O[j]] = 1;
+    const int64_t KN = K - nO;
+
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *row = src + r * ld;
+
+        /* a = absolute maximum over the normal channels only. */
+        float a = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            if (is_outlier[k]) continue;
+            float v = fabsf(orc_bf16_to_f32(row[k]));
+            if (v > a) a = v;
+        }
+        float s = a / 7.0f;
+        if (a == 0.0f) s = 0.0f;
+        scale[r] = s;
+
+        /* Codes of the normal channels, in ascending channel order. */
+        int64_t j = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            if (is_outlier[k]) continue;
+            int q = 0;
+            if (a != 0.0f) {
+                float x = orc_bf16_to_f32(row[k]);
+                float t = x / s;
+                q = (int)nearbyintf(t); /* default mode: nearest, ties to even */
+                if (q > ORC_QMAX) q = ORC_QMAX;
+                if (q < -ORC_QMAX) q = -ORC_QMAX;
+            }
+            codes[r * KN + j] = (int8_t)q;
+            ++j;
+        }
+
+        /* Compact outlier tensor: bit copies of the channels in O. */
+        for (int64_t jo = 0; jo < nO; ++jo) outl[r * nO + jo] = row[O[jo]];
+    }
+    free(is_outlier);
+    return 0;
+}
+
+/*
+ * Storage layout of the packed 4-bit normal part: row r occupies `row_bytes`
+ * bytes; byte j holds code 2j in its low nibble and code 2j+1 in its high
+ * nibble, each as 4-bit two's complement; bytes past the codes are zero.
+ */
+int orc_pack_int4(const int8_t *codes, int64_t rows, int64_t KN, int64_t row_bytes,
+                  uint8_t *packed)
+{
+    if (row_bytes * 2 < KN) return -1;
+    for (int64_t r = 0; r < rows; ++r) {
+        uint8_t *dst = packed + r * row_bytes;
+        memset(dst, 0, (size_t)row_bytes);
+        for (int64_t j = 0; j < KN; ++j) {
+            uint8_t nib = (uint8_t)(codes[r * KN + j]) & 0x0F;
+            if (j % 2 == 0)
+                dst[j / 2] |= nib;
+            else
+                dst[j / 2] |= (uint8_t)(nib << 4);
+        }
+    }
+    return 0;
+}
+
+/*
+ * Static channel table (the pages' "static mask", one word per 8 channels):
+ * word c = (number of outlier channels below 8c) << 8 | bit e set when
+ * channel 8c+e is an outlier.  K must be a multiple of 8.
+ */
+int orc_chan_table(const int32_t *O, int64_t nO, int64_t K, uint32_t *table)
+{
+    if (orc_validate_outliers(O, nO, K) != 0 || K % 8 != 0) return -1;
+    for (int64_t c = 0; c < K / 8; ++c) {
+        uint32_t below = 0, mask = 0;
+        for (int64_t j = 0; j < nO; ++j) {
+            if (O[j] < 8 * c) ++below;
+            else if (O[j] < 8 * c + 8) mask |= 1u << (O[j] - 8 * c);
+        }
+        table[c] = (below << 8) | mask;
+    }
+    return 0;
+}
+
+/*
+ * Dual-path products for `Mr` activation rows against all N weight rows.
+ * Inputs are the outputs of orc_quantize_rows for X and for W.
+ *   acc_i [Mr, N]  exact integer dot product of the codes (int64)
+ *   acc_o [Mr, N]  16-bit branch: sum of X_O * W_O in fp64
+ *   y     [Mr, N]  acc_i * s_x * s_w + acc_o in fp64 (no final rounding)
+ */
+int orc_dual_linear_rows(const int8_t *qx, const float *sx, const uint16_t *xo, int64_t Mr,
+                         const int8_t *qw, const float *sw, const uint16_t *wo, int64_t N,
+                         int64_t KN, int64_t nO,
+                         int64_t *acc_i, double *acc_o, double *y)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < Mr; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t ai = 0;
+            for (int64_t j = 0; j < KN; ++j)
+                ai += (int64_t)qx[m * KN + j] * (int64_t)qw[n * KN + j];
+            double ao = 0.0;
+            for (int64_t j = 0; j < nO; ++j)
+                ao += (double)orc_bf16_to_f32(xo[m * nO + j]) *
+                      (double)orc_bf16_to_f32(wo[n * nO + j]);
+            acc_i[m * N + n] = ai;
+            acc_o[m * N + n] = ao;
+            y[m * N + n] = (double)ai * (double)sx[m] * (double)sw[n] + ao;
+        }
+    }
+    return 0;
+}
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+/* Number of host threads the parallel loops above use. */
+int orc_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

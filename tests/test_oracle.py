@@ -1,0 +1,318 @@
+"""Pins for the CPU oracle (no GPU).
+
+Each test ties the oracle to something other than itself: hand-worked golden
+cases, exact rational arithmetic, closed-form reductions to library routines
+(numpy integer / fp64 matmul), brute force on tiny inputs, and invariants of
+the quantizer (bound, split reconstruction, power-of-two scaling, sign
+symmetry, channel-permutation invariance).
+"""
+from __future__ import annotations
+
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------- helpers
+def bf16_bits_of(values) -> np.ndarray:
+    t = torch.tensor(values, dtype=torch.float32)
+    b = t.to(torch.bfloat16)
+    assert torch.equal(b.float(), t), "golden values must be exact in bf16"
+    return b.view(torch.int16).numpy().view(np.uint16)
+
+
+def bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def f32_round(q: Fraction) -> Fraction:
+    """Round a rational to the nearest IEEE binary32 value, ties to even."""
+    if q == 0:
+        return Fraction(0)
+    sign = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    e = max(e, -126)
+    quantum = Fraction(2) ** (e - 23)
+    n = a / quantum
+    fl = n.numerator // n.denominator
+    rem = n - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return sign * fl * quantum
+
+
+def exact_quant_row(xs: list[Fraction], normal: list[int]):
+    """Independent statement of the quantizer in exact rational arithmetic."""
+    a = max((abs(xs[k]) for k in normal), default=Fraction(0))
+    if a == 0:
+        return Fraction(0), [0] * len(normal)
+    s = f32_round(a / 7)
+    codes = []
+    for k in normal:
+        t = f32_round(xs[k] / s)
+        q = round(t)  # Fraction.__round__ rounds half to even
+        codes.append(max(-7, min(7, q)))
+    return s, codes
+
+
+def parse_cases(path):
+    cases, cur = [], None
+    for raw in open(path):
+        line = raw.split("#", 1)[0].strip()
+        if not line:
+            continue
+        key, *rest = line.split()
+        if key == "case":
+            cur = {"name": rest[0]}
+            cases.append(cur)
+        else:
+            cur[key] = rest
+    return cases
+
+
+# ----------------------------------------------------------------- golden
+@pytest.mark.parametrize("case", parse_cases(os.path.join(GOLDEN, "quant_rows.txt")),
+                         ids=lambda c: c["name"])
+def test_golden_quant_rows(case):
+    K = int(case["K"][0])
+    O = [int(v) for v in case.get("O", [])]
+    x = [float(v) for v in case["x"]]
+    codes, scale, outl = oracle.quantize_rows(bf16_bits_of([x]), K, O)
+    assert scale[0] == np.float32(float.fromhex(case["scale"][0]))
+    assert codes[0].tolist() == [int(v) for v in case.get("codes", [])]
+    assert outl[0].tolist() == bf16_bits_of([[float(v) for v in case.get("outl", [])]] if case.get("outl") else [[]]).reshape(-1).tolist()
+
+
+def test_golden_dual_linear():
+    case = {}
+    for raw in open(os.path.join(GOLDEN, "dual_linear.txt")):
+        line = raw.split("#", 1)[0].strip()
+        if line:
+            key, *rest = line.split()
+            case.setdefault(key, []).append(rest)
+    K = int(case["K"][0][0])
+    O = [int(v) for v in case["O"][0]]
+    X = bf16_bits_of([[float(v) for v in r] for r in case["X"]])
+    W = bf16_bits_of([[float(v) for v in r] for r in case["W"]])
+    r = oracle.linear(X, W, O)
+    assert r["acc_i"].tolist() == [[int(v) for v in row] for row in case["acc_i"]]
+    assert r["y"].tolist() == [[float(v) for v in row] for row in case["y"]]
+    assert K == X.shape[1]
+
+
+# ----------------------------------------------------------------- exact arithmetic
+def _tie_heavy_rows(rng, rows, K):
+    """bf16 rows whose entries sit on or next to rounding ties of x/s."""
+    out = []
+    for _ in range(rows):
+        a = float(2.0 ** rng.integers(-6, 6)) * float(rng.choice([1.0, 1.5, 1.25, 1.75]))
+        halves = rng.integers(-14, 15, size=K).astype(np.float64) / 2.0  # multiples of 0.5 in [-7, 7]
+        xs = halves * (a / 7.0)
+        xs[rng.integers(0, K)] = a * rng.choice([-1.0, 1.0])
+        out.append(xs)
+    b = torch.tensor(np.array(out), dtype=torch.float32).to(torch.bfloat16)
+    return b.view(torch.int16).numpy().view(np.uint16)
+
+
+@pytest.mark.parametrize("kind", ["gauss", "ties"])
+def test_quantizer_matches_exact_rational(kind):
+    rng = np.random.default_rng(7)
+    K, nO = 48, 5
+    O = np.sort(rng.choice(K, nO, replace=False)).astype(np.int32)
+    if kind == "gauss":
+        bits = workloads.bf16_bits(workloads.activations(64, K, torch.from_numpy(O), sigma=30.0, seed=11))
+    else:
+        bits = _tie_heavy_rows(rng, 64, K)
+    codes, scale, outl = oracle.quantize_rows(bits, K, O)
+    normal = [k for k in range(K) if k not in set(O.tolist())]
+    xf = bits_to_f64(bits)
+    for r in range(bits.shape[0]):
+        xs = [Fraction(float(v)) for v in xf[r]]
+        s, q = exact_quant_row(xs, normal)
+        assert Fraction(float(scale[r])) == s
+        assert codes[r].tolist() == q
+        assert outl[r].tolist() == bits[r, O].tolist()
+
+
+# ----------------------------------------------------------------- invariants
+def _tiny():
+    w = workloads.TINY
+    O, X, W = workloads.make(w)
+    return w, O.numpy(), workloads.bf16_bits(X), workloads.bf16_bits(W)
+
+
+def test_quantizer_bound_and_range():
+    w, O, Xb, Wb = _tiny()
+    for bits in (Xb, Wb):
+        codes, scale, _ = oracle.quantize_rows(bits, w.K, O)
+        normal = np.setdiff1d(np.arange(w.K), O)
+        x = bits_to_f64(bits)[:, normal]
+        s = scale.astype(np.float64)[:, None]
+        assert codes.min() >= -7 and codes.max() <= 7
+        err = np.abs(x - s * codes)
+        assert np.all(err <= s / 2 * (1 + 2.0 ** -20))
+        amax = np.argmax(np.abs(x), axis=1)
+        assert np.all(np.abs(codes[np.arange(len(x)), amax]) == 7)
+
+
+def test_split_reconstruction_is_exact():
+    w, O, Xb, _ = _tiny()
+    codes, scale, outl = oracle.quantize_rows(Xb, w.K, O)
+    # Scatter the compact outlier tensor back: bit-identical to X on O.
+    back = np.zeros_like(Xb)
+    back[:, O] = outl
+    assert np.array_equal(back[:, O], Xb[:, O])
+    assert np.all(back[:, np.setdiff1d(np.arange(w.K), O)] == 0)
+    # Every channel lands in exactly one part.
+    assert codes.shape[1] + outl.shape[1] == w.K
+    # Scatter the dequantized normal part back: it approximates X off O
+    # (within half a step) and is exactly zero on O.
+    normal = np.setdiff1d(np.arange(w.K), O)
+    deq = np.zeros((Xb.shape[0], w.K))
+    deq[:, normal] = scale[:, None].astype(np.float64) * codes
+    x = bits_to_f64(Xb)
+    assert np.all(deq[:, O] == 0)
+    assert np.all(np.abs(deq[:, normal] - x[:, normal]) <= scale[:, None] / 2 * (1 + 2.0 ** -20))
+
+
+@pytest.mark.parametrize("e", [-3, 1, 5])
+def test_power_of_two_scaling(e):
+    w, O, Xb, _ = _tiny()
+    codes, scale, _ = oracle.quantize_rows(Xb, w.K, O)
+    Xs = (torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).float() * 2.0 ** e).to(torch.bfloat16)
+    codes2, scale2, _ = oracle.quantize_rows(workloads.bf16_bits(Xs), w.K, O)
+    assert np.array_equal(codes, codes2)
+    assert np.array_equal(scale.astype(np.float64) * 2.0 ** e, scale2.astype(np.float64))
+
+
+def test_sign_symmetry():
+    w, O, Xb, _ = _tiny()
+    codes, scale, outl = oracle.quantize_rows(Xb, w.K, O)
+    neg = Xb ^ np.uint16(0x8000)
+    codes_n, scale_n, outl_n = oracle.quantize_rows(neg, w.K, O)
+    assert np.array_equal(codes_n, -codes)
+    assert np.array_equal(scale_n, scale)
+    assert np.array_equal(outl_n, outl ^ np.uint16(0x8000))
+
+
+def test_channel_permutation_invariance():
+    w, O, Xb, Wb = _tiny()
+    r0 = oracle.linear(Xb, Wb, O)
+    perm = np.random.default_rng(3).permutation(w.K)          # new channel j <- old perm[j]
+    inv = np.argsort(perm)
+    O2 = np.sort(inv[O]).astype(np.int32)
+    r1 = oracle.linear(Xb[:, perm], Wb[:, perm], O2)
+    assert np.array_equal(r0["acc_i"], r1["acc_i"])
+    assert np.array_equal(r0["sx"], r1["sx"]) and np.array_equal(r0["sw"], r1["sw"])
+    np.testing.assert_allclose(r1["y"], r0["y"], rtol=1e-12, atol=1e-12)
+
+
+# ----------------------------------------------------------------- reductions
+def test_empty_outlier_set_is_plain_w4a4():
+    w = workloads.Workload("t", 32, 128, 48, 0)
+    O, X, W = workloads.make(w)
+    Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
+    r = oracle.linear(Xb, Wb, O.numpy())
+    assert r["xo"].shape == (32, 0) and r["wo"].shape == (48, 0)
+    ref = r["qx"].astype(np.int64) @ r["qw"].astype(np.int64).T
+    assert np.array_equal(r["acc_i"], ref)
+    assert np.all(r["acc_o"] == 0)
+    y = ref.astype(np.float64) * r["sx"].astype(np.float64)[:, None] * r["sw"].astype(np.float64)[None, :]
+    assert np.array_equal(r["y"], y)
+
+
+def test_all_channels_outliers_is_bf16_gemm():
+    w = workloads.Workload("t", 24, 64, 40, 64)
+    O, X, W = workloads.make(w)
+    Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
+    r = oracle.linear(Xb, Wb, O.numpy())
+    assert r["qx"].shape == (24, 0) and np.all(r["sx"] == 0) and np.all(r["sw"] == 0)
+    ref = bits_to_f64(Xb) @ bits_to_f64(Wb).T
+    np.testing.assert_allclose(r["y"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_bruteforce_triple_loop():
+    rng = np.random.default_rng(5)
+    M, N, K = 3, 4, 16
+    O = np.sort(rng.choice(K, 3, replace=False)).astype(np.int32)
+    X = torch.from_numpy(rng.standard_normal((M, K)).astype(np.float32)).to(torch.bfloat16)
+    W = torch.from_numpy(rng.standard_normal((N, K)).astype(np.float32)).to(torch.bfloat16)
+    Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
+    r = oracle.linear(Xb, Wb, O)
+    x, wt = bits_to_f64(Xb), bits_to_f64(Wb)
+    normal = [k for k in range(K) if k not in set(O.tolist())]
+    for m in range(M):
+        sx, qx = exact_quant_row([Fraction(float(v)) for v in x[m]], normal)
+        for n in range(N):
+            sw, qw = exact_quant_row([Fraction(float(v)) for v in wt[n]], normal)
+            low = sum(qx[j] * qw[j] for j in range(len(normal)))
+            high = sum(Fraction(float(x[m, k])) * Fraction(float(wt[n, k])) for k in O)
+            exact = Fraction(low) * sx * sw + high
+            assert r["acc_i"][m, n] == low
+            assert abs(r["y"][m, n] - float(exact)) <= 1e-12 * max(1.0, abs(float(exact)))
+
+
+# ----------------------------------------------------------------- storage formats
+def test_pack_layout_matches_definition():
+    rng = np.random.default_rng(1)
+    codes = rng.integers(-7, 8, size=(5, 37)).astype(np.int8)
+    packed = oracle.pack_int4(codes, 64)
+    for r in range(5):
+        expect = bytearray(64)
+        for j, c in enumerate(codes[r].tolist()):
+            nib = c & 0xF
+            expect[j // 2] |= nib if j % 2 == 0 else nib << 4
+        assert bytes(packed[r]) == bytes(expect)
+    # two's complement nibbles: 0x9 is -7, 0x8 (-8) never appears
+    lo = (packed & 0xF).astype(np.int16)
+    assert not np.any((lo == 8))
+
+
+def test_chan_table_definition():
+    K = 64
+    O = [0, 5, 7, 8, 31, 32, 63]
+    tab = oracle.chan_table(O, K)
+    for c in range(K // 8):
+        below = sum(1 for o in O if o < 8 * c)
+        mask = sum(1 << (o - 8 * c) for o in O if 8 * c <= o < 8 * c + 8)
+        assert int(tab[c]) == (below << 8) | mask
+
+
+def test_outlier_set_validation():
+    assert oracle.validate_outliers([1, 4, 9], 10)
+    assert oracle.validate_outliers([], 10)
+    assert not oracle.validate_outliers([4, 1], 10)
+    assert not oracle.validate_outliers([1, 1], 10)
+    assert not oracle.validate_outliers([10], 10)
+    assert not oracle.validate_outliers([-1], 10)
+    with pytest.raises(ValueError):
+        oracle.quantize_rows(np.zeros((1, 8), np.uint16), 8, [3, 2])
+
+
+# ----------------------------------------------------------------- method sanity
+def test_outlier_channels_reduce_error():
+    """Routing the true outlier channels through the 16-bit branch must cut the
+    error against the exact fp64 product (the point of the channel split)."""
+    w = workloads.TINY
+    O, X, W = workloads.make(w)
+    Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
+    exact = bits_to_f64(Xb) @ bits_to_f64(Wb).T
+    err = {}
+    for name, o in (("none", np.zeros(0, np.int32)), ("true", O.numpy())):
+        y = oracle.linear(Xb, Wb, o)["y"]
+        err[name] = np.linalg.norm(y - exact) / np.linalg.norm(exact)
+    assert err["true"] < 0.25 * err["none"]
+    assert err["true"] < 0.2
