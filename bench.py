@@ -1,0 +1,379 @@
+#!/usr/bin/env python
+"""Benchmark of the dual-path W4A4 + BF16 linear layer on B200.
+
+One step = one pass of the online hot path over one batch of tokens:
+quantize-and-gather of X (per-token scales, packed INT4 codes, compact bf16
+outlier channels) followed by the dual-path GEMM with its fused epilogue.
+The offline weight preparation is done once before timing.
+
+Default workload: the Llama-3-8B fused QKV projection shape
+(M=2048 tokens, K=4096, N=6144, |O|=256 outlier channels).
+
+Output: one JSON line on rank 0 (see the keys written in ``main``).
+  value        whole-job TOPS = 2*M*N*K per step (all MACs of both paths), device-timed
+  e2e          same metric through sq_linear with pinned host buffers, copies included
+  roofline     the GEMM kernel against the dense tensor roofline of its two paths
+  quant_gather the quantize-and-gather kernel against the HBM copy bandwidth
+  cpu_baseline the CPU oracle on a bounded sample of the same workload
+
+``--impl reference`` times the CPU oracle (the reference arm) instead.
+Multi-GPU: one process per GPU (torchrun); every rank runs its own batch of
+tokens against a replica of the layer (data parallel over tokens, no
+collective on the data path); value = all ranks' work / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import workloads  # noqa: E402
+
+DEFAULT_WORKLOAD = workloads.LLAMA8B_QKV.name
+METRIC = "dual-path W4A4+BF16 GEMM TOPS & % tensor peak; quant-gather HBM GB/s"
+INT8_PER_BF16 = 2.0   # nominal dense int8 : bf16 tensor rate on B200 (4.5 : 2.25 POPS)
+
+
+# ----------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "mixed_precision_gemm_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernels are unchanged since."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_hash") != source_hash():
+        return None
+    return d.get("workloads", {}).get(workload, {}).get(kernel)
+
+
+def gemm_bytes(M, N, K, nO):
+    KN = K - nO
+    return N * KN / 2 + 2 * N * nO + 4 * N + M * KN / 2 + 2 * M * nO + 4 * M + 2 * M * N
+
+
+def quant_gather_bytes(M, K, nO):
+    KN = K - nO
+    return 2 * M * K + M * KN / 2 + 2 * M * nO + 4 * M
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return None
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------- CPU oracle timing
+def time_oracle(w, O, X, W, target_s: float, max_rows: int | None = None):
+    """Time the oracle on a bounded sample of token rows (weights quantized beforehand,
+    as the offline step is on the GPU side).  Returns (TOPS, rows, seconds, cores)."""
+    import oracle
+    Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
+    O = O.numpy()
+    qw, sw, wo = oracle.quantize_rows(Wb, w.K, O)
+
+    def run(rows):
+        t0 = time.perf_counter()
+        qx, sx, xo = oracle.quantize_rows(Xb[:rows], w.K, O)
+        oracle.dual_linear_rows(qx, sx, xo, qw, sw, wo)
+        return time.perf_counter() - t0
+
+    probe = min(8, w.M)
+    t = run(probe)
+    rows = int(min(max_rows or w.M, w.M, max(probe, probe * target_s / max(t, 1e-6))))
+    t = run(rows)
+    return 2.0 * rows * w.N * w.K / t / 1e12, rows, t, oracle.num_threads()
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(args, w, rank, world):
+    if rank != 0:
+        return 0
+    O, X, W = workloads.make(w)
+    import oracle
+    Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
+    On = O.numpy()
+    qw, sw, wo = oracle.quantize_rows(Wb, w.K, On)
+    rows = args.ref_rows
+
+    def step():
+        qx, sx, xo = oracle.quantize_rows(Xb[:rows], w.K, On)
+        oracle.dual_linear_rows(qx, sx, xo, qw, sw, wo)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / args.steps
+    tops = 2.0 * rows * w.N * w.K / dt / 1e12
+    sample = f"{rows} token rows of the workload per step (weights quantized before timing)"
+    line = {"impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64", "data": "synthetic",
+            "config": w.describe(),
+            "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="sq", choices=["sq", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-rows", type=int, default=8, help="token rows per reference-arm step")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = workloads.CONFIGS[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, w, rank, world)
+
+    import torch.distributed as dist
+    import mixed_precision_gemm_b200 as sq
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = load_peaks()
+    O, X, W = workloads.make(w)
+    M, N, K, nO = w.M, w.N, w.K, w.nO
+    kn_pad, no_pad = sq.sq_kn_pad(K, nO), sq.sq_no_pad(nO)
+
+    # Rotating input sets so that every step reads operands that are not L2-resident.
+    Xd = X.to(dev)
+    pw0 = sq.prepare_weights(W.to(dev), O)
+    foot = (2 * M * K + pw0.W_N.numel() + 2 * pw0.W_O.numel() + 4 * N + 2 * M * N
+            + sq.sq_linear_workspace_bytes(M, K, nO))
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    n_sets = max(2, math.ceil(3 * l2 / foot))
+    sets = []
+    for i in range(n_sets):
+        pw = pw0 if i == 0 else sq.PreparedWeights(N, K, nO, pw0.W_N.clone(), pw0.s_w.clone(), pw0.W_O.clone(),
+                                                      pw0.chan_tab.clone())
+        sets.append({
+            "X": Xd if i == 0 else Xd.clone(), "pw": pw,
+            "X_N": torch.empty(M, kn_pad // 2, dtype=torch.uint8, device=dev),
+            "s_x": torch.empty(M, dtype=torch.float32, device=dev),
+            "X_O": torch.empty(M, no_pad, dtype=torch.bfloat16, device=dev),
+            "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+        })
+    stream = torch.cuda.current_stream(dev)
+
+    def step(s, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sq.sq_quant_gather(s["X"], s["pw"].chan_tab, nO, s["X_N"], s["s_x"], s["X_O"], stream)
+        if ev is not None:
+            ev[1].record(stream)
+        pw = s["pw"]
+        sq.sq_gemm(s["X_N"], s["s_x"], s["X_O"], pw.W_N, pw.s_w, pw.W_O, M, N, K, nO, s["Y"], None, None, stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for i in range(args.warmup):
+        step(sets[i % n_sets])
+    torch.cuda.synchronize(dev)
+    sq.sq_check(stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev.index if dev.index is not None else 0) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(sets[i % n_sets], evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    sq.sq_check(stream)
+    ms_step = max_over_ranks(t_start.elapsed_time(t_end) / args.steps)
+    ms_qg = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    ms_gemm = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    clocks = clk.summary()
+
+    flops = 2.0 * M * N * K
+    value = world * flops / (ms_step * 1e-3) / 1e12
+
+    # roofline of the GEMM: int8 path at 2x the bf16 peak, bf16 path at the bf16 peak (burst: timed alone)
+    p_bf = peaks["bf16_tflops"]
+    p_i8 = INT8_PER_BF16 * p_bf
+    t_roof_s = (2.0 * M * N * (K - nO)) / (p_i8 * 1e12) + (2.0 * M * N * nO) / (p_bf * 1e12)
+    peak_eff = flops / t_roof_s / 1e12
+    gemm_tops = flops / (ms_gemm * 1e-3) / 1e12
+    qg_bytes = quant_gather_bytes(M, K, nO)
+    qg_gbs = qg_bytes / (ms_qg * 1e-3) / 1e9
+
+    # end to end through sq_linear with pinned host buffers (copies inside the timed region)
+    X_host = X.pin_memory()
+    Y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    e2e_sets = sets[:2]
+    ws = [torch.empty(sq.sq_linear_workspace_bytes(M, K, nO), dtype=torch.uint8, device=dev) for _ in e2e_sets]
+
+    def e2e_step(i):
+        s = e2e_sets[i % len(e2e_sets)]
+        s["X"].copy_(X_host, non_blocking=True)
+        pw = s["pw"]
+        sq.sq_linear(s["X"], pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, N, nO, s["Y"], ws[i % len(ws)], stream)
+        Y_host.copy_(s["Y"], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    sq.sq_check(stream)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+    e2e_value = world * flops / (ms_e2e * 1e-3) / 1e12
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tops, rows, secs, cores = time_oracle(w, O, X, W, args.cpu_seconds)
+        cpu = {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle",
+               "sample": f"{rows} of {M} token rows x all {N} outputs ({secs:.1f} s; weights quantized beforehand)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "s4*s4->s32 + bf16*bf16->f32", "data": "synthetic",
+            "config": {**w.describe(), "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": f"{n_sets} rotating input sets of {foot / 1e6:.0f} MB (> L2 {l2 / 1e6:.0f} MB)"},
+            "roofline": {"bound": "tensor", "achieved": gemm_tops, "peak": peak_eff, "unit": "TFLOP/s",
+                         "frac": gemm_tops / peak_eff, "traffic": recorded_traffic(w.name, "dual_gemm"),
+                         "kernel": "dual_gemm_kernel", "ms": ms_gemm,
+                         "peak_basis": f"{peaks['source']} bf16 {p_bf:.0f} TFLOP/s (burst), int8 = {INT8_PER_BF16:g}x",
+                         "algorithmic_bytes": gemm_bytes(M, N, K, nO)},
+            "quant_gather": {"bound": "hbm", "achieved": qg_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": qg_gbs / peaks["hbm_gbs"], "ms": ms_qg, "algorithmic_bytes": qg_bytes,
+                             "traffic": recorded_traffic(w.name, "rowquant")},
+            "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": 2 * M * K,
+                    "d2h_bytes_per_step": 2 * M * N, "ms_per_step": ms_e2e},
+            "cpu_baseline": cpu,
+            "clocks": clocks,
+            "gpu_launches": 2 * args.steps,
+        }
+        print(json.dumps(line), flush=True)
+
+    for s in sets:
+        s.clear()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,172 @@
+/*
+ * sq.h -- C ABI of the dual-path sparse-quantized linear layer on B200 (sm_100a).
+ *
+ *   Y[m,n] = s_x[m] * s_w[n] * sum_{k not in O} q4(X)[m,k] * q4(W)[n,k]
+ *          +                   sum_{k in O}     X[m,k]    * W[n,k]
+ *
+ * The layer follows two pages:
+ *   - OSC: Hardware Efficient W4A4 Quantization via Outlier Separation in
+ *     Channel Dimension (arXiv:2604.12782), abstract and technical framework:
+ *     an offline step fixes the outlier channels O; online, the scattered
+ *     outlier channels are coalesced into a compact dense tensor for a 16-bit
+ *     branch GEMM while all other channels take a 4-bit GEMM; the two results
+ *     are fused.
+ *   - SQ-format (arXiv:2512.05409) write-up, section 9: symmetric quantization
+ *     of the low-precision part (INT4 codes in [-7, 7]) and reordering of the
+ *     weight columns by the static mask; section 5: the static mask is chosen
+ *     offline so no runtime top-k is needed.
+ *
+ * Scales: one fp32 scale per token row of X (computed online by
+ * sq_quant_gather) and one per output channel of W (computed offline by
+ * sq_prepare_weights): s = max_{k not in O} |x_k| / 7 (IEEE fp32 division),
+ * code = clamp(rint(x / s), -7, 7) with the fp32 quotient, ties to even;
+ * a row whose normal channels are all zero gets s = 0 and zero codes.
+ *
+ * Conventions for every call
+ *   - Memory: every buffer is allocated by the caller.  The library keeps
+ *     only a per-device error word; it never allocates device memory.
+ *   - Pointers named "dev" are device pointers, "host" host pointers.  All
+ *     device pointers must be 16-byte aligned (SQ_ERR_MISALIGNED otherwise).
+ *   - Matrices are row-major.  bf16 buffers are passed as void* holding IEEE
+ *     bfloat16 bit patterns (uint16).
+ *   - Asynchrony: calls enqueue work on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and return without waiting, except
+ *     sq_prepare_weights, which waits for its own work (it is an offline step).
+ *     Argument errors are returned before anything is enqueued.
+ *   - Errors: SQ_ERR_INVALID_ARG / SQ_ERR_MISALIGNED / SQ_ERR_UNSUPPORTED are
+ *     returned synchronously; SQ_ERR_CUDA reports a failed launch or copy.
+ *     A kernel whose bounded wait ran out records it in the device error word
+ *     and exits cleanly; sq_check() reports it as SQ_ERR_TIMEOUT.
+ *     sq_last_error_detail() returns a text for the last failing call on the
+ *     calling thread.
+ *
+ * Storage formats (all produced by this library, all zero-padded; padding is
+ * exact because zero codes and zero bf16 values add nothing):
+ *   - KN = K - nO normal channels, ascending channel order; kn_pad = sq_kn_pad.
+ *   - Packed INT4 part, [rows, kn_pad/2] bytes: byte j holds code 2j in its
+ *     low nibble and code 2j+1 in its high nibble, 4-bit two's complement;
+ *     code -8 is never produced.
+ *   - Compact outlier part, [rows, no_pad] bf16: column j is channel O[j].
+ *   - Channel table, [K/8] uint32 ("static mask"): word c holds
+ *     (number of channels of O below 8c) << 8 | (bit e set when channel
+ *     8c+e is in O).
+ */
+#ifndef SQ_B200_H
+#define SQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *sq_stream_t;
+
+typedef enum {
+    SQ_OK = 0,
+    SQ_ERR_INVALID_ARG = 1,  /* a size, a stride or the outlier set is invalid */
+    SQ_ERR_UNSUPPORTED = 2,  /* no sm_100 device, or a size beyond the limits below */
+    SQ_ERR_MISALIGNED = 3,   /* a device pointer is not 16-byte aligned */
+    SQ_ERR_CUDA = 4,         /* a CUDA launch or copy failed */
+    SQ_ERR_TIMEOUT = 5       /* a kernel's bounded wait ran out (see sq_check) */
+} sq_status;
+
+/* Limits: 8 <= K <= 65536, K % 8 == 0, 0 <= nO <= K, N % 8 == 0, M >= 0. */
+#define SQ_MAX_K 65536
+
+const char *sq_status_string(sq_status status);
+const char *sq_last_error_detail(void);
+
+/* Layout queries (pure functions, no device access). */
+int64_t sq_kn_pad(int64_t K, int64_t nO);            /* roundup(K - nO, 128) codes   */
+int64_t sq_no_pad(int64_t nO);                       /* roundup(nO, 64) bf16 columns */
+int64_t sq_chan_table_words(int64_t K);              /* K / 8                        */
+/* Bytes of the sq_linear workspace: packed X part, s_x and compact X_O, each
+ * 256-byte aligned. */
+size_t sq_linear_workspace_bytes(int64_t M, int64_t K, int64_t nO);
+
+/*
+ * Offline step (SQ-format write-up sections 5 and 9; OSC "offline grouping"):
+ * from the outlier channel list and the bf16 weights, build the static
+ * channel table and the weight operands of both paths.
+ *
+ *   W        dev  bf16 [N, ldw]     weights, one row per output channel
+ *   O        host int32 [nO]        strictly increasing channels in [0, K)
+ *   W_N      dev  u8   [N, kn_pad/2] packed INT4 codes of the normal channels
+ *   s_w      dev  f32  [N]          per-output-channel scales
+ *   W_O      dev  bf16 [N, no_pad]  compact outlier columns (may be NULL if nO == 0)
+ *   chan_tab dev  u32  [K/8]        static channel table
+ * Waits for the stream before returning (the table is copied from host memory).
+ */
+sq_status sq_prepare_weights(const void *W, int64_t N, int64_t K, int64_t ldw,
+                             const int32_t *O, int64_t nO,
+                             void *W_N, float *s_w, void *W_O, uint32_t *chan_tab,
+                             sq_stream_t stream);
+
+/*
+ * Online quantize-and-gather of the activations (OSC technical framework:
+ * "structured sub-tensor extraction" of the outlier channels into a compact
+ * dense tensor; the rest quantized to INT4 with a per-token scale).  One pass
+ * over X; memory-bound.
+ *
+ *   X        dev bf16 [M, ldx]       activations, ldx >= K, ldx % 8 == 0
+ *   chan_tab dev u32  [K/8]          from sq_prepare_weights
+ *   X_N      dev u8   [M, kn_pad/2]  packed INT4 codes (may be NULL if kn_pad == 0)
+ *   s_x      dev f32  [M]            per-token scales
+ *   X_O      dev bf16 [M, no_pad]    compact outlier channels (may be NULL if nO == 0)
+ */
+sq_status sq_quant_gather(const void *X, int64_t M, int64_t K, int64_t ldx,
+                          const uint32_t *chan_tab, int64_t nO,
+                          void *X_N, float *s_x, void *X_O, sq_stream_t stream);
+
+/*
+ * Dual-path GEMM with fused epilogue (OSC abstract: 4-bit GEMM path plus a
+ * 16-bit branch GEMM, results fused):
+ *   acc_i[m,n] = sum_j codeX[m,j] * codeW[n,j]         (exact, int32)
+ *   acc_f[m,n] = sum_j X_O[m,j] * W_O[n,j]             (fp32 accumulate)
+ *   Y[m,n]     = bf16_rn( (float)acc_i * s_x[m] * s_w[n] + acc_f )
+ *
+ *   Y            dev bf16 [M, ldy]   ldy >= N, ldy % 8 == 0
+ *   dbg_acc_i32  dev i32  [M, N]     optional (NULL): the exact integer sums
+ *   dbg_acc_f32  dev f32  [M, N]     optional (NULL): the 16-bit branch sums
+ * Other operands as produced by the two calls above.
+ */
+sq_status sq_gemm(const void *X_N, const float *s_x, const void *X_O,
+                  const void *W_N, const float *s_w, const void *W_O,
+                  int64_t M, int64_t N, int64_t K, int64_t nO,
+                  void *Y, int64_t ldy,
+                  int32_t *dbg_acc_i32, float *dbg_acc_f32, sq_stream_t stream);
+
+/*
+ * The whole online layer: sq_quant_gather into `workspace`, then sq_gemm,
+ * both on `stream`.  workspace: dev, ws_bytes >= sq_linear_workspace_bytes.
+ */
+sq_status sq_linear(const void *X, int64_t M, int64_t K, int64_t ldx,
+                    const uint32_t *chan_tab,
+                    const void *W_N, const float *s_w, const void *W_O,
+                    int64_t N, int64_t nO, void *Y, int64_t ldy,
+                    void *workspace, size_t ws_bytes, sq_stream_t stream);
+
+/*
+ * Waits for `stream`, then reports (and clears) the device error word of the
+ * current device: SQ_ERR_TIMEOUT if a kernel's bounded wait ran out,
+ * SQ_ERR_CUDA on a pending CUDA error, SQ_OK otherwise.
+ */
+sq_status sq_check(sq_stream_t stream);
+
+/*
+ * Failure-detection self test: launches one single-thread kernel that waits
+ * on a barrier nothing will ever complete, with a bounded wait of about
+ * `timeout_ms` milliseconds (1..10000).  The kernel records the timeout in
+ * the device error word and exits; sq_check() then returns SQ_ERR_TIMEOUT
+ * and the context stays usable.
+ */
+sq_status sq_selftest_watchdog(int timeout_ms, sq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SQ_B200_H */

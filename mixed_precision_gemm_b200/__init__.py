@@ -1,0 +1,288 @@
+"""Dual-path sparse-quantized linear layer on B200 (sm_100a).
+
+    Y = s_x[m] * s_w[n] * sum_{k not in O} q4(X)[m,k] * q4(W)[n,k]  +  sum_{k in O} X[m,k] * W[n,k]
+
+A thin Python binding of the C ABI in ``include/sq.h`` (library
+``libsq_b200.so``, built from ``csrc/``).  Every step of the layer runs in the
+library's CUDA kernels; this module only checks tensor metadata, marshals
+pointers and sizes, and allocates buffers with torch.  There is no CPU
+fallback: if the library is missing the calls raise.
+
+The ABI calls keep their C names (``sq_prepare_weights``, ``sq_quant_gather``,
+``sq_gemm``, ``sq_linear``, ...).  ``prepare_weights`` / ``SQLinear`` are
+small conveniences that allocate the buffers and call them.
+
+Method: OSC (arXiv:2604.12782, abstract and technical framework) -- static
+outlier channels coalesced into a compact bf16 tensor for a 16-bit branch
+GEMM, all other channels through a 4-bit GEMM, results fused; SQ-format
+write-up of arXiv:2512.05409, sections 5 and 9 -- static mask chosen offline,
+symmetric quantization, weight columns reordered by the mask.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import re
+from typing import Optional, Sequence
+
+import torch
+
+from . import _build
+
+__all__ = [
+    "SQError", "load", "library_path", "header_functions",
+    "sq_status_string", "sq_kn_pad", "sq_no_pad", "sq_chan_table_words", "sq_linear_workspace_bytes",
+    "sq_prepare_weights", "sq_quant_gather", "sq_gemm", "sq_linear", "sq_check", "sq_selftest_watchdog",
+    "PreparedWeights", "prepare_weights", "quant_gather", "gemm", "SQLinear",
+]
+
+SQ_OK = 0
+SQ_ERR_INVALID_ARG = 1
+SQ_ERR_UNSUPPORTED = 2
+SQ_ERR_MISALIGNED = 3
+SQ_ERR_CUDA = 4
+SQ_ERR_TIMEOUT = 5
+
+HEADER = os.path.join(_build.ROOT, "include", "sq.h")
+
+
+class SQError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS_NAMES.get(status, status)}: {detail}")
+
+
+_STATUS_NAMES = {0: "SQ_OK", 1: "SQ_ERR_INVALID_ARG", 2: "SQ_ERR_UNSUPPORTED",
+                 3: "SQ_ERR_MISALIGNED", 4: "SQ_ERR_CUDA", 5: "SQ_ERR_TIMEOUT"}
+
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB_PATH
+
+
+def load():
+    """Load libsq_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = _build.LIB_PATH
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"CUDA library {path} is missing; build it with "
+            "`python -m mixed_precision_gemm_b200._build` (or __graft_entry__.build())")
+    lib = ctypes.CDLL(path)
+    P, I, Z, F = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_int
+    lib.sq_status_string.argtypes = [F]
+    lib.sq_status_string.restype = ctypes.c_char_p
+    lib.sq_last_error_detail.argtypes = []
+    lib.sq_last_error_detail.restype = ctypes.c_char_p
+    lib.sq_kn_pad.argtypes = [I, I]
+    lib.sq_kn_pad.restype = I
+    lib.sq_no_pad.argtypes = [I]
+    lib.sq_no_pad.restype = I
+    lib.sq_chan_table_words.argtypes = [I]
+    lib.sq_chan_table_words.restype = I
+    lib.sq_linear_workspace_bytes.argtypes = [I, I, I]
+    lib.sq_linear_workspace_bytes.restype = Z
+    lib.sq_prepare_weights.argtypes = [P, I, I, I, P, I, P, P, P, P, P]
+    lib.sq_quant_gather.argtypes = [P, I, I, I, P, I, P, P, P, P]
+    lib.sq_gemm.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P, P, P]
+    lib.sq_linear.argtypes = [P, I, I, I, P, P, P, P, I, I, P, I, P, Z, P]
+    lib.sq_check.argtypes = [P]
+    lib.sq_selftest_watchdog.argtypes = [F, P]
+    for f in (lib.sq_prepare_weights, lib.sq_quant_gather, lib.sq_gemm, lib.sq_linear, lib.sq_check,
+              lib.sq_selftest_watchdog):
+        f.restype = F
+    _lib = lib
+    return lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions include/sq.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sq_[a-z0-9_]+)\s*\(", text)))
+
+
+def _raise(st: int, where: str):
+    if st != SQ_OK:
+        detail = load().sq_last_error_detail().decode(errors="replace")
+        raise SQError(st, where, detail)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None or t.numel() == 0:
+        return None
+    if not t.is_cuda:
+        raise ValueError("device tensor expected")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _rowmajor(t: torch.Tensor, name: str, dtype=None):
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name}: expected a 2-D row-major tensor (unit inner stride)")
+    return t
+
+
+# ----------------------------------------------------------------- pure queries
+def sq_status_string(st: int) -> str:
+    return load().sq_status_string(st).decode()
+
+
+def sq_kn_pad(K: int, nO: int) -> int:
+    return int(load().sq_kn_pad(K, nO))
+
+
+def sq_no_pad(nO: int) -> int:
+    return int(load().sq_no_pad(nO))
+
+
+def sq_chan_table_words(K: int) -> int:
+    return int(load().sq_chan_table_words(K))
+
+
+def sq_linear_workspace_bytes(M: int, K: int, nO: int) -> int:
+    return int(load().sq_linear_workspace_bytes(M, K, nO))
+
+
+# ----------------------------------------------------------------- ABI calls
+def sq_prepare_weights(W: torch.Tensor, O, W_N: torch.Tensor, s_w: torch.Tensor, W_O: Optional[torch.Tensor],
+                       chan_tab: torch.Tensor, stream=None) -> None:
+    """Offline weight step: static channel table + both weight operands (waits for the stream)."""
+    _rowmajor(W, "W", torch.bfloat16)
+    N, K = W.shape
+    O_host = torch.as_tensor(O, dtype=torch.int32).reshape(-1).contiguous().cpu()
+    nO = O_host.numel()
+    st = load().sq_prepare_weights(_ptr(W), N, K, W.stride(0),
+                                   ctypes.c_void_p(O_host.data_ptr()) if nO else None, nO,
+                                   _ptr(W_N), _ptr(s_w), _ptr(W_O), _ptr(chan_tab), _stream(stream))
+    _raise(st, "sq_prepare_weights")
+
+
+def sq_quant_gather(X: torch.Tensor, chan_tab: torch.Tensor, nO: int, X_N: Optional[torch.Tensor],
+                    s_x: torch.Tensor, X_O: Optional[torch.Tensor], stream=None) -> None:
+    _rowmajor(X, "X", torch.bfloat16)
+    M, K = X.shape
+    st = load().sq_quant_gather(_ptr(X), M, K, X.stride(0), _ptr(chan_tab), nO, _ptr(X_N), _ptr(s_x), _ptr(X_O),
+                                _stream(stream))
+    _raise(st, "sq_quant_gather")
+
+
+def sq_gemm(X_N, s_x, X_O, W_N, s_w, W_O, M: int, N: int, K: int, nO: int, Y: torch.Tensor,
+            dbg_acc_i32: Optional[torch.Tensor] = None, dbg_acc_f32: Optional[torch.Tensor] = None,
+            stream=None) -> None:
+    _rowmajor(Y, "Y", torch.bfloat16)
+    st = load().sq_gemm(_ptr(X_N), _ptr(s_x), _ptr(X_O), _ptr(W_N), _ptr(s_w), _ptr(W_O), M, N, K, nO,
+                        _ptr(Y), Y.stride(0), _ptr(dbg_acc_i32), _ptr(dbg_acc_f32), _stream(stream))
+    _raise(st, "sq_gemm")
+
+
+def sq_linear(X: torch.Tensor, chan_tab: torch.Tensor, W_N, s_w, W_O, N: int, nO: int, Y: torch.Tensor,
+              workspace: torch.Tensor, stream=None) -> None:
+    _rowmajor(X, "X", torch.bfloat16)
+    _rowmajor(Y, "Y", torch.bfloat16)
+    M, K = X.shape
+    st = load().sq_linear(_ptr(X), M, K, X.stride(0), _ptr(chan_tab), _ptr(W_N), _ptr(s_w), _ptr(W_O), N, nO,
+                          _ptr(Y), Y.stride(0), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                          _stream(stream))
+    _raise(st, "sq_linear")
+
+
+def sq_check(stream=None) -> None:
+    _raise(load().sq_check(_stream(stream)), "sq_check")
+
+
+def sq_selftest_watchdog(timeout_ms: int, stream=None) -> None:
+    _raise(load().sq_selftest_watchdog(timeout_ms, _stream(stream)), "sq_selftest_watchdog")
+
+
+# ----------------------------------------------------------------- conveniences
+@dataclasses.dataclass
+class PreparedWeights:
+    """Offline artefacts of one layer: the static channel table and both weight operands."""
+    N: int
+    K: int
+    nO: int
+    W_N: torch.Tensor        # uint8 [N, kn_pad/2]
+    s_w: torch.Tensor        # float32 [N]
+    W_O: torch.Tensor        # bf16 [N, no_pad]
+    chan_tab: torch.Tensor   # int32 view of uint32 [K/8]
+
+    def state_dict(self) -> dict:
+        return {"N": self.N, "K": self.K, "nO": self.nO, "W_N": self.W_N, "s_w": self.s_w,
+                "W_O": self.W_O, "chan_tab": self.chan_tab}
+
+    @classmethod
+    def from_state_dict(cls, d: dict, device=None) -> "PreparedWeights":
+        mv = (lambda t: t.to(device)) if device is not None else (lambda t: t)
+        return cls(int(d["N"]), int(d["K"]), int(d["nO"]), mv(d["W_N"]), mv(d["s_w"]), mv(d["W_O"]),
+                   mv(d["chan_tab"]))
+
+
+def prepare_weights(W: torch.Tensor, O: Sequence[int], stream=None) -> PreparedWeights:
+    N, K = W.shape
+    nO = len(torch.as_tensor(O).reshape(-1))
+    dev = W.device
+    W_N = torch.zeros(N, sq_kn_pad(K, nO) // 2, dtype=torch.uint8, device=dev)
+    s_w = torch.zeros(N, dtype=torch.float32, device=dev)
+    W_O = torch.zeros(N, sq_no_pad(nO), dtype=torch.bfloat16, device=dev)
+    tab = torch.zeros(sq_chan_table_words(K), dtype=torch.int32, device=dev)
+    sq_prepare_weights(W, O, W_N, s_w, W_O, tab, stream)
+    return PreparedWeights(N, K, nO, W_N, s_w, W_O, tab)
+
+
+def quant_gather(X: torch.Tensor, pw: PreparedWeights, stream=None):
+    M, K = X.shape
+    dev = X.device
+    X_N = torch.empty(M, sq_kn_pad(K, pw.nO) // 2, dtype=torch.uint8, device=dev)
+    s_x = torch.empty(M, dtype=torch.float32, device=dev)
+    X_O = torch.empty(M, sq_no_pad(pw.nO), dtype=torch.bfloat16, device=dev)
+    sq_quant_gather(X, pw.chan_tab, pw.nO, X_N, s_x, X_O, stream)
+    return X_N, s_x, X_O
+
+
+def gemm(X_N, s_x, X_O, pw: PreparedWeights, Y: Optional[torch.Tensor] = None, debug: bool = False, stream=None):
+    M = s_x.shape[0]
+    if Y is None:
+        Y = torch.empty(M, pw.N, dtype=torch.bfloat16, device=s_x.device)
+    dbg_i = dbg_f = None
+    if debug:
+        dbg_i = torch.empty(M, pw.N, dtype=torch.int32, device=s_x.device)
+        dbg_f = torch.empty(M, pw.N, dtype=torch.float32, device=s_x.device)
+    sq_gemm(X_N, s_x, X_O, pw.W_N, pw.s_w, pw.W_O, M, pw.N, pw.K, pw.nO, Y, dbg_i, dbg_f, stream)
+    return (Y, dbg_i, dbg_f) if debug else Y
+
+
+class SQLinear:
+    """A prepared dual-path linear layer: ``y = layer(x)`` for bf16 x [M, K] on the GPU."""
+
+    def __init__(self, W: torch.Tensor, O: Sequence[int], stream=None):
+        self.weights = prepare_weights(W, O, stream)
+        self._ws = None
+
+    def workspace(self, M: int, device) -> torch.Tensor:
+        need = sq_linear_workspace_bytes(M, self.weights.K, self.weights.nO)
+        if self._ws is None or self._ws.numel() < need or self._ws.device != torch.device(device):
+            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+        return self._ws
+
+    def __call__(self, X: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        pw = self.weights
+        M = X.shape[0]
+        if out is None:
+            out = torch.empty(M, pw.N, dtype=torch.bfloat16, device=X.device)
+        sq_linear(X, pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, pw.N, pw.nO, out, self.workspace(M, X.device), stream)
+        return out

@@ -1,0 +1,453 @@
+// C ABI of the dual-path sparse-quantized linear layer (declared in include/sq.h).
+//
+// Host side only: argument validation, layout arithmetic, TMA tensor-map
+// encoding and kernel launches.  Every kernel lives in the .cuh files included
+// below so that the whole library is one translation unit (one device error
+// word per device).
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/sq.h"
+#include "sq_device.cuh"
+#include "sq_gemm.cuh"
+#include "sq_rowquant.cuh"
+
+namespace {
+
+thread_local std::string g_detail;
+
+sq_status fail(sq_status st, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_detail = buf;
+    return st;
+}
+
+sq_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(SQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+constexpr int kMaxDevices = 64;
+
+struct DevInfo {
+    bool ready = false;
+    bool sm100 = false;
+    int sms = 0;
+};
+
+DevInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+sq_status device_info(DevInfo &out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(SQ_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DevInfo &d = g_dev[dev];
+    if (!d.ready) {
+        int major = 0, sms = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return cuda_fail(e, "cudaDeviceGetAttribute");
+        d.sm100 = (major == 10);
+        d.sms = sms;
+        d.ready = true;
+    }
+    out = d;
+    if (!out.sm100) return fail(SQ_ERR_UNSUPPORTED, "this library needs an sm_100 (B200-class) device");
+    return SQ_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+sq_status get_encode(PFN_cuTensorMapEncodeTiled_v12000 &fn)
+{
+    std::call_once(g_encode_once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    fn = g_encode;
+    if (!fn) return fail(SQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    return SQ_OK;
+}
+
+// 2-D row-major tensor: `inner` elements per row (contiguous), `outer` rows,
+// rows `row_bytes` apart; box of box_inner x box_outer elements.
+sq_status make_map(CUtensorMap &map, const void *base, CUtensorMapDataType dt, uint64_t inner,
+                   uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                   CUtensorMapSwizzle swz)
+{
+    PFN_cuTensorMapEncodeTiled_v12000 enc;
+    sq_status st = get_encode(enc);
+    if (st != SQ_OK) return st;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return SQ_OK;
+}
+
+// ---------------------------------------------------------------- row quantizer
+template <int T, int CPT>
+sq_status launch_rowquant_t(const DevInfo &di, const uint16_t *src, int64_t rows, int K, int64_t ld,
+                            const uint32_t *tab, int nO, int kn_pad, int no_pad, uint8_t *dn, float *ds,
+                            uint16_t *dout, cudaStream_t stream)
+{
+    auto kern = sqq::rowquant_kernel<T, CPT>;
+    const size_t smem = static_cast<size_t>(kn_pad) + 2u * static_cast<size_t>(no_pad);
+    cudaError_t e;
+    if (smem > 48 * 1024) {
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))) !=
+            cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute(rowquant)");
+    }
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, T, smem)) != cudaSuccess)
+        return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+    if (per_sm < 1) per_sm = 1;
+    const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * di.sms);
+    kern<<<static_cast<unsigned>(grid), T, smem, stream>>>(src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds, dout);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "rowquant launch");
+    return SQ_OK;
+}
+
+sq_status launch_rowquant(const uint16_t *src, int64_t rows, int64_t K, int64_t ld, const uint32_t *tab,
+                          int64_t nO, uint8_t *dn, float *ds, uint16_t *dout, cudaStream_t stream)
+{
+    if (rows == 0) return SQ_OK;
+    DevInfo di;
+    sq_status st = device_info(di);
+    if (st != SQ_OK) return st;
+    const int kn_pad = static_cast<int>(sq_kn_pad(K, nO));
+    const int no_pad = static_cast<int>(sq_no_pad(nO));
+    const int64_t nchunk = K / 8;
+    const int k = static_cast<int>(K), no = static_cast<int>(nO);
+    if (nchunk <= 256) return launch_rowquant_t<256, 1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 512) return launch_rowquant_t<256, 2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 1024) return launch_rowquant_t<256, 4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 2048) return launch_rowquant_t<256, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 4096) return launch_rowquant_t<512, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    return launch_rowquant_t<1024, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+}
+
+// ---------------------------------------------------------------- GEMM
+template <class C>
+sq_status launch_gemm_t(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
+                        const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
+                        int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+{
+    const int64_t kn_pad = sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
+    CUtensorMap m_xn{}, m_wn{}, m_xo{}, m_wo{};
+    sq_status st;
+    if (kn_pad > 0) {
+        if ((st = make_map(m_xn, X_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, M, kn_pad / 2, sqg::PROWB, sqg::BM,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
+            return st;
+        if ((st = make_map(m_wn, W_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, N, kn_pad / 2, sqg::PROWB, C::BN,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
+            return st;
+    }
+    if (no_pad > 0) {
+        if ((st = make_map(m_xo, X_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, M, no_pad * 2, sqg::KB_BF, sqg::BM,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
+            return st;
+        if ((st = make_map(m_wo, W_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, N, no_pad * 2, sqg::KB_BF, C::BN,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
+            return st;
+    }
+    sqg::GemmArgs a;
+    a.s_x = s_x;
+    a.s_w = s_w;
+    a.Y = static_cast<uint16_t *>(Y);
+    a.dbg_i = dbg_i;
+    a.dbg_f = dbg_f;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.ldy = ldy;
+    a.nkb_i = static_cast<int>(kn_pad / sqg::KB_I8);
+    a.nkb_o = static_cast<int>(no_pad / sqg::KB_BF);
+    a.tiles_m = static_cast<int>((M + sqg::BM - 1) / sqg::BM);
+    a.tiles_n = static_cast<int>((N + C::BN - 1) / C::BN);
+    a.group_m = 8;
+    const int64_t ntiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
+    const bool dbg = dbg_i || dbg_f;
+    auto kern = dbg ? sqg::dual_gemm_kernel<C, true> : sqg::dual_gemm_kernel<C, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
+    kern<<<static_cast<unsigned>(ntiles), sqg::NUM_THREADS, C::SMEM_BYTES, stream>>>(m_xn, m_wn, m_xo, m_wo, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "gemm launch");
+    return SQ_OK;
+}
+
+using CfgN256 = sqg::Cfg<256, 3, 2>;
+using CfgN128 = sqg::Cfg<128, 4, 3>;
+using CfgN64 = sqg::Cfg<64, 4, 3>;
+
+sq_status gemm_impl(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
+                    const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
+                    int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+{
+    if (M == 0 || N == 0) return SQ_OK;
+    DevInfo di;
+    sq_status st = device_info(di);
+    if (st != SQ_OK) return st;
+    const int64_t tiles_m = (M + sqg::BM - 1) / sqg::BM;
+    if (tiles_m * ((N + 255) / 256) >= 2 * di.sms)
+        return launch_gemm_t<CfgN256>(X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    if (tiles_m * ((N + 127) / 128) >= di.sms)
+        return launch_gemm_t<CfgN128>(X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    return launch_gemm_t<CfgN64>(X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+}
+
+// ---------------------------------------------------------------- validation
+sq_status check_K_nO(int64_t K, int64_t nO)
+{
+    if (K < 8 || K > SQ_MAX_K || K % 8 != 0)
+        return fail(SQ_ERR_INVALID_ARG, "K=%lld must be a multiple of 8 in [8, %d]", (long long)K, SQ_MAX_K);
+    if (nO < 0 || nO > K) return fail(SQ_ERR_INVALID_ARG, "nO=%lld must lie in [0, K]", (long long)nO);
+    return SQ_OK;
+}
+
+sq_status check_ptr(const void *p, bool needed, const char *name)
+{
+    if (!needed) return SQ_OK;
+    if (!p) return fail(SQ_ERR_INVALID_ARG, "%s is NULL", name);
+    if (!aligned16(p)) return fail(SQ_ERR_MISALIGNED, "%s is not 16-byte aligned", name);
+    return SQ_OK;
+}
+
+#define SQ_TRY(expr)                 \
+    do {                             \
+        sq_status st_ = (expr);      \
+        if (st_ != SQ_OK) return st_; \
+    } while (0)
+
+sq_status quant_gather_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, int64_t nO,
+                            void *X_N, float *s_x, void *X_O, cudaStream_t stream)
+{
+    SQ_TRY(check_K_nO(K, nO));
+    if (M < 0) return fail(SQ_ERR_INVALID_ARG, "M < 0");
+    if (ldx < K || ldx % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldx must be >= K and a multiple of 8");
+    if (M == 0) return SQ_OK;
+    const int64_t kn_pad = sq_kn_pad(K, nO);
+    SQ_TRY(check_ptr(X, true, "X"));
+    SQ_TRY(check_ptr(chan_tab, true, "chan_tab"));
+    SQ_TRY(check_ptr(X_N, kn_pad > 0, "X_N"));
+    SQ_TRY(check_ptr(s_x, true, "s_x"));
+    SQ_TRY(check_ptr(X_O, nO > 0, "X_O"));
+    return launch_rowquant(static_cast<const uint16_t *>(X), M, K, ldx, chan_tab, nO, static_cast<uint8_t *>(X_N), s_x,
+                           static_cast<uint16_t *>(X_O), stream);
+}
+
+sq_status gemm_checked(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
+                       const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
+                       int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+{
+    SQ_TRY(check_K_nO(K, nO));
+    if (M < 0 || M > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "M out of range");
+    if (N < 0 || N % 8 != 0 || N > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "N must be a non-negative multiple of 8");
+    if (ldy < N || ldy % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldy must be >= N and a multiple of 8");
+    if (M == 0 || N == 0) return SQ_OK;
+    const int64_t kn_pad = sq_kn_pad(K, nO);
+    SQ_TRY(check_ptr(X_N, kn_pad > 0, "X_N"));
+    SQ_TRY(check_ptr(W_N, kn_pad > 0, "W_N"));
+    SQ_TRY(check_ptr(X_O, nO > 0, "X_O"));
+    SQ_TRY(check_ptr(W_O, nO > 0, "W_O"));
+    SQ_TRY(check_ptr(s_x, true, "s_x"));
+    SQ_TRY(check_ptr(s_w, true, "s_w"));
+    SQ_TRY(check_ptr(Y, true, "Y"));
+    if (dbg_i && !aligned16(dbg_i)) return fail(SQ_ERR_MISALIGNED, "dbg_acc_i32 is not 16-byte aligned");
+    if (dbg_f && !aligned16(dbg_f)) return fail(SQ_ERR_MISALIGNED, "dbg_acc_f32 is not 16-byte aligned");
+    return gemm_impl(X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+}
+
+// Single-thread kernel that waits on a barrier nobody completes, with a
+// bounded wait, then records the timeout and exits.
+__global__ void watchdog_selftest_kernel(unsigned long long limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = sqd::smem_u32(&bar);
+    sqd::mbar_init(b, 1);
+    sqd::fence_barrier_init();
+    const unsigned long long t0 = sqd::globaltimer();
+    while (!sqd::mbar_try_wait(b, 0)) {
+        if (sqd::globaltimer() - t0 > limit_ns) {
+            atomicCAS(&g_sq_dev_error, 0u, 0x7E57u);
+            return;
+        }
+    }
+}
+
+}  // namespace
+
+// ================================================================ C ABI
+extern "C" {
+
+const char *sq_status_string(sq_status s)
+{
+    switch (s) {
+    case SQ_OK: return "SQ_OK";
+    case SQ_ERR_INVALID_ARG: return "SQ_ERR_INVALID_ARG";
+    case SQ_ERR_UNSUPPORTED: return "SQ_ERR_UNSUPPORTED";
+    case SQ_ERR_MISALIGNED: return "SQ_ERR_MISALIGNED";
+    case SQ_ERR_CUDA: return "SQ_ERR_CUDA";
+    case SQ_ERR_TIMEOUT: return "SQ_ERR_TIMEOUT";
+    }
+    return "SQ_ERR_UNKNOWN";
+}
+
+const char *sq_last_error_detail(void) { return g_detail.c_str(); }
+
+int64_t sq_kn_pad(int64_t K, int64_t nO) { return round_up(K - nO, 128); }
+
+int64_t sq_no_pad(int64_t nO) { return round_up(nO, 64); }
+
+int64_t sq_chan_table_words(int64_t K) { return K / 8; }
+
+size_t sq_linear_workspace_bytes(int64_t M, int64_t K, int64_t nO)
+{
+    if (M <= 0) return 0;
+    const int64_t xn = round_up(M * (sq_kn_pad(K, nO) / 2), 256);
+    const int64_t sx = round_up(M * 4, 256);
+    const int64_t xo = round_up(M * sq_no_pad(nO) * 2, 256);
+    return static_cast<size_t>(xn + sx + xo);
+}
+
+sq_status sq_prepare_weights(const void *W, int64_t N, int64_t K, int64_t ldw, const int32_t *O, int64_t nO,
+                             void *W_N, float *s_w, void *W_O, uint32_t *chan_tab, sq_stream_t stream)
+{
+    g_detail.clear();
+    SQ_TRY(check_K_nO(K, nO));
+    if (N < 0) return fail(SQ_ERR_INVALID_ARG, "N < 0");
+    if (ldw < K || ldw % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldw must be >= K and a multiple of 8");
+    if (nO > 0 && !O) return fail(SQ_ERR_INVALID_ARG, "O is NULL");
+    for (int64_t j = 0; j < nO; ++j) {
+        if (O[j] < 0 || O[j] >= K) return fail(SQ_ERR_INVALID_ARG, "O[%lld]=%d outside [0, K)", (long long)j, O[j]);
+        if (j > 0 && O[j] <= O[j - 1]) return fail(SQ_ERR_INVALID_ARG, "O must be strictly increasing (index %lld)", (long long)j);
+    }
+    SQ_TRY(check_ptr(chan_tab, true, "chan_tab"));
+    const int64_t kn_pad = sq_kn_pad(K, nO);
+    if (N > 0) {
+        SQ_TRY(check_ptr(W, true, "W"));
+        SQ_TRY(check_ptr(W_N, kn_pad > 0, "W_N"));
+        SQ_TRY(check_ptr(s_w, true, "s_w"));
+        SQ_TRY(check_ptr(W_O, nO > 0, "W_O"));
+    }
+    DevInfo di;
+    SQ_TRY(device_info(di));
+
+    // Static channel table: one word per 8 channels.
+    std::vector<uint32_t> tab(static_cast<size_t>(K / 8), 0u);
+    for (int64_t j = 0; j < nO; ++j) tab[O[j] / 8] |= 1u << (O[j] % 8);
+    uint32_t below = 0;
+    for (int64_t c = 0; c < K / 8; ++c) {
+        const uint32_t mask = tab[c];
+        tab[c] = (below << 8) | mask;
+        below += static_cast<uint32_t>(__builtin_popcount(mask));
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(chan_tab, tab.data(), tab.size() * sizeof(uint32_t), cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copy of the channel table");
+    SQ_TRY(launch_rowquant(static_cast<const uint16_t *>(W), N, K, ldw, chan_tab, nO, static_cast<uint8_t *>(W_N), s_w,
+                           static_cast<uint16_t *>(W_O), s));
+    if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "sq_prepare_weights");
+    return SQ_OK;
+}
+
+sq_status sq_quant_gather(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, int64_t nO,
+                          void *X_N, float *s_x, void *X_O, sq_stream_t stream)
+{
+    g_detail.clear();
+    return quant_gather_impl(X, M, K, ldx, chan_tab, nO, X_N, s_x, X_O, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_gemm(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
+                  const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
+                  int32_t *dbg_acc_i32, float *dbg_acc_f32, sq_stream_t stream)
+{
+    g_detail.clear();
+    return gemm_checked(X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_acc_i32, dbg_acc_f32,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_linear(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, const void *W_N,
+                    const float *s_w, const void *W_O, int64_t N, int64_t nO, void *Y, int64_t ldy, void *workspace,
+                    size_t ws_bytes, sq_stream_t stream)
+{
+    g_detail.clear();
+    SQ_TRY(check_K_nO(K, nO));
+    if (M < 0) return fail(SQ_ERR_INVALID_ARG, "M < 0");
+    if (M == 0) return SQ_OK;
+    const size_t need = sq_linear_workspace_bytes(M, K, nO);
+    if (ws_bytes < need) return fail(SQ_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+    SQ_TRY(check_ptr(workspace, true, "workspace"));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const int64_t kn_pad = sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
+    uint8_t *X_N = ws;
+    float *s_x = reinterpret_cast<float *>(ws + round_up(M * (kn_pad / 2), 256));
+    uint16_t *X_O = reinterpret_cast<uint16_t *>(ws + round_up(M * (kn_pad / 2), 256) + round_up(M * 4, 256));
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    SQ_TRY(quant_gather_impl(X, M, K, ldx, chan_tab, nO, kn_pad > 0 ? X_N : nullptr, s_x, no_pad > 0 ? X_O : nullptr, s));
+    return gemm_checked(kn_pad > 0 ? X_N : nullptr, s_x, no_pad > 0 ? X_O : nullptr, W_N, s_w, W_O, M, N, K, nO, Y, ldy,
+                        nullptr, nullptr, s);
+}
+
+sq_status sq_check(sq_stream_t stream)
+{
+    g_detail.clear();
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "sq_check");
+    unsigned int word = 0;
+    if ((e = cudaMemcpyFromSymbol(&word, g_sq_dev_error, sizeof word)) != cudaSuccess)
+        return cuda_fail(e, "reading the device error word");
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if ((e = cudaMemcpyToSymbol(g_sq_dev_error, &zero, sizeof zero)) != cudaSuccess)
+            return cuda_fail(e, "clearing the device error word");
+        return fail(SQ_ERR_TIMEOUT, "a bounded wait ran out (site 0x%x)", word);
+    }
+    return SQ_OK;
+}
+
+sq_status sq_selftest_watchdog(int timeout_ms, sq_stream_t stream)
+{
+    g_detail.clear();
+    if (timeout_ms < 1 || timeout_ms > 10000) return fail(SQ_ERR_INVALID_ARG, "timeout_ms must lie in [1, 10000]");
+    DevInfo di;
+    SQ_TRY(device_info(di));
+    watchdog_selftest_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<unsigned long long>(timeout_ms) * 1000000ull);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "watchdog self-test launch");
+    return SQ_OK;
+}
+
+}  // extern "C"
