@@ -61,13 +61,13 @@ def run_gpu(O, X: torch.Tensor, W: torch.Tensor, ldy_extra: int = 0):
     Xd = X.to(dev)
     X_N, s_x, X_O = sq.quant_gather(Xd, pw)
     M, N = X.shape[0], W.shape[0]
-    guard = torch.full((M + 1, N + ldy_extra), -777.0, dtype=torch.bfloat16, device=dev)
+    guard = torch.full((M + 1, N + ldy_extra), -1024.0, dtype=torch.bfloat16, device=dev)
     Y = guard[:M, :N]
     _, dbg_i, dbg_f = sq.gemm(X_N, s_x, X_O, pw, Y=Y, debug=True)
     torch.cuda.synchronize()
     sq.sq_check()
     g = guard.float().cpu()
-    assert torch.all(g[M] == -777.0) and torch.all(g[:, N:] == -777.0), "write outside Y"
+    assert torch.all(g[M] == -1024.0) and torch.all(g[:, N:] == -1024.0), "write outside Y"
     return pw, (X_N, s_x, X_O), Y, dbg_i, dbg_f
 
 
