@@ -150,6 +150,38 @@ sq_status sq_linear(const void *X, int64_t M, int64_t K, int64_t ldx,
                     void *workspace, size_t ws_bytes, sq_stream_t stream);
 
 /*
+ * sq_linear without a caller workspace.  (No counterpart in the papers: this
+ * is a deployment convenience of this library.)
+ *
+ * Some callers cannot allocate device memory for the workspace sq_linear
+ * needs: a plugin or inference server that hands out all device memory from
+ * its own pool and forbids allocations once it has started, or a
+ * latency-bound serving loop where cudaMalloc/cudaFree would synchronize the
+ * device and stall other streams.  This entry point takes the same inputs and
+ * outputs as sq_linear but keeps its scratch in a fixed array inside the
+ * library, so it allocates nothing and calls no allocating routine.
+ *
+ *   - Limit: sq_linear_workspace_bytes(M, K, nO) must not exceed
+ *     SQ_NOALLOC_WS_BYTES (16 MiB; e.g. M <= 4096 tokens at K = 4096, nO = 256);
+ *     larger requests return SQ_ERR_UNSUPPORTED before anything is enqueued.
+ *   - Every device that loads the library holds this 16 MiB until the process
+ *     exits.
+ *   - The first call on a device looks up the array's device address once;
+ *     make that first call before any stream capture begins.
+ *   - All calls share the one array and it keeps the previous call's
+ *     contents.  Nothing in it has to start at zero (the quantize-and-gather
+ *     kernel writes every byte the GEMM reads), but calls whose work overlaps
+ *     on the GPU (different streams, or different host threads) race on it:
+ *     serialize them.
+ */
+#define SQ_NOALLOC_WS_BYTES (16u * 1024u * 1024u)
+sq_status sq_linear_noalloc(const void *X, int64_t M, int64_t K, int64_t ldx,
+                            const uint32_t *chan_tab,
+                            const void *W_N, const float *s_w, const void *W_O,
+                            int64_t N, int64_t nO, void *Y, int64_t ldy,
+                            sq_stream_t stream);
+
+/*
  * Waits for `stream`, then reports (and clears) the device error word of the
  * current device: SQ_ERR_TIMEOUT if a kernel's bounded wait ran out,
  * SQ_ERR_CUDA on a pending CUDA error, SQ_OK otherwise.

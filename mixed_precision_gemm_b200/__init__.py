@@ -33,7 +33,8 @@ from . import _build
 __all__ = [
     "SQError", "load", "library_path", "header_functions",
     "sq_status_string", "sq_kn_pad", "sq_no_pad", "sq_chan_table_words", "sq_linear_workspace_bytes",
-    "sq_prepare_weights", "sq_quant_gather", "sq_gemm", "sq_linear", "sq_check", "sq_selftest_watchdog",
+    "sq_prepare_weights", "sq_quant_gather", "sq_gemm", "sq_linear", "sq_linear_noalloc", "sq_check",
+    "sq_selftest_watchdog",
     "PreparedWeights", "prepare_weights", "quant_gather", "gemm", "SQLinear",
 ]
 
@@ -91,10 +92,11 @@ def load():
     lib.sq_quant_gather.argtypes = [P, I, I, I, P, I, P, P, P, P]
     lib.sq_gemm.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P, P, P]
     lib.sq_linear.argtypes = [P, I, I, I, P, P, P, P, I, I, P, I, P, Z, P]
+    lib.sq_linear_noalloc.argtypes = [P, I, I, I, P, P, P, P, I, I, P, I, P]
     lib.sq_check.argtypes = [P]
     lib.sq_selftest_watchdog.argtypes = [F, P]
     for f in (lib.sq_prepare_weights, lib.sq_quant_gather, lib.sq_gemm, lib.sq_linear, lib.sq_check,
-              lib.sq_selftest_watchdog):
+              lib.sq_selftest_watchdog, lib.sq_linear_noalloc):
         f.restype = F
     _lib = lib
     return lib
@@ -199,6 +201,23 @@ def sq_linear(X: torch.Tensor, chan_tab: torch.Tensor, W_N, s_w, W_O, N: int, nO
                           _ptr(Y), Y.stride(0), _ptr(workspace), workspace.numel() * workspace.element_size(),
                           _stream(stream))
     _raise(st, "sq_linear")
+
+
+def sq_linear_noalloc(X: torch.Tensor, chan_tab: torch.Tensor, W_N, s_w, W_O, N: int, nO: int, Y: torch.Tensor,
+                      stream=None) -> None:
+    """sq_linear for callers that cannot allocate device memory for a workspace.
+
+    The scratch lives in a fixed 16 MiB array inside the library (see
+    SQ_NOALLOC_WS_BYTES in include/sq.h): calls that need more raise
+    SQError(SQ_ERR_UNSUPPORTED), and calls that overlap on the GPU race on the
+    shared array, so serialize them.
+    """
+    _rowmajor(X, "X", torch.bfloat16)
+    _rowmajor(Y, "Y", torch.bfloat16)
+    M, K = X.shape
+    st = load().sq_linear_noalloc(_ptr(X), M, K, X.stride(0), _ptr(chan_tab), _ptr(W_N), _ptr(s_w), _ptr(W_O), N, nO,
+                                  _ptr(Y), Y.stride(0), _stream(stream))
+    _raise(st, "sq_linear_noalloc")
 
 
 def sq_check(stream=None) -> None:

@@ -451,3 +451,55 @@ sq_status sq_selftest_watchdog(int timeout_ms, sq_stream_t stream)
 }
 
 }  // extern "C"
+
+// ================================================================ workspace-free sq_linear
+// Scratch for sq_linear_noalloc: a fixed array in the library, one per device
+// that loads it.  Host code must not hand this symbol to a kernel directly
+// (on the host it names a stand-in, not device memory); the device address is
+// looked up once per device below.
+static __device__ __align__(256) uint8_t g_sq_noalloc_ws[SQ_NOALLOC_WS_BYTES];
+
+namespace {
+
+void *g_noalloc_addr[kMaxDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device (looked up on the
+// first call for each device, with that device current).
+sq_status noalloc_scratch(void **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(SQ_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_sq_noalloc_ws);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        g_noalloc_addr[dev] = p;
+    }
+    *out = g_noalloc_addr[dev];
+    return SQ_OK;
+}
+
+}  // namespace
+
+extern "C" sq_status sq_linear_noalloc(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab,
+                                       const void *W_N, const float *s_w, const void *W_O, int64_t N, int64_t nO,
+                                       void *Y, int64_t ldy, sq_stream_t stream)
+{
+    g_detail.clear();
+    SQ_TRY(check_K_nO(K, nO));
+    if (M < 0) return fail(SQ_ERR_INVALID_ARG, "M < 0");
+    if (M == 0) return SQ_OK;
+    const size_t need = sq_linear_workspace_bytes(M, K, nO);
+    if (need > SQ_NOALLOC_WS_BYTES)
+        return fail(SQ_ERR_UNSUPPORTED,
+                    "sq_linear_noalloc: M=%lld, K=%lld, nO=%lld need %zu scratch bytes but the built-in scratch "
+                    "holds %u; split the tokens into smaller calls or use sq_linear with a workspace",
+                    (long long)M, (long long)K, (long long)nO, need, SQ_NOALLOC_WS_BYTES);
+    void *ws = nullptr;
+    SQ_TRY(noalloc_scratch(&ws));
+    return sq_linear(X, M, K, ldx, chan_tab, W_N, s_w, W_O, N, nO, Y, ldy, ws, SQ_NOALLOC_WS_BYTES, stream);
+}
