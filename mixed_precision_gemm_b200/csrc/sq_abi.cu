@@ -16,6 +16,7 @@
 #include "../../include/sq.h"
 #include "sq_device.cuh"
 #include "sq_gemm.cuh"
+#include "sq_gemm_pair.cuh"
 #include "sq_rowquant.cuh"
 
 namespace {
@@ -122,7 +123,8 @@ sq_status launch_rowquant_t(const DevInfo &di, const uint16_t *src, int64_t rows
                             uint16_t *dout, cudaStream_t stream)
 {
     auto kern = sqq::rowquant_kernel<T, CPT>;
-    const size_t smem = static_cast<size_t>(kn_pad) + 2u * static_cast<size_t>(no_pad);
+    // two alternating (code buffer + outlier buffer) pairs
+    const size_t smem = 2u * (static_cast<size_t>(kn_pad) + 2u * static_cast<size_t>(no_pad));
     cudaError_t e;
     if (smem > 48 * 1024) {
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))) !=
@@ -152,29 +154,21 @@ sq_status launch_rowquant(const uint16_t *src, int64_t rows, int64_t K, int64_t 
     const int k = static_cast<int>(K), no = static_cast<int>(nO);
     if (nchunk <= 256) return launch_rowquant_t<256, 1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
     if (nchunk <= 512) return launch_rowquant_t<256, 2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 1024) return launch_rowquant_t<256, 4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 2048) return launch_rowquant_t<256, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 4096) return launch_rowquant_t<512, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 1024) return launch_rowquant_t<512, 2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 2048) return launch_rowquant_t<1024, 2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 4096) return launch_rowquant_t<1024, 4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
     return launch_rowquant_t<1024, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
 }
 
 // ---------------------------------------------------------------- GEMM
 template <class C>
-sq_status launch_gemm_t(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
-                        const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
-                        int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+sq_status launch_gemm_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O, const void *W_N,
+                        const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y,
+                        int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
 {
     const int64_t kn_pad = sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
-    CUtensorMap m_xn{}, m_wn{}, m_xo{}, m_wo{};
+    CUtensorMap m_xo{}, m_wo{};
     sq_status st;
-    if (kn_pad > 0) {
-        if ((st = make_map(m_xn, X_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, M, kn_pad / 2, sqg::PROWB, sqg::BM,
-                           CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
-            return st;
-        if ((st = make_map(m_wn, W_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, N, kn_pad / 2, sqg::PROWB, C::BN,
-                           CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
-            return st;
-    }
     if (no_pad > 0) {
         if ((st = make_map(m_xo, X_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, M, no_pad * 2, sqg::KB_BF, sqg::BM,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
@@ -184,6 +178,9 @@ sq_status launch_gemm_t(const void *X_N, const float *s_x, const void *X_O, cons
             return st;
     }
     sqg::GemmArgs a;
+    a.xn = static_cast<const uint8_t *>(X_N);
+    a.wn = static_cast<const uint8_t *>(W_N);
+    a.row_bytes = kn_pad / 2;
     a.s_x = s_x;
     a.s_w = s_w;
     a.Y = static_cast<uint16_t *>(Y);
@@ -198,18 +195,74 @@ sq_status launch_gemm_t(const void *X_N, const float *s_x, const void *X_O, cons
     a.tiles_n = static_cast<int>((N + C::BN - 1) / C::BN);
     a.group_m = 8;
     const int64_t ntiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
+    const int64_t grid = std::min<int64_t>(ntiles, di.sms);
     const bool dbg = dbg_i || dbg_f;
     auto kern = dbg ? sqg::dual_gemm_kernel<C, true> : sqg::dual_gemm_kernel<C, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-    kern<<<static_cast<unsigned>(ntiles), sqg::NUM_THREADS, C::SMEM_BYTES, stream>>>(m_xn, m_wn, m_xo, m_wo, a);
+    kern<<<static_cast<unsigned>(grid), sqg::NUM_THREADS, C::SMEM_BYTES, stream>>>(m_xo, m_wo, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "gemm launch");
     return SQ_OK;
 }
 
-using CfgN256 = sqg::Cfg<256, 3, 2>;
-using CfgN128 = sqg::Cfg<128, 4, 3>;
-using CfgN64 = sqg::Cfg<64, 4, 3>;
+// Pair (cta_group::2) kernel: 256 x 256 tiles over clusters of two CTAs.
+template <class C>
+sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O, const void *W_N,
+                             const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y,
+                             int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+{
+    const int64_t kn_pad = sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
+    CUtensorMap m_xo{}, m_wo{}, m_xn{}, m_wn{};
+    sq_status st;
+    if (kn_pad > 0) {
+        if ((st = make_map(m_xn, X_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, M, kn_pad / 2, sqg::PROWB, 128,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
+            return st;
+        if ((st = make_map(m_wn, W_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, N, kn_pad / 2, sqg::PROWB, 128,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
+            return st;
+    }
+    if (no_pad > 0) {
+        if ((st = make_map(m_xo, X_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, M, no_pad * 2, sqg::KB_BF, 128,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
+            return st;
+        if ((st = make_map(m_wo, W_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, N, no_pad * 2, sqg::KB_BF, 128,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
+            return st;
+    }
+    sqg::GemmArgs a;
+    a.xn = static_cast<const uint8_t *>(X_N);
+    a.wn = static_cast<const uint8_t *>(W_N);
+    a.row_bytes = kn_pad / 2;
+    a.s_x = s_x;
+    a.s_w = s_w;
+    a.Y = static_cast<uint16_t *>(Y);
+    a.dbg_i = dbg_i;
+    a.dbg_f = dbg_f;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.ldy = ldy;
+    a.nkb_i = static_cast<int>(kn_pad / sqg::KB_I8);
+    a.nkb_o = static_cast<int>(no_pad / sqg::KB_BF);
+    a.tiles_m = static_cast<int>((M + sqg::PAIR_BM - 1) / sqg::PAIR_BM);
+    a.tiles_n = static_cast<int>((N + sqg::PAIR_BN - 1) / sqg::PAIR_BN);
+    a.group_m = 4;
+    const int64_t ntiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
+    const int64_t clusters = std::min<int64_t>(ntiles, di.sms / 2);
+    const bool dbg = dbg_i || dbg_f;
+    auto kern = dbg ? sqg::dual_gemm_pair_kernel<C, true> : sqg::dual_gemm_pair_kernel<C, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
+    kern<<<static_cast<unsigned>(2 * clusters), sqg::NUM_THREADS, C::SMEM_BYTES, stream>>>(m_xo, m_wo, m_xn, m_wn, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "gemm pair launch");
+    return SQ_OK;
+}
+
+using CfgPair = sqg::CfgPair<4, 6>;
+
+using CfgN256 = sqg::Cfg<256, 4>;
+using CfgN128 = sqg::Cfg<128, 6>;
+using CfgN64 = sqg::Cfg<64, 8>;
 
 sq_status gemm_impl(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
                     const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
@@ -220,11 +273,14 @@ sq_status gemm_impl(const void *X_N, const float *s_x, const void *X_O, const vo
     sq_status st = device_info(di);
     if (st != SQ_OK) return st;
     const int64_t tiles_m = (M + sqg::BM - 1) / sqg::BM;
+    const int64_t pair_tiles = ((M + sqg::PAIR_BM - 1) / sqg::PAIR_BM) * ((N + sqg::PAIR_BN - 1) / sqg::PAIR_BN);
+    if (M >= 256 && pair_tiles >= di.sms / 2)
+        return launch_gemm_pair_t<CfgPair>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (tiles_m * ((N + 255) / 256) >= 2 * di.sms)
-        return launch_gemm_t<CfgN256>(X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+        return launch_gemm_t<CfgN256>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (tiles_m * ((N + 127) / 128) >= di.sms)
-        return launch_gemm_t<CfgN128>(X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
-    return launch_gemm_t<CfgN64>(X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+        return launch_gemm_t<CfgN128>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    return launch_gemm_t<CfgN64>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
 }
 
 // ---------------------------------------------------------------- validation

@@ -2,20 +2,28 @@
 //
 // OSC (arXiv:2604.12782), abstract: inference runs a low-precision 4-bit GEMM
 // path and a high-precision 16-bit branch GEMM on the compact outlier tensor,
-// and fuses the two results.  Here both run inside one kernel per 128 x BN
-// output tile, each into its own tensor-memory (TMEM) accumulator:
+// and fuses the two results.  Here both run inside one persistent kernel; each
+// 128 x BN output tile owns two tensor-memory (TMEM) accumulators:
 //
-//   acc_f (fp32, TMEM columns [0, BN))   += X_O . W_O^T   (tcgen05 kind::f16, bf16 inputs)
+//   acc_f (fp32, TMEM columns [0, BN))    += X_O . W_O^T          (tcgen05 kind::f16, bf16 inputs)
 //   acc_i (int32, TMEM columns [BN, 2BN)) += codes_X . codes_W^T  (tcgen05 kind::i8)
-//   Y = bf16_rn( (float)acc_i * s_x[m] * s_w[n] + acc_f )         (one epilogue)
+//   Y = bf16_rn( (float)acc_i * s_x[m] * s_w[n] + acc_f )           (one epilogue)
 //
-// Warp roles (6 warps):
-//   warp 0      TMA producer: compact bf16 tiles straight into the operand
-//               ring (128-byte swizzle, consumable by the MMA), packed INT4
-//               tiles into a staging ring.
+// Warp roles (14 warps, one CTA per SM, tiles handed out round-robin):
+//   warp 0      idle after set-up.
 //   warp 1      allocates TMEM; one lane issues every MMA and commits.
-//   warps 2..5  expand packed INT4 tiles into int8 operand tiles, then run
-//               the epilogue (each warp owns one 32-lane TMEM sub-partition).
+//   warps 2..5  epilogue: tcgen05.ld of both accumulators (each warp owns one
+//               32-lane TMEM sub-partition), scale, fuse, bf16 stores.  They
+//               hand TMEM back as soon as the last column block is read.
+//   warps 6..13 operand producers, in the MMA's order of ring uses: for a
+//               bf16 block one lane issues the two TMA tile loads (128-byte
+//               swizzle, consumable by the MMA as they land); for an INT4
+//               block every thread stores its share of the expanded int8
+//               tile.  Packed INT4 rows come from global memory straight into
+//               registers, two INT4 blocks ahead, so packed bytes never pass
+//               through shared memory.  A single producer group keeps every
+//               ring slot's uses strictly in order, which the mbarrier phase
+//               parity protocol needs.
 //
 // INT4 expansion.  A packed 32-bit word holds 8 codes c0..c7 (c0 in the low
 // nibble).  (w << 4) & 0xF0F0F0F0 gives the bytes 16*c0, 16*c2, 16*c4, 16*c6
@@ -38,37 +46,42 @@ constexpr int ROWB = 128;       // operand bytes per row per K-block (one 128-by
 constexpr int PROWB = 64;       // packed INT4 bytes per row per K-block
 constexpr int KB_I8 = 128;      // int8 K elements per block
 constexpr int KB_BF = 64;       // bf16 K elements per block
-constexpr int NUM_THREADS = 192;
-constexpr int NUM_EXP_WARPS = 4;
+constexpr int NUM_EPI_WARPS = 4;
+constexpr int NUM_EXP_WARPS = 8;
+constexpr int EPI_WARP0 = 2;
+constexpr int EXP_WARP0 = EPI_WARP0 + NUM_EPI_WARPS;
+constexpr int NUM_THREADS = 32 * (EXP_WARP0 + NUM_EXP_WARPS);
+constexpr int EXP_THREADS = 32 * NUM_EXP_WARPS;
 
 enum : unsigned {
-    SITE_PROD_OP = 0x101, SITE_PROD_STG = 0x102, SITE_EXP_STG = 0x201, SITE_EXP_OP = 0x202,
-    SITE_MMA = 0x301, SITE_EPI = 0x401
+    SITE_EXP_OP = 0x202, SITE_MMA_FULL = 0x301, SITE_MMA_ACC = 0x302, SITE_EPI = 0x401
 };
 
-template <int BN_, int OPS_, int STG_>
+template <int BN_, int OPS_>
 struct Cfg {
-    static constexpr int BN = BN_, OPS = OPS_, STG = STG_;
+    static constexpr int BN = BN_, OPS = OPS_;
     static constexpr int A_BYTES = BM * ROWB;
     static constexpr int B_BYTES = BN * ROWB;
     static constexpr int OP_BYTES = A_BYTES + B_BYTES;
-    static constexpr int PA_BYTES = BM * PROWB;
-    static constexpr int PB_BYTES = BN * PROWB;
-    static constexpr int STG_BYTES = PA_BYTES + PB_BYTES;
     static constexpr int OFF_OP = 0;
-    static constexpr int OFF_STG = OPS * OP_BYTES;
-    static constexpr int OFF_BAR = OFF_STG + STG * STG_BYTES;
-    // barriers: stg_full[STG] stg_empty[STG] opx_full[OPS] opt_full[OPS] op_empty[OPS] acc_full drain
-    static constexpr int NBAR = 2 * STG + 3 * OPS + 2;
+    static constexpr int OFF_BAR = OPS * OP_BYTES;
+    // barriers: op_full[OPS] op_empty[OPS] acc_full acc_empty drain
+    static constexpr int NBAR = 2 * OPS + 3;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
     static constexpr int TMEM_COLS = 2 * BN;
+    // packed 16-byte chunks per K-block and per expansion thread
+    static constexpr int EXP_CHUNKS = (BM + BN) * (PROWB / 16) / EXP_THREADS;
     static_assert(BN == 64 || BN == 128 || BN == 256, "BN");
     static_assert(OP_BYTES % 1024 == 0, "operand tiles must stay 1024-byte aligned");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert((BM + BN) * (PROWB / 16) % EXP_THREADS == 0, "expansion work split");
 };
 
 struct GemmArgs {
+    const uint8_t *xn;   // packed X part [M, row_bytes]
+    const uint8_t *wn;   // packed W part [N, row_bytes]
+    long long row_bytes; // kn_pad / 2
     const float *s_x;
     const float *s_w;
     uint16_t *Y;
@@ -76,18 +89,31 @@ struct GemmArgs {
     float *dbg_f;
     int M, N;
     long long ldy;
-    int nkb_i;    // packed INT4 K-blocks (kn_pad / 128)
-    int nkb_o;    // bf16 K-blocks (no_pad / 64)
+    int nkb_i;    // INT4 K-blocks per tile (kn_pad / 128)
+    int nkb_o;    // bf16 K-blocks per tile (no_pad / 64)
     int tiles_m, tiles_n, group_m;
 };
 
+// Tile t -> (M-tile, N-tile): groups of `group_m` M-tiles sweep all N-tiles,
+// so the CTAs working at the same time share a few X tiles and a band of W
+// tiles in L2.
+__device__ __forceinline__ void tile_coords(const GemmArgs &a, int t, int &tmi, int &tni)
+{
+    const int gsz = a.group_m * a.tiles_n;
+    const int g = t / gsz;
+    const int first_m = g * a.group_m;
+    const int gm = min(a.tiles_m - first_m, a.group_m);
+    const int idx = t - g * gsz;
+    tmi = first_m + idx % gm;
+    tni = idx / gm;
+}
+
 template <class C, bool DBG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_xn, const __grid_constant__ CUtensorMap tm_wn,
-                 const __grid_constant__ CUtensorMap tm_xo, const __grid_constant__ CUtensorMap tm_wo,
+dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_constant__ CUtensorMap tm_wo,
                  const GemmArgs args)
 {
-    constexpr int BN = C::BN, OPS = C::OPS, STG = C::STG;
+    constexpr int BN = C::BN, OPS = C::OPS, EC = C::EXP_CHUNKS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = sqd::smem_u32(smem);
@@ -95,52 +121,33 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_xn, const __grid_constan
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // Tile coordinates: groups of `group_m` M-tiles sweep all N-tiles so that a
-    // wave of CTAs shares a few X tiles and a band of W tiles in L2.
-    int tmi, tni;
-    {
-        const int bid = blockIdx.x;
-        const int gsz = args.group_m * args.tiles_n;
-        const int g = bid / gsz;
-        const int first_m = g * args.group_m;
-        const int gm = min(args.tiles_m - first_m, args.group_m);
-        const int idx = bid - g * gsz;
-        tmi = first_m + idx % gm;
-        tni = idx / gm;
-    }
-
     const uint32_t bar0 = sbase + C::OFF_BAR;
-    auto stg_full = [&](int s) { return bar0 + 8u * s; };
-    auto stg_empty = [&](int s) { return bar0 + 8u * (STG + s); };
-    auto opx_full = [&](int e) { return bar0 + 8u * (2 * STG + e); };
-    auto opt_full = [&](int e) { return bar0 + 8u * (2 * STG + OPS + e); };
-    auto op_empty = [&](int e) { return bar0 + 8u * (2 * STG + 2 * OPS + e); };
-    const uint32_t acc_full = bar0 + 8u * (2 * STG + 3 * OPS);
-    const uint32_t drain = acc_full + 8u;
+    auto op_full = [&](int e) { return bar0 + 8u * e; };
+    auto op_empty = [&](int e) { return bar0 + 8u * (OPS + e); };
+    const uint32_t acc_full = bar0 + 8u * (2 * OPS);
+    const uint32_t acc_empty = acc_full + 8u;
+    const uint32_t drain = acc_full + 16u;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC + 4);
     auto op_a = [&](int e) { return sbase + C::OFF_OP + e * C::OP_BYTES; };
-    auto stg_a = [&](int s) { return sbase + C::OFF_STG + s * C::STG_BYTES; };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STG; ++s) {
-            sqd::mbar_init(stg_full(s), 1);
-            sqd::mbar_init(stg_empty(s), NUM_EXP_WARPS);
-        }
         for (int e = 0; e < OPS; ++e) {
-            sqd::mbar_init(opx_full(e), NUM_EXP_WARPS);
-            sqd::mbar_init(opt_full(e), 1);
+            // One arrival per producer warp; for bf16 blocks the first
+            // producer's arrival also carries the TMA byte count.
+            sqd::mbar_init(op_full(e), NUM_EXP_WARPS);
             sqd::mbar_init(op_empty(e), 1);
         }
         sqd::mbar_init(acc_full, 1);
+        sqd::mbar_init(acc_empty, NUM_EPI_WARPS);
         sqd::mbar_init(drain, 1);
         *abort_flag = 0u;
         sqd::fence_barrier_init();
         sqd::fence_proxy_async_smem();
     }
-    if (warp == 0 && lane == 0) {
-        if (args.nkb_i > 0) { sqd::prefetch_tensormap(&tm_xn); sqd::prefetch_tensormap(&tm_wn); }
-        if (args.nkb_o > 0) { sqd::prefetch_tensormap(&tm_xo); sqd::prefetch_tensormap(&tm_wo); }
+    if (warp == EXP_WARP0 && lane == 0 && args.nkb_o > 0) {
+        sqd::prefetch_tensormap(&tm_xo);
+        sqd::prefetch_tensormap(&tm_wo);
     }
     if (warp == 1) {
         sqd::tmem_alloc(sqd::smem_u32(tmem_slot), C::TMEM_COLS);
@@ -152,94 +159,94 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_xn, const __grid_constan
     const uint32_t tmem = *tmem_slot;
 
     const int nkb_i = args.nkb_i, nkb_o = args.nkb_o;
-    const int ntot = nkb_o + nkb_i;
+    const int per_tile = nkb_o + nkb_i;
+    const int num_tiles = args.tiles_m * args.tiles_n;
+    const int my_tiles = (num_tiles - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                         static_cast<int>(gridDim.x);
 
     if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            int i = 0;
-            int armed_o = 0, armed_s = 0;
-            bool ok = true;
-            for (int kb = 0; kb < nkb_o && ok; ++kb, ++i) {
-                const int e = i % OPS;
-                const uint32_t ph = (i / OPS) & 1;
-                if (!sqd::mbar_wait(op_empty(e), ph ^ 1u, abort_flag, SITE_PROD_OP)) { ok = false; break; }
-                sqd::mbar_arrive_expect_tx(opt_full(e), C::OP_BYTES);
-                sqd::tma_load_2d(op_a(e), &tm_xo, opt_full(e), kb * KB_BF, tmi * BM);
-                sqd::tma_load_2d(op_a(e) + C::A_BYTES, &tm_wo, opt_full(e), kb * KB_BF, tni * BN);
-                armed_o = kb + 1;
-            }
-            for (int kb = 0; kb < nkb_i && ok; ++kb) {
-                const int s = kb % STG;
-                const uint32_t ph = (kb / STG) & 1;
-                if (!sqd::mbar_wait(stg_empty(s), ph ^ 1u, abort_flag, SITE_PROD_STG)) { ok = false; break; }
-                sqd::mbar_arrive_expect_tx(stg_full(s), C::STG_BYTES);
-                sqd::tma_load_2d(stg_a(s), &tm_xn, stg_full(s), kb * PROWB, tmi * BM);
-                sqd::tma_load_2d(stg_a(s) + C::PA_BYTES, &tm_wn, stg_full(s), kb * PROWB, tni * BN);
-                armed_s = kb + 1;
-            }
-            if (!ok) {
-                // Let every copy that was issued land before the CTA exits.
-                for (int kb = (armed_o > OPS ? armed_o - OPS : 0); kb < armed_o; ++kb)
-                    sqd::mbar_drain(opt_full(kb % OPS), (kb / OPS) & 1);
-                for (int kb = (armed_s > STG ? armed_s - STG : 0); kb < armed_s; ++kb)
-                    sqd::mbar_drain(stg_full(kb % STG), (kb / STG) & 1);
-            }
-        }
+        // idle
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_bf = sqd::make_idesc(false, BM, BN);
             constexpr uint32_t idesc_i8 = sqd::make_idesc(true, BM, BN);
             bool ok = true;
-            for (int i = 0; i < ntot; ++i) {
-                const int e = i % OPS;
-                const bool is_bf = i < nkb_o;
-                // opt_full(e) completes once per bf16 use of slot e and
-                // opx_full(e) once per INT4 use, so each has its own phase.
-                const uint32_t ph = is_bf ? ((i / OPS) & 1) : (((i - nkb_o) / OPS) & 1);
-                if (!sqd::mbar_wait(is_bf ? opt_full(e) : opx_full(e), ph, abort_flag, SITE_MMA)) { ok = false; break; }
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                // the epilogue must have read the previous tile's accumulators
+                if (!sqd::mbar_wait(acc_empty, (lt & 1) ^ 1u, abort_flag, SITE_MMA_ACC)) { ok = false; break; }
                 sqd::tc_fence_after();
-                const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
-                const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
-                const uint32_t d = tmem + (is_bf ? 0u : static_cast<uint32_t>(BN));
-                const bool first = is_bf ? (i == 0) : (i == nkb_o);
+                for (int i = 0; i < per_tile; ++i) {
+                    const int u = lt * per_tile + i;
+                    const int e = u % OPS;
+                    if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_MMA_FULL)) { ok = false; break; }
+                    sqd::tc_fence_after();
+                    const bool is_bf = i < nkb_o;
+                    const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
+                    const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
+                    const uint32_t d = tmem + (is_bf ? 0u : static_cast<uint32_t>(BN));
+                    const bool first = (i == 0) || (i == nkb_o);
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    // each step advances 32 bytes along K inside the swizzle row
-                    const uint32_t acc = (first && k == 0) ? 0u : 1u;
-                    if (is_bf) sqd::mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc_bf, acc);
-                    else sqd::mma_s8(d, adesc + 2 * k, bdesc + 2 * k, idesc_i8, acc);
+                    for (int k = 0; k < 4; ++k) {
+                        // each step advances 32 bytes along K inside the swizzle row
+                        const uint32_t acc = (first && k == 0) ? 0u : 1u;
+                        if (is_bf) sqd::mma_bf16(d, adesc + 2 * k, bdesc + 2 * k, idesc_bf, acc);
+                        else sqd::mma_s8(d, adesc + 2 * k, bdesc + 2 * k, idesc_i8, acc);
+                    }
+                    sqd::mma_commit(op_empty(e));
                 }
-                sqd::mma_commit(op_empty(e));
+                if (ok) sqd::mma_commit(acc_full);
             }
-            if (ok) {
-                sqd::mma_commit(acc_full);
-            } else {
+            if (!ok) {
                 sqd::mma_commit(drain);
                 sqd::mbar_drain(drain, 0);
             }
         }
-    } else {
+    } else if (warp >= EXP_WARP0) {
         // ------------------------------------------------------------ expansion
-        const int et = threadIdx.x - 64;  // 0..127
-        constexpr int ROWS = BM + BN;
-        for (int kb = 0; kb < nkb_i; ++kb) {
-            const int s = kb % STG;
-            const uint32_t sph = (kb / STG) & 1;
-            const int i = nkb_o + kb;
-            const int e = i % OPS;
-            const uint32_t eph = (i / OPS) & 1;
-            if (!sqd::mbar_wait(stg_full(s), sph, abort_flag, SITE_EXP_STG)) break;
-            if (!sqd::mbar_wait(op_empty(e), eph ^ 1u, abort_flag, SITE_EXP_OP)) break;
-            const uint32_t src = stg_a(s);
-            const uint32_t dst = op_a(e);
-            for (int q = et; q < ROWS * 4; q += NUM_EXP_WARPS * 32) {
+        const int et = threadIdx.x - EXP_WARP0 * 32;
+        const int F = my_tiles * nkb_i;  // INT4 K-blocks this CTA expands, over all its tiles
+        const long long rb = args.row_bytes;
+
+        auto load = [&](int f, uint4 (&buf)[EC]) {
+            const int lt = f / nkb_i;
+            const int kb = f - lt * nkb_i;
+            int tmi, tni;
+            tile_coords(args, static_cast<int>(blockIdx.x) + lt * static_cast<int>(gridDim.x), tmi, tni);
+#pragma unroll
+            for (int c = 0; c < EC; ++c) {
+                const int q = et + c * EXP_THREADS;
                 const int r = q >> 2;
                 const int j = q & 3;
-                const uint4 w = sqd::lds128(src + r * PROWB + j * 16);
+                const uint8_t *p;
+                bool ok;
+                if (r < BM) {
+                    const int row = tmi * BM + r;
+                    ok = row < args.M;
+                    p = args.xn + static_cast<long long>(row) * rb;
+                } else {
+                    const int row = tni * BN + (r - BM);
+                    ok = row < args.N;
+                    p = args.wn + static_cast<long long>(row) * rb;
+                }
+                buf[c] = ok ? sqd::ld_nc_v4(p + kb * PROWB + j * 16) : make_uint4(0, 0, 0, 0);
+            }
+        };
+        auto store = [&](int f, const uint4 (&buf)[EC]) -> bool {
+            const int lt = f / nkb_i;
+            const int kb = f - lt * nkb_i;
+            const int u = lt * per_tile + nkb_o + kb;
+            const int e = u % OPS;
+            if (!sqd::mbar_wait(op_empty(e), ((u / OPS) & 1) ^ 1u, abort_flag, SITE_EXP_OP)) return false;
+            const uint32_t dst = op_a(e);
+#pragma unroll
+            for (int c = 0; c < EC; ++c) {
+                const int q = et + c * EXP_THREADS;
+                const int r = q >> 2;
+                const uint32_t j = static_cast<uint32_t>(q & 3);
                 const uint32_t sw = static_cast<uint32_t>(r & 7);
                 const uint32_t row = dst + r * ROWB;
+                const uint4 w = buf[c];
                 sqd::sts128(row + (((2u * j) ^ sw) << 4),
                             (w.x << 4) & 0xF0F0F0F0u, w.x & 0xF0F0F0F0u,
                             (w.y << 4) & 0xF0F0F0F0u, w.y & 0xF0F0F0F0u);
@@ -249,30 +256,90 @@ dual_gemm_kernel(const __grid_constant__ CUtensorMap tm_xn, const __grid_constan
             }
             sqd::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                sqd::mbar_arrive(stg_empty(s));
-                sqd::mbar_arrive(opx_full(e));
+            if (lane == 0) sqd::mbar_arrive(op_full(e));
+            return true;
+        };
+
+        // bf16 blocks of tile lt: the first producer thread issues the TMA
+        // loads with the expected byte count; every other warp adds one plain
+        // arrival (op_full counts one arrival per producer warp).
+        const bool tma_thread = (et == 0);
+        int last_armed = -1;
+        auto produce_bf16 = [&](int lt) -> bool {
+            int tmi, tni;
+            tile_coords(args, static_cast<int>(blockIdx.x) + lt * static_cast<int>(gridDim.x), tmi, tni);
+            for (int kb = 0; kb < nkb_o; ++kb) {
+                const int u = lt * per_tile + kb;
+                const int e = u % OPS;
+                if (!sqd::mbar_wait(op_empty(e), ((u / OPS) & 1) ^ 1u, abort_flag, SITE_EXP_OP)) return false;
+                if (tma_thread) {
+                    sqd::mbar_arrive_expect_tx(op_full(e), C::OP_BYTES);
+                    sqd::tma_load_2d(op_a(e), &tm_xo, op_full(e), kb * KB_BF, tmi * BM);
+                    sqd::tma_load_2d(op_a(e) + C::A_BYTES, &tm_wo, op_full(e), kb * KB_BF, tni * BN);
+                    last_armed = u;
+                } else if (lane == 0) {
+                    sqd::mbar_arrive(op_full(e));
+                }
+            }
+            return true;
+        };
+
+        bool ok = true;
+        if (nkb_i == 0) {
+            for (int lt = 0; lt < my_tiles && ok; ++lt) ok = produce_bf16(lt);
+        } else {
+            // INT4 block f starts tile f / nkb_i when f % nkb_i == 0: its bf16
+            // blocks come first in the ring.
+            auto step = [&](int f, const uint4 (&buf)[EC]) -> bool {
+                if (nkb_o > 0 && f % nkb_i == 0 && !produce_bf16(f / nkb_i)) return false;
+                return store(f, buf);
+            };
+            uint4 b0[EC], b1[EC], b2[EC];
+            if (F > 0) load(0, b0);
+            if (F > 1) load(1, b1);
+            for (int f = 0; f < F; f += 3) {
+                if (f + 2 < F) load(f + 2, b2);
+                if (!(ok = step(f, b0))) break;
+                if (f + 1 >= F) break;
+                if (f + 3 < F) load(f + 3, b0);
+                if (!(ok = step(f + 1, b1))) break;
+                if (f + 2 >= F) break;
+                if (f + 4 < F) load(f + 4, b1);
+                if (!(ok = step(f + 2, b2))) break;
             }
         }
-
+        if (!ok && tma_thread && last_armed >= 0) {
+            // Let the last copies that were issued land before the CTA exits.
+            sqd::mbar_drain(op_full(last_armed % OPS), (last_armed / OPS) & 1);
+        }
+    } else {
         // ------------------------------------------------------------ epilogue
-        if (sqd::mbar_wait(acc_full, 0, abort_flag, SITE_EPI)) {
+        const int sub = warp & 3;  // TMEM lane sub-partition of this warp
+        const uint32_t tl = tmem + (static_cast<uint32_t>(sub * 32) << 16);
+        const bool has_i = nkb_i > 0, has_o = nkb_o > 0;
+        for (int lt = 0; lt < my_tiles; ++lt) {
+            int tmi, tni;
+            tile_coords(args, static_cast<int>(blockIdx.x) + lt * static_cast<int>(gridDim.x), tmi, tni);
+            if (!sqd::mbar_wait(acc_full, lt & 1, abort_flag, SITE_EPI)) break;
             sqd::tc_fence_after();
-            const int sub = warp & 3;                 // TMEM lane sub-partition of this warp
             const int m = tmi * BM + sub * 32 + lane;
             const bool row_ok = m < args.M;
             const float sx = row_ok ? args.s_x[m] : 0.0f;
-            const uint32_t tl = tmem + (static_cast<uint32_t>(sub * 32) << 16);
-            const bool has_i = nkb_i > 0, has_o = nkb_o > 0;
+            uint16_t *yrow = args.Y + static_cast<long long>(row_ok ? m : 0) * args.ldy;
 #pragma unroll 1
             for (int c = 0; c < BN; c += 32) {
                 uint32_t vi[32], vf[32];
                 if (has_i) sqd::tmem_ld_32x32b_x32(tl + BN + c, vi);
                 if (has_o) sqd::tmem_ld_32x32b_x32(tl + c, vf);
                 sqd::tmem_wait_ld();
+                if (c + 32 == BN) {
+                    // Accumulators fully read: the next tile's MMAs may start.
+                    sqd::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) sqd::mbar_arrive(acc_empty);
+                }
                 const int n0 = tni * BN + c;
                 if (!row_ok || n0 >= args.N) continue;
-                uint16_t *yrow = args.Y + static_cast<long long>(m) * args.ldy;
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     const int n = n0 + 8 * g;

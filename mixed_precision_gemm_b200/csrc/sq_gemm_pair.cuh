@@ -1,0 +1,341 @@
+// Dual-path GEMM on CTA pairs (tcgen05 cta_group::2): the same computation as
+// sq_gemm.cuh (OSC, arXiv:2604.12782, abstract: a 4-bit GEMM path plus a
+// 16-bit branch GEMM on the compact outlier tensor, fused), with 256 x 256
+// output tiles shared by the two CTAs of a cluster.
+//
+// In a pair MMA each CTA supplies half of A (its 128 token rows) and half of
+// B (128 of the 256 output channels) from its own shared memory, and receives
+// its 128 rows x 256 columns of D in its own tensor memory.  Per SM that is
+// the 128 x 256 tile of the single-CTA kernel with a third fewer operand bytes
+// to fetch and expand, which is what the INT4 -> int8 expansion is bound by.
+//
+// Roles (14 warps per CTA, one cluster of 2 CTAs per SM pair, tiles handed
+// out round-robin to clusters):
+//   warp 0 (each CTA)        TMA producer of the packed INT4 tiles (this CTA's
+//                            X rows and W rows) into a staging ring.
+//   warp 1 of the first CTA  issues every pair MMA; its commits arrive on the
+//                            barriers of both CTAs (multicast commit).
+//   warps 2..5 (each CTA)    epilogue of the CTA's 128 rows; they report to the
+//                            first CTA's acc_empty barrier when TMEM is read.
+//   warps 6..13 (each CTA)   operand producers for the CTA's halves, in ring
+//                            order: bf16 blocks by TMA (.cta_group::2 form, no
+//                            multicast, completion bytes counted on the first
+//                            CTA's barrier); INT4 blocks expanded from the
+//                            staging ring into int8 operand tiles (see
+//                            sq_gemm.cuh).  Every producer warp of both CTAs
+//                            arrives on the first CTA's op_full.
+// The packed tiles travel by TMA into a staging ring (asynchronous, six
+// K-blocks deep) and are expanded from shared memory, so no producer thread
+// has long global loads outstanding when it publishes a tile.
+// TMEM per CTA: acc_f in columns [0, 256), acc_i in [256, 512).
+#pragma once
+
+#include "sq_gemm.cuh"
+
+namespace sqg {
+
+constexpr int PAIR_BM = 256;     // tile rows of the pair (128 per CTA)
+constexpr int PAIR_BN = 256;     // tile columns (128 W rows per CTA)
+
+template <int OPS_, int STG_>
+struct CfgPair {
+    static constexpr int OPS = OPS_;                  // operand ring stages (expanded int8 or bf16 tiles)
+    static constexpr int STG = STG_;                  // staging ring stages (packed INT4 tiles)
+    static constexpr int A_BYTES = 128 * ROWB;        // this CTA's X rows
+    static constexpr int B_BYTES = 128 * ROWB;        // this CTA's W rows
+    static constexpr int OP_BYTES = A_BYTES + B_BYTES;
+    static constexpr int PA_BYTES = 128 * PROWB;      // packed X rows of one K-block
+    static constexpr int STG_BYTES = 256 * PROWB;     // packed X + W rows of one K-block
+    static constexpr int OFF_OP = 0;
+    static constexpr int OFF_STG = OPS * OP_BYTES;
+    static constexpr int OFF_BAR = OFF_STG + STG * STG_BYTES;
+    // barriers: op_full[OPS] op_empty[OPS] stg_full[STG] stg_empty[STG] acc_full acc_empty drain
+    static constexpr int NBAR = 2 * OPS + 2 * STG + 3;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int EXP_CHUNKS = 256 * (PROWB / 16) / EXP_THREADS;  // 4
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+template <class C, bool DBG>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_constant__ CUtensorMap tm_wo,
+                      const __grid_constant__ CUtensorMap tm_xn, const __grid_constant__ CUtensorMap tm_wn,
+                      const GemmArgs args)
+{
+    constexpr int OPS = C::OPS, EC = C::EXP_CHUNKS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = sqd::smem_u32(smem);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = sqd::cluster_ctarank();
+    const bool leader = (rank == 0);
+
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto op_full = [&](int e) { return bar0 + 8u * e; };
+    auto op_empty = [&](int e) { return bar0 + 8u * (OPS + e); };
+    constexpr int STG = C::STG;
+    auto stg_full = [&](int i) { return bar0 + 8u * (2 * OPS + i); };
+    auto stg_empty = [&](int i) { return bar0 + 8u * (2 * OPS + STG + i); };
+    const uint32_t acc_full = bar0 + 8u * (2 * OPS + 2 * STG);
+    const uint32_t acc_empty = acc_full + 8u;
+    const uint32_t drain = acc_full + 16u;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC + 4);
+    auto op_a = [&](int e) { return sbase + C::OFF_OP + e * C::OP_BYTES; };
+    auto stg_a = [&](int i) { return sbase + C::OFF_STG + i * C::STG_BYTES; };
+
+    if (threadIdx.x == 0) {
+        for (int e = 0; e < OPS; ++e) {
+            sqd::mbar_init(op_full(e), 2 * NUM_EXP_WARPS);  // every producer warp of both CTAs (first CTA's copy)
+            sqd::mbar_init(op_empty(e), 1);                 // multicast commit
+        }
+        for (int i = 0; i < STG; ++i) {
+            sqd::mbar_init(stg_full(i), 1);                 // this CTA's staging TMA (expect-tx)
+            sqd::mbar_init(stg_empty(i), NUM_EXP_WARPS);    // this CTA's expansion warps
+        }
+        sqd::mbar_init(acc_full, 1);                        // multicast commit
+        sqd::mbar_init(acc_empty, 2 * NUM_EPI_WARPS);       // epilogue warps of both CTAs (first CTA's copy)
+        sqd::mbar_init(drain, 1);
+        *abort_flag = 0u;
+        sqd::fence_barrier_init();
+        sqd::fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        if (args.nkb_o > 0) {
+            sqd::prefetch_tensormap(&tm_xo);
+            sqd::prefetch_tensormap(&tm_wo);
+        }
+        if (args.nkb_i > 0) {
+            sqd::prefetch_tensormap(&tm_xn);
+            sqd::prefetch_tensormap(&tm_wn);
+        }
+    }
+    if (warp == 1) {
+        sqd::tmem_alloc_pair(sqd::smem_u32(tmem_slot), C::TMEM_COLS);
+        sqd::tmem_relinquish_pair();
+    }
+    sqd::tc_fence_before();
+    sqd::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
+    sqd::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int nkb_i = args.nkb_i, nkb_o = args.nkb_o;
+    const int per_tile = nkb_o + nkb_i;
+    const int num_tiles = args.tiles_m * args.tiles_n;
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int num_pairs = static_cast<int>(gridDim.x >> 1);
+    const int my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ staging producer (each CTA)
+        // Packed INT4 tiles of this CTA's X rows and W rows, one K-block per
+        // stage, in the order the expansion warps consume them.
+        if (lane == 0 && nkb_i > 0) {
+            const int F = my_tiles * nkb_i;
+            const int r0 = static_cast<int>(rank) * 128;
+            int last_armed = -1;
+            bool ok = true;
+            for (int f = 0; f < F; ++f) {
+                const int lt = f / nkb_i;
+                const int kb = f - lt * nkb_i;
+                int tmi, tni;
+                tile_coords(args, pair + lt * num_pairs, tmi, tni);
+                const int si = f % STG;
+                if (!sqd::mbar_wait(stg_empty(si), ((f / STG) & 1) ^ 1u, abort_flag, SITE_EXP_OP)) { ok = false; break; }
+                sqd::mbar_arrive_expect_tx(stg_full(si), C::STG_BYTES);
+                sqd::tma_load_2d(stg_a(si), &tm_xn, stg_full(si), kb * PROWB, tmi * PAIR_BM + r0);
+                sqd::tma_load_2d(stg_a(si) + C::PA_BYTES, &tm_wn, stg_full(si), kb * PROWB, tni * PAIR_BN + r0);
+                last_armed = f;
+            }
+            if (!ok && last_armed >= 0) sqd::mbar_drain(stg_full(last_armed % STG), (last_armed / STG) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (first CTA)
+        if (leader && lane == 0) {
+            constexpr uint32_t idesc_bf = sqd::make_idesc(false, PAIR_BM, PAIR_BN);
+            constexpr uint32_t idesc_i8 = sqd::make_idesc(true, PAIR_BM, PAIR_BN);
+            bool ok = true;
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                if (!sqd::mbar_wait(acc_empty, (lt & 1) ^ 1u, abort_flag, SITE_MMA_ACC)) { ok = false; break; }
+                sqd::tc_fence_after();
+                for (int i = 0; i < per_tile; ++i) {
+                    const int u = lt * per_tile + i;
+                    const int e = u % OPS;
+                    if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_MMA_FULL)) { ok = false; break; }
+                    sqd::tc_fence_after();
+                    const bool is_bf = i < nkb_o;
+                    const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
+                    const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
+                    const uint32_t d = tmem + (is_bf ? 0u : static_cast<uint32_t>(PAIR_BN));
+                    const bool first = (i == 0) || (i == nkb_o);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t acc = (first && k == 0) ? 0u : 1u;
+                        if (is_bf) sqd::mma_bf16_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_bf, acc);
+                        else sqd::mma_s8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_i8, acc);
+                    }
+                    sqd::mma_commit_pair_multicast(op_empty(e), 0x3);
+                }
+                if (ok) sqd::mma_commit_pair_multicast(acc_full, 0x3);
+            }
+            if (!ok) {
+                sqd::mma_commit_pair(drain);
+                sqd::mbar_drain(drain, 0);
+            }
+        }
+    } else if (warp >= EXP_WARP0) {
+        // ------------------------------------------------------------ operand producers
+        const int et = threadIdx.x - EXP_WARP0 * 32;
+        const int F = my_tiles * nkb_i;
+        const uint32_t r0 = rank * 128u;  // this CTA's row offset inside the pair tile
+
+        // INT4 block f: packed rows from staging stage f % STG -> int8 rows in
+        // operand stage e (the tile's X rows, then its W rows).
+        auto store = [&](int f) -> bool {
+            const int lt = f / nkb_i;
+            const int kb = f - lt * nkb_i;
+            const int u = lt * per_tile + nkb_o + kb;
+            const int e = u % OPS;
+            const int si = f % STG;
+            if (!sqd::mbar_wait(stg_full(si), (f / STG) & 1, abort_flag, SITE_EXP_OP)) return false;
+            if (!sqd::mbar_wait(op_empty(e), ((u / OPS) & 1) ^ 1u, abort_flag, SITE_EXP_OP)) return false;
+            const uint32_t src = stg_a(si);
+            const uint32_t dst = op_a(e);
+            uint4 w[EC];
+#pragma unroll
+            for (int c = 0; c < EC; ++c) {
+                const int q = et + c * EXP_THREADS;
+                w[c] = sqd::lds128(src + (q >> 2) * PROWB + (q & 3) * 16);
+            }
+#pragma unroll
+            for (int c = 0; c < EC; ++c) {
+                const int q = et + c * EXP_THREADS;
+                const int r = q >> 2;
+                const uint32_t j = static_cast<uint32_t>(q & 3);
+                const uint32_t sw = static_cast<uint32_t>(r & 7);
+                const uint32_t row = dst + r * ROWB;
+                sqd::sts128(row + (((2u * j) ^ sw) << 4),
+                            (w[c].x << 4) & 0xF0F0F0F0u, w[c].x & 0xF0F0F0F0u,
+                            (w[c].y << 4) & 0xF0F0F0F0u, w[c].y & 0xF0F0F0F0u);
+                sqd::sts128(row + (((2u * j + 1u) ^ sw) << 4),
+                            (w[c].z << 4) & 0xF0F0F0F0u, w[c].z & 0xF0F0F0F0u,
+                            (w[c].w << 4) & 0xF0F0F0F0u, w[c].w & 0xF0F0F0F0u);
+            }
+            sqd::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                sqd::mbar_arrive(stg_empty(si));
+                sqd::mbar_arrive_cluster(sqd::map_to_cta(op_full(e), 0));
+            }
+            return true;
+        };
+
+        const bool tma_thread = (et == 0);
+        int last_armed = -1;
+        auto produce_bf16 = [&](int lt) -> bool {
+            int tmi, tni;
+            tile_coords(args, pair + lt * num_pairs, tmi, tni);
+            for (int kb = 0; kb < nkb_o; ++kb) {
+                const int u = lt * per_tile + kb;
+                const int e = u % OPS;
+                if (!sqd::mbar_wait(op_empty(e), ((u / OPS) & 1) ^ 1u, abort_flag, SITE_EXP_OP)) return false;
+                const uint32_t full_leader = sqd::map_to_cta(op_full(e), 0);
+                if (tma_thread) {
+                    sqd::mbar_arrive_expect_tx_cluster(full_leader, C::OP_BYTES);
+                    sqd::tma_load_2d_pair(op_a(e), &tm_xo, full_leader, kb * KB_BF,
+                                          tmi * PAIR_BM + static_cast<int>(r0));
+                    sqd::tma_load_2d_pair(op_a(e) + C::A_BYTES, &tm_wo, full_leader, kb * KB_BF,
+                                          tni * PAIR_BN + static_cast<int>(r0));
+                    last_armed = u;
+                } else if (lane == 0) {
+                    sqd::mbar_arrive_cluster(full_leader);
+                }
+            }
+            return true;
+        };
+
+        bool ok = true;
+        if (nkb_i == 0) {
+            for (int lt = 0; lt < my_tiles && ok; ++lt) ok = produce_bf16(lt);
+        } else {
+            for (int f = 0; f < F && ok; ++f) {
+                if (nkb_o > 0 && f % nkb_i == 0 && !produce_bf16(f / nkb_i)) { ok = false; break; }
+                ok = store(f);
+            }
+        }
+        if (!ok && tma_thread && last_armed >= 0 && leader) {
+            // Let the last copies that were issued land before the CTA exits.
+            sqd::mbar_drain(op_full(last_armed % OPS), (last_armed / OPS) & 1);
+        }
+    } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + NUM_EPI_WARPS) {
+        // ------------------------------------------------------------ epilogue (each CTA: its 128 rows)
+        const int sub = warp & 3;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(sub * 32) << 16);
+        const bool has_i = nkb_i > 0, has_o = nkb_o > 0;
+        const uint32_t empty_leader = sqd::map_to_cta(acc_empty, 0);
+        for (int lt = 0; lt < my_tiles; ++lt) {
+            int tmi, tni;
+            tile_coords(args, pair + lt * num_pairs, tmi, tni);
+            if (!sqd::mbar_wait(acc_full, lt & 1, abort_flag, SITE_EPI)) break;
+            sqd::tc_fence_after();
+            const int m = tmi * PAIR_BM + static_cast<int>(rank) * 128 + sub * 32 + lane;
+            const bool row_ok = m < args.M;
+            const float sx = row_ok ? args.s_x[m] : 0.0f;
+            uint16_t *yrow = args.Y + static_cast<long long>(row_ok ? m : 0) * args.ldy;
+#pragma unroll 1
+            for (int c = 0; c < PAIR_BN; c += 32) {
+                uint32_t vi[32], vf[32];
+                if (has_i) sqd::tmem_ld_32x32b_x32(tl + PAIR_BN + c, vi);
+                if (has_o) sqd::tmem_ld_32x32b_x32(tl + c, vf);
+                sqd::tmem_wait_ld();
+                if (c + 32 == PAIR_BN) {
+                    sqd::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) sqd::mbar_arrive_cluster(empty_leader);
+                }
+                const int n0 = tni * PAIR_BN + c;
+                if (!row_ok || n0 >= args.N) continue;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int n = n0 + 8 * g;
+                    if (n >= args.N) break;
+                    const float4 sw0 = __ldg(reinterpret_cast<const float4 *>(args.s_w + n));
+                    const float4 sw1 = __ldg(reinterpret_cast<const float4 *>(args.s_w + n + 4));
+                    const float swv[8] = {sw0.x, sw0.y, sw0.z, sw0.w, sw1.x, sw1.y, sw1.z, sw1.w};
+                    uint32_t out[4];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        float y2[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int t = 8 * g + 2 * h + u;
+                            const int ai = has_i ? (static_cast<int>(vi[t]) >> 8) : 0;
+                            const float af = has_o ? __uint_as_float(vf[t]) : 0.0f;
+                            y2[u] = __fadd_rn(__fmul_rn(__fmul_rn(static_cast<float>(ai), sx), swv[2 * h + u]), af);
+                            if constexpr (DBG) {
+                                if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + 2 * h + u] = ai;
+                                if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n + 2 * h + u] = af;
+                            }
+                        }
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
+                        out[h] = *reinterpret_cast<const uint32_t *>(&b2);
+                    }
+                    *reinterpret_cast<uint4 *>(yrow + n) = make_uint4(out[0], out[1], out[2], out[3]);
+                }
+            }
+        }
+    }
+
+    sqd::tc_fence_before();
+    sqd::cluster_sync();  // every pair MMA and every TMEM read of both CTAs is done
+    if (warp == 1) {
+        sqd::tc_fence_after();
+        sqd::tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace sqg

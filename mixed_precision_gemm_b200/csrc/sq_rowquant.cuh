@@ -5,61 +5,88 @@
 // write-up, section 9: symmetric quantization, columns reordered by the
 // static mask).
 //
-// One CTA handles one row at a time (grid-stride over rows).  The row is read
-// once from HBM with 16-byte loads held in registers; a block reduction gives
-// the absolute maximum over the normal channels; each element then goes
-// either to a code byte in shared memory (at its rank among the normal
-// channels) or to the compact outlier buffer (at its rank in O); finally the
-// codes are packed two per byte and both parts are written with 16-byte
-// stores.  Memory-bound: bytes per row = 2K read + kn_pad/2 + 2 no_pad + 4
-// written.
+// One CTA handles one row at a time (grid-stride over rows) and prefetches
+// its next row into registers while it works on the current one.  Per row:
+//   1. absolute maximum over the normal channels, on packed bf16 magnitude
+//      bits (exact; outlier channels masked out), block reduction;
+//   2. codes of every 8-channel chunk (see quant8 below) scattered as bytes
+//      into shared memory at their rank among the normal channels, outliers
+//      copied to a shared compact buffer at their rank in O;
+//   3. codes packed two per byte and both parts written with 16-byte stores.
+// Shared buffers alternate between consecutive rows, so two block barriers
+// per row suffice.  Memory-bound: bytes per row = 2K read + kn_pad/2 +
+// 2 no_pad + 4 written.
 #pragma once
 
 #include "sq_device.cuh"
 
 namespace sqq {
 
-// Code of x for scale s (s > 0): clamp(rint(fl(x / s)), -7, 7) with the IEEE
-// fp32 quotient fl(x / s).  The quotient is first estimated as x * fl(1/s),
-// which is within 2^-19 of fl(x / s) for |x / s| <= 7.  When the estimate is
-// farther than 2^-16 from every half-integer, both round to the same integer
-// and the estimate is used; otherwise the correctly rounded division decides.
-__device__ __forceinline__ int quant_code(float x, float s, float inv_s, bool fast_ok)
+constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: x + kMagic rounds x to an integer (ties to even)
+
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b)
 {
-    float t;
-    if (fast_ok) {
-        const float r = x * inv_s;
-        const float fr = r - floorf(r);
-        if (fabsf(fr - 0.5f) > 1.52587890625e-05f) {  // 2^-16
-            t = r;
-        } else {
-            t = __fdiv_rn(x, s);
-        }
-    } else {
-        t = __fdiv_rn(x, s);
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Low bytes of four words -> one word (byte i = low byte of word i).
+__device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Exact code: clamp(rint(fl(x / s)), -7, 7) with the IEEE fp32 quotient.
+__device__ __forceinline__ uint32_t exact_code_byte(float x, float s)
+{
+    int q = __float2int_rn(__fdiv_rn(x, s));
+    q = q > 7 ? 7 : (q < -7 ? -7 : q);
+    return static_cast<uint32_t>(q) & 0xFFu;
+}
+
+// Codes of the 8 channels of one chunk as 8 int8 bytes (lo: channels 0..3,
+// hi: 4..7).  Fast path: t = fma(x, inv_s, 1.5*2^23) rounds the exact product
+// x * fl(1/s) to the nearest integer q, whose int8 value is the low byte of t.
+// |x*fl(1/s) - x/s| and |fl(x/s) - x/s| are both below 7 * 2^-24 for
+// |x/s| <= 7, so when the residual x*fl(1/s) - q stays 2^-16 away from +-1/2
+// no half-integer separates x*fl(1/s) from fl(x/s) and q = rint(fl(x/s)).
+// Otherwise (or when 1/s is not safely finite) the correctly rounded
+// division decides.  Codes of outlier channels in the chunk are computed but
+// never used.  For |x| <= a = 7s the result never exceeds 7 in magnitude.
+__device__ __forceinline__ void quant8(const uint4 &v, float s, float inv_s, bool fast_ok, uint32_t &lo,
+                                       uint32_t &hi)
+{
+    const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    uint32_t t[8];
+    float worst = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const float tf = fmaf(x[e], inv_s, kMagic);
+        const float q = tf - kMagic;
+        worst = fmaxf(worst, fabsf(fmaf(x[e], inv_s, -q)));
+        t[e] = __float_as_uint(tf);
     }
-    int q = __float2int_rn(t);
-    q = q > 7 ? 7 : q;
-    q = q < -7 ? -7 : q;
-    return q;
+    if (!fast_ok || worst > 0.49998474121f) {  // 1/2 - 2^-16
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = exact_code_byte(x[e], s);
+    }
+    lo = low_bytes4(t[0], t[1], t[2], t[3]);
+    hi = low_bytes4(t[4], t[5], t[6], t[7]);
 }
 
-__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b)
-{
-    return __uint_as_float(b << 16);
-}
-
-// Packs 32 code bytes (int8, values in [-7, 7]) into 16 bytes, two codes per
-// byte, even code in the low nibble.
+// Packs 8 code bytes (lo4: codes 0..3, hi4: codes 4..7) into 4 bytes, two
+// codes per byte, the even code in the low nibble.
 __device__ __forceinline__ uint32_t pack8_codes(uint32_t lo4, uint32_t hi4)
 {
-    // lo4 holds codes 0..3 (one per byte), hi4 codes 4..7.
-    uint32_t a = lo4 & 0x0F0F0F0Fu;           // nibbles in the low half of each byte
-    uint32_t b = hi4 & 0x0F0F0F0Fu;
-    // byte k of a: code k.  Want nibble 2i = code 2i (low), 2i+1 = code 2i+1 (high).
-    uint32_t pa = (a & 0x000F000Fu) | ((a & 0x0F000F00u) >> 4);  // bytes 0,2: code0|code1<<4, code2|code3<<4
-    uint32_t pb = (b & 0x000F000Fu) | ((b & 0x0F000F00u) >> 4);
-    // pa: byte0 = c0|c1<<4, byte2 = c2|c3<<4 ; pb similarly for c4..c7
+    const uint32_t a = lo4 & 0x0F0F0F0Fu;
+    const uint32_t b = hi4 & 0x0F0F0F0Fu;
+    const uint32_t pa = (a & 0x000F000Fu) | ((a & 0x0F000F00u) >> 4);  // bytes 0, 2: c0|c1<<4, c2|c3<<4
+    const uint32_t pb = (b & 0x000F000Fu) | ((b & 0x0F000F00u) >> 4);
     return __byte_perm(pa, pb, 0x6420);
 }
 
@@ -70,110 +97,126 @@ __global__ void __launch_bounds__(T) rowquant_kernel(
     uint8_t *__restrict__ dst_n, float *__restrict__ dst_s, uint16_t *__restrict__ dst_o)
 {
     extern __shared__ __align__(16) uint8_t rq_smem[];
-    int8_t *qbuf = reinterpret_cast<int8_t *>(rq_smem);                  // [kn_pad] codes
-    uint16_t *obuf = reinterpret_cast<uint16_t *>(rq_smem + kn_pad);     // [no_pad] bf16 bits
-    __shared__ uint32_t red[T / 32];
+    __shared__ uint32_t red[2][T / 32];
+    const int buf_bytes = kn_pad + 2 * no_pad;  // one code buffer + one outlier buffer
 
     const int tid = threadIdx.x;
     const int KN = K - nO;
     const int nchunk = K >> 3;
 
-    // Padding positions are never written by the row loop: zero them once.
-    for (int i = KN + tid; i < kn_pad; i += T) qbuf[i] = 0;
-    for (int i = nO + tid; i < no_pad; i += T) obuf[i] = 0;
+    // Padding positions are never written by the row loop: zero them once in both buffers.
+    for (int b = 0; b < 2; ++b) {
+        int8_t *qb = reinterpret_cast<int8_t *>(rq_smem + b * buf_bytes);
+        uint16_t *ob = reinterpret_cast<uint16_t *>(rq_smem + b * buf_bytes + kn_pad);
+        for (int i = KN + tid; i < kn_pad; i += T) qb[i] = 0;
+        for (int i = nO + tid; i < no_pad; i += T) ob[i] = 0;
+    }
 
-    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    // The channel table is the same for every row: keep this thread's words.
+    uint32_t tb[CPT];
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = tid + i * T;
+        tb[i] = c < nchunk ? __ldg(chan_tab + c) : 0xFFu;
+    }
+
+    uint4 nxt[CPT];
+    auto load_row = [&](int64_t r) {
         const uint16_t *row = src + r * ld;
-        uint4 v[CPT];
-        uint32_t tb[CPT];
 #pragma unroll
         for (int i = 0; i < CPT; ++i) {
             const int c = tid + i * T;
-            if (c < nchunk) {
-                v[i] = sqd::ld_nc_v4(row + 8 * c);
-                tb[i] = __ldg(chan_tab + c);
-            } else {
-                v[i] = make_uint4(0, 0, 0, 0);
-                tb[i] = 0xFFu;  // all outliers: excluded from everything below
-            }
+            nxt[i] = c < nchunk ? sqd::ld_nc_v4(row + 8 * c) : make_uint4(0, 0, 0, 0);
         }
+    };
 
-        // Absolute maximum over the normal channels, on bf16 magnitude bits
-        // (monotone in the value for finite inputs, and exact).
-        uint32_t amax = 0;
+    int64_t r = blockIdx.x;
+    if (r < rows) load_row(r);
+    int parity = 0;
+    for (; r < rows; r += gridDim.x, parity ^= 1) {
+        uint4 v[CPT];
+#pragma unroll
+        for (int i = 0; i < CPT; ++i) v[i] = nxt[i];
+        if (r + gridDim.x < rows) load_row(r + gridDim.x);
+
+        int8_t *qbuf = reinterpret_cast<int8_t *>(rq_smem + parity * buf_bytes);
+        uint16_t *obuf = reinterpret_cast<uint16_t *>(rq_smem + parity * buf_bytes + kn_pad);
+
+        // 1. absolute maximum over the normal channels (bf16 magnitude bits)
+        uint32_t am2 = 0;
 #pragma unroll
         for (int i = 0; i < CPT; ++i) {
-            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+            const uint32_t mask = tb[i] & 0xFFu;
+            uint32_t w[4] = {v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu, v[i].z & 0x7FFF7FFFu, v[i].w & 0x7FFF7FFFu};
+            if (mask) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const uint32_t bits = (w[e >> 1] >> ((e & 1) * 16)) & 0x7FFFu;
-                if (!((tb[i] >> e) & 1u)) amax = bits > amax ? bits : amax;
+                for (int p = 0; p < 4; ++p) {
+                    const uint32_t keep = (((mask >> (2 * p)) & 1u) ? 0u : 0x0000FFFFu) |
+                                          (((mask >> (2 * p + 1)) & 1u) ? 0u : 0xFFFF0000u);
+                    w[p] &= keep;
+                }
             }
+            am2 = max_u16x2(am2, max_u16x2(max_u16x2(w[0], w[1]), max_u16x2(w[2], w[3])));
         }
+        uint32_t amax = max(am2 & 0xFFFFu, am2 >> 16);
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const uint32_t o = __shfl_xor_sync(0xFFFFFFFFu, amax, off);
-            amax = o > amax ? o : amax;
-        }
-        if ((tid & 31) == 0) red[tid >> 5] = amax;
+        for (int off = 16; off > 0; off >>= 1) amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        if ((tid & 31) == 0) red[parity][tid >> 5] = amax;
         __syncthreads();
-        amax = red[0];
+        amax = red[parity][0];
 #pragma unroll
-        for (int wi = 1; wi < T / 32; ++wi) amax = red[wi] > amax ? red[wi] : amax;
+        for (int wi = 1; wi < T / 32; ++wi) amax = max(amax, red[parity][wi]);
 
-        const float a = bf16_bits_to_f32(amax);
+        const float a = __uint_as_float(amax << 16);
         const float s = __fdiv_rn(a, 7.0f);
         const bool zero = (amax == 0u);
         const float inv_s = zero ? 0.0f : __frcp_rn(s);
-        const bool fast_ok = s >= 7.888609052210118e-31f;  // 2^-100: 1/s stays finite
+        const bool fast_ok = zero || s >= 7.888609052210118e-31f;  // 2^-100: 1/s stays finite
         if (tid == 0) dst_s[r] = zero ? 0.0f : s;
 
-        // Scatter: codes to qbuf at their normal rank, outliers to obuf at
-        // their rank in O.
+        // 2. codes -> qbuf at their normal rank, outliers -> obuf at their rank in O
 #pragma unroll
         for (int i = 0; i < CPT; ++i) {
             const int c = tid + i * T;
             if (c >= nchunk) continue;
             const uint32_t mask = tb[i] & 0xFFu;
             const int below = static_cast<int>(tb[i] >> 8);
-            const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+            uint32_t lo, hi;
+            quant8(v[i], s, inv_s, fast_ok, lo, hi);
+            const int p = 8 * c - below;
             if (mask == 0u) {
-                // No outlier in this chunk: 8 consecutive normal ranks.
-                uint32_t packed_lo = 0, packed_hi = 0;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float x = bf16_bits_to_f32((w[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
-                    const int q = zero ? 0 : quant_code(x, s, inv_s, fast_ok);
-                    const uint32_t byte = static_cast<uint32_t>(q) & 0xFFu;
-                    if (e < 4) packed_lo |= byte << (8 * e);
-                    else packed_hi |= byte << (8 * (e - 4));
-                }
-                const int p = 8 * c - below;
                 if ((p & 7) == 0) {
-                    *reinterpret_cast<uint2 *>(qbuf + p) = make_uint2(packed_lo, packed_hi);
+                    *reinterpret_cast<uint2 *>(qbuf + p) = make_uint2(lo, hi);
+                } else if ((p & 3) == 0) {
+                    *reinterpret_cast<uint32_t *>(qbuf + p) = lo;
+                    *reinterpret_cast<uint32_t *>(qbuf + p + 4) = hi;
+                } else if ((p & 1) == 0) {
+                    *reinterpret_cast<uint16_t *>(qbuf + p) = static_cast<uint16_t>(lo);
+                    *reinterpret_cast<uint16_t *>(qbuf + p + 2) = static_cast<uint16_t>(lo >> 16);
+                    *reinterpret_cast<uint16_t *>(qbuf + p + 4) = static_cast<uint16_t>(hi);
+                    *reinterpret_cast<uint16_t *>(qbuf + p + 6) = static_cast<uint16_t>(hi >> 16);
                 } else {
 #pragma unroll
                     for (int e = 0; e < 8; ++e)
-                        qbuf[p + e] = static_cast<int8_t>(((e < 4 ? packed_lo : packed_hi) >> (8 * (e & 3))) & 0xFFu);
+                        qbuf[p + e] = static_cast<int8_t>(((e < 4 ? lo : hi) >> (8 * (e & 3))) & 0xFFu);
                 }
             } else {
+                const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
                 int nlow = 0;  // outliers of this chunk before element e
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const uint32_t bits = (w[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu;
                     if ((mask >> e) & 1u) {
-                        obuf[below + nlow] = static_cast<uint16_t>(bits);
+                        obuf[below + nlow] = static_cast<uint16_t>(w[e >> 1] >> ((e & 1) * 16));
                         ++nlow;
                     } else {
-                        const int q = zero ? 0 : quant_code(bf16_bits_to_f32(bits), s, inv_s, fast_ok);
-                        qbuf[8 * c - below + (e - nlow)] = static_cast<int8_t>(q);
+                        qbuf[p + e - nlow] = static_cast<int8_t>(((e < 4 ? lo : hi) >> (8 * (e & 3))) & 0xFFu);
                     }
                 }
             }
         }
         __syncthreads();
 
-        // Pack and store: 32 codes -> 16 bytes per thread-iteration.
+        // 3. pack and store: 32 codes -> 16 bytes per item; outliers 8 per item
         uint8_t *out_n = dst_n + r * static_cast<int64_t>(kn_pad >> 1);
         for (int j = tid; j < (kn_pad >> 5); j += T) {
             const uint4 c0 = *reinterpret_cast<const uint4 *>(qbuf + 32 * j);
@@ -186,10 +229,10 @@ __global__ void __launch_bounds__(T) rowquant_kernel(
             *reinterpret_cast<uint4 *>(out_n + 16 * j) = o;
         }
         uint16_t *out_o = dst_o + r * static_cast<int64_t>(no_pad);
-        for (int j = tid; j < (no_pad >> 3); j += T) {
+        for (int j = tid; j < (no_pad >> 3); j += T)
             *reinterpret_cast<uint4 *>(out_o + 8 * j) = *reinterpret_cast<const uint4 *>(obuf + 8 * j);
-        }
-        __syncthreads();  // qbuf, obuf and red are reused by the next row
+        // No barrier here: the next row fills the other buffers; this row's
+        // buffers are reused two rows later, after that row's two barriers.
     }
 }
 

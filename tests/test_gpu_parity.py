@@ -126,6 +126,26 @@ def test_edge_shapes(M, K, N, nO):
     check_layer(O.numpy(), X, W, ldy_extra=16)
 
 
+# Shapes that take the CTA-pair kernel (256 x 256 tiles over two SMs): ragged
+# M and N, more outlier blocks than ring slots, and both degenerate outlier sets.
+PAIR_EDGE = [
+    # (M, K, N, nO)
+    (1000, 768, 4872, 200),
+    (520, 2048, 9480, 1500),
+    (512, 256, 9728, 256),
+    (768, 512, 6400, 0),
+]
+
+
+@pytest.mark.parametrize("M,K,N,nO", PAIR_EDGE, ids=lambda v: str(v))
+def test_pair_kernel_edge_shapes(M, K, N, nO):
+    O = workloads.outlier_channels(K, nO, seed=M + K + 1)
+    X = workloads.activations(M, K, O, seed=M + 1)
+    W = workloads.weights(N, K, seed=N + 1)
+    rows = np.unique(np.concatenate([sampled_rows(M, 40), np.arange(248, 264), np.arange(M - 8, M)]))
+    check_layer(O.numpy(), X, W, rows=rows, ldy_extra=8)
+
+
 def test_zero_rows_and_ties():
     M, K, N, nO = 40, 512, 128, 16
     O = workloads.outlier_channels(K, nO, seed=3)
