@@ -37,10 +37,13 @@ namespace sqg {
 constexpr int PAIR_BM = 256;     // tile rows of the pair (128 per CTA)
 constexpr int PAIR_BN = 256;     // tile columns (128 W rows per CTA)
 
-template <int OPS_, int STG_>
+template <int OPS_, int STG_, int NG_>
 struct CfgPair {
     static constexpr int OPS = OPS_;                  // operand ring stages (expanded int8 or bf16 tiles)
     static constexpr int STG = STG_;                  // staging ring stages (packed INT4 tiles)
+    static constexpr int NG = NG_;                    // producer groups; group g owns ring uses u = g mod NG
+    static constexpr int GW = NUM_EXP_WARPS / NG;     // warps per producer group
+    static constexpr int GT = 32 * GW;                // threads per producer group
     static constexpr int A_BYTES = 128 * ROWB;        // this CTA's X rows
     static constexpr int B_BYTES = 128 * ROWB;        // this CTA's W rows
     static constexpr int OP_BYTES = A_BYTES + B_BYTES;
@@ -54,8 +57,9 @@ struct CfgPair {
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
     static constexpr int TMEM_COLS = 512;
-    static constexpr int EXP_CHUNKS = 256 * (PROWB / 16) / EXP_THREADS;  // 4
+    static constexpr int EXP_CHUNKS = 256 * (PROWB / 16) / GT;  // packed 16-byte chunks per thread per K-block
     static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(NUM_EXP_WARPS % NG == 0 && OPS % NG == 0, "every ring slot must belong to one group");
 };
 
 template <class C, bool DBG>
@@ -90,12 +94,12 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
 
     if (threadIdx.x == 0) {
         for (int e = 0; e < OPS; ++e) {
-            sqd::mbar_init(op_full(e), 2 * NUM_EXP_WARPS);  // every producer warp of both CTAs (first CTA's copy)
+            sqd::mbar_init(op_full(e), 2 * C::GW);          // the owning group's warps in both CTAs (first CTA's copy)
             sqd::mbar_init(op_empty(e), 1);                 // multicast commit
         }
         for (int i = 0; i < STG; ++i) {
             sqd::mbar_init(stg_full(i), 1);                 // this CTA's staging TMA (expect-tx)
-            sqd::mbar_init(stg_empty(i), NUM_EXP_WARPS);    // this CTA's expansion warps
+            sqd::mbar_init(stg_empty(i), C::GW);            // the consuming group's warps
         }
         sqd::mbar_init(acc_full, 1);                        // multicast commit
         sqd::mbar_init(acc_empty, 2 * NUM_EPI_WARPS);       // epilogue warps of both CTAs (first CTA's copy)
@@ -189,8 +193,8 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         }
     } else if (warp >= EXP_WARP0) {
         // ------------------------------------------------------------ operand producers
-        const int et = threadIdx.x - EXP_WARP0 * 32;
-        const int F = my_tiles * nkb_i;
+        const int gi = (warp - EXP_WARP0) / C::GW;              // producer group
+        const int et = threadIdx.x - (EXP_WARP0 + gi * C::GW) * 32;  // thread index inside the group
         const uint32_t r0 = rank * 128u;  // this CTA's row offset inside the pair tile
 
         // INT4 block f: packed rows from staging stage f % STG -> int8 rows in
@@ -208,12 +212,12 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             uint4 w[EC];
 #pragma unroll
             for (int c = 0; c < EC; ++c) {
-                const int q = et + c * EXP_THREADS;
+                const int q = et + c * C::GT;
                 w[c] = sqd::lds128(src + (q >> 2) * PROWB + (q & 3) * 16);
             }
 #pragma unroll
             for (int c = 0; c < EC; ++c) {
-                const int q = et + c * EXP_THREADS;
+                const int q = et + c * C::GT;
                 const int r = q >> 2;
                 const uint32_t j = static_cast<uint32_t>(q & 3);
                 const uint32_t sw = static_cast<uint32_t>(r & 7);
@@ -236,36 +240,34 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
 
         const bool tma_thread = (et == 0);
         int last_armed = -1;
-        auto produce_bf16 = [&](int lt) -> bool {
+        // bf16 block kb of tile lt: the group's first thread issues the two TMA
+        // loads with their byte count; every other warp of the group arrives.
+        auto produce_bf16 = [&](int lt, int kb) -> bool {
             int tmi, tni;
             tile_coords(args, pair + lt * num_pairs, tmi, tni);
-            for (int kb = 0; kb < nkb_o; ++kb) {
-                const int u = lt * per_tile + kb;
-                const int e = u % OPS;
-                if (!sqd::mbar_wait(op_empty(e), ((u / OPS) & 1) ^ 1u, abort_flag, SITE_EXP_OP)) return false;
-                const uint32_t full_leader = sqd::map_to_cta(op_full(e), 0);
-                if (tma_thread) {
-                    sqd::mbar_arrive_expect_tx_cluster(full_leader, C::OP_BYTES);
-                    sqd::tma_load_2d_pair(op_a(e), &tm_xo, full_leader, kb * KB_BF,
-                                          tmi * PAIR_BM + static_cast<int>(r0));
-                    sqd::tma_load_2d_pair(op_a(e) + C::A_BYTES, &tm_wo, full_leader, kb * KB_BF,
-                                          tni * PAIR_BN + static_cast<int>(r0));
-                    last_armed = u;
-                } else if (lane == 0) {
-                    sqd::mbar_arrive_cluster(full_leader);
-                }
+            const int u = lt * per_tile + kb;
+            const int e = u % OPS;
+            if (!sqd::mbar_wait(op_empty(e), ((u / OPS) & 1) ^ 1u, abort_flag, SITE_EXP_OP)) return false;
+            const uint32_t full_leader = sqd::map_to_cta(op_full(e), 0);
+            if (tma_thread) {
+                sqd::mbar_arrive_expect_tx_cluster(full_leader, C::OP_BYTES);
+                sqd::tma_load_2d_pair(op_a(e), &tm_xo, full_leader, kb * KB_BF, tmi * PAIR_BM + static_cast<int>(r0));
+                sqd::tma_load_2d_pair(op_a(e) + C::A_BYTES, &tm_wo, full_leader, kb * KB_BF,
+                                      tni * PAIR_BN + static_cast<int>(r0));
+                last_armed = u;
+            } else if (lane == 0) {
+                sqd::mbar_arrive_cluster(full_leader);
             }
             return true;
         };
 
+        // Ring uses of this group, in order: u = gi, gi + NG, ...
         bool ok = true;
-        if (nkb_i == 0) {
-            for (int lt = 0; lt < my_tiles && ok; ++lt) ok = produce_bf16(lt);
-        } else {
-            for (int f = 0; f < F && ok; ++f) {
-                if (nkb_o > 0 && f % nkb_i == 0 && !produce_bf16(f / nkb_i)) { ok = false; break; }
-                ok = store(f);
-            }
+        const int total = my_tiles * per_tile;
+        for (int u = gi; u < total && ok; u += C::NG) {
+            const int lt = u / per_tile;
+            const int i = u - lt * per_tile;
+            ok = (i < nkb_o) ? produce_bf16(lt, i) : store(lt * nkb_i + (i - nkb_o));
         }
         if (!ok && tma_thread && last_armed >= 0 && leader) {
             // Let the last copies that were issued land before the CTA exits.
