@@ -152,11 +152,15 @@ sq_status launch_rowquant(const uint16_t *src, int64_t rows, int64_t K, int64_t 
     const int no_pad = static_cast<int>(sq_no_pad(nO));
     const int64_t nchunk = K / 8;
     const int k = static_cast<int>(K), no = static_cast<int>(nO);
-    if (nchunk <= 256) return launch_rowquant_t<256, 1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 512) return launch_rowquant_t<256, 2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 1024) return launch_rowquant_t<512, 2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 2048) return launch_rowquant_t<1024, 2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 4096) return launch_rowquant_t<1024, 4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    // Few threads per row and many channels per thread: the per-row reduction
+    // and barriers are amortised over up to 64 elements per thread.
+    if (nchunk <= 64) return launch_rowquant_t<64, 1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 128) return launch_rowquant_t<64, 2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 256) return launch_rowquant_t<64, 4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 512) return launch_rowquant_t<64, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 1024) return launch_rowquant_t<128, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 2048) return launch_rowquant_t<256, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (nchunk <= 4096) return launch_rowquant_t<512, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
     return launch_rowquant_t<1024, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
 }
 
@@ -253,7 +257,7 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
     auto kern = dbg ? sqg::dual_gemm_pair_kernel<C, true> : sqg::dual_gemm_pair_kernel<C, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
-    kern<<<static_cast<unsigned>(2 * clusters), sqg::NUM_THREADS, C::SMEM_BYTES, stream>>>(m_xo, m_wo, m_xn, m_wn, a);
+    kern<<<static_cast<unsigned>(2 * clusters), sqg::PAIR_THREADS, C::SMEM_BYTES, stream>>>(m_xo, m_wo, m_xn, m_wn, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "gemm pair launch");
     return SQ_OK;
 }

@@ -9,15 +9,16 @@
 // the 128 x 256 tile of the single-CTA kernel with a third fewer operand bytes
 // to fetch and expand, which is what the INT4 -> int8 expansion is bound by.
 //
-// Roles (14 warps per CTA, one cluster of 2 CTAs per SM pair, tiles handed
+// Roles (18 warps per CTA, one cluster of 2 CTAs per SM pair, tiles handed
 // out round-robin to clusters):
 //   warp 0 (each CTA)        TMA producer of the packed INT4 tiles (this CTA's
 //                            X rows and W rows) into a staging ring.
 //   warp 1 of the first CTA  issues every pair MMA; its commits arrive on the
 //                            barriers of both CTAs (multicast commit).
-//   warps 2..5 (each CTA)    epilogue of the CTA's 128 rows; they report to the
-//                            first CTA's acc_empty barrier when TMEM is read.
-//   warps 6..13 (each CTA)   operand producers for the CTA's halves, in ring
+//   warps 2..9 (each CTA)    epilogue of the CTA's 128 rows (two warps per TMEM
+//                            lane quarter); they report to the first CTA's
+//                            acc_empty barrier when TMEM is read.
+//   warps 10..17 (each CTA)  operand producers for the CTA's halves, in ring
 //                            order: bf16 blocks by TMA (.cta_group::2 form, no
 //                            multicast, completion bytes counted on the first
 //                            CTA's barrier); INT4 blocks expanded from the
@@ -36,6 +37,10 @@ namespace sqg {
 
 constexpr int PAIR_BM = 256;     // tile rows of the pair (128 per CTA)
 constexpr int PAIR_BN = 256;     // tile columns (128 W rows per CTA)
+constexpr int PAIR_EPI_WARP0 = 2;
+constexpr int PAIR_EPI_WARPS = 8;  // two per TMEM lane quarter, each half of the columns
+constexpr int PAIR_EXP_WARP0 = PAIR_EPI_WARP0 + PAIR_EPI_WARPS;
+constexpr int PAIR_THREADS = 32 * (PAIR_EXP_WARP0 + NUM_EXP_WARPS);
 
 template <int OPS_, int STG_, int NG_>
 struct CfgPair {
@@ -63,7 +68,7 @@ struct CfgPair {
 };
 
 template <class C, bool DBG>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
 dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_constant__ CUtensorMap tm_wo,
                       const __grid_constant__ CUtensorMap tm_xn, const __grid_constant__ CUtensorMap tm_wn,
                       const GemmArgs args)
@@ -102,7 +107,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             sqd::mbar_init(stg_empty(i), C::GW);            // the consuming group's warps
         }
         sqd::mbar_init(acc_full, 1);                        // multicast commit
-        sqd::mbar_init(acc_empty, 2 * NUM_EPI_WARPS);       // epilogue warps of both CTAs (first CTA's copy)
+        sqd::mbar_init(acc_empty, 2 * PAIR_EPI_WARPS);      // epilogue warps of both CTAs (first CTA's copy)
         sqd::mbar_init(drain, 1);
         *abort_flag = 0u;
         sqd::fence_barrier_init();
@@ -191,10 +196,10 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                 sqd::mbar_drain(drain, 0);
             }
         }
-    } else if (warp >= EXP_WARP0) {
+    } else if (warp >= PAIR_EXP_WARP0) {
         // ------------------------------------------------------------ operand producers
-        const int gi = (warp - EXP_WARP0) / C::GW;              // producer group
-        const int et = threadIdx.x - (EXP_WARP0 + gi * C::GW) * 32;  // thread index inside the group
+        const int gi = (warp - PAIR_EXP_WARP0) / C::GW;              // producer group
+        const int et = threadIdx.x - (PAIR_EXP_WARP0 + gi * C::GW) * 32;  // thread index inside the group
         const uint32_t r0 = rank * 128u;  // this CTA's row offset inside the pair tile
 
         // INT4 block f: packed rows from staging stage f % STG -> int8 rows in
@@ -273,12 +278,18 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             // Let the last copies that were issued land before the CTA exits.
             sqd::mbar_drain(op_full(last_armed % OPS), (last_armed / OPS) & 1);
         }
-    } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + NUM_EPI_WARPS) {
+    } else if (warp >= PAIR_EPI_WARP0 && warp < PAIR_EPI_WARP0 + PAIR_EPI_WARPS) {
         // ------------------------------------------------------------ epilogue (each CTA: its 128 rows)
+        // Warp w reads TMEM lane quarter w % 4 and half (w - 2) / 4 of the 256
+        // columns, 16 columns at a time; the load of the next 16 columns is in
+        // flight while the current ones are scaled, fused and stored.
         const int sub = warp & 3;
+        const int half = (warp - PAIR_EPI_WARP0) >> 2;
         const uint32_t tl = tmem + (static_cast<uint32_t>(sub * 32) << 16);
         const bool has_i = nkb_i > 0, has_o = nkb_o > 0;
         const uint32_t empty_leader = sqd::map_to_cta(acc_empty, 0);
+        constexpr int CW = 16;                   // columns per TMEM load
+        constexpr int NCH = (PAIR_BN / 2) / CW;  // 8 loads per accumulator per warp
         for (int lt = 0; lt < my_tiles; ++lt) {
             int tmi, tni;
             tile_coords(args, pair + lt * num_pairs, tmi, tni);
@@ -288,45 +299,56 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             const bool row_ok = m < args.M;
             const float sx = row_ok ? args.s_x[m] : 0.0f;
             uint16_t *yrow = args.Y + static_cast<long long>(row_ok ? m : 0) * args.ldy;
-#pragma unroll 1
-            for (int c = 0; c < PAIR_BN; c += 32) {
-                uint32_t vi[32], vf[32];
-                if (has_i) sqd::tmem_ld_32x32b_x32(tl + PAIR_BN + c, vi);
-                if (has_o) sqd::tmem_ld_32x32b_x32(tl + c, vf);
-                sqd::tmem_wait_ld();
-                if (c + 32 == PAIR_BN) {
-                    sqd::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) sqd::mbar_arrive_cluster(empty_leader);
-                }
-                const int n0 = tni * PAIR_BN + c;
-                if (!row_ok || n0 >= args.N) continue;
+            const int c_base = half * (PAIR_BN / 2);
+            uint32_t vi[2][CW] = {}, vf[2][CW] = {};
+            auto issue = [&](int ch, int b) {
+                if (has_i) sqd::tmem_ld_32x32b_x16(tl + PAIR_BN + c_base + ch * CW, vi[b]);
+                if (has_o) sqd::tmem_ld_32x32b_x16(tl + c_base + ch * CW, vf[b]);
+            };
+            issue(0, 0);
+            sqd::tmem_wait_ld_dep(vi[0], vf[0]);
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const int n = n0 + 8 * g;
-                    if (n >= args.N) break;
-                    const float4 sw0 = __ldg(reinterpret_cast<const float4 *>(args.s_w + n));
-                    const float4 sw1 = __ldg(reinterpret_cast<const float4 *>(args.s_w + n + 4));
-                    const float swv[8] = {sw0.x, sw0.y, sw0.z, sw0.w, sw1.x, sw1.y, sw1.z, sw1.w};
-                    uint32_t out[4];
+            for (int ch = 0; ch < NCH; ++ch) {
+                const int b = ch & 1;
+                if (ch + 1 < NCH) issue(ch + 1, b ^ 1);
+                const int n0 = tni * PAIR_BN + c_base + ch * CW;
+                if (row_ok && n0 < args.N) {
 #pragma unroll
-                    for (int h = 0; h < 4; ++h) {
-                        float y2[2];
+                    for (int g = 0; g < CW / 8; ++g) {
+                        const int n = n0 + 8 * g;
+                        if (n >= args.N) break;
+                        const float4 sw0 = __ldg(reinterpret_cast<const float4 *>(args.s_w + n));
+                        const float4 sw1 = __ldg(reinterpret_cast<const float4 *>(args.s_w + n + 4));
+                        const float swv[8] = {sw0.x, sw0.y, sw0.z, sw0.w, sw1.x, sw1.y, sw1.z, sw1.w};
+                        uint32_t out[4];
 #pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int t = 8 * g + 2 * h + u;
-                            const int ai = has_i ? (static_cast<int>(vi[t]) >> 8) : 0;
-                            const float af = has_o ? __uint_as_float(vf[t]) : 0.0f;
-                            y2[u] = __fadd_rn(__fmul_rn(__fmul_rn(static_cast<float>(ai), sx), swv[2 * h + u]), af);
-                            if constexpr (DBG) {
-                                if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + 2 * h + u] = ai;
-                                if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n + 2 * h + u] = af;
+                        for (int h = 0; h < 4; ++h) {
+                            float y2[2];
+#pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int t = 8 * g + 2 * h + u;
+                                const int ai = has_i ? (static_cast<int>(vi[b][t]) >> 8) : 0;
+                                const float af = has_o ? __uint_as_float(vf[b][t]) : 0.0f;
+                                y2[u] = __fadd_rn(__fmul_rn(__fmul_rn(static_cast<float>(ai), sx), swv[2 * h + u]), af);
+                                if constexpr (DBG) {
+                                    if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + 2 * h + u] = ai;
+                                    if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n + 2 * h + u] = af;
+                                }
                             }
+                            const __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
+                            out[h] = *reinterpret_cast<const uint32_t *>(&b2);
                         }
-                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
-                        out[h] = *reinterpret_cast<const uint32_t *>(&b2);
+                        *reinterpret_cast<uint4 *>(yrow + n) = make_uint4(out[0], out[1], out[2], out[3]);
                     }
-                    *reinterpret_cast<uint4 *>(yrow + n) = make_uint4(out[0], out[1], out[2], out[3]);
+                }
+                if (ch + 1 < NCH) {
+                    sqd::tmem_wait_ld_dep(vi[b ^ 1], vf[b ^ 1]);
+                    if (ch + 2 == NCH) {
+                        // Last load of this warp landed: the accumulators may be reused.
+                        sqd::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) sqd::mbar_arrive_cluster(empty_leader);
+                    }
                 }
             }
         }

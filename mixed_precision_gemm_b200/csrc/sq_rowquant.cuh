@@ -5,8 +5,11 @@
 // write-up, section 9: symmetric quantization, columns reordered by the
 // static mask).
 //
-// One CTA handles one row at a time (grid-stride over rows) and prefetches
-// its next row into registers while it works on the current one.  Per row:
+// One small CTA (64 threads for K <= 4096) handles one row at a time
+// (grid-stride over rows), so each thread holds up to 8 chunks of 8 channels
+// and the per-row fixed work (reduction, scale, barriers, packing set-up) is
+// spread over many elements; with few chunks per thread it also prefetches
+// its next row into registers.  Per row:
 //   1. absolute maximum over the normal channels, on packed bf16 magnitude
 //      bits (exact; outlier channels masked out), block reduction;
 //   2. codes of every 8-channel chunk (see quant8 below) scattered as bytes
@@ -48,6 +51,22 @@ __device__ __forceinline__ uint32_t exact_code_byte(float x, float s)
     return static_cast<uint32_t>(q) & 0xFFu;
 }
 
+__device__ __forceinline__ float bf16_lo(uint32_t w);
+__device__ __forceinline__ float bf16_hi(uint32_t w);
+__device__ __forceinline__ uint32_t low_bytes4(uint32_t a, uint32_t b, uint32_t c, uint32_t d);
+
+// The 8 codes of a chunk by correctly rounded division (rare path, kept out
+// of line so that the common path stays small).
+__device__ __noinline__ uint2 quant8_exact(uint4 v, float s)
+{
+    const float x[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                        bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+    uint32_t t[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) t[e] = exact_code_byte(x[e], s);
+    return make_uint2(low_bytes4(t[0], t[1], t[2], t[3]), low_bytes4(t[4], t[5], t[6], t[7]));
+}
+
 // Codes of the 8 channels of one chunk as 8 int8 bytes (lo: channels 0..3,
 // hi: 4..7).  Fast path: t = fma(x, inv_s, 1.5*2^23) rounds the exact product
 // x * fl(1/s) to the nearest integer q, whose int8 value is the low byte of t.
@@ -72,8 +91,10 @@ __device__ __forceinline__ void quant8(const uint4 &v, float s, float inv_s, boo
         t[e] = __float_as_uint(tf);
     }
     if (!fast_ok || worst > 0.49998474121f) {  // 1/2 - 2^-16
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = exact_code_byte(x[e], s);
+        const uint2 ex = quant8_exact(v, s);
+        lo = ex.x;
+        hi = ex.y;
+        return;
     }
     lo = low_bytes4(t[0], t[1], t[2], t[3]);
     hi = low_bytes4(t[4], t[5], t[6], t[7]);
@@ -91,7 +112,7 @@ __device__ __forceinline__ uint32_t pack8_codes(uint32_t lo4, uint32_t hi4)
 }
 
 template <int T, int CPT>
-__global__ void __launch_bounds__(T) rowquant_kernel(
+__global__ void __launch_bounds__(T, (T >= 512 ? 1 : 512 / T)) rowquant_kernel(
     const uint16_t *__restrict__ src, int64_t rows, int K, int64_t ld,
     const uint32_t *__restrict__ chan_tab, int nO, int kn_pad, int no_pad,
     uint8_t *__restrict__ dst_n, float *__restrict__ dst_s, uint16_t *__restrict__ dst_o)
@@ -120,24 +141,31 @@ __global__ void __launch_bounds__(T) rowquant_kernel(
         tb[i] = c < nchunk ? __ldg(chan_tab + c) : 0xFFu;
     }
 
-    uint4 nxt[CPT];
-    auto load_row = [&](int64_t r) {
+    constexpr bool kPrefetch = CPT <= 4;  // registers allow holding the next row too
+    uint4 nxt[kPrefetch ? CPT : 1];
+    auto load_row = [&](int64_t r, uint4 *dst) {
         const uint16_t *row = src + r * ld;
 #pragma unroll
         for (int i = 0; i < CPT; ++i) {
             const int c = tid + i * T;
-            nxt[i] = c < nchunk ? sqd::ld_nc_v4(row + 8 * c) : make_uint4(0, 0, 0, 0);
+            dst[i] = c < nchunk ? sqd::ld_nc_v4(row + 8 * c) : make_uint4(0, 0, 0, 0);
         }
     };
 
     int64_t r = blockIdx.x;
-    if (r < rows) load_row(r);
+    if constexpr (kPrefetch) {
+        if (r < rows) load_row(r, nxt);
+    }
     int parity = 0;
     for (; r < rows; r += gridDim.x, parity ^= 1) {
         uint4 v[CPT];
+        if constexpr (kPrefetch) {
 #pragma unroll
-        for (int i = 0; i < CPT; ++i) v[i] = nxt[i];
-        if (r + gridDim.x < rows) load_row(r + gridDim.x);
+            for (int i = 0; i < CPT; ++i) v[i] = nxt[i];
+            if (r + gridDim.x < rows) load_row(r + gridDim.x, nxt);
+        } else {
+            load_row(r, v);
+        }
 
         int8_t *qbuf = reinterpret_cast<int8_t *>(rq_smem + parity * buf_bytes);
         uint16_t *obuf = reinterpret_cast<uint16_t *>(rq_smem + parity * buf_bytes + kn_pad);
