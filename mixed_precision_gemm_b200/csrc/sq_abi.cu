@@ -262,7 +262,7 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
     return SQ_OK;
 }
 
-using CfgPair = sqg::CfgPair<4, 6, 2>;
+using CfgPair = sqg::CfgPair<4, 5, 2>;
 
 using CfgN256 = sqg::Cfg<256, 4>;
 using CfgN128 = sqg::Cfg<128, 6>;

@@ -60,7 +60,8 @@ struct CfgPair {
     // barriers: op_full[OPS] op_empty[OPS] stg_full[STG] stg_empty[STG] acc_full acc_empty drain
     static constexpr int NBAR = 2 * OPS + 2 * STG + 3;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
-    static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+    static constexpr int OFF_SW = (OFF_MISC + 16 + 15) / 16 * 16;   // per epilogue warp: its 128 s_w values
+    static constexpr int SMEM_BYTES = OFF_SW + PAIR_EPI_WARPS * 128 * 4 + 1024;
     static constexpr int TMEM_COLS = 512;
     static constexpr int EXP_CHUNKS = 256 * (PROWB / 16) / GT;  // packed 16-byte chunks per thread per K-block
     static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -293,13 +294,22 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         for (int lt = 0; lt < my_tiles; ++lt) {
             int tmi, tni;
             tile_coords(args, pair + lt * num_pairs, tmi, tni);
-            if (!sqd::mbar_wait(acc_full, lt & 1, abort_flag, SITE_EPI)) break;
-            sqd::tc_fence_after();
             const int m = tmi * PAIR_BM + static_cast<int>(rank) * 128 + sub * 32 + lane;
             const bool row_ok = m < args.M;
+            const int c_base = half * (PAIR_BN / 2);
+            // Scales of this warp's 128 columns and of this lane's row, fetched
+            // while the tile's MMAs still run.
+            const int ncol = tni * PAIR_BN + c_base + 4 * lane;
+            const float4 swp = ncol < args.N ? __ldg(reinterpret_cast<const float4 *>(args.s_w + ncol))
+                                             : make_float4(0.f, 0.f, 0.f, 0.f);
             const float sx = row_ok ? args.s_x[m] : 0.0f;
             uint16_t *yrow = args.Y + static_cast<long long>(row_ok ? m : 0) * args.ldy;
-            const int c_base = half * (PAIR_BN / 2);
+            if (!sqd::mbar_wait(acc_full, lt & 1, abort_flag, SITE_EPI)) break;
+            sqd::tc_fence_after();
+            const uint32_t sw_smem = sbase + C::OFF_SW + (warp - PAIR_EPI_WARP0) * 512;
+            sqd::sts128(sw_smem + 16 * lane, __float_as_uint(swp.x), __float_as_uint(swp.y), __float_as_uint(swp.z),
+                        __float_as_uint(swp.w));
+            __syncwarp();
             uint32_t vi[2][CW] = {}, vf[2][CW] = {};
             auto issue = [&](int ch, int b) {
                 if (has_i) sqd::tmem_ld_32x32b_x16(tl + PAIR_BN + c_base + ch * CW, vi[b]);
@@ -317,9 +327,11 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                     for (int g = 0; g < CW / 8; ++g) {
                         const int n = n0 + 8 * g;
                         if (n >= args.N) break;
-                        const float4 sw0 = __ldg(reinterpret_cast<const float4 *>(args.s_w + n));
-                        const float4 sw1 = __ldg(reinterpret_cast<const float4 *>(args.s_w + n + 4));
-                        const float swv[8] = {sw0.x, sw0.y, sw0.z, sw0.w, sw1.x, sw1.y, sw1.z, sw1.w};
+                        const uint4 sw0 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g));
+                        const uint4 sw1 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g + 4));
+                        const float swv[8] = {__uint_as_float(sw0.x), __uint_as_float(sw0.y), __uint_as_float(sw0.z),
+                                              __uint_as_float(sw0.w), __uint_as_float(sw1.x), __uint_as_float(sw1.y),
+                                              __uint_as_float(sw1.z), __uint_as_float(sw1.w)};
                         uint32_t out[4];
 #pragma unroll
                         for (int h = 0; h < 4; ++h) {
