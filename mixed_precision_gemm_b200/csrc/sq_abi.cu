@@ -123,8 +123,8 @@ sq_status launch_rowquant_t(const DevInfo &di, const uint16_t *src, int64_t rows
                             uint16_t *dout, cudaStream_t stream)
 {
     auto kern = sqq::rowquant_kernel<T, CPT>;
-    // two alternating (code buffer + outlier buffer) pairs
-    const size_t smem = 2u * (static_cast<size_t>(kn_pad) + 2u * static_cast<size_t>(no_pad));
+    // two alternating (packed code row + outlier row) pairs, selector and keep tables
+    const size_t smem = 2u * (static_cast<size_t>(kn_pad / 2) + 16u + 2u * static_cast<size_t>(no_pad)) + 256u * 24u;
     cudaError_t e;
     if (smem > 48 * 1024) {
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))) !=

@@ -12,10 +12,14 @@
 // its next row into registers.  Per row:
 //   1. absolute maximum over the normal channels, on packed bf16 magnitude
 //      bits (exact; outlier channels masked out), block reduction;
-//   2. codes of every 8-channel chunk (see quant8 below) scattered as bytes
-//      into shared memory at their rank among the normal channels, outliers
-//      copied to a shared compact buffer at their rank in O;
-//   3. codes packed two per byte and both parts written with 16-byte stores.
+//   2. codes of every 8-channel chunk (see quant8_pairs below) packed into one
+//      32-bit nibble word -- the normal channels' codes first moved to the
+//      front with a byte permutation from a 256-entry table, the same steps
+//      for every chunk -- and OR-ed into a packed row in shared memory at
+//      their rank among the normal channels (two shared atomics, so
+//      neighbouring chunks never race); outliers go to a shared compact
+//      buffer at their rank in O (in step 1, before the maximum);
+//   3. both rows written out with 16-byte stores.
 // Shared buffers alternate between consecutive rows, so two block barriers
 // per row suffice.  Memory-bound: bytes per row = 2K read + kn_pad/2 +
 // 2 no_pad + 4 written.
@@ -111,26 +115,126 @@ __device__ __forceinline__ uint32_t pack8_codes(uint32_t lo4, uint32_t hi4)
     return __byte_perm(pa, pb, 0x6420);
 }
 
+// ---------------------------------------------------------------- paired fp32 arithmetic
+// sm_100 executes two fp32 operations per instruction on register pairs.
+__device__ __forceinline__ uint64_t f2_pack(uint32_t lo, uint32_t hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, uint32_t &lo, uint32_t &hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// Per-row quantizer constants, as fp32 pairs.
+struct RowScale {
+    uint64_t inv2;   // (fl(1/s), fl(1/s))
+    uint64_t negs2;  // (-s, -s)
+    uint64_t magic2; // (1.5 * 2^23, 1.5 * 2^23)
+};
+
+// Codes of the 8 channels of a chunk as int8 bytes (lo: channels 0..3, hi:
+// 4..7).  The fp32 quotient fl(x / s) is obtained with Markstein's correction
+// (P. Markstein, "Computation of elementary functions on the IBM RISC
+// System/6000 processor", IBM J. Res. Dev. 34(1), 1990; restated as the
+// "correcting the quotient" theorem in Muller et al., Handbook of
+// Floating-Point Arithmetic): with y = fl(1/s) and q0 = fl(x * y), which is
+// within one ulp of x / s, the residual r = x - s * q0 is exact in one fused
+// multiply-add and fl(q0 + r * y) is the correctly rounded quotient.  Adding
+// 1.5 * 2^23 then rounds it to the nearest integer, ties to even, and the
+// low byte of the sum is that integer as int8.  Needs 1/s finite and no
+// underflow near a rounding tie (tiny |x / s| rounds to 0 either way); rows
+// with s < 2^-100 take the division path instead.  |x| <= 7 s keeps the code
+// within [-7, 7].
+__device__ __forceinline__ void quant8_pairs(const uint4 &v, const RowScale &rs, uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t t[8];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const uint64_t x = f2_pack(w[p] << 16, w[p] & 0xFFFF0000u);
+        const uint64_t q0 = f2_mul(x, rs.inv2);
+        const uint64_t r = f2_fma(q0, rs.negs2, x);
+        const uint64_t q1 = f2_fma(r, rs.inv2, q0);
+        f2_unpack(f2_add(q1, rs.magic2), t[2 * p], t[2 * p + 1]);
+    }
+    lo = low_bytes4(t[0], t[1], t[2], t[3]);
+    hi = low_bytes4(t[4], t[5], t[6], t[7]);
+}
+
+// Byte-compaction selectors: for an 8-bit outlier mask m, the byte_perm
+// selectors (low word, high word) that move the codes of the normal channels
+// of a chunk to the front, in channel order.
+__device__ __forceinline__ uint2 compaction_selectors(uint32_t m)
+{
+    uint32_t sel[2] = {0u, 0u};
+    int t = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        if (!((m >> e) & 1u)) {
+            sel[t >> 2] |= static_cast<uint32_t>(e) << (4 * (t & 3));
+            ++t;
+        }
+    }
+    return make_uint2(sel[0], sel[1]);
+}
+
+// Keep masks for an 8-bit outlier mask: word p clears the bf16 halves of
+// pair p that are outliers.
+__device__ __forceinline__ uint4 keep_words(uint32_t m)
+{
+    uint32_t k[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+        k[p] = (((m >> (2 * p)) & 1u) ? 0u : 0x0000FFFFu) | (((m >> (2 * p + 1)) & 1u) ? 0u : 0xFFFF0000u);
+    return make_uint4(k[0], k[1], k[2], k[3]);
+}
+
 template <int T, int CPT>
 __global__ void __launch_bounds__(T, (T >= 512 ? 1 : 512 / T)) rowquant_kernel(
     const uint16_t *__restrict__ src, int64_t rows, int K, int64_t ld,
     const uint32_t *__restrict__ chan_tab, int nO, int kn_pad, int no_pad,
     uint8_t *__restrict__ dst_n, float *__restrict__ dst_s, uint16_t *__restrict__ dst_o)
 {
+    // Shared memory: two alternating (packed code row [kn_pad/2 + 16 bytes] +
+    // outlier row [2 no_pad bytes]) pairs, then 256 compaction selectors and
+    // 256 keep masks.
     extern __shared__ __align__(16) uint8_t rq_smem[];
     __shared__ uint32_t red[2][T / 32];
-    const int buf_bytes = kn_pad + 2 * no_pad;  // one code buffer + one outlier buffer
+    const int pk_bytes = kn_pad >> 1;
+    const int pk_alloc = pk_bytes + 16;  // room for the second OR of the last chunk
+    const int buf_bytes = pk_alloc + 2 * no_pad;
+    uint2 *sel_tab = reinterpret_cast<uint2 *>(rq_smem + 2 * buf_bytes);
+    uint4 *keep_tab = reinterpret_cast<uint4 *>(rq_smem + 2 * buf_bytes + 256 * 8);
 
     const int tid = threadIdx.x;
-    const int KN = K - nO;
     const int nchunk = K >> 3;
 
-    // Padding positions are never written by the row loop: zero them once in both buffers.
-    for (int b = 0; b < 2; ++b) {
-        int8_t *qb = reinterpret_cast<int8_t *>(rq_smem + b * buf_bytes);
-        uint16_t *ob = reinterpret_cast<uint16_t *>(rq_smem + b * buf_bytes + kn_pad);
-        for (int i = KN + tid; i < kn_pad; i += T) qb[i] = 0;
-        for (int i = nO + tid; i < no_pad; i += T) ob[i] = 0;
+    for (int i = tid; i < 2 * buf_bytes / 16; i += T)
+        reinterpret_cast<uint4 *>(rq_smem)[i] = make_uint4(0, 0, 0, 0);
+    for (int m = tid; m < 256; m += T) {
+        sel_tab[m] = compaction_selectors(static_cast<uint32_t>(m));
+        keep_tab[m] = keep_words(static_cast<uint32_t>(m));
     }
 
     // The channel table is the same for every row: keep this thread's words.
@@ -156,6 +260,7 @@ __global__ void __launch_bounds__(T, (T >= 512 ? 1 : 512 / T)) rowquant_kernel(
     if constexpr (kPrefetch) {
         if (r < rows) load_row(r, nxt);
     }
+    __syncthreads();  // zeroed buffers and tables visible
     int parity = 0;
     for (; r < rows; r += gridDim.x, parity ^= 1) {
         uint4 v[CPT];
@@ -167,24 +272,32 @@ __global__ void __launch_bounds__(T, (T >= 512 ? 1 : 512 / T)) rowquant_kernel(
             load_row(r, v);
         }
 
-        int8_t *qbuf = reinterpret_cast<int8_t *>(rq_smem + parity * buf_bytes);
-        uint16_t *obuf = reinterpret_cast<uint16_t *>(rq_smem + parity * buf_bytes + kn_pad);
+        uint32_t *pbuf = reinterpret_cast<uint32_t *>(rq_smem + parity * buf_bytes);          // packed codes
+        uint16_t *obuf = reinterpret_cast<uint16_t *>(rq_smem + parity * buf_bytes + pk_alloc);  // outliers
 
-        // 1. absolute maximum over the normal channels (bf16 magnitude bits)
+        // 1. outliers to obuf at their rank in O and cleared from the chunk;
+        //    absolute maximum over what is left (bf16 magnitude bits)
         uint32_t am2 = 0;
 #pragma unroll
         for (int i = 0; i < CPT; ++i) {
             const uint32_t mask = tb[i] & 0xFFu;
-            uint32_t w[4] = {v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu, v[i].z & 0x7FFF7FFFu, v[i].w & 0x7FFF7FFFu};
-            if (mask) {
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    const uint32_t keep = (((mask >> (2 * p)) & 1u) ? 0u : 0x0000FFFFu) |
-                                          (((mask >> (2 * p + 1)) & 1u) ? 0u : 0xFFFF0000u);
-                    w[p] &= keep;
+            if (mask && tid + i * T < nchunk) {
+                const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+                uint32_t mm = mask;
+                int j = static_cast<int>(tb[i] >> 8);
+                while (mm) {
+                    const int e = __ffs(mm) - 1;
+                    mm &= mm - 1;
+                    obuf[j++] = static_cast<uint16_t>(w[e >> 1] >> ((e & 1) * 16));
                 }
+                const uint4 kp = keep_tab[mask];
+                v[i].x &= kp.x;
+                v[i].y &= kp.y;
+                v[i].z &= kp.z;
+                v[i].w &= kp.w;
             }
-            am2 = max_u16x2(am2, max_u16x2(max_u16x2(w[0], w[1]), max_u16x2(w[2], w[3])));
+            am2 = max_u16x2(am2, max_u16x2(max_u16x2(v[i].x & 0x7FFF7FFFu, v[i].y & 0x7FFF7FFFu),
+                                           max_u16x2(v[i].z & 0x7FFF7FFFu, v[i].w & 0x7FFF7FFFu)));
         }
         uint32_t amax = max(am2 & 0xFFFFu, am2 >> 16);
 #pragma unroll
@@ -201,8 +314,13 @@ __global__ void __launch_bounds__(T, (T >= 512 ? 1 : 512 / T)) rowquant_kernel(
         const float inv_s = zero ? 0.0f : __frcp_rn(s);
         const bool fast_ok = zero || s >= 7.888609052210118e-31f;  // 2^-100: 1/s stays finite
         if (tid == 0) dst_s[r] = zero ? 0.0f : s;
+        RowScale rs;
+        rs.inv2 = f2_pack(__float_as_uint(inv_s), __float_as_uint(inv_s));
+        rs.negs2 = f2_pack(__float_as_uint(-s), __float_as_uint(-s));
+        rs.magic2 = f2_pack(__float_as_uint(kMagic), __float_as_uint(kMagic));
 
-        // 2. codes -> qbuf at their normal rank, outliers -> obuf at their rank in O
+        // 2. each chunk: codes, normal codes moved to the front, packed into
+        //    one nibble word, OR-ed into the packed row at their rank
 #pragma unroll
         for (int i = 0; i < CPT; ++i) {
             const int c = tid + i * T;
@@ -210,57 +328,38 @@ __global__ void __launch_bounds__(T, (T >= 512 ? 1 : 512 / T)) rowquant_kernel(
             const uint32_t mask = tb[i] & 0xFFu;
             const int below = static_cast<int>(tb[i] >> 8);
             uint32_t lo, hi;
-            quant8(v[i], s, inv_s, fast_ok, lo, hi);
-            const int p = 8 * c - below;
-            if (mask == 0u) {
-                if ((p & 7) == 0) {
-                    *reinterpret_cast<uint2 *>(qbuf + p) = make_uint2(lo, hi);
-                } else if ((p & 3) == 0) {
-                    *reinterpret_cast<uint32_t *>(qbuf + p) = lo;
-                    *reinterpret_cast<uint32_t *>(qbuf + p + 4) = hi;
-                } else if ((p & 1) == 0) {
-                    *reinterpret_cast<uint16_t *>(qbuf + p) = static_cast<uint16_t>(lo);
-                    *reinterpret_cast<uint16_t *>(qbuf + p + 2) = static_cast<uint16_t>(lo >> 16);
-                    *reinterpret_cast<uint16_t *>(qbuf + p + 4) = static_cast<uint16_t>(hi);
-                    *reinterpret_cast<uint16_t *>(qbuf + p + 6) = static_cast<uint16_t>(hi >> 16);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        qbuf[p + e] = static_cast<int8_t>(((e < 4 ? lo : hi) >> (8 * (e & 3))) & 0xFFu);
-                }
+            if (fast_ok) {
+                quant8_pairs(v[i], rs, lo, hi);
             } else {
-                const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-                int nlow = 0;  // outliers of this chunk before element e
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    if ((mask >> e) & 1u) {
-                        obuf[below + nlow] = static_cast<uint16_t>(w[e >> 1] >> ((e & 1) * 16));
-                        ++nlow;
-                    } else {
-                        qbuf[p + e - nlow] = static_cast<int8_t>(((e < 4 ? lo : hi) >> (8 * (e & 3))) & 0xFFu);
-                    }
-                }
+                const uint2 ex = quant8_exact(v[i], s);
+                lo = ex.x;
+                hi = ex.y;
             }
+            const uint2 sel = sel_tab[mask];
+            const uint32_t clo = __byte_perm(lo, hi, sel.x);
+            const uint32_t chi = __byte_perm(lo, hi, sel.y);
+            const int n = 8 - __popc(mask);
+            const uint32_t V = pack8_codes(clo, chi) & static_cast<uint32_t>((1ull << (4 * n)) - 1ull);
+            const int p = 8 * c - below;   // rank of the chunk's first normal channel
+            const int sh = (p & 7) * 4;
+            uint32_t *dst = pbuf + (p >> 3);
+            atomicOr(dst, V << sh);
+            atomicOr(dst + 1, sh ? (V >> (32 - sh)) : 0u);
         }
         __syncthreads();
 
-        // 3. pack and store: 32 codes -> 16 bytes per item; outliers 8 per item
-        uint8_t *out_n = dst_n + r * static_cast<int64_t>(kn_pad >> 1);
-        for (int j = tid; j < (kn_pad >> 5); j += T) {
-            const uint4 c0 = *reinterpret_cast<const uint4 *>(qbuf + 32 * j);
-            const uint4 c1 = *reinterpret_cast<const uint4 *>(qbuf + 32 * j + 16);
-            uint4 o;
-            o.x = pack8_codes(c0.x, c0.y);
-            o.y = pack8_codes(c0.z, c0.w);
-            o.z = pack8_codes(c1.x, c1.y);
-            o.w = pack8_codes(c1.z, c1.w);
-            *reinterpret_cast<uint4 *>(out_n + 16 * j) = o;
+        // 3. copy out, clearing the packed row for its next use (two rows on)
+        uint4 *pk16 = reinterpret_cast<uint4 *>(pbuf);
+        uint4 *out_n = reinterpret_cast<uint4 *>(dst_n + r * static_cast<int64_t>(pk_bytes));
+        for (int j = tid; j < (pk_alloc >> 4); j += T) {
+            if (j < (pk_bytes >> 4)) out_n[j] = pk16[j];
+            pk16[j] = make_uint4(0, 0, 0, 0);
         }
         uint16_t *out_o = dst_o + r * static_cast<int64_t>(no_pad);
         for (int j = tid; j < (no_pad >> 3); j += T)
             *reinterpret_cast<uint4 *>(out_o + 8 * j) = *reinterpret_cast<const uint4 *>(obuf + 8 * j);
-        // No barrier here: the next row fills the other buffers; this row's
-        // buffers are reused two rows later, after that row's two barriers.
+        // No barrier here: the next row uses the other buffers; these are
+        // reused two rows later, after that row's two barriers.
     }
 }
 
