@@ -153,6 +153,22 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples), "source": "nvml"}
 
 
+# ----------------------------------------------------------------- multi-rank aggregation
+def max_over_ranks(v: float, world: int, device=None) -> float:
+    """Largest value over all ranks (device time of the slowest rank)."""
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tops(ops_per_rank_step: float, ms_per_step_max: float, world: int) -> float:
+    """Throughput of the whole job: every rank's work divided by the slowest rank's time."""
+    return world * ops_per_rank_step / (ms_per_step_max * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------- CPU oracle timing
 def time_oracle(w, O, X, W, target_s: float, max_rows: int | None = None):
     """Time the oracle on a bounded sample of token rows (weights quantized beforehand,
@@ -245,13 +261,6 @@ def main():
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     peaks = load_peaks()
     O, X, W = workloads.make(w)
     M, N, K, nO = w.M, w.N, w.K, w.nO
@@ -307,13 +316,13 @@ def main():
         torch.cuda.synchronize(dev)
     barrier()
     sq.sq_check(stream)
-    ms_step = max_over_ranks(t_start.elapsed_time(t_end) / args.steps)
+    ms_step = max_over_ranks(t_start.elapsed_time(t_end) / args.steps, world, dev)
     ms_qg = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     ms_gemm = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
     clocks = clk.summary()
 
     flops = 2.0 * M * N * K
-    value = world * flops / (ms_step * 1e-3) / 1e12
+    value = whole_job_tops(flops, ms_step, world)
 
     # roofline of the GEMM: int8 path at 2x the bf16 peak, bf16 path at the bf16 peak (burst: timed alone)
     p_bf = peaks["bf16_tflops"]
@@ -349,8 +358,8 @@ def main():
     torch.cuda.synchronize(dev)
     barrier()
     sq.sq_check(stream)
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-    e2e_value = world * flops / (ms_e2e * 1e-3) / 1e12
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    e2e_value = whole_job_tops(flops, ms_e2e, world)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -165,6 +165,19 @@ sq_status launch_rowquant(const uint16_t *src, int64_t rows, int64_t K, int64_t 
 }
 
 // ---------------------------------------------------------------- GEMM
+// Raster band height (in M-tiles).  Tiles are handed out M-fastest within a
+// band, so the CTAs at work together share a band of X rows and a few W
+// tiles.  The band takes as many M-tiles as keep its X operands within about
+// 48 MB of L2: when all of X fits, each W tile is fetched from HBM once.
+int raster_group(int tiles_m, int tile_rows, int64_t kn_pad, int64_t no_pad)
+{
+    const int64_t band_bytes = static_cast<int64_t>(tile_rows) * (kn_pad / 2 + 2 * no_pad);
+    int64_t g = band_bytes > 0 ? (48ll << 20) / band_bytes : tiles_m;
+    if (g < 1) g = 1;
+    if (g > tiles_m) g = tiles_m;
+    return static_cast<int>(g);
+}
+
 template <class C>
 sq_status launch_gemm_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O, const void *W_N,
                         const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y,
@@ -197,7 +210,7 @@ sq_status launch_gemm_t(const DevInfo &di, const void *X_N, const float *s_x, co
     a.nkb_o = static_cast<int>(no_pad / sqg::KB_BF);
     a.tiles_m = static_cast<int>((M + sqg::BM - 1) / sqg::BM);
     a.tiles_n = static_cast<int>((N + C::BN - 1) / C::BN);
-    a.group_m = 8;
+    a.group_m = raster_group(a.tiles_m, sqg::BM, kn_pad, no_pad);
     const int64_t ntiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
     const int64_t grid = std::min<int64_t>(ntiles, di.sms);
     const bool dbg = dbg_i || dbg_f;
@@ -250,7 +263,7 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
     a.nkb_o = static_cast<int>(no_pad / sqg::KB_BF);
     a.tiles_m = static_cast<int>((M + sqg::PAIR_BM - 1) / sqg::PAIR_BM);
     a.tiles_n = static_cast<int>((N + sqg::PAIR_BN - 1) / sqg::PAIR_BN);
-    a.group_m = 4;
+    a.group_m = raster_group(a.tiles_m, sqg::PAIR_BM, kn_pad, no_pad);
     const int64_t ntiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
     const int64_t clusters = std::min<int64_t>(ntiles, di.sms / 2);
     const bool dbg = dbg_i || dbg_f;
@@ -262,7 +275,7 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
     return SQ_OK;
 }
 
-using CfgPair = sqg::CfgPair<4, 5, 2>;
+using CfgPair = sqg::CfgPair<4, 4, 2>;
 
 using CfgN256 = sqg::Cfg<256, 4>;
 using CfgN128 = sqg::Cfg<128, 6>;

@@ -65,7 +65,13 @@ struct CfgPair {
     static constexpr int TMEM_COLS = 512;
     static constexpr int EXP_CHUNKS = 256 * (PROWB / 16) / GT;  // packed 16-byte chunks per thread per K-block
     static_assert(SMEM_BYTES <= 232448, "shared memory");
-    static_assert(NUM_EXP_WARPS % NG == 0 && OPS % NG == 0, "every ring slot must belong to one group");
+    // Each slot of both rings must be used by a single producer group: a group
+    // waiting on a slot only knows that its own earlier blocks have landed, and
+    // bulk copies may complete out of order, so a slot shared by two groups
+    // could still hold (or be receiving) the other group's block when the
+    // phase-parity wait passes.
+    static_assert(NUM_EXP_WARPS % NG == 0 && OPS % NG == 0 && STG % NG == 0,
+                  "every ring slot must belong to one producer group");
 };
 
 template <class C, bool DBG>
