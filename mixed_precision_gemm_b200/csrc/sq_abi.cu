@@ -290,8 +290,7 @@ sq_status gemm_impl(const void *X_N, const float *s_x, const void *X_O, const vo
     sq_status st = device_info(di);
     if (st != SQ_OK) return st;
     const int64_t tiles_m = (M + sqg::BM - 1) / sqg::BM;
-    const int64_t pair_tiles = ((M + sqg::PAIR_BM - 1) / sqg::PAIR_BM) * ((N + sqg::PAIR_BN - 1) / sqg::PAIR_BN);
-    if (M >= 256 && pair_tiles >= di.sms / 2)
+    if (M > 128)
         return launch_gemm_pair_t<CfgPair>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (tiles_m * ((N + 255) / 256) >= 2 * di.sms)
         return launch_gemm_t<CfgN256>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
