@@ -15,8 +15,9 @@
 
 #include "../../include/sq.h"
 #include "sq_device.cuh"
-#include "sq_gemm.cuh"
+#include "sq_gemm_common.cuh"
 #include "sq_gemm_pair.cuh"
+#include "sq_gemm_skinny.cuh"
 #include "sq_rowquant.cuh"
 
 namespace {
@@ -77,6 +78,42 @@ sq_status device_info(DevInfo &out)
     return SQ_OK;
 }
 
+// ---------------------------------------------------------------- per-kernel launch set-up
+// The dynamic shared-memory opt-in and the occupancy of each kernel are set
+// and queried once per device and size; later calls (including calls made
+// while a stream is captured into a CUDA graph) only look them up.
+struct KernelSetup {
+    const void *fn;
+    int dev;
+    size_t smem;
+    int threads;
+    int per_sm;
+};
+std::vector<KernelSetup> g_setups;
+std::mutex g_setup_mu;
+
+sq_status kernel_setup(const void *fn, int threads, size_t smem, int &per_sm, const char *what)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lk(g_setup_mu);
+    for (const KernelSetup &k : g_setups)
+        if (k.fn == fn && k.dev == dev && k.smem == smem && k.threads == threads) {
+            per_sm = k.per_sm;
+            return SQ_OK;
+        }
+    if (smem > 48 * 1024 &&
+        (e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))) !=
+            cudaSuccess)
+        return cuda_fail(e, what);
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem)) != cudaSuccess)
+        return cuda_fail(e, what);
+    if (per_sm < 1) return fail(SQ_ERR_UNSUPPORTED, "%s: kernel does not fit on an SM", what);
+    g_setups.push_back({fn, dev, smem, threads, per_sm});
+    return SQ_OK;
+}
+
 // ---------------------------------------------------------------- tensor maps
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -125,16 +162,10 @@ sq_status launch_rowquant_t(const DevInfo &di, const uint16_t *src, int64_t rows
     auto kern = sqq::rowquant_kernel<T, CPT>;
     // two alternating (packed code row + outlier row) pairs, selector and keep tables
     const size_t smem = 2u * (static_cast<size_t>(kn_pad / 2) + 16u + 2u * static_cast<size_t>(no_pad)) + 256u * 24u;
-    cudaError_t e;
-    if (smem > 48 * 1024) {
-        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))) !=
-            cudaSuccess)
-            return cuda_fail(e, "cudaFuncSetAttribute(rowquant)");
-    }
     int per_sm = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, T, smem)) != cudaSuccess)
-        return cuda_fail(e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
-    if (per_sm < 1) per_sm = 1;
+    sq_status st = kernel_setup(reinterpret_cast<const void *>(kern), T, smem, per_sm, "rowquant set-up");
+    if (st != SQ_OK) return st;
+    cudaError_t e;
     const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * di.sms);
     kern<<<static_cast<unsigned>(grid), T, smem, stream>>>(src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds, dout);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "rowquant launch");
@@ -178,50 +209,6 @@ int raster_group(int tiles_m, int tile_rows, int64_t kn_pad, int64_t no_pad)
     return static_cast<int>(g);
 }
 
-template <class C>
-sq_status launch_gemm_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O, const void *W_N,
-                        const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y,
-                        int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
-{
-    const int64_t kn_pad = sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
-    CUtensorMap m_xo{}, m_wo{};
-    sq_status st;
-    if (no_pad > 0) {
-        if ((st = make_map(m_xo, X_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, M, no_pad * 2, sqg::KB_BF, sqg::BM,
-                           CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
-            return st;
-        if ((st = make_map(m_wo, W_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, N, no_pad * 2, sqg::KB_BF, C::BN,
-                           CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
-            return st;
-    }
-    sqg::GemmArgs a;
-    a.xn = static_cast<const uint8_t *>(X_N);
-    a.wn = static_cast<const uint8_t *>(W_N);
-    a.row_bytes = kn_pad / 2;
-    a.s_x = s_x;
-    a.s_w = s_w;
-    a.Y = static_cast<uint16_t *>(Y);
-    a.dbg_i = dbg_i;
-    a.dbg_f = dbg_f;
-    a.M = static_cast<int>(M);
-    a.N = static_cast<int>(N);
-    a.ldy = ldy;
-    a.nkb_i = static_cast<int>(kn_pad / sqg::KB_I8);
-    a.nkb_o = static_cast<int>(no_pad / sqg::KB_BF);
-    a.tiles_m = static_cast<int>((M + sqg::BM - 1) / sqg::BM);
-    a.tiles_n = static_cast<int>((N + C::BN - 1) / C::BN);
-    a.group_m = raster_group(a.tiles_m, sqg::BM, kn_pad, no_pad);
-    const int64_t ntiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
-    const int64_t grid = std::min<int64_t>(ntiles, di.sms);
-    const bool dbg = dbg_i || dbg_f;
-    auto kern = dbg ? sqg::dual_gemm_kernel<C, true> : sqg::dual_gemm_kernel<C, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm)");
-    kern<<<static_cast<unsigned>(grid), sqg::NUM_THREADS, C::SMEM_BYTES, stream>>>(m_xo, m_wo, a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "gemm launch");
-    return SQ_OK;
-}
-
 // Pair (cta_group::2) kernel: 256 x 256 tiles over clusters of two CTAs.
 template <class C>
 sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O, const void *W_N,
@@ -248,9 +235,6 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
             return st;
     }
     sqg::GemmArgs a;
-    a.xn = static_cast<const uint8_t *>(X_N);
-    a.wn = static_cast<const uint8_t *>(W_N);
-    a.row_bytes = kn_pad / 2;
     a.s_x = s_x;
     a.s_w = s_w;
     a.Y = static_cast<uint16_t *>(Y);
@@ -268,18 +252,92 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
     const int64_t clusters = std::min<int64_t>(ntiles, di.sms / 2);
     const bool dbg = dbg_i || dbg_f;
     auto kern = dbg ? sqg::dual_gemm_pair_kernel<C, true> : sqg::dual_gemm_pair_kernel<C, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(gemm pair)");
+    int per_sm = 0;
+    if ((st = kernel_setup(reinterpret_cast<const void *>(kern), sqg::PAIR_THREADS, C::SMEM_BYTES, per_sm, "gemm pair set-up")) != SQ_OK)
+        return st;
+    cudaError_t e;
     kern<<<static_cast<unsigned>(2 * clusters), sqg::PAIR_THREADS, C::SMEM_BYTES, stream>>>(m_xo, m_wo, m_xn, m_wn, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "gemm pair launch");
     return SQ_OK;
 }
 
-using CfgPair = sqg::CfgPair<4, 4, 2>;
+// Swapped-operand split-K kernel for M <= 128: tiles of 128 W rows x MP
+// tokens; the K-blocks of each tile are spread over a cluster of S CTAs.
+template <class C>
+sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O,
+                               const void *W_N, const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K,
+                               int64_t nO, void *Y, int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+{
+    const int64_t kn_pad = sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
+    CUtensorMap m_xo{}, m_wo{}, m_xn{}, m_wn{};
+    sq_status st;
+    if (kn_pad > 0) {
+        // 128-byte boxes (two INT4 K-blocks) with the 128-byte swizzle.
+        if ((st = make_map(m_xn, X_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, M, kn_pad / 2, 2 * sqg::PROWB, C::MP,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
+            return st;
+        if ((st = make_map(m_wn, W_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, N, kn_pad / 2, 2 * sqg::PROWB, 128,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
+            return st;
+    }
+    if (no_pad > 0) {
+        if ((st = make_map(m_xo, X_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, M, no_pad * 2, sqg::KB_BF, C::MP,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
+            return st;
+        if ((st = make_map(m_wo, W_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, N, no_pad * 2, sqg::KB_BF, 128,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
+            return st;
+    }
+    sqg::SkinnyArgs a;
+    a.s_x = s_x;
+    a.s_w = s_w;
+    a.Y = static_cast<uint16_t *>(Y);
+    a.dbg_i = dbg_i;
+    a.dbg_f = dbg_f;
+    a.M = static_cast<int>(M);
+    a.N = static_cast<int>(N);
+    a.ldy = ldy;
+    a.nkb_i = static_cast<int>(kn_pad / sqg::KB_I8);
+    a.nkb_o = static_cast<int>(no_pad / sqg::KB_BF);
+    const int64_t tiles_n = (N + 127) / 128;
+    // As many K ranges per W tile as fill the SMs once, at most 8 (portable
+    // cluster size) and at most half the tile's byte count in 64-byte units,
+    // so that every range holds at least one K-block.
+    const int cost = a.nkb_i + 2 * a.nkb_o;
+    int64_t S = tiles_n >= di.sms ? 1 : di.sms / tiles_n;
+    S = std::min<int64_t>(S, sqg::SK_MAX_SPLITS);
+    S = std::min<int64_t>(S, std::max(1, cost / 2));
+    S = std::max<int64_t>(S, 1);
+    a.splits = static_cast<int>(S);
+    const bool dbg = dbg_i || dbg_f;
+    auto kern = dbg ? sqg::dual_gemm_skinny_kernel<C, true> : sqg::dual_gemm_skinny_kernel<C, false>;
+    int per_sm = 0;
+    if ((st = kernel_setup(reinterpret_cast<const void *>(kern), sqg::SK_THREADS, C::SMEM_BYTES, per_sm, "gemm skinny set-up")) != SQ_OK)
+        return st;
+    cudaError_t e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(tiles_n * S), 1, 1);
+    cfg.blockDim = dim3(sqg::SK_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((e = cudaLaunchKernelEx(&cfg, kern, m_xo, m_wo, m_xn, m_wn, a)) != cudaSuccess)
+        return cuda_fail(e, "gemm skinny launch");
+    return SQ_OK;
+}
 
-using CfgN256 = sqg::Cfg<256, 4>;
-using CfgN128 = sqg::Cfg<128, 6>;
-using CfgN64 = sqg::Cfg<64, 8>;
+using CfgPair = sqg::CfgPair<4, 4, 2>;
+using CfgSk16 = sqg::CfgSkinny<16, 8, 3>;
+using CfgSk32 = sqg::CfgSkinny<32, 7, 3>;
+using CfgSk64 = sqg::CfgSkinny<64, 6, 2>;
+using CfgSk128 = sqg::CfgSkinny<128, 4, 2>;
+
 
 sq_status gemm_impl(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
                     const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
@@ -289,14 +347,15 @@ sq_status gemm_impl(const void *X_N, const float *s_x, const void *X_O, const vo
     DevInfo di;
     sq_status st = device_info(di);
     if (st != SQ_OK) return st;
-    const int64_t tiles_m = (M + sqg::BM - 1) / sqg::BM;
     if (M > 128)
         return launch_gemm_pair_t<CfgPair>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
-    if (tiles_m * ((N + 255) / 256) >= 2 * di.sms)
-        return launch_gemm_t<CfgN256>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
-    if (tiles_m * ((N + 127) / 128) >= di.sms)
-        return launch_gemm_t<CfgN128>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
-    return launch_gemm_t<CfgN64>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    if (M <= 16)
+        return launch_gemm_skinny_t<CfgSk16>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    if (M <= 32)
+        return launch_gemm_skinny_t<CfgSk32>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    if (M <= 64)
+        return launch_gemm_skinny_t<CfgSk64>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    return launch_gemm_skinny_t<CfgSk128>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
 }
 
 // ---------------------------------------------------------------- validation

@@ -1,5 +1,5 @@
 // Dual-path GEMM on CTA pairs (tcgen05 cta_group::2): the same computation as
-// sq_gemm.cuh (OSC, arXiv:2604.12782, abstract: a 4-bit GEMM path plus a
+// sq_gemm_common.cuh (OSC, arXiv:2604.12782, abstract: a 4-bit GEMM path plus a
 // 16-bit branch GEMM on the compact outlier tensor, fused), with 256 x 256
 // output tiles shared by the two CTAs of a cluster.
 //
@@ -23,7 +23,7 @@
 //                            multicast, completion bytes counted on the first
 //                            CTA's barrier); INT4 blocks expanded from the
 //                            staging ring into int8 operand tiles (see
-//                            sq_gemm.cuh).  Every producer warp of both CTAs
+//                            sq_gemm_common.cuh).  Every producer warp of both CTAs
 //                            arrives on the first CTA's op_full.
 // The packed tiles travel by TMA into a staging ring (asynchronous, six
 // K-blocks deep) and are expanded from shared memory, so no producer thread
@@ -31,7 +31,7 @@
 // TMEM per CTA: acc_f in columns [0, 256), acc_i in [256, 512).
 #pragma once
 
-#include "sq_gemm.cuh"
+#include "sq_gemm_common.cuh"
 
 namespace sqg {
 

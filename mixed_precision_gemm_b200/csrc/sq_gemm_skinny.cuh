@@ -1,0 +1,383 @@
+// Dual-path GEMM for few tokens (M <= 128): swapped operands, K split over a
+// cluster.  Same computation as sq_gemm_pair.cuh (OSC, arXiv:2604.12782,
+// abstract: a 4-bit GEMM path plus a 16-bit branch GEMM on the compact
+// outlier tensor, fused).
+//
+// With few tokens the layer is a stream over the weights: every packed W byte
+// is read once and the arithmetic per byte is small.  Three choices follow.
+//
+// Swapped operands.  The MMA computes D^T = W . X^T: the 128 W rows of a tile
+// are the MMA's M side (the TMEM lanes) and the MP tokens (MP = M rounded up
+// to 16, 32, 64 or 128) are its N side, so no MMA work is spent on token rows
+// that do not exist.  D holds 128 output channels x MP tokens.
+//
+// Split K.  The K-blocks of one 128-row W tile (INT4 blocks of 128 channels
+// first, then bf16 blocks of 64 outlier channels, weighted 1 and 2 by their
+// bytes) are divided into S contiguous ranges of equal byte count, one per
+// CTA of a cluster of S (S <= 8), so that tiles_n * S CTAs stream W at once.
+// The S partial accumulators are summed through distributed shared memory:
+// CTA r of the cluster owns rows [r*RP, (r+1)*RP) of the tile (RP =
+// ceil(128/S)); every CTA sends the owner its int32 and fp32 partials of
+// those rows; the owner adds them (int32 exactly, fp32 in rank order) and
+// writes Y.  The reduction buffer reuses the rings, which are idle once every
+// MMA of the cluster has completed (first cluster barrier).
+//
+// Wide loads, deep ring.  Weight rows are fetched 128 bytes at a time (two
+// packed INT4 K-blocks, or one bf16 K-block) with the 128-byte swizzle, into
+// a staging ring of about 144 KB, which keeps enough bytes in flight per SM
+// to stream HBM.  bf16 stages are read by the MMA where they land; INT4
+// stages are expanded into a small ring of int8 operand tiles.
+//
+// Roles (6 warps, one tile-split per CTA):
+//   warp 0      TMA producer of the staging ring: for each stage, 128 W rows
+//               and MP token rows of 128 bytes.
+//   warp 1      allocates TMEM; one lane issues every MMA and commits.
+//   warps 2..5  expand INT4 stages (both K-blocks at once, eight threads per
+//               128-byte row) into the operand ring, in order; afterwards
+//               they run the epilogue.
+// Stage order is every INT4 stage, then every bf16 stage.  The INT4 stages
+// are consumed by the expansion warps and the bf16 stages by the MMA issuer;
+// because all INT4 stages come first, each consumer's earlier uses of a slot
+// were its own or were consumed before it reached the slot, so the
+// phase-parity waits cannot alias.
+// TMEM: acc_i (int32) in columns [0, MP), acc_f (fp32) in [MP, 2 MP).
+#pragma once
+
+#include "sq_gemm_common.cuh"
+
+namespace sqg {
+
+constexpr int SK_PROD_WARP0 = 2;
+constexpr int SK_PROD_WARPS = 4;
+constexpr int SK_THREADS = 32 * (SK_PROD_WARP0 + SK_PROD_WARPS);
+constexpr int SK_PT = 32 * SK_PROD_WARPS;  // expansion threads (= TMEM lanes)
+constexpr int SK_MAX_SPLITS = 8;
+
+enum : unsigned { SITE_SK_STG = 0x501, SITE_SK_OP = 0x502, SITE_SK_MMA = 0x503, SITE_SK_EPI = 0x504 };
+
+template <int MP_, int NST_, int OPS_>
+struct CfgSkinny {
+    static constexpr int MP = MP_;                    // token columns of D (MMA N)
+    static constexpr int NST = NST_;                  // staging ring stages
+    static constexpr int OPS = OPS_;                  // expanded int8 operand ring stages
+    static constexpr int ROWS = 128 + MP;             // W rows, then token rows, in every tile
+    static constexpr int A_BYTES = 128 * ROWB;
+    static constexpr int TILE_BYTES = ROWS * ROWB;    // one stage = one operand tile (128-byte rows)
+    static constexpr int OFF_STG = 0;
+    static constexpr int OFF_OP = NST * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_OP + OPS * TILE_BYTES;
+    // barriers: stg_full[NST] stg_empty[NST] op_full[OPS] op_empty[OPS] acc_full drain
+    static constexpr int NBAR = 2 * NST + 2 * OPS + 2;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_CNT = OFF_MISC + 16;           // per staging slot: expansion warps done
+    static constexpr int SMEM_BYTES = OFF_CNT + NST * 4 + 1024;
+    static constexpr int TMEM_COLS = 2 * MP < 32 ? 32 : 2 * MP;
+    static constexpr int EXP_CHUNKS = ROWS * 8 / SK_PT;   // 16-byte packed chunks per thread per stage
+    // Reduction buffer (aliases the rings): int32 and fp32 regions of
+    // S * RP <= 128 + S - 1 partial rows, RSTRIDE words apart.
+    static constexpr int RSTRIDE = MP + 4;
+    static constexpr int RED_ROWS = 128 + SK_MAX_SPLITS - 1;
+    static constexpr int OFF_RED_I = 0;
+    static constexpr int OFF_RED_F = RED_ROWS * RSTRIDE * 4;
+    static_assert(MP == 16 || MP == 32 || MP == 64 || MP == 128, "MP");
+    static_assert(TILE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned");
+    static_assert(ROWS * 8 % SK_PT == 0, "expansion work split");
+    static_assert(OPS >= 2, "an INT4 stage fills two operand tiles");
+    static_assert(2 * RED_ROWS * RSTRIDE * 4 <= OFF_BAR, "reduction buffer must fit in the rings");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+struct SkinnyArgs {
+    const float *s_x;
+    const float *s_w;
+    uint16_t *Y;
+    int32_t *dbg_i;
+    float *dbg_f;
+    int M, N;
+    long long ldy;
+    int nkb_i;   // INT4 K-blocks (kn_pad / 128)
+    int nkb_o;   // bf16 K-blocks (no_pad / 64)
+    int splits;  // CTAs per cluster = K ranges per W tile
+};
+
+// First K-block of split r of S: blocks 0..nkb_i-1 are INT4 (64 bytes per W
+// row), then nkb_o bf16 blocks (128 bytes per W row); the split points are
+// the block boundaries at or after r/S of the total bytes.
+__device__ __forceinline__ int skinny_first_block(int r, int S, int nkb_i, int nkb_o)
+{
+    const int cost = nkb_i + 2 * nkb_o;
+    const int c = static_cast<int>(static_cast<long long>(cost) * r / S);
+    return c <= nkb_i ? c : nkb_i + (c - nkb_i + 1) / 2;
+}
+
+template <class C, bool DBG>
+__global__ void __launch_bounds__(SK_THREADS, 1)
+dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_constant__ CUtensorMap tm_wo,
+                        const __grid_constant__ CUtensorMap tm_xn, const __grid_constant__ CUtensorMap tm_wn,
+                        const SkinnyArgs args)
+{
+    constexpr int MP = C::MP, NST = C::NST, OPS = C::OPS, EC = C::EXP_CHUNKS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = sqd::smem_u32(smem);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int S = args.splits;
+    const int rank = static_cast<int>(sqd::cluster_ctarank());
+    const int n0 = static_cast<int>(blockIdx.x) / S * 128;
+
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto stg_full = [&](int s) { return bar0 + 8u * s; };
+    auto stg_empty = [&](int s) { return bar0 + 8u * (NST + s); };
+    auto op_full = [&](int e) { return bar0 + 8u * (2 * NST + e); };
+    auto op_empty = [&](int e) { return bar0 + 8u * (2 * NST + OPS + e); };
+    const uint32_t acc_full = bar0 + 8u * (2 * NST + 2 * OPS);
+    const uint32_t drain = acc_full + 8u;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC + 4);
+    uint32_t *stg_done = reinterpret_cast<uint32_t *>(smem + C::OFF_CNT);
+    auto stg_a = [&](int s) { return sbase + C::OFF_STG + s * C::TILE_BYTES; };
+    auto op_a = [&](int e) { return sbase + C::OFF_OP + e * C::TILE_BYTES; };
+
+    // This CTA's K range: INT4 blocks [i_lo, i_lo + n_i) in ns_i stages of
+    // two, then bf16 blocks [o_lo, o_lo + n_o), one stage each.
+    const int nkb_i = args.nkb_i, nkb_o = args.nkb_o;
+    const int b_lo = skinny_first_block(rank, S, nkb_i, nkb_o);
+    const int b_hi = skinny_first_block(rank + 1, S, nkb_i, nkb_o);
+    const int i_lo = min(b_lo, nkb_i);
+    const int n_i = min(b_hi, nkb_i) - i_lo;
+    const int o_lo = max(b_lo, nkb_i) - nkb_i;
+    const int n_o = max(b_hi, nkb_i) - nkb_i - o_lo;
+    const int ns_i = (n_i + 1) / 2;
+    const int ns = ns_i + n_o;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            sqd::mbar_init(stg_full(s), 1);   // TMA producer (expect-tx)
+            sqd::mbar_init(stg_empty(s), 1);  // the last expansion warp, or the MMA commit
+            stg_done[s] = 0u;
+        }
+        for (int e = 0; e < OPS; ++e) {
+            sqd::mbar_init(op_full(e), SK_PROD_WARPS);
+            sqd::mbar_init(op_empty(e), 1);
+        }
+        sqd::mbar_init(acc_full, 1);
+        sqd::mbar_init(drain, 1);
+        *abort_flag = 0u;
+        sqd::fence_barrier_init();
+        sqd::fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        if (n_o > 0) {
+            sqd::prefetch_tensormap(&tm_xo);
+            sqd::prefetch_tensormap(&tm_wo);
+        }
+        if (n_i > 0) {
+            sqd::prefetch_tensormap(&tm_xn);
+            sqd::prefetch_tensormap(&tm_wn);
+        }
+    }
+    if (warp == 1) {
+        sqd::tmem_alloc(sqd::smem_u32(tmem_slot), C::TMEM_COLS);
+        sqd::tmem_relinquish();
+    }
+    sqd::tc_fence_before();
+    __syncthreads();
+    sqd::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ staging producer
+        if (lane == 0) {
+            int last_armed = -1;
+            bool ok = true;
+            for (int t = 0; t < ns; ++t) {
+                const int s = t % NST;
+                if (!sqd::mbar_wait(stg_empty(s), ((t / NST) & 1) ^ 1u, abort_flag, SITE_SK_STG)) { ok = false; break; }
+                sqd::mbar_arrive_expect_tx(stg_full(s), C::TILE_BYTES);
+                if (t < ns_i) {
+                    const int x = (i_lo + 2 * t) * PROWB;  // byte offset of the stage's first K-block
+                    sqd::tma_load_2d(stg_a(s), &tm_wn, stg_full(s), x, n0);
+                    sqd::tma_load_2d(stg_a(s) + C::A_BYTES, &tm_xn, stg_full(s), x, 0);
+                } else {
+                    const int x = (o_lo + t - ns_i) * KB_BF;
+                    sqd::tma_load_2d(stg_a(s), &tm_wo, stg_full(s), x, n0);
+                    sqd::tma_load_2d(stg_a(s) + C::A_BYTES, &tm_xo, stg_full(s), x, 0);
+                }
+                last_armed = t;
+            }
+            if (!ok && last_armed >= 0) sqd::mbar_drain(stg_full(last_armed % NST), (last_armed / NST) & 1);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_bf = sqd::make_idesc(false, 128, MP);
+            constexpr uint32_t idesc_i8 = sqd::make_idesc(true, 128, MP);
+            bool ok = true;
+            for (int u = 0; u < n_i && ok; ++u) {  // INT4 blocks from the operand ring
+                const int e = u % OPS;
+                if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_SK_MMA)) { ok = false; break; }
+                sqd::tc_fence_after();
+                const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
+                const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    sqd::mma_s8(tmem, adesc + 2 * k, bdesc + 2 * k, idesc_i8, (u == 0 && k == 0) ? 0u : 1u);
+                sqd::mma_commit(op_empty(e));
+            }
+            for (int t = ns_i; t < ns && ok; ++t) {  // bf16 blocks straight from the staging ring
+                const int s = t % NST;
+                if (!sqd::mbar_wait(stg_full(s), (t / NST) & 1, abort_flag, SITE_SK_MMA)) { ok = false; break; }
+                sqd::tc_fence_after();
+                const uint64_t adesc = sqd::make_sw128_desc(stg_a(s));
+                const uint64_t bdesc = sqd::make_sw128_desc(stg_a(s) + C::A_BYTES);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    sqd::mma_bf16(tmem + MP, adesc + 2 * k, bdesc + 2 * k, idesc_bf, (t == ns_i && k == 0) ? 0u : 1u);
+                sqd::mma_commit(stg_empty(s));
+            }
+            if (ok) {
+                sqd::mma_commit(acc_full);  // also when this split has no blocks
+            } else {
+                sqd::mma_commit(drain);
+                sqd::mbar_drain(drain, 0);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ INT4 expansion
+        // Thread q of a stage handles 16-byte chunk q & 7 of row q >> 3: chunk
+        // c holds packed K-block c >> 2 of the stage, and stored chunk c of
+        // row r sits at position c ^ (r & 7) (128-byte swizzle).  Eight
+        // threads read one whole row, so the loads are conflict-free.
+        const int et = threadIdx.x - SK_PROD_WARP0 * 32;
+        bool ok = true;
+        for (int t = 0; t < ns_i && ok; ++t) {
+            const int s = t % NST;
+            const int nblk = min(2, n_i - 2 * t);
+            const int u0 = 2 * t;  // operand ring uses u0, u0 + 1
+            if (!sqd::mbar_wait(stg_full(s), (t / NST) & 1, abort_flag, SITE_SK_OP)) { ok = false; break; }
+            for (int j = 0; j < nblk; ++j) {
+                if (!sqd::mbar_wait(op_empty((u0 + j) % OPS), (((u0 + j) / OPS) & 1) ^ 1u, abort_flag, SITE_SK_OP)) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (!ok) break;
+            const uint32_t src = stg_a(s);
+            uint4 w[EC];
+#pragma unroll
+            for (int c = 0; c < EC; ++c) {
+                const int q = et + c * SK_PT;
+                const int r = q >> 3;
+                w[c] = sqd::lds128(src + r * ROWB + (((q & 7) ^ (r & 7)) << 4));
+            }
+#pragma unroll
+            for (int c = 0; c < EC; ++c) {
+                const int q = et + c * SK_PT;
+                const int r = q >> 3;
+                const int j = (q >> 2) & 1;  // K-block of the stage
+                if (j < nblk) {
+                    const uint32_t sw = static_cast<uint32_t>(r & 7);
+                    const uint32_t jj = static_cast<uint32_t>(q & 3);
+                    const uint32_t row = op_a((u0 + j) % OPS) + r * ROWB;
+                    const uint32_t a0 = row + (((2u * jj) ^ sw) << 4);
+                    const uint32_t a1 = row + (((2u * jj + 1u) ^ sw) << 4);
+                    const uint32_t lo0 = (w[c].x << 4) & 0xF0F0F0F0u, hi0 = w[c].x & 0xF0F0F0F0u;
+                    const uint32_t lo1 = (w[c].y << 4) & 0xF0F0F0F0u, hi1 = w[c].y & 0xF0F0F0F0u;
+                    const uint32_t lo2 = (w[c].z << 4) & 0xF0F0F0F0u, hi2 = w[c].z & 0xF0F0F0F0u;
+                    const uint32_t lo3 = (w[c].w << 4) & 0xF0F0F0F0u, hi3 = w[c].w & 0xF0F0F0F0u;
+                    // The two K-blocks' threads of a row store in opposite
+                    // order, so the eight stores of a phase hit distinct banks.
+                    if (j == 0) {
+                        sqd::sts128(a0, lo0, hi0, lo1, hi1);
+                        sqd::sts128(a1, lo2, hi2, lo3, hi3);
+                    } else {
+                        sqd::sts128(a1, lo2, hi2, lo3, hi3);
+                        sqd::sts128(a0, lo0, hi0, lo1, hi1);
+                    }
+                }
+            }
+            sqd::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                for (int j = 0; j < nblk; ++j) sqd::mbar_arrive(op_full((u0 + j) % OPS));
+                // The stage is released by the last of the four warps to have
+                // read it (a running count per slot, never reset).
+                if ((atomicAdd(&stg_done[s], 1u) + 1u) % SK_PROD_WARPS == 0u) sqd::mbar_arrive(stg_empty(s));
+            }
+        }
+        if (sqd::mbar_wait(acc_full, 0, abort_flag, SITE_SK_EPI)) sqd::tc_fence_after();
+        // The rings are reused by the generic proxy below.
+        sqd::fence_proxy_async_smem();
+    }
+
+    // ---------------------------------------------------------------- split reduction
+    __syncwarp();
+    sqd::tc_fence_before();
+    sqd::cluster_sync();  // every MMA of every CTA of the cluster is complete: rings are free
+
+    const int RP = (128 + S - 1) / S;
+    if (warp >= SK_PROD_WARP0) {
+        // Send this CTA's partial rows to their owners.  TMEM lane quarter
+        // warp % 4 holds W rows t = 32 * (warp % 4) + lane.
+        const int quarter = warp & 3;
+        const int t = quarter * 32 + lane;
+        const int owner = t / RP;
+        const int rl = t - owner * RP;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const uint32_t off = static_cast<uint32_t>(((rank * RP + rl) * C::RSTRIDE) * 4);
+        const uint32_t dst_i = sqd::map_to_cta(sbase + C::OFF_RED_I + off, static_cast<uint32_t>(owner));
+        const uint32_t dst_f = sqd::map_to_cta(sbase + C::OFF_RED_F + off, static_cast<uint32_t>(owner));
+        const bool has_i = n_i > 0 && !*abort_flag, has_f = n_o > 0 && !*abort_flag;
+#pragma unroll 1
+        for (int ch = 0; ch < MP / 16; ++ch) {
+            uint32_t vi[16] = {}, vf[16] = {};
+            if (has_i) sqd::tmem_ld_32x32b_x16(tl + ch * 16, vi);
+            if (has_f) sqd::tmem_ld_32x32b_x16(tl + MP + ch * 16, vf);
+            sqd::tmem_wait_ld_dep(vi, vf);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                sqd::st_cluster_v4(dst_i + (ch * 16 + 4 * g) * 4, vi[4 * g], vi[4 * g + 1], vi[4 * g + 2], vi[4 * g + 3]);
+                sqd::st_cluster_v4(dst_f + (ch * 16 + 4 * g) * 4, vf[4 * g], vf[4 * g + 1], vf[4 * g + 2], vf[4 * g + 3]);
+            }
+        }
+    }
+    sqd::tc_fence_before();
+    sqd::cluster_sync();  // all partials delivered
+
+    if (warp >= SK_PROD_WARP0) {
+        // Owned rows [rank * RP, rank * RP + R): sum the S partials, fuse, store.
+        const int et = threadIdx.x - SK_PROD_WARP0 * 32;
+        const int r0 = rank * RP;
+        const int R = max(0, min(128 - r0, RP));
+        const int32_t *red_i = reinterpret_cast<const int32_t *>(smem + C::OFF_RED_I);
+        const float *red_f = reinterpret_cast<const float *>(smem + C::OFF_RED_F);
+        for (int idx = et; idx < R * MP; idx += SK_PT) {
+            const int rl = idx % R;
+            const int m = idx / R;
+            const int n = n0 + r0 + rl;
+            if (m >= args.M || n >= args.N) continue;
+            int32_t si = 0;
+            float sf = 0.0f;
+            for (int s = 0; s < S; ++s) {
+                const int w = (s * RP + rl) * C::RSTRIDE + m;
+                si += red_i[w];
+                sf = __fadd_rn(sf, red_f[w]);
+            }
+            const int ai = si >> 8;
+            const float y = __fadd_rn(__fmul_rn(__fmul_rn(static_cast<float>(ai), args.s_x[m]), args.s_w[n]), sf);
+            args.Y[static_cast<long long>(m) * args.ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+            if constexpr (DBG) {
+                if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n] = ai;
+                if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n] = sf;
+            }
+        }
+    }
+    if (warp == 1) {
+        sqd::tc_fence_after();
+        sqd::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace sqg

@@ -146,6 +146,30 @@ def test_pair_kernel_edge_shapes(M, K, N, nO):
     check_layer(O.numpy(), X, W, rows=rows, ldy_extra=8)
 
 
+# Shapes that take the swapped-operand split-K kernel (M <= 128): every token
+# width class (16, 32, 64, 128), K split over clusters of 2..8 CTAs, ragged N,
+# a single K-block, and both degenerate outlier sets.
+SKINNY_EDGE = [
+    # (M, K, N, nO)
+    (16, 8192, 8192, 4096),
+    (5, 4096, 1040, 100),
+    (2, 64, 16, 0),
+    (32, 1024, 384, 0),
+    (33, 2048, 640, 2048),
+    (100, 3072, 2176, 320),
+    (128, 14336, 4096, 1792),
+]
+
+
+@pytest.mark.parametrize("M,K,N,nO", SKINNY_EDGE, ids=lambda v: str(v))
+def test_skinny_kernel_edge_shapes(M, K, N, nO):
+    O = workloads.outlier_channels(K, nO, seed=M + K + 2)
+    X = workloads.activations(M, K, O, seed=M + 2)
+    W = workloads.weights(N, K, seed=N + 2)
+    rows = None if M * N * K <= 2 ** 31 else np.unique(np.concatenate([sampled_rows(M, 24), [M - 1]]))
+    check_layer(O.numpy(), X, W, rows=rows, ldy_extra=8)
+
+
 def test_zero_rows_and_ties():
     M, K, N, nO = 40, 512, 128, 16
     O = workloads.outlier_channels(K, nO, seed=3)
