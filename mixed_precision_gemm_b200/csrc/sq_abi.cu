@@ -19,6 +19,7 @@
 #include "sq_gemm_pair.cuh"
 #include "sq_gemm_skinny.cuh"
 #include "sq_rowquant.cuh"
+#include "sq_rowquant_stream.cuh"
 
 namespace {
 
@@ -79,9 +80,16 @@ sq_status device_info(DevInfo &out)
 }
 
 // ---------------------------------------------------------------- per-kernel launch set-up
-// The dynamic shared-memory opt-in and the occupancy of each kernel are set
-// and queried once per device and size; later calls (including calls made
-// while a stream is captured into a CUDA graph) only look them up.
+// The dynamic shared-memory opt-in of each kernel (a per-function limit:
+// only ever raised, to the largest size launched so far) and its occupancy
+// per launch shape are set and queried once per device; later calls
+// (including calls made while a stream is captured into a CUDA graph) only
+// look them up.
+struct KernelLimit {
+    const void *fn;
+    int dev;
+    size_t smem_max;
+};
 struct KernelSetup {
     const void *fn;
     int dev;
@@ -89,6 +97,7 @@ struct KernelSetup {
     int threads;
     int per_sm;
 };
+std::vector<KernelLimit> g_limits;
 std::vector<KernelSetup> g_setups;
 std::mutex g_setup_mu;
 
@@ -98,15 +107,24 @@ sq_status kernel_setup(const void *fn, int threads, size_t smem, int &per_sm, co
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     std::lock_guard<std::mutex> lk(g_setup_mu);
+    KernelLimit *lim = nullptr;
+    for (KernelLimit &l : g_limits)
+        if (l.fn == fn && l.dev == dev) lim = &l;
+    if (!lim) {
+        g_limits.push_back({fn, dev, 48 * 1024});
+        lim = &g_limits.back();
+    }
+    if (smem > lim->smem_max) {
+        if ((e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))) !=
+            cudaSuccess)
+            return cuda_fail(e, what);
+        lim->smem_max = smem;
+    }
     for (const KernelSetup &k : g_setups)
         if (k.fn == fn && k.dev == dev && k.smem == smem && k.threads == threads) {
             per_sm = k.per_sm;
             return SQ_OK;
         }
-    if (smem > 48 * 1024 &&
-        (e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem))) !=
-            cudaSuccess)
-        return cuda_fail(e, what);
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem)) != cudaSuccess)
         return cuda_fail(e, what);
     if (per_sm < 1) return fail(SQ_ERR_UNSUPPORTED, "%s: kernel does not fit on an SM", what);
@@ -154,21 +172,62 @@ sq_status make_map(CUtensorMap &map, const void *base, CUtensorMapDataType dt, u
 }
 
 // ---------------------------------------------------------------- row quantizer
-template <int T, int CPT>
+template <int G, int CPT>
 sq_status launch_rowquant_t(const DevInfo &di, const uint16_t *src, int64_t rows, int K, int64_t ld,
                             const uint32_t *tab, int nO, int kn_pad, int no_pad, uint8_t *dn, float *ds,
                             uint16_t *dout, cudaStream_t stream)
 {
-    auto kern = sqq::rowquant_kernel<T, CPT>;
-    // two alternating (packed code row + outlier row) pairs, selector and keep tables
-    const size_t smem = 2u * (static_cast<size_t>(kn_pad / 2) + 16u + 2u * static_cast<size_t>(no_pad)) + 256u * 24u;
+    auto kern = sqq::rowquant_kernel<G, CPT>;
+    constexpr int T = 32 * G;
+    // constant tables, outlier channel list, two alternating packed code rows
+    const size_t smem = sizeof(sqq::QuantTables) + ((2u * static_cast<size_t>(no_pad) + 15u) & ~size_t(15)) +
+                        2u * (static_cast<size_t>(kn_pad / 2) + 16u);
     int per_sm = 0;
     sq_status st = kernel_setup(reinterpret_cast<const void *>(kern), T, smem, per_sm, "rowquant set-up");
     if (st != SQ_OK) return st;
-    cudaError_t e;
     const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * di.sms);
     kern<<<static_cast<unsigned>(grid), T, smem, stream>>>(src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds, dout);
+    cudaError_t e;
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "rowquant launch");
+    return SQ_OK;
+}
+
+template <int G>
+sq_status launch_rowquant_g(const DevInfo &di, const uint16_t *src, int64_t rows, int K, int64_t ld,
+                            const uint32_t *tab, int nO, int kn_pad, int no_pad, uint8_t *dn, float *ds,
+                            uint16_t *dout, cudaStream_t stream)
+{
+    const int cpt = (K / 8 + 32 * G - 1) / (32 * G);  // chunks of 8 channels per thread
+    if (cpt <= 1) return launch_rowquant_t<G, 1>(di, src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds, dout, stream);
+    if (cpt <= 2) return launch_rowquant_t<G, 2>(di, src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds, dout, stream);
+    if (cpt <= 4) return launch_rowquant_t<G, 4>(di, src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds, dout, stream);
+    if (cpt <= 8) return launch_rowquant_t<G, 8>(di, src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds, dout, stream);
+    return launch_rowquant_t<G, 16>(di, src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds, dout, stream);
+}
+
+// Rows streamed through shared memory (K <= 16384): as many consumer groups
+// of G warps as the shared memory holds (two row slots each), one CTA per SM.
+template <int G>
+sq_status launch_rowquant_stream(const DevInfo &di, const uint16_t *src, int64_t rows, int K, int64_t ld,
+                                 const uint32_t *tab, int nO, int kn_pad, int no_pad, uint8_t *dn, float *ds,
+                                 uint16_t *dout, cudaStream_t stream)
+{
+    constexpr int kSmemLimit = 232448 - 1024;
+    int ngrp = sqq::stream_max_groups(G);
+    while (ngrp > 1 && sqq::StreamLayout(K, kn_pad, no_pad, ngrp).bytes > kSmemLimit) --ngrp;
+    const size_t smem = static_cast<size_t>(sqq::StreamLayout(K, kn_pad, no_pad, ngrp).bytes);
+    if (smem > static_cast<size_t>(kSmemLimit))
+        return fail(SQ_ERR_UNSUPPORTED, "quantize-gather: K=%d, nO=%d do not fit in shared memory", K, nO);
+    auto kern = sqq::rowquant_stream_kernel<G>;
+    const int threads = 32 * (1 + ngrp * G);
+    int per_sm = 0;
+    sq_status st = kernel_setup(reinterpret_cast<const void *>(kern), threads, smem, per_sm, "rowquant stream set-up");
+    if (st != SQ_OK) return st;
+    const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * di.sms);
+    kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds,
+                                                                  dout, ngrp);
+    cudaError_t e;
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "rowquant stream launch");
     return SQ_OK;
 }
 
@@ -181,18 +240,22 @@ sq_status launch_rowquant(const uint16_t *src, int64_t rows, int64_t K, int64_t 
     if (st != SQ_OK) return st;
     const int kn_pad = static_cast<int>(sq_kn_pad(K, nO));
     const int no_pad = static_cast<int>(sq_no_pad(nO));
-    const int64_t nchunk = K / 8;
     const int k = static_cast<int>(K), no = static_cast<int>(nO);
-    // Few threads per row and many channels per thread: the per-row reduction
-    // and barriers are amortised over up to 64 elements per thread.
-    if (nchunk <= 64) return launch_rowquant_t<64, 1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 128) return launch_rowquant_t<64, 2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 256) return launch_rowquant_t<64, 4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 512) return launch_rowquant_t<64, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 1024) return launch_rowquant_t<128, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 2048) return launch_rowquant_t<256, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (nchunk <= 4096) return launch_rowquant_t<512, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    return launch_rowquant_t<1024, 8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (K <= sqq::kStreamMaxK) {
+        // 2048 channels per warp (8 chunks of 8 per thread)
+        if (K <= 2048) return launch_rowquant_stream<1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+        if (K <= 4096) return launch_rowquant_stream<2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+        if (K <= 8192) return launch_rowquant_stream<4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+        return launch_rowquant_stream<8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    }
+    // One warp per row up to 2048 channels (8 chunks of 8 per thread), then
+    // as many warps as keep a thread at 8 chunks or fewer.
+    const int64_t per_warp = 32 * sqq::kChunksPerThread * 8;
+    if (K <= per_warp) return launch_rowquant_g<1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (K <= 2 * per_warp) return launch_rowquant_g<2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (K <= 4 * per_warp) return launch_rowquant_g<4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (K <= 8 * per_warp) return launch_rowquant_g<8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    return launch_rowquant_g<16>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
 }
 
 // ---------------------------------------------------------------- GEMM

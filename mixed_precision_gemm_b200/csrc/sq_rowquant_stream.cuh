@@ -1,0 +1,245 @@
+// Quantize-and-gather with rows streamed through shared memory (K <= 16384).
+// Same computation and output layout as rowquant_kernel (sq_rowquant.cuh);
+// the difference is how rows reach the threads.
+//
+// A persistent CTA (one per SM) owns rows b, b + grid, b + 2 grid, ...  One
+// thread of warp 0 copies whole rows (2K bytes, one bulk asynchronous copy
+// each) into a ring of shared-memory slots, completion counted on an
+// mbarrier per slot; NGRP groups of G consumer warps take the CTA's rows in
+// turn (row i of the CTA goes to group i % NGRP), two slots per group, so a
+// group's next row is in flight while it works on the current one.  The ring
+// holds 2 * NGRP rows, which keeps enough bytes in flight per SM to stream
+// HBM without spending registers on them.
+//
+// A group works on a row in two passes over the slot: (1) absolute maximum
+// over the normal channels (outlier halves cleared with the keep masks),
+// group-wide maximum (shuffles; a named barrier when G > 1), scale; (2) codes
+// of every chunk, packed and OR-ed into the group's packed row (as in
+// rowquant_kernel), and the compact outlier row gathered from the slot.  The
+// slot is then released and the packed row written out.
+//
+// Every wait is bounded; after a timeout the abort flag makes the remaining
+// waits return at once, and every group still walks through the same rows
+// and named barriers, so the CTA always finishes.
+#pragma once
+
+#include "sq_rowquant.cuh"
+
+namespace sqq {
+
+constexpr int kStreamMaxK = 16384;
+constexpr int kStreamChunks = 8;  // most 8-channel chunks per thread and row: K <= 2048 G
+
+enum : unsigned { SITE_RQ_PROD = 0x601, SITE_RQ_CONS = 0x602 };
+
+// Shared-memory layout, computed identically on the host and the device.
+struct StreamLayout {
+    int row_bytes;   // 2K, rounded up to 128
+    int pk_alloc;    // kn_pad / 2 + 16
+    int off_pl, off_olist, off_pbuf, off_bar, off_misc, off_ring, bytes;
+
+    __host__ __device__ StreamLayout(int K, int kn_pad, int no_pad, int ngrp)
+    {
+        row_bytes = (2 * K + 127) & ~127;
+        pk_alloc = kn_pad / 2 + 16;
+        off_pl = static_cast<int>(sizeof(QuantTables));
+        off_olist = off_pl + ((4 * (K / 8) + 15) & ~15);
+        off_pbuf = off_olist + ((2 * no_pad + 15) & ~15);
+        off_bar = off_pbuf + ngrp * ((pk_alloc + 15) & ~15);
+        off_misc = off_bar + 2 * (2 * ngrp) * 8;
+        off_ring = (off_misc + 16 + 8 * ngrp * 4 + 127) & ~127;   // + per-group reduction words
+        bytes = off_ring + 2 * ngrp * row_bytes;
+    }
+};
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Most consumer groups per CTA for G warps per row (shared memory holds
+// two row slots per group; more warps per row raise the warps per SM
+// without more shared memory).
+__host__ __device__ constexpr int stream_max_groups(int G) { return G <= 2 ? 10 : G == 4 ? 6 : 3; }
+
+template <int G>
+__global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowquant_stream_kernel(
+    const uint16_t *__restrict__ src, int64_t rows, int K, int64_t ld,
+    const uint32_t *__restrict__ chan_tab, int nO, int kn_pad, int no_pad,
+    uint8_t *__restrict__ dst_n, float *__restrict__ dst_s, uint16_t *__restrict__ dst_o, int ngrp)
+{
+    extern __shared__ __align__(128) uint8_t rs_smem[];
+    const StreamLayout L(K, kn_pad, no_pad, ngrp);
+    QuantTables *tabs = reinterpret_cast<QuantTables *>(rs_smem);
+    uint32_t *pl_tab = reinterpret_cast<uint32_t *>(rs_smem + L.off_pl);
+    uint16_t *olist = reinterpret_cast<uint16_t *>(rs_smem + L.off_olist);
+    const uint32_t sbase = sqd::smem_u32(rs_smem);
+    const int nslot = 2 * ngrp;
+    auto full = [&](int s) { return sbase + L.off_bar + 8u * s; };
+    auto empty = [&](int s) { return sbase + L.off_bar + 8u * (nslot + s); };
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(rs_smem + L.off_misc);
+    uint32_t *red = reinterpret_cast<uint32_t *>(rs_smem + L.off_misc + 16);   // [ngrp][8]
+
+    const int tid = threadIdx.x;
+    const int nthr = blockDim.x;
+    const int nchunk = K >> 3;
+
+    // ---------------------------------------------------------------- set-up
+    if (tid == 0) {
+        for (int s = 0; s < nslot; ++s) {
+            sqd::mbar_init(full(s), 1);   // producer's expect-tx arrival + the copy's bytes
+            sqd::mbar_init(empty(s), G);  // one arrival per warp of the consuming group
+        }
+        *abort_flag = 0u;
+        sqd::fence_barrier_init();
+    }
+    for (int i = tid; i < static_cast<int>(sizeof(QuantTables) / 16); i += nthr)
+        reinterpret_cast<uint4 *>(tabs)[i] = __ldg(reinterpret_cast<const uint4 *>(&g_qtab) + i);
+    for (int i = tid; i < ngrp * ((L.pk_alloc + 15) / 16); i += nthr)
+        reinterpret_cast<uint4 *>(rs_smem + L.off_pbuf)[i] = make_uint4(0, 0, 0, 0);
+    for (int j = nO + tid; j < no_pad; j += nthr) olist[j] = kNoChannel;
+    // Per chunk: outlier mask, packed word and nibble shift of its first
+    // code (see rowquant_kernel); its outliers enter the list O.
+    for (int c = tid; c < nchunk; c += nthr) {
+        const uint32_t tb = __ldg(chan_tab + c);
+        const uint32_t below = tb >> 8;
+        const uint32_t p = 8u * static_cast<uint32_t>(c) - below;
+        pl_tab[c] = (tb & 0xFFu) | ((p & 7u) << 8) | ((p >> 3) << 11);
+        for (uint32_t mm = tb & 0xFFu, j = below; mm; mm &= mm - 1, ++j)
+            olist[j] = static_cast<uint16_t>(8 * c + __ffs(mm) - 1);
+    }
+    __syncthreads();
+
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    if (warp == 0) {
+        // ------------------------------------------------------------ row copies
+        if (lane == 0) {
+            int64_t issued = 0;
+            for (int64_t i = 0;; ++i) {
+                const int64_t r = blockIdx.x + i * gridDim.x;
+                if (r >= rows) break;
+                const int s = static_cast<int>(i % nslot);
+                if (!sqd::mbar_wait(empty(s), static_cast<uint32_t>((i / nslot) & 1) ^ 1u, abort_flag, SITE_RQ_PROD))
+                    break;
+                sqd::mbar_arrive_expect_tx(full(s), static_cast<uint32_t>(2 * K));
+                sqd::bulk_load(sbase + L.off_ring + s * L.row_bytes, src + r * ld, static_cast<uint32_t>(2 * K), full(s));
+                issued = i + 1;
+            }
+            if (*abort_flag) {
+                // Let the copies still in flight land before the CTA exits.
+                for (int64_t i = issued > nslot ? issued - nslot : 0; i < issued; ++i)
+                    sqd::mbar_drain(full(static_cast<int>(i % nslot)), static_cast<uint32_t>((i / nslot) & 1));
+            }
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumer groups
+    const int gi = (warp - 1) / G;       // group
+    const int gt = tid - 32 - gi * 32 * G;  // thread index inside the group
+    const int GT = 32 * G;
+    const int bar_id = 1 + gi;
+    uint32_t *pbuf = reinterpret_cast<uint32_t *>(rs_smem + L.off_pbuf + gi * L.pk_alloc);
+    const uint32_t *ol2 = reinterpret_cast<const uint32_t *>(olist);
+    const int pk_bytes = kn_pad >> 1;
+    const float y7 = __frcp_rn(7.0f);
+    const RowScale rs_const = [] {
+        RowScale r{};
+        r.magic2 = f2_pack(__float_as_uint(kMagic), __float_as_uint(kMagic));
+        r.up2 = f2_pack(__float_as_uint(kUpScale), __float_as_uint(kUpScale));
+        return r;
+    }();
+
+    for (int64_t i = gi;; i += ngrp) {
+        const int64_t r = blockIdx.x + i * gridDim.x;
+        if (r >= rows) break;
+        const int s = static_cast<int>(i % nslot);
+        // A timed-out wait only raises the abort flag: the group goes on with
+        // whatever the slot holds, so that every barrier below is still met.
+        sqd::mbar_wait(full(s), static_cast<uint32_t>((i / nslot) & 1), abort_flag, SITE_RQ_CONS);
+
+        // 1. absolute maximum over the normal channels
+        uint32_t am = 0u;
+#pragma unroll
+        for (int k = 0; k < kStreamChunks; ++k) {
+            const int c = gt + k * GT;
+            if (c >= nchunk) break;
+            const uint4 v = *reinterpret_cast<const uint4 *>(rs_smem + L.off_ring + s * L.row_bytes + 16 * c);
+            const uint4 kp = *reinterpret_cast<const uint4 *>(tabs->keep[chunk_mask(pl_tab[c])]);
+            am = maxabs_bf16x2(am, maxabs_bf16x2(maxabs_bf16x2(v.x & kp.x, v.y & kp.y),
+                                                 maxabs_bf16x2(v.z & kp.z, v.w & kp.w)));
+        }
+        uint32_t amax = max(am & 0x7FFFu, (am >> 16) & 0x7FFFu);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
+        if constexpr (G > 1) {
+            if (lane == 0) red[gi * 8 + (gt >> 5)] = amax;
+            named_bar_sync(bar_id, GT);
+            amax = red[gi * 8];
+#pragma unroll
+            for (int w = 1; w < G; ++w) amax = max(amax, red[gi * 8 + w]);
+        }
+
+        // 2. scale and quantizer constants
+        const bool zero = (amax == 0u);
+        const float sc = zero ? 0.0f : row_scale(__uint_as_float(amax << 16), y7);
+        const bool up = !zero && sc < kTinyScale;
+        const float s1 = up ? sc * kUpScale : sc;
+        const float inv_s = zero ? 0.0f : __frcp_rn(s1);
+        if (gt == 0) dst_s[r] = sc;
+        RowScale rs = rs_const;
+        rs.inv2 = f2_pack(__float_as_uint(inv_s), __float_as_uint(inv_s));
+        rs.negs2 = f2_pack(__float_as_uint(-s1), __float_as_uint(-s1));
+
+        // 3. codes of each chunk, normal ones packed and OR-ed into the row
+#pragma unroll
+        for (int k = 0; k < kStreamChunks; ++k) {
+            const int c = gt + k * GT;
+            if (c >= nchunk) break;
+            const uint4 v = *reinterpret_cast<const uint4 *>(rs_smem + L.off_ring + s * L.row_bytes + 16 * c);
+            const uint32_t pl = pl_tab[c];
+            uint32_t lo, hi;
+            if (!up) quant8_pairs<false>(v, rs, lo, hi);
+            else quant8_pairs<true>(v, rs, lo, hi);
+            const uint4 pk = *reinterpret_cast<const uint4 *>(tabs->pack[chunk_mask(pl)]);
+            const uint32_t ev = __byte_perm(lo, hi, pk.x);  // normal codes 0, 2, 4, 6
+            const uint32_t od = __byte_perm(lo, hi, pk.y);  // normal codes 1, 3, 5, 7
+            const uint32_t V = ((ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u)) & pk.z;
+            const uint32_t sh = 4u * chunk_nib(pl);
+            uint32_t *dst = pbuf + chunk_word(pl);
+            atomicOr(dst, V << sh);
+            if (sh) atomicOr(dst + 1, V >> (32u - sh));
+        }
+
+        // 4. compact outlier row X_O[r, j] = X[r, O[j]], read from the slot
+        if (nO > 0) {
+            const uint16_t *xrow = reinterpret_cast<const uint16_t *>(rs_smem + L.off_ring + s * L.row_bytes);
+            uint32_t *out_o = reinterpret_cast<uint32_t *>(dst_o + r * static_cast<int64_t>(no_pad));
+#pragma unroll 4
+            for (int jp = gt; jp < (no_pad >> 1); jp += GT) {
+                const uint32_t e2 = ol2[jp];
+                const uint32_t e0 = e2 & 0xFFFFu, e1 = e2 >> 16;
+                const uint32_t x0 = e0 != kNoChannel ? xrow[e0] : 0u;
+                const uint32_t x1 = e1 != kNoChannel ? xrow[e1] : 0u;
+                out_o[jp] = x0 | (x1 << 16);
+            }
+        }
+        // The slot has been read by this warp: hand it back.
+        __syncwarp();
+        if (lane == 0) sqd::mbar_arrive(empty(s));
+        if constexpr (G > 1) named_bar_sync(bar_id, GT);
+        else __syncwarp();
+
+        // 5. packed row out, cleared for the group's next row
+        uint4 *pk16 = reinterpret_cast<uint4 *>(pbuf);
+        uint4 *out_n = reinterpret_cast<uint4 *>(dst_n + r * static_cast<int64_t>(pk_bytes));
+        for (int j = gt; j < (L.pk_alloc >> 4); j += GT) {
+            if (j < (pk_bytes >> 4)) out_n[j] = pk16[j];
+            pk16[j] = make_uint4(0, 0, 0, 0);
+        }
+        if constexpr (G == 1) __syncwarp();
+    }
+}
+
+}  // namespace sqq

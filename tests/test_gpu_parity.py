@@ -170,6 +170,23 @@ def test_skinny_kernel_edge_shapes(M, K, N, nO):
     check_layer(O.numpy(), X, W, rows=rows, ldy_extra=8)
 
 
+# Rows wider than 16384 channels take the register-resident quantizer (a group
+# of 16 warps per row); narrower rows are streamed through shared memory.
+WIDE_K = [
+    # (M, K, N, nO)
+    (40, 20480, 256, 300),
+    (24, 40960, 128, 5000),
+]
+
+
+@pytest.mark.parametrize("M,K,N,nO", WIDE_K, ids=lambda v: str(v))
+def test_wide_rows(M, K, N, nO):
+    O = workloads.outlier_channels(K, nO, seed=K + 5)
+    X = workloads.activations(M, K, O, seed=M + 5)
+    W = workloads.weights(N, K, seed=N + 5)
+    check_layer(O.numpy(), X, W, ldy_extra=8)
+
+
 def test_zero_rows_and_ties():
     M, K, N, nO = 40, 512, 128, 16
     O = workloads.outlier_channels(K, nO, seed=3)
@@ -183,6 +200,24 @@ def test_zero_rows_and_ties():
     X[3, normal] = X[2, normal] * 0.125
     W = workloads.weights(N, K, seed=5).float()
     W[7] = 0.0
+    check_layer(O.numpy(), X.to(torch.bfloat16), W.to(torch.bfloat16))
+
+
+def test_tiny_and_huge_row_scales():
+    """Rows scaled by powers of two from the bf16 subnormal range (scale below
+    2^-100: the quantizer's prescaled path) up to 2^100: codes and scales
+    bit-exact, and Y within tolerance."""
+    exps = [-140, -136, -133, -130, -127, -124, -120, -112, -104, -100, -96, -60, 0, 40, 80, 100]
+    M, K, N, nO = len(exps) * 2, 1024, 128, 40
+    O = workloads.outlier_channels(K, nO, seed=11)
+    X = workloads.activations(M, K, O, seed=12).float()
+    for i, e in enumerate(exps):
+        X[2 * i] *= 2.0 ** e
+        X[2 * i + 1] *= 2.0 ** e
+        X[2 * i + 1, O.long()] = 1.0     # outliers of ordinary size beside a tiny or huge normal part
+    W = workloads.weights(N, K, seed=13).float()
+    W[3] *= 2.0 ** -120
+    W[4] *= 2.0 ** -133
     check_layer(O.numpy(), X.to(torch.bfloat16), W.to(torch.bfloat16))
 
 
