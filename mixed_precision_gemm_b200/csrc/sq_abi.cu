@@ -171,6 +171,37 @@ sq_status make_map(CUtensorMap &map, const void *base, CUtensorMapDataType dt, u
     return SQ_OK;
 }
 
+// ---------------------------------------------------------------- launches
+// Every kernel goes out with programmatic stream serialization: it may start
+// its set-up while the previous kernel in the stream finishes, and waits for
+// it (griddepcontrol.wait) before touching memory that kernel may own.
+// cluster_x > 0 also sets the cluster shape (cluster_x, 1, 1).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                     unsigned cluster_x, Args &&...args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+    if (cluster_x > 0) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ---------------------------------------------------------------- row quantizer
 template <int G, int CPT>
 sq_status launch_rowquant_t(const DevInfo &di, const uint16_t *src, int64_t rows, int K, int64_t ld,
@@ -186,9 +217,9 @@ sq_status launch_rowquant_t(const DevInfo &di, const uint16_t *src, int64_t rows
     sq_status st = kernel_setup(reinterpret_cast<const void *>(kern), T, smem, per_sm, "rowquant set-up");
     if (st != SQ_OK) return st;
     const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * di.sms);
-    kern<<<static_cast<unsigned>(grid), T, smem, stream>>>(src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds, dout);
-    cudaError_t e;
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "rowquant launch");
+    cudaError_t e = launch_k(kern, dim3(static_cast<unsigned>(grid)), dim3(T), smem, stream, 0u, src, rows, K, ld, tab,
+                             nO, kn_pad, no_pad, dn, ds, dout);
+    if (e != cudaSuccess) return cuda_fail(e, "rowquant launch");
     return SQ_OK;
 }
 
@@ -224,10 +255,9 @@ sq_status launch_rowquant_stream(const DevInfo &di, const uint16_t *src, int64_t
     sq_status st = kernel_setup(reinterpret_cast<const void *>(kern), threads, smem, per_sm, "rowquant stream set-up");
     if (st != SQ_OK) return st;
     const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * di.sms);
-    kern<<<static_cast<unsigned>(grid), threads, smem, stream>>>(src, rows, K, ld, tab, nO, kn_pad, no_pad, dn, ds,
-                                                                  dout, ngrp);
-    cudaError_t e;
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "rowquant stream launch");
+    cudaError_t e = launch_k(kern, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream, 0u, src, rows, K, ld,
+                             tab, nO, kn_pad, no_pad, dn, ds, dout, ngrp);
+    if (e != cudaSuccess) return cuda_fail(e, "rowquant stream launch");
     return SQ_OK;
 }
 
@@ -242,9 +272,10 @@ sq_status launch_rowquant(const uint16_t *src, int64_t rows, int64_t K, int64_t 
     const int no_pad = static_cast<int>(sq_no_pad(nO));
     const int k = static_cast<int>(K), no = static_cast<int>(nO);
     if (K <= sqq::kStreamMaxK) {
-        // 2048 channels per warp (8 chunks of 8 per thread)
-        if (K <= 2048) return launch_rowquant_stream<1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-        if (K <= 4096) return launch_rowquant_stream<2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+        // up to 2048 channels per warp (8 chunks of 8 per thread); narrow rows
+        // take more warps per row, so that each SM runs more warps
+        if (K <= 1024) return launch_rowquant_stream<1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+        if (K <= 2048) return launch_rowquant_stream<2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
         if (K <= 8192) return launch_rowquant_stream<4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
         return launch_rowquant_stream<8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
     }
@@ -319,8 +350,9 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
     if ((st = kernel_setup(reinterpret_cast<const void *>(kern), sqg::PAIR_THREADS, C::SMEM_BYTES, per_sm, "gemm pair set-up")) != SQ_OK)
         return st;
     cudaError_t e;
-    kern<<<static_cast<unsigned>(2 * clusters), sqg::PAIR_THREADS, C::SMEM_BYTES, stream>>>(m_xo, m_wo, m_xn, m_wn, a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_fail(e, "gemm pair launch");
+    if ((e = launch_k(kern, dim3(static_cast<unsigned>(2 * clusters)), dim3(sqg::PAIR_THREADS), C::SMEM_BYTES, stream, 0u,
+                      m_xo, m_wo, m_xn, m_wn, a)) != cudaSuccess)
+        return cuda_fail(e, "gemm pair launch");
     return SQ_OK;
 }
 
@@ -378,19 +410,8 @@ sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *
     if ((st = kernel_setup(reinterpret_cast<const void *>(kern), sqg::SK_THREADS, C::SMEM_BYTES, per_sm, "gemm skinny set-up")) != SQ_OK)
         return st;
     cudaError_t e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(tiles_n * S), 1, 1);
-    cfg.blockDim = dim3(sqg::SK_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(S);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if ((e = cudaLaunchKernelEx(&cfg, kern, m_xo, m_wo, m_xn, m_wn, a)) != cudaSuccess)
+    if ((e = launch_k(kern, dim3(static_cast<unsigned>(tiles_n * S)), dim3(sqg::SK_THREADS), C::SMEM_BYTES, stream,
+                      static_cast<unsigned>(S), m_xo, m_wo, m_xn, m_wn, a)) != cudaSuccess)
         return cuda_fail(e, "gemm skinny launch");
     return SQ_OK;
 }

@@ -389,6 +389,15 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
                  : "memory");
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Kernels are launched with programmatic stream serialization: the next
+// kernel in the stream may start (and run its set-up) before this one ends.
+// pdl_launch_dependents() lets it; pdl_wait() blocks until every kernel this
+// one depends on has completed and its memory is visible.  Without the
+// launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // 16-byte store to a shared::cluster address (any CTA of the cluster).
 __device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
 {

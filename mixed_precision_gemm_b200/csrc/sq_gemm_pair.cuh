@@ -89,6 +89,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
     const int lane = threadIdx.x & 31;
     const uint32_t rank = sqd::cluster_ctarank();
     const bool leader = (rank == 0);
+    sqd::pdl_launch_dependents();
 
     const uint32_t bar0 = sbase + C::OFF_BAR;
     auto op_full = [&](int e) { return bar0 + 8u * e; };
@@ -138,6 +139,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
     sqd::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated in both
     sqd::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    sqd::pdl_wait();  // operands and Y may belong to the previous kernel
 
     const int nkb_i = args.nkb_i, nkb_o = args.nkb_o;
     const int per_tile = nkb_o + nkb_i;

@@ -126,6 +126,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
     const int S = args.splits;
     const int rank = static_cast<int>(sqd::cluster_ctarank());
     const int n0 = static_cast<int>(blockIdx.x) / S * 128;
+    sqd::pdl_launch_dependents();
 
     const uint32_t bar0 = sbase + C::OFF_BAR;
     auto stg_full = [&](int s) { return bar0 + 8u * s; };
@@ -186,6 +187,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
     __syncthreads();
     sqd::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    sqd::pdl_wait();  // operands and Y may belong to the previous kernel
 
     if (warp == 0) {
         // ------------------------------------------------------------ staging producer

@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(32 * G, 512 / (32 * G)) rowquant_kernel(
     const int nchunk = K >> 3;
     const bool has_o = nO > 0;
 
-    // First row's loads go out before anything else.
+    sqd::pdl_launch_dependents();
     constexpr bool kPrefetch = CPT <= 8;  // registers allow holding the next row too
     uint4 nxt[kPrefetch ? CPT : 1];
     auto load_row = [&](int64_t r, uint4 *dst) {
@@ -252,10 +252,7 @@ __global__ void __launch_bounds__(32 * G, 512 / (32 * G)) rowquant_kernel(
                                  : load_chunk<false>(row + 8 * c);
         }
     };
-    if constexpr (kPrefetch) {
-        if (blockIdx.x < rows) load_row(blockIdx.x, nxt);
-    }
-
+    // Set-up (runs while the previous kernel in the stream may still be finishing).
     for (int i = tid; i < static_cast<int>(sizeof(QuantTables) / 16); i += T)
         reinterpret_cast<uint4 *>(tabs)[i] = __ldg(reinterpret_cast<const uint4 *>(&g_qtab) + i);
     for (int i = tid; i < 2 * pk_alloc / 16; i += T)
@@ -281,6 +278,10 @@ __global__ void __launch_bounds__(32 * G, 512 / (32 * G)) rowquant_kernel(
     }
     const float y7 = __frcp_rn(7.0f);
     __syncthreads();  // tables, outlier list and zeroed buffers visible
+    sqd::pdl_wait();  // X and the outputs may belong to the previous kernel
+    if constexpr (kPrefetch) {
+        if (blockIdx.x < rows) load_row(blockIdx.x, nxt);
+    }
 
     int parity = 0;
     for (int64_t r = blockIdx.x; r < rows; r += gridDim.x, parity ^= 1) {

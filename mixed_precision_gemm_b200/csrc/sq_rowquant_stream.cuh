@@ -60,7 +60,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads)
 // Most consumer groups per CTA for G warps per row (shared memory holds
 // two row slots per group; more warps per row raise the warps per SM
 // without more shared memory).
-__host__ __device__ constexpr int stream_max_groups(int G) { return G <= 2 ? 10 : G == 4 ? 6 : 3; }
+__host__ __device__ constexpr int stream_max_groups(int G) { return G <= 2 ? 10 : G == 4 ? 7 : 3; }
 
 template <int G>
 __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowquant_stream_kernel(
@@ -83,8 +83,10 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
     const int tid = threadIdx.x;
     const int nthr = blockDim.x;
     const int nchunk = K >> 3;
+    sqd::pdl_launch_dependents();
 
     // ---------------------------------------------------------------- set-up
+    // (runs while the previous kernel in the stream may still be finishing)
     if (tid == 0) {
         for (int s = 0; s < nslot; ++s) {
             sqd::mbar_init(full(s), 1);   // producer's expect-tx arrival + the copy's bytes
@@ -109,6 +111,7 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
             olist[j] = static_cast<uint16_t>(8 * c + __ffs(mm) - 1);
     }
     __syncthreads();
+    sqd::pdl_wait();  // X and the outputs may belong to the previous kernel
 
     const int warp = tid >> 5;
     const int lane = tid & 31;
