@@ -11,7 +11,9 @@ is described in the C file's header: the OSC page (arXiv:2604.12782, abstract
 and technical framework: static outlier channels, compact gather, 4-bit GEMM
 plus 16-bit branch GEMM, fused sum) and the SQ-format write-up of
 arXiv:2512.05409 (section 9: symmetric quantization, column reordering by the
-static mask).
+static mask).  The FP8 functions follow the same page's FP8 fallback for the
+inputs of W2 (E4M3 low path, scale = absolute maximum / 448; readings in the C
+file).
 """
 from __future__ import annotations
 
@@ -57,8 +59,14 @@ def _load():
             lib.orc_chan_table.argtypes = [P, I, I, P]
             lib.orc_dual_linear_rows.argtypes = [P, P, P, I, P, P, P, I, I, I, P, P, P]
             lib.orc_num_threads.argtypes = []
+            lib.orc_e4m3_encode_array.argtypes = [P, I, P]
+            lib.orc_e4m3_decode_array.argtypes = [P, I, P]
+            lib.orc_quantize_rows_fp8.argtypes = [P, I, I, I, P, I, P, P, P]
+            lib.orc_dual_linear_rows_fp8.argtypes = [P, P, P, I, P, P, P, I, I, I, P, P, P]
             for f in (lib.orc_validate_outliers, lib.orc_quantize_rows, lib.orc_pack_int4,
-                      lib.orc_chan_table, lib.orc_dual_linear_rows, lib.orc_num_threads):
+                      lib.orc_chan_table, lib.orc_dual_linear_rows, lib.orc_num_threads,
+                      lib.orc_e4m3_encode_array, lib.orc_e4m3_decode_array, lib.orc_quantize_rows_fp8,
+                      lib.orc_dual_linear_rows_fp8):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -155,3 +163,71 @@ def linear(X_bits: np.ndarray, W_bits: np.ndarray, O, rows=None):
     qw, sw, wo = quantize_rows(W_bits, K, O)
     acc_i, acc_o, y = dual_linear_rows(qx, sx, xo, qw, sw, wo)
     return dict(qx=qx, sx=sx, xo=xo, qw=qw, sw=sw, wo=wo, acc_i=acc_i, acc_o=acc_o, y=y)
+
+
+# ---------------------------------------------------------------- FP8 low path
+E4M3_MAX = 448.0  # largest finite E4M3 value
+
+
+def e4m3_encode(t) -> np.ndarray:
+    """E4M3 codes (uint8) nearest to float32 values, ties to even, saturating at 448."""
+    t = np.ascontiguousarray(t, np.float32).reshape(-1)
+    out = np.zeros(t.size, np.uint8)
+    _load().orc_e4m3_encode_array(_ptr(t), t.size, _ptr(out))
+    return out
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 values of E4M3 codes."""
+    c = np.ascontiguousarray(codes, np.uint8).reshape(-1)
+    out = np.zeros(c.size, np.float64)
+    _load().orc_e4m3_decode_array(_ptr(c), c.size, _ptr(out))
+    return out
+
+
+def quantize_rows_fp8(src_bits: np.ndarray, K: int, O):
+    """FP8 quantize-and-gather: (codes uint8 E4M3 [rows, K-nO], scale float32 [rows], outl uint16 [rows, nO])."""
+    src = np.ascontiguousarray(src_bits, dtype=np.uint16)
+    if src.ndim != 2 or src.shape[1] < K:
+        raise ValueError("src must be [rows, ld>=K]")
+    O = _as_O(O)
+    rows, ld = src.shape
+    KN = K - O.size
+    codes = np.zeros((rows, KN), np.uint8)
+    scale = np.zeros(rows, np.float32)
+    outl = np.zeros((rows, O.size), np.uint16)
+    rc = _load().orc_quantize_rows_fp8(_ptr(src), rows, K, ld, _ptr(O), O.size,
+                                       _ptr(codes), _ptr(scale), _ptr(outl))
+    if rc != 0:
+        raise ValueError("invalid outlier channel set")
+    return codes, scale, outl
+
+
+def dual_linear_rows_fp8(qx, sx, xo, qw, sw, wo):
+    """(acc_8 float64, acc_o float64, y float64), each [rows of qx, rows of qw]."""
+    qx = np.ascontiguousarray(qx, np.uint8)
+    qw = np.ascontiguousarray(qw, np.uint8)
+    sx = np.ascontiguousarray(sx, np.float32)
+    sw = np.ascontiguousarray(sw, np.float32)
+    xo = np.ascontiguousarray(xo, np.uint16)
+    wo = np.ascontiguousarray(wo, np.uint16)
+    Mr, KN = qx.shape
+    N = qw.shape[0]
+    nO = xo.shape[1]
+    assert qw.shape[1] == KN and wo.shape == (N, nO) and xo.shape[0] == Mr
+    acc_8 = np.zeros((Mr, N), np.float64)
+    acc_o = np.zeros((Mr, N), np.float64)
+    y = np.zeros((Mr, N), np.float64)
+    _load().orc_dual_linear_rows_fp8(_ptr(qx), _ptr(sx), _ptr(xo), Mr, _ptr(qw), _ptr(sw), _ptr(wo),
+                                     N, KN, nO, _ptr(acc_8), _ptr(acc_o), _ptr(y))
+    return acc_8, acc_o, y
+
+
+def linear_fp8(X_bits: np.ndarray, W_bits: np.ndarray, O, rows=None):
+    """Whole layer with the FP8 low path for the selected activation rows (all when None)."""
+    K = W_bits.shape[1]
+    Xs = X_bits if rows is None else X_bits[np.asarray(rows)]
+    qx, sx, xo = quantize_rows_fp8(Xs, K, O)
+    qw, sw, wo = quantize_rows_fp8(W_bits, K, O)
+    acc_8, acc_o, y = dual_linear_rows_fp8(qx, sx, xo, qw, sw, wo)
+    return dict(qx=qx, sx=sx, xo=xo, qw=qw, sw=sw, wo=wo, acc_8=acc_8, acc_o=acc_o, y=y)

@@ -202,6 +202,132 @@ int orc_dual_linear_rows(const int8_t *qx, const float *sx, const uint16_t *xo, 
     return 0;
 }
 
+/* ------------------------------------------------------------------ FP8 low path
+ * OSC (arXiv:2604.12782), abstract and "technical framework": for the inputs
+ * of W2 (the down projection), where outlier clustering is less pronounced,
+ * the 4-bit path falls back to FP8.  The pages fix nothing further; the
+ * reading taken here keeps the rest of the layer unchanged:
+ *   - format E4M3 (4 exponent bits, bias 7, 3 mantissa bits, subnormals
+ *     m * 2^-9, largest finite value 448, no infinities);
+ *   - s = a / 448 with a the absolute maximum over the normal channels (fp32,
+ *     IEEE division), one scale per token row of X and per output row of W;
+ *   - code = E4M3 nearest to the fp32 quotient t = x / s, ties to the even
+ *     code, magnitudes above 448 saturate to 448 (t can exceed 448 by a
+ *     rounding error at the absolute-maximum element);
+ *   - the sign follows the quotient, as in any IEEE-style conversion: a
+ *     negative t that rounds to zero gives -0 (0x80);
+ *   - a == 0: s = 0 and every code is 0x00;
+ *   - the outlier channels still run through the 16-bit branch (nO = 0 gives
+ *     a plain FP8 GEMM).
+ */
+#define ORC_E4M3_MAX 448.0
+
+/* Value of an E4M3 code (sign bit 7, exponent bits 6..3, mantissa bits 2..0). */
+double orc_e4m3_decode(uint8_t code)
+{
+    const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Nearest E4M3 code to t (finite), ties to the even code, saturating at
+ * 448.  The non-negative finite codes 0x00..0x7E are increasing in value, so
+ * the neighbours of |t| are found by bisection over them. */
+uint8_t orc_e4m3_encode(float t)
+{
+    const uint8_t sign = signbit(t) ? 0x80 : 0x00;
+    const double v = fabs((double)t);
+    if (v >= ORC_E4M3_MAX) return (uint8_t)(sign | 0x7E);
+    int lo = 0, hi = 0x7E; /* decode(lo) <= v < decode(hi) */
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) / 2;
+        if (orc_e4m3_decode((uint8_t)mid) <= v) lo = mid; else hi = mid;
+    }
+    const double dl = v - orc_e4m3_decode((uint8_t)lo), dh = orc_e4m3_decode((uint8_t)hi) - v;
+    const int code = (dl < dh) ? lo : (dh < dl) ? hi : ((lo % 2 == 0) ? lo : hi);
+    return (uint8_t)(sign | code); /* a negative value that rounds to zero gives -0 (0x80) */
+}
+
+int orc_e4m3_encode_array(const float *t, int64_t n, uint8_t *codes)
+{
+    for (int64_t i = 0; i < n; ++i) codes[i] = orc_e4m3_encode(t[i]);
+    return 0;
+}
+
+int orc_e4m3_decode_array(const uint8_t *codes, int64_t n, double *v)
+{
+    for (int64_t i = 0; i < n; ++i) v[i] = orc_e4m3_decode(codes[i]);
+    return 0;
+}
+
+/* Quantize-and-gather with the FP8 low path; outputs as orc_quantize_rows,
+ * with E4M3 codes (uint8) in place of the INT4 codes. */
+int orc_quantize_rows_fp8(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                          const int32_t *O, int64_t nO,
+                          uint8_t *codes, float *scale, uint16_t *outl)
+{
+    if (orc_validate_outliers(O, nO, K) != 0 || ld < K) return -1;
+    char *is_outlier = (char *)calloc((size_t)K, 1);
+    if (!is_outlier) return -1;
+    for (int64_t j = 0; j < nO; ++j) is_outlier[O[j]] = 1;
+    const int64_t KN = K - nO;
+
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *row = src + r * ld;
+        float a = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            if (is_outlier[k]) continue;
+            float v = fabsf(orc_bf16_to_f32(row[k]));
+            if (v > a) a = v;
+        }
+        float s = a / 448.0f;
+        if (a == 0.0f) s = 0.0f;
+        scale[r] = s;
+        int64_t j = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            if (is_outlier[k]) continue;
+            uint8_t q = 0;
+            if (a != 0.0f) {
+                float t = orc_bf16_to_f32(row[k]) / s;
+                q = orc_e4m3_encode(t);
+            }
+            codes[r * KN + j] = q;
+            ++j;
+        }
+        for (int64_t jo = 0; jo < nO; ++jo) outl[r * nO + jo] = row[O[jo]];
+    }
+    free(is_outlier);
+    return 0;
+}
+
+/* Dual-path products with the FP8 low path:
+ *   acc_8 [Mr, N]  sum of decoded E4M3 products, fp64 (each product exact)
+ *   acc_o [Mr, N]  16-bit branch, fp64
+ *   y     [Mr, N]  acc_8 * s_x * s_w + acc_o, fp64 */
+int orc_dual_linear_rows_fp8(const uint8_t *qx, const float *sx, const uint16_t *xo, int64_t Mr,
+                             const uint8_t *qw, const float *sw, const uint16_t *wo, int64_t N,
+                             int64_t KN, int64_t nO,
+                             double *acc_8, double *acc_o, double *y)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < Mr; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double a8 = 0.0;
+            for (int64_t j = 0; j < KN; ++j)
+                a8 += orc_e4m3_decode(qx[m * KN + j]) * orc_e4m3_decode(qw[n * KN + j]);
+            double ao = 0.0;
+            for (int64_t j = 0; j < nO; ++j)
+                ao += (double)orc_bf16_to_f32(xo[m * nO + j]) *
+                      (double)orc_bf16_to_f32(wo[n * nO + j]);
+            acc_8[m * N + n] = a8;
+            acc_o[m * N + n] = ao;
+            y[m * N + n] = a8 * (double)sx[m] * (double)sw[n] + ao;
+        }
+    }
+    return 0;
+}
+
 #ifdef _OPENMP
 #include <omp.h>
 #endif

@@ -316,3 +316,134 @@ def test_outlier_channels_reduce_error():
         err[name] = np.linalg.norm(y - exact) / np.linalg.norm(exact)
     assert err["true"] < 0.25 * err["none"]
     assert err["true"] < 0.2
+
+
+# ----------------------------------------------------------------- FP8 low path (OSC: FP8 fallback for W2 inputs)
+def _finite_e4m3_codes():
+    c = np.arange(256, dtype=np.uint8)
+    return c[(c & 0x7F) != 0x7F]  # 0x7F / 0xFF are NaN in E4M3
+
+
+def test_e4m3_decode_matches_library():
+    """Every finite E4M3 code decodes to the value torch's float8_e4m3fn gives it."""
+    c = _finite_e4m3_codes()
+    ref = torch.from_numpy(c.copy()).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(oracle.e4m3_decode(c), ref)
+    assert oracle.e4m3_decode(np.array([0x7E], np.uint8))[0] == 448.0
+    assert oracle.e4m3_decode(np.array([0x01], np.uint8))[0] == 2.0 ** -9
+
+
+def test_e4m3_encode_matches_library():
+    """Nearest-even encoding of in-range values agrees with torch's conversion,
+    including every midpoint between neighbouring codes (the ties)."""
+    vals = oracle.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)
+    rng = np.random.default_rng(7)
+    rnd = np.concatenate([rng.standard_normal(50000) * 30, rng.standard_normal(20000) * 2.0 ** -7,
+                          rng.uniform(-448, 448, 20000)]).astype(np.float32)
+    t = np.concatenate([mids, -mids, vals.astype(np.float32), rnd])
+    t = t[np.abs(t) <= 448]
+    ref = torch.from_numpy(t.copy()).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode(t), ref)
+
+
+def test_e4m3_ties_saturation_and_signed_zero():
+    t = np.array([1.0625, 1.1875, 448.5, 1000.0, -1000.0, 2.0 ** -10, 3 * 2.0 ** -10, -2.0 ** -11, 0.0, -0.0],
+                 np.float32)
+    want = [0x38,  # tie between 1.0 (m=0) and 1.125 (m=1): even code
+            0x3A,  # tie between 1.125 and 1.25: 1.25 (m=2)
+            0x7E, 0x7E, 0xFE,  # saturation to +-448
+            0x00,  # tie between 0 and 2^-9: even code 0
+            0x02,  # tie between 2^-9 (code 1) and 2^-8 (code 2): code 2
+            0x80,  # negative value rounding to zero keeps its sign
+            0x00, 0x80]
+    assert list(oracle.e4m3_encode(t)) == want
+
+
+def _fp8_case(M=48, K=512, nO=24, seed=3):
+    O = workloads.outlier_channels(K, nO, seed=seed)
+    X = workloads.activations(M, K, O, seed=seed + 1)
+    return O.numpy(), workloads.bf16_bits(X)
+
+
+def test_fp8_quantizer_invariants():
+    O, Xb = _fp8_case()
+    K = Xb.shape[1]
+    q, s, xo = oracle.quantize_rows_fp8(Xb, K, O)
+    normal = np.setdiff1d(np.arange(K), O)
+    x = (Xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)[:, normal]
+    d = oracle.e4m3_decode(q).reshape(q.shape)
+    # the absolute-maximum element of each row lands on +-448 exactly
+    am = np.argmax(np.abs(x), axis=1)
+    assert np.all(np.abs(d[np.arange(len(am)), am]) == 448.0)
+    assert np.all(np.abs(d) <= 448.0)
+    # error of a 3-bit mantissa: half an ulp relative (normals), 2^-10 s absolute (subnormals)
+    err = np.abs(d * s[:, None].astype(np.float64) - x)
+    assert np.all(err <= 2.0 ** -4 * np.abs(x) * (1 + 2.0 ** -20) + 2.0 ** -10 * s[:, None] * (1 + 2.0 ** -20))
+    # outliers are exact bit copies
+    assert np.array_equal(xo, Xb[:, O])
+
+
+@pytest.mark.parametrize("e", [-20, -3, 5, 30])
+def test_fp8_power_of_two_scaling(e):
+    O, Xb = _fp8_case(seed=5)
+    K = Xb.shape[1]
+    x = (Xb.astype(np.uint32) << 16).view(np.float32) * np.float32(2.0 ** e)
+    Xe = (x.view(np.uint32) >> 16).astype(np.uint16)
+    q0, s0, _ = oracle.quantize_rows_fp8(Xb, K, O)
+    q1, s1, _ = oracle.quantize_rows_fp8(Xe, K, O)
+    assert np.array_equal(q0, q1)
+    assert np.array_equal(s1, (s0 * np.float32(2.0 ** e)).astype(np.float32))
+
+
+def test_fp8_sign_symmetry():
+    O, Xb = _fp8_case(seed=9)
+    K = Xb.shape[1]
+    q0, s0, _ = oracle.quantize_rows_fp8(Xb, K, O)
+    q1, s1, _ = oracle.quantize_rows_fp8(Xb ^ np.uint16(0x8000), K, O)
+    assert np.array_equal(s0, s1)
+    assert np.array_equal(q1, q0 ^ np.uint8(0x80))
+
+
+def test_fp8_products_exact_rational():
+    """acc_8 equals the exact rational sum of decoded products (small K: exact in fp64)."""
+    O, Xb = _fp8_case(M=6, K=256, nO=8, seed=11)
+    Wb = workloads.bf16_bits(workloads.weights(5, 256, seed=12))
+    ref = oracle.linear_fp8(Xb, Wb, O)
+    for m in range(6):
+        for n in range(5):
+            exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in
+                        zip(oracle.e4m3_decode(ref["qx"][m]), oracle.e4m3_decode(ref["qw"][n])))
+            assert Fraction(ref["acc_8"][m, n]) == exact
+
+
+def test_fp8_reductions():
+    """nO = 0: a plain FP8 GEMM (numpy matmul of the decoded codes); nO = K: a plain bf16 GEMM."""
+    M, K, N = 32, 384, 40
+    X = workloads.activations(M, K, workloads.outlier_channels(K, 0, seed=1), seed=2)
+    W = workloads.weights(N, K, seed=3)
+    Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
+    r0 = oracle.linear_fp8(Xb, Wb, np.zeros(0, np.int32))
+    dx = oracle.e4m3_decode(r0["qx"]).reshape(r0["qx"].shape)
+    dw = oracle.e4m3_decode(r0["qw"]).reshape(r0["qw"].shape)
+    y0 = (dx @ dw.T) * r0["sx"][:, None].astype(np.float64) * r0["sw"][None, :].astype(np.float64)
+    assert np.allclose(r0["y"], y0, rtol=1e-12, atol=1e-12)
+    rK = oracle.linear_fp8(Xb, Wb, np.arange(K, dtype=np.int32))
+    xf = (Xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    wf = (Wb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.allclose(rK["y"], xf @ wf.T, rtol=1e-12, atol=1e-12)
+    assert np.all(rK["sx"] == 0) and rK["qx"].shape == (M, 0)
+
+
+def test_fp8_path_tracks_the_exact_product():
+    """Method sanity (information): on a down-projection-like input (products of
+    two Gaussians, outlier channels x40) the FP8 low path with the outlier
+    branch stays within a few percent of the exact X W^T, closer than INT4."""
+    w = workloads.Workload("t", 64, 1024, 96, 128, x_kind="swiglu", sigma=40.0)
+    O, X, W = workloads.make(w)
+    Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
+    exact = (Xb.astype(np.uint32) << 16).view(np.float32).astype(np.float64) @ \
+        (Wb.astype(np.uint32) << 16).view(np.float32).astype(np.float64).T
+    e8 = np.linalg.norm(oracle.linear_fp8(Xb, Wb, O.numpy())["y"] - exact) / np.linalg.norm(exact)
+    e4 = np.linalg.norm(oracle.linear(Xb, Wb, O.numpy())["y"] - exact) / np.linalg.norm(exact)
+    assert e8 < 0.05 and e8 < e4
