@@ -43,7 +43,7 @@ import workloads  # noqa: E402
 
 DEFAULT_WORKLOAD = workloads.LLAMA8B_QKV.name
 METRIC = "dual-path W4A4+BF16 GEMM TOPS & % tensor peak; quant-gather HBM GB/s"
-INT8_PER_BF16 = 2.0   # nominal dense int8 : bf16 tensor rate on B200 (4.5 : 2.25 POPS)
+INT8_PER_BF16 = 2.0   # nominal dense int8 (and fp8) : bf16 tensor rate on B200 (4.5 : 2.25 POPS)
 
 
 # ----------------------------------------------------------------- helpers
@@ -78,14 +78,15 @@ def recorded_traffic(workload: str, kernel: str):
     return d.get("workloads", {}).get(workload, {}).get(kernel)
 
 
-def gemm_bytes(M, N, K, nO):
+def gemm_bytes(M, N, K, nO, cb=0.5):
+    """Algorithmic GEMM bytes; cb = bytes per low-path code (0.5 INT4, 1 E4M3)."""
     KN = K - nO
-    return N * KN / 2 + 2 * N * nO + 4 * N + M * KN / 2 + 2 * M * nO + 4 * M + 2 * M * N
+    return N * KN * cb + 2 * N * nO + 4 * N + M * KN * cb + 2 * M * nO + 4 * M + 2 * M * N
 
 
-def quant_gather_bytes(M, K, nO):
+def quant_gather_bytes(M, K, nO, cb=0.5):
     KN = K - nO
-    return 2 * M * K + M * KN / 2 + 2 * M * nO + 4 * M
+    return 2 * M * K + M * KN * cb + 2 * M * nO + 4 * M
 
 
 class ClockSampler:
@@ -170,18 +171,26 @@ def whole_job_tops(ops_per_rank_step: float, ms_per_step_max: float, world: int)
 
 
 # ----------------------------------------------------------------- CPU oracle timing
-def time_oracle(w, O, X, W, target_s: float, max_rows: int | None = None):
+def oracle_fns(fp8: bool):
+    import oracle
+    if fp8:
+        return oracle.quantize_rows_fp8, oracle.dual_linear_rows_fp8
+    return oracle.quantize_rows, oracle.dual_linear_rows
+
+
+def time_oracle(w, O, X, W, target_s: float, max_rows: int | None = None, fp8: bool = False):
     """Time the oracle on a bounded sample of token rows (weights quantized beforehand,
     as the offline step is on the GPU side).  Returns (TOPS, rows, seconds, cores)."""
     import oracle
+    quantize, dual = oracle_fns(fp8)
     Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
     O = O.numpy()
-    qw, sw, wo = oracle.quantize_rows(Wb, w.K, O)
+    qw, sw, wo = quantize(Wb, w.K, O)
 
     def run(rows):
         t0 = time.perf_counter()
-        qx, sx, xo = oracle.quantize_rows(Xb[:rows], w.K, O)
-        oracle.dual_linear_rows(qx, sx, xo, qw, sw, wo)
+        qx, sx, xo = quantize(Xb[:rows], w.K, O)
+        dual(qx, sx, xo, qw, sw, wo)
         return time.perf_counter() - t0
 
     probe = min(8, w.M)
@@ -197,14 +206,15 @@ def run_reference(args, w, rank, world):
         return 0
     O, X, W = workloads.make(w)
     import oracle
+    quantize, dual = oracle_fns(args.low == "fp8")
     Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
     On = O.numpy()
-    qw, sw, wo = oracle.quantize_rows(Wb, w.K, On)
+    qw, sw, wo = quantize(Wb, w.K, On)
     rows = args.ref_rows
 
     def step():
-        qx, sx, xo = oracle.quantize_rows(Xb[:rows], w.K, On)
-        oracle.dual_linear_rows(qx, sx, xo, qw, sw, wo)
+        qx, sx, xo = quantize(Xb[:rows], w.K, On)
+        dual(qx, sx, xo, qw, sw, wo)
 
     for _ in range(args.warmup):
         step()
@@ -216,8 +226,8 @@ def run_reference(args, w, rank, world):
     sample = f"{rows} token rows of the workload per step (weights quantized before timing)"
     line = {"impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64", "data": "synthetic",
-            "config": w.describe(),
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64" if args.low == "fp8" else "int64+f64",
+            "data": "synthetic", "config": {**w.describe(), "low_path": args.low},
             "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -236,6 +246,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=8, help="token rows per reference-arm step")
+    ap.add_argument("--low", default="int4", choices=["int4", "fp8"],
+                    help="low path: INT4 (default) or FP8 E4M3 (the pages' fallback for the inputs of W2)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -267,29 +279,34 @@ def main():
     kn_pad, no_pad = sq.sq_kn_pad(K, nO), sq.sq_no_pad(nO)
 
     # Rotating input sets so that every step reads operands that are not L2-resident.
+    fp8 = args.low == "fp8"
+    cb = 1.0 if fp8 else 0.5  # bytes per low-path code
+    ws_bytes = sq.sq_linear_workspace_bytes_fp8 if fp8 else sq.sq_linear_workspace_bytes
+    quant_gather_fn = sq.sq_quant_gather_fp8 if fp8 else sq.sq_quant_gather
+    gemm_fn = sq.sq_gemm_fp8 if fp8 else sq.sq_gemm
+    linear_fn = sq.sq_linear_fp8 if fp8 else sq.sq_linear
     Xd = X.to(dev)
-    pw0 = sq.prepare_weights(W.to(dev), O)
-    foot = (2 * M * K + pw0.W_N.numel() + 2 * pw0.W_O.numel() + 4 * N + 2 * M * N
-            + sq.sq_linear_workspace_bytes(M, K, nO))
+    pw0 = sq.prepare_weights(W.to(dev), O, fp8=fp8)
+    foot = (2 * M * K + pw0.W_N.numel() + 2 * pw0.W_O.numel() + 4 * N + 2 * M * N + ws_bytes(M, K, nO))
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     n_sets = max(2, math.ceil(3 * l2 / foot))
     sets = []
     for i in range(n_sets):
         pw = pw0 if i == 0 else sq.PreparedWeights(N, K, nO, pw0.W_N.clone(), pw0.s_w.clone(), pw0.W_O.clone(),
-                                                      pw0.chan_tab.clone())
+                                                      pw0.chan_tab.clone(), fp8)
         sets.append({
             "X": Xd if i == 0 else Xd.clone(), "pw": pw,
-            "X_N": torch.empty(M, kn_pad // 2, dtype=torch.uint8, device=dev),
+            "X_N": torch.empty(M, pw0.code_bytes(K), dtype=torch.uint8, device=dev),
             "s_x": torch.empty(M, dtype=torch.float32, device=dev),
             "X_O": torch.empty(M, no_pad, dtype=torch.bfloat16, device=dev),
             "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
         })
     def quant(s, stream):
-        sq.sq_quant_gather(s["X"], s["pw"].chan_tab, nO, s["X_N"], s["s_x"], s["X_O"], stream)
+        quant_gather_fn(s["X"], s["pw"].chan_tab, nO, s["X_N"], s["s_x"], s["X_O"], stream)
 
     def gemm(s, stream):
         pw = s["pw"]
-        sq.sq_gemm(s["X_N"], s["s_x"], s["X_O"], pw.W_N, pw.s_w, pw.W_O, M, N, K, nO, s["Y"], None, None, stream)
+        gemm_fn(s["X_N"], s["s_x"], s["X_O"], pw.W_N, pw.s_w, pw.W_O, M, N, K, nO, s["Y"], None, None, stream)
 
     def step(s, stream):
         quant(s, stream)
@@ -356,7 +373,7 @@ def main():
     t_roof_s = (2.0 * M * N * (K - nO)) / (p_i8 * 1e12) + (2.0 * M * N * nO) / (p_bf * 1e12)
     peak_eff = flops / t_roof_s / 1e12
     gemm_tops = flops / (ms_gemm * 1e-3) / 1e12
-    g_bytes = gemm_bytes(M, N, K, nO)
+    g_bytes = gemm_bytes(M, N, K, nO, cb)
     t_hbm_s = g_bytes / (peaks["hbm_gbs"] * 1e9)
     if t_hbm_s > t_roof_s:
         # few tokens: the GEMM is bound by streaming the weights, not by the tensor cores
@@ -366,21 +383,22 @@ def main():
     else:
         gemm_roof = {"bound": "tensor", "achieved": gemm_tops, "peak": peak_eff, "unit": "TFLOP/s",
                      "frac": gemm_tops / peak_eff,
-                     "peak_basis": f"{peaks['source']} bf16 {p_bf:.0f} TFLOP/s (burst), int8 = {INT8_PER_BF16:g}x"}
-    qg_bytes = quant_gather_bytes(M, K, nO)
+                     "peak_basis": f"{peaks['source']} bf16 {p_bf:.0f} TFLOP/s (burst), "
+                                   f"{'fp8' if fp8 else 'int8'} = {INT8_PER_BF16:g}x"}
+    qg_bytes = quant_gather_bytes(M, K, nO, cb)
     qg_gbs = qg_bytes / (ms_qg * 1e-3) / 1e9
 
     # end to end through sq_linear with pinned host buffers (copies inside the timed region)
     X_host = X.pin_memory()
     Y_host = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
     e2e_sets = sets[:2]
-    ws = [torch.empty(sq.sq_linear_workspace_bytes(M, K, nO), dtype=torch.uint8, device=dev) for _ in e2e_sets]
+    ws = [torch.empty(ws_bytes(M, K, nO), dtype=torch.uint8, device=dev) for _ in e2e_sets]
 
     def e2e_step(i):
         s = e2e_sets[i % len(e2e_sets)]
         s["X"].copy_(X_host, non_blocking=True)
         pw = s["pw"]
-        sq.sq_linear(s["X"], pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, N, nO, s["Y"], ws[i % len(ws)], stream)
+        linear_fn(s["X"], pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, N, nO, s["Y"], ws[i % len(ws)], stream)
         Y_host.copy_(s["Y"], non_blocking=True)
 
     for i in range(args.warmup):
@@ -400,7 +418,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tops, rows, secs, cores = time_oracle(w, O, X, W, args.cpu_seconds)
+        tops, rows, secs, cores = time_oracle(w, O, X, W, args.cpu_seconds, fp8=fp8)
         cpu = {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle",
                "sample": f"{rows} of {M} token rows x all {N} outputs ({secs:.1f} s; weights quantized beforehand)"}
 
@@ -408,8 +426,10 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "s4*s4->s32 + bf16*bf16->f32", "data": "synthetic",
-            "config": {**w.describe(), "parallelism": f"dp{world}" if world > 1 else "single",
+            "vs_baseline": None,
+            "dtype": "e4m3*e4m3->f32 + bf16*bf16->f32" if fp8 else "s4*s4->s32 + bf16*bf16->f32",
+            "data": "synthetic",
+            "config": {**w.describe(), "low_path": args.low, "parallelism": f"dp{world}" if world > 1 else "single",
                        "l2": f"{n_sets} rotating input sets of {foot / 1e6:.0f} MB (> L2 {l2 / 1e6:.0f} MB)",
                        "timing": "K steps replayed from one CUDA graph; per-kernel times from graphs of K launches"},
             "roofline": {**gemm_roof, "traffic": recorded_traffic(w.name, "dual_gemm"),

@@ -181,6 +181,55 @@ sq_status sq_linear_noalloc(const void *X, int64_t M, int64_t K, int64_t ldx,
                             int64_t N, int64_t nO, void *Y, int64_t ldy,
                             sq_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * FP8 low path.
+ *
+ * OSC (arXiv:2604.12782), abstract and "technical framework": for the inputs
+ * of W2 (the down projection), where outlier clustering is less pronounced,
+ * the 4-bit path falls back to FP8.  These calls are the four above with the
+ * normal (non-outlier) channels in FP8 E4M3 instead of INT4:
+ *
+ *   Y[m,n] = s_x[m] * s_w[n] * sum_{k not in O} e(X)[m,k] * e(W)[n,k]
+ *          +                   sum_{k in O}     X[m,k]   * W[n,k]
+ *
+ *   - s = a / 448 (fp32, IEEE), a = absolute maximum over the normal
+ *     channels of the row; a == 0 gives s = 0 and all-zero codes.
+ *   - e(x) = the E4M3 code nearest to the fp32 quotient x / s, ties to the
+ *     even code, magnitudes above 448 saturated to 448, the sign kept (a
+ *     negative value that rounds to zero gives -0, byte 0x80).
+ *   - Layout: W_N8 / X_N8 are u8 [rows, sq_kn_pad(K, nO)], one E4M3 byte per
+ *     normal channel in ascending channel order, zero bytes past K - nO.
+ *     s_w, s_x, W_O, X_O and the channel table are as for INT4.
+ *   - The products run on the tensor cores as E4M3 x E4M3 with fp32
+ *     accumulation (tcgen05 kind::f8f6f4); the epilogue is
+ *     Y = bf16_rn(((float)acc_8 * s_x) * s_w + acc_f).
+ *   - Supported for K <= 16384 (SQ_ERR_UNSUPPORTED above).
+ *   - dbg_acc_8 (nullable, [M, N] fp32): the low-path accumulator.
+ * Error behaviour, ownership and stream ordering are those of the INT4 calls.
+ * ------------------------------------------------------------------------ */
+size_t sq_linear_workspace_bytes_fp8(int64_t M, int64_t K, int64_t nO);
+
+sq_status sq_prepare_weights_fp8(const void *W, int64_t N, int64_t K, int64_t ldw,
+                                 const int32_t *O, int64_t nO,
+                                 void *W_N8, float *s_w, void *W_O, uint32_t *chan_tab,
+                                 sq_stream_t stream);
+
+sq_status sq_quant_gather_fp8(const void *X, int64_t M, int64_t K, int64_t ldx,
+                              const uint32_t *chan_tab, int64_t nO,
+                              void *X_N8, float *s_x, void *X_O, sq_stream_t stream);
+
+sq_status sq_gemm_fp8(const void *X_N8, const float *s_x, const void *X_O,
+                      const void *W_N8, const float *s_w, const void *W_O,
+                      int64_t M, int64_t N, int64_t K, int64_t nO,
+                      void *Y, int64_t ldy,
+                      float *dbg_acc_8, float *dbg_acc_f32, sq_stream_t stream);
+
+sq_status sq_linear_fp8(const void *X, int64_t M, int64_t K, int64_t ldx,
+                        const uint32_t *chan_tab,
+                        const void *W_N8, const float *s_w, const void *W_O,
+                        int64_t N, int64_t nO, void *Y, int64_t ldy,
+                        void *workspace, size_t ws_bytes, sq_stream_t stream);
+
 /*
  * Waits for `stream`, then reports (and clears) the device error word of the
  * current device: SQ_ERR_TIMEOUT if a kernel's bounded wait ran out,

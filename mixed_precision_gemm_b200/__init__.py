@@ -34,7 +34,8 @@ __all__ = [
     "SQError", "load", "library_path", "header_functions",
     "sq_status_string", "sq_kn_pad", "sq_no_pad", "sq_chan_table_words", "sq_linear_workspace_bytes",
     "sq_prepare_weights", "sq_quant_gather", "sq_gemm", "sq_linear", "sq_linear_noalloc", "sq_check",
-    "sq_selftest_watchdog",
+    "sq_selftest_watchdog", "sq_linear_workspace_bytes_fp8", "sq_prepare_weights_fp8", "sq_quant_gather_fp8",
+    "sq_gemm_fp8", "sq_linear_fp8",
     "PreparedWeights", "prepare_weights", "quant_gather", "gemm", "SQLinear",
 ]
 
@@ -95,8 +96,15 @@ def load():
     lib.sq_linear_noalloc.argtypes = [P, I, I, I, P, P, P, P, I, I, P, I, P]
     lib.sq_check.argtypes = [P]
     lib.sq_selftest_watchdog.argtypes = [F, P]
+    lib.sq_linear_workspace_bytes_fp8.argtypes = [I, I, I]
+    lib.sq_linear_workspace_bytes_fp8.restype = Z
+    lib.sq_prepare_weights_fp8.argtypes = [P, I, I, I, P, I, P, P, P, P, P]
+    lib.sq_quant_gather_fp8.argtypes = [P, I, I, I, P, I, P, P, P, P]
+    lib.sq_gemm_fp8.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P, P, P]
+    lib.sq_linear_fp8.argtypes = [P, I, I, I, P, P, P, P, I, I, P, I, P, Z, P]
     for f in (lib.sq_prepare_weights, lib.sq_quant_gather, lib.sq_gemm, lib.sq_linear, lib.sq_check,
-              lib.sq_selftest_watchdog, lib.sq_linear_noalloc):
+              lib.sq_selftest_watchdog, lib.sq_linear_noalloc, lib.sq_prepare_weights_fp8, lib.sq_quant_gather_fp8,
+              lib.sq_gemm_fp8, lib.sq_linear_fp8):
         f.restype = F
     _lib = lib
     return lib
@@ -220,6 +228,53 @@ def sq_linear_noalloc(X: torch.Tensor, chan_tab: torch.Tensor, W_N, s_w, W_O, N:
     _raise(st, "sq_linear_noalloc")
 
 
+# FP8 low path (OSC: FP8 fallback for the inputs of W2): the same calls with
+# one E4M3 byte per normal channel (u8 [rows, kn_pad]) instead of packed INT4.
+def sq_linear_workspace_bytes_fp8(M: int, K: int, nO: int) -> int:
+    return int(load().sq_linear_workspace_bytes_fp8(M, K, nO))
+
+
+def sq_prepare_weights_fp8(W: torch.Tensor, O, W_N8: torch.Tensor, s_w: torch.Tensor, W_O: Optional[torch.Tensor],
+                           chan_tab: torch.Tensor, stream=None) -> None:
+    _rowmajor(W, "W", torch.bfloat16)
+    N, K = W.shape
+    O_host = torch.as_tensor(O, dtype=torch.int32).reshape(-1).contiguous().cpu()
+    nO = O_host.numel()
+    st = load().sq_prepare_weights_fp8(_ptr(W), N, K, W.stride(0),
+                                       ctypes.c_void_p(O_host.data_ptr()) if nO else None, nO,
+                                       _ptr(W_N8), _ptr(s_w), _ptr(W_O), _ptr(chan_tab), _stream(stream))
+    _raise(st, "sq_prepare_weights_fp8")
+
+
+def sq_quant_gather_fp8(X: torch.Tensor, chan_tab: torch.Tensor, nO: int, X_N8: Optional[torch.Tensor],
+                        s_x: torch.Tensor, X_O: Optional[torch.Tensor], stream=None) -> None:
+    _rowmajor(X, "X", torch.bfloat16)
+    M, K = X.shape
+    st = load().sq_quant_gather_fp8(_ptr(X), M, K, X.stride(0), _ptr(chan_tab), nO, _ptr(X_N8), _ptr(s_x),
+                                    _ptr(X_O), _stream(stream))
+    _raise(st, "sq_quant_gather_fp8")
+
+
+def sq_gemm_fp8(X_N8, s_x, X_O, W_N8, s_w, W_O, M: int, N: int, K: int, nO: int, Y: torch.Tensor,
+                dbg_acc_8: Optional[torch.Tensor] = None, dbg_acc_f32: Optional[torch.Tensor] = None,
+                stream=None) -> None:
+    _rowmajor(Y, "Y", torch.bfloat16)
+    st = load().sq_gemm_fp8(_ptr(X_N8), _ptr(s_x), _ptr(X_O), _ptr(W_N8), _ptr(s_w), _ptr(W_O), M, N, K, nO,
+                            _ptr(Y), Y.stride(0), _ptr(dbg_acc_8), _ptr(dbg_acc_f32), _stream(stream))
+    _raise(st, "sq_gemm_fp8")
+
+
+def sq_linear_fp8(X: torch.Tensor, chan_tab: torch.Tensor, W_N8, s_w, W_O, N: int, nO: int, Y: torch.Tensor,
+                  workspace: torch.Tensor, stream=None) -> None:
+    _rowmajor(X, "X", torch.bfloat16)
+    _rowmajor(Y, "Y", torch.bfloat16)
+    M, K = X.shape
+    st = load().sq_linear_fp8(_ptr(X), M, K, X.stride(0), _ptr(chan_tab), _ptr(W_N8), _ptr(s_w), _ptr(W_O), N, nO,
+                              _ptr(Y), Y.stride(0), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(stream))
+    _raise(st, "sq_linear_fp8")
+
+
 def sq_check(stream=None) -> None:
     _raise(load().sq_check(_stream(stream)), "sq_check")
 
@@ -235,65 +290,78 @@ class PreparedWeights:
     N: int
     K: int
     nO: int
-    W_N: torch.Tensor        # uint8 [N, kn_pad/2]
+    W_N: torch.Tensor        # uint8 [N, kn_pad/2] packed INT4, or [N, kn_pad] E4M3 when fp8
     s_w: torch.Tensor        # float32 [N]
     W_O: torch.Tensor        # bf16 [N, no_pad]
     chan_tab: torch.Tensor   # int32 view of uint32 [K/8]
+    fp8: bool = False        # low path in FP8 E4M3 (the W2 fallback) instead of INT4
 
     def state_dict(self) -> dict:
         return {"N": self.N, "K": self.K, "nO": self.nO, "W_N": self.W_N, "s_w": self.s_w,
-                "W_O": self.W_O, "chan_tab": self.chan_tab}
+                "W_O": self.W_O, "chan_tab": self.chan_tab, "fp8": self.fp8}
 
     @classmethod
     def from_state_dict(cls, d: dict, device=None) -> "PreparedWeights":
         mv = (lambda t: t.to(device)) if device is not None else (lambda t: t)
         return cls(int(d["N"]), int(d["K"]), int(d["nO"]), mv(d["W_N"]), mv(d["s_w"]), mv(d["W_O"]),
-                   mv(d["chan_tab"]))
+                   mv(d["chan_tab"]), bool(d.get("fp8", False)))
+
+    def code_bytes(self, K: int) -> int:
+        kn = sq_kn_pad(K, self.nO)
+        return kn if self.fp8 else kn // 2
 
 
-def prepare_weights(W: torch.Tensor, O: Sequence[int], stream=None) -> PreparedWeights:
+def prepare_weights(W: torch.Tensor, O: Sequence[int], stream=None, fp8: bool = False) -> PreparedWeights:
+    """Offline weight step; fp8=True prepares the FP8 (E4M3) low path instead of INT4."""
     N, K = W.shape
     nO = len(torch.as_tensor(O).reshape(-1))
     dev = W.device
-    W_N = torch.zeros(N, sq_kn_pad(K, nO) // 2, dtype=torch.uint8, device=dev)
+    kn = sq_kn_pad(K, nO)
+    W_N = torch.zeros(N, kn if fp8 else kn // 2, dtype=torch.uint8, device=dev)
     s_w = torch.zeros(N, dtype=torch.float32, device=dev)
     W_O = torch.zeros(N, sq_no_pad(nO), dtype=torch.bfloat16, device=dev)
     tab = torch.zeros(sq_chan_table_words(K), dtype=torch.int32, device=dev)
-    sq_prepare_weights(W, O, W_N, s_w, W_O, tab, stream)
-    return PreparedWeights(N, K, nO, W_N, s_w, W_O, tab)
+    (sq_prepare_weights_fp8 if fp8 else sq_prepare_weights)(W, O, W_N, s_w, W_O, tab, stream)
+    return PreparedWeights(N, K, nO, W_N, s_w, W_O, tab, fp8)
 
 
 def quant_gather(X: torch.Tensor, pw: PreparedWeights, stream=None):
     M, K = X.shape
     dev = X.device
-    X_N = torch.empty(M, sq_kn_pad(K, pw.nO) // 2, dtype=torch.uint8, device=dev)
+    X_N = torch.empty(M, pw.code_bytes(K), dtype=torch.uint8, device=dev)
     s_x = torch.empty(M, dtype=torch.float32, device=dev)
     X_O = torch.empty(M, sq_no_pad(pw.nO), dtype=torch.bfloat16, device=dev)
-    sq_quant_gather(X, pw.chan_tab, pw.nO, X_N, s_x, X_O, stream)
+    (sq_quant_gather_fp8 if pw.fp8 else sq_quant_gather)(X, pw.chan_tab, pw.nO, X_N, s_x, X_O, stream)
     return X_N, s_x, X_O
 
 
 def gemm(X_N, s_x, X_O, pw: PreparedWeights, Y: Optional[torch.Tensor] = None, debug: bool = False, stream=None):
+    """Dual GEMM.  With debug=True also returns the two accumulators: the low
+    path's (int32 for INT4, fp32 for FP8) and the bf16 branch's (fp32)."""
     M = s_x.shape[0]
     if Y is None:
         Y = torch.empty(M, pw.N, dtype=torch.bfloat16, device=s_x.device)
     dbg_i = dbg_f = None
     if debug:
-        dbg_i = torch.empty(M, pw.N, dtype=torch.int32, device=s_x.device)
+        dbg_i = torch.empty(M, pw.N, dtype=torch.float32 if pw.fp8 else torch.int32, device=s_x.device)
         dbg_f = torch.empty(M, pw.N, dtype=torch.float32, device=s_x.device)
-    sq_gemm(X_N, s_x, X_O, pw.W_N, pw.s_w, pw.W_O, M, pw.N, pw.K, pw.nO, Y, dbg_i, dbg_f, stream)
+    (sq_gemm_fp8 if pw.fp8 else sq_gemm)(X_N, s_x, X_O, pw.W_N, pw.s_w, pw.W_O, M, pw.N, pw.K, pw.nO, Y, dbg_i, dbg_f,
+                                         stream)
     return (Y, dbg_i, dbg_f) if debug else Y
 
 
 class SQLinear:
-    """A prepared dual-path linear layer: ``y = layer(x)`` for bf16 x [M, K] on the GPU."""
+    """A prepared dual-path linear layer: ``y = layer(x)`` for bf16 x [M, K] on the GPU.
 
-    def __init__(self, W: torch.Tensor, O: Sequence[int], stream=None):
-        self.weights = prepare_weights(W, O, stream)
+    fp8=True runs the low path in FP8 E4M3 (OSC's fallback for the inputs of W2)."""
+
+    def __init__(self, W: torch.Tensor, O: Sequence[int], stream=None, fp8: bool = False):
+        self.weights = prepare_weights(W, O, stream, fp8)
         self._ws = None
 
     def workspace(self, M: int, device) -> torch.Tensor:
-        need = sq_linear_workspace_bytes(M, self.weights.K, self.weights.nO)
+        ws_fn = sq_linear_workspace_bytes_fp8 if self.weights.fp8 else sq_linear_workspace_bytes
+        need = ws_fn(M, self.weights.K, self.weights.nO)
         if self._ws is None or self._ws.numel() < need or self._ws.device != torch.device(device):
             self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
         return self._ws
@@ -303,5 +371,6 @@ class SQLinear:
         M = X.shape[0]
         if out is None:
             out = torch.empty(M, pw.N, dtype=torch.bfloat16, device=X.device)
-        sq_linear(X, pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, pw.N, pw.nO, out, self.workspace(M, X.device), stream)
+        (sq_linear_fp8 if pw.fp8 else sq_linear)(X, pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, pw.N, pw.nO, out,
+                                                 self.workspace(M, X.device), stream)
         return out

@@ -10,6 +10,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>
+#include <type_traits>
 #include <string>
 #include <vector>
 
@@ -238,18 +239,18 @@ sq_status launch_rowquant_g(const DevInfo &di, const uint16_t *src, int64_t rows
 
 // Rows streamed through shared memory (K <= 16384): as many consumer groups
 // of G warps as the shared memory holds (two row slots each), one CTA per SM.
-template <int G>
+template <int G, bool FP8>
 sq_status launch_rowquant_stream(const DevInfo &di, const uint16_t *src, int64_t rows, int K, int64_t ld,
                                  const uint32_t *tab, int nO, int kn_pad, int no_pad, uint8_t *dn, float *ds,
                                  uint16_t *dout, cudaStream_t stream)
 {
     constexpr int kSmemLimit = 232448 - 1024;
     int ngrp = sqq::stream_max_groups(G);
-    while (ngrp > 1 && sqq::StreamLayout(K, kn_pad, no_pad, ngrp).bytes > kSmemLimit) --ngrp;
-    const size_t smem = static_cast<size_t>(sqq::StreamLayout(K, kn_pad, no_pad, ngrp).bytes);
+    while (ngrp > 1 && sqq::StreamLayout(K, kn_pad, no_pad, ngrp, FP8).bytes > kSmemLimit) --ngrp;
+    const size_t smem = static_cast<size_t>(sqq::StreamLayout(K, kn_pad, no_pad, ngrp, FP8).bytes);
     if (smem > static_cast<size_t>(kSmemLimit))
         return fail(SQ_ERR_UNSUPPORTED, "quantize-gather: K=%d, nO=%d do not fit in shared memory", K, nO);
-    auto kern = sqq::rowquant_stream_kernel<G>;
+    auto kern = sqq::rowquant_stream_kernel<G, FP8>;
     const int threads = 32 * (1 + ngrp * G);
     int per_sm = 0;
     sq_status st = kernel_setup(reinterpret_cast<const void *>(kern), threads, smem, per_sm, "rowquant stream set-up");
@@ -261,8 +262,22 @@ sq_status launch_rowquant_stream(const DevInfo &di, const uint16_t *src, int64_t
     return SQ_OK;
 }
 
+template <bool FP8>
+sq_status launch_rowquant_streamed(const DevInfo &di, const uint16_t *src, int64_t rows, int k, int64_t ld,
+                                   const uint32_t *tab, int no, int kn_pad, int no_pad, uint8_t *dn, float *ds,
+                                   uint16_t *dout, cudaStream_t stream)
+{
+    // up to 2048 channels per warp (8 chunks of 8 per thread); narrow rows
+    // take more warps per row, so that each SM runs more warps
+    if (k <= 1024) return launch_rowquant_stream<1, FP8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (k <= 2048) return launch_rowquant_stream<2, FP8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (k <= 8192) return launch_rowquant_stream<4, FP8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    return launch_rowquant_stream<8, FP8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+}
+
+// fp8: E4M3 codes (the FP8 low path) instead of packed INT4 codes.
 sq_status launch_rowquant(const uint16_t *src, int64_t rows, int64_t K, int64_t ld, const uint32_t *tab,
-                          int64_t nO, uint8_t *dn, float *ds, uint16_t *dout, cudaStream_t stream)
+                          int64_t nO, uint8_t *dn, float *ds, uint16_t *dout, cudaStream_t stream, bool fp8 = false)
 {
     if (rows == 0) return SQ_OK;
     DevInfo di;
@@ -271,21 +286,15 @@ sq_status launch_rowquant(const uint16_t *src, int64_t rows, int64_t K, int64_t 
     const int kn_pad = static_cast<int>(sq_kn_pad(K, nO));
     const int no_pad = static_cast<int>(sq_no_pad(nO));
     const int k = static_cast<int>(K), no = static_cast<int>(nO);
-    if (K <= sqq::kStreamMaxK) {
-        // up to 2048 channels per warp (8 chunks of 8 per thread); narrow rows
-        // take more warps per row, so that each SM runs more warps
-        if (K <= 1024) return launch_rowquant_stream<1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-        if (K <= 2048) return launch_rowquant_stream<2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-        if (K <= 8192) return launch_rowquant_stream<4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-        return launch_rowquant_stream<8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (fp8) {
+        if (K > sqq::kStreamMaxK)
+            return fail(SQ_ERR_UNSUPPORTED, "the FP8 low path supports K <= %d (K=%lld)", sqq::kStreamMaxK, (long long)K);
+        return launch_rowquant_streamed<true>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
     }
-    // One warp per row up to 2048 channels (8 chunks of 8 per thread), then
-    // as many warps as keep a thread at 8 chunks or fewer.
-    const int64_t per_warp = 32 * sqq::kChunksPerThread * 8;
-    if (K <= per_warp) return launch_rowquant_g<1>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (K <= 2 * per_warp) return launch_rowquant_g<2>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (K <= 4 * per_warp) return launch_rowquant_g<4>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
-    if (K <= 8 * per_warp) return launch_rowquant_g<8>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    if (K <= sqq::kStreamMaxK)
+        return launch_rowquant_streamed<false>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
+    // Wider rows stay in registers: a group of 16 warps per row, 8 or 16
+    // chunks of 8 channels per thread.
     return launch_rowquant_g<16>(di, src, rows, k, ld, tab, no, kn_pad, no_pad, dn, ds, dout, stream);
 }
 
@@ -304,7 +313,10 @@ int raster_group(int tiles_m, int tile_rows, int64_t kn_pad, int64_t no_pad)
 }
 
 // Pair (cta_group::2) kernel: 256 x 256 tiles over clusters of two CTAs.
-template <class C>
+// FP8: E4M3 low path (kn_pad bytes per row, tiles loaded straight into the
+// operand ring with the 128-byte swizzle); otherwise packed INT4 (kn_pad / 2
+// bytes per row, 64-byte staging boxes).
+template <class C, bool FP8>
 sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O, const void *W_N,
                              const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y,
                              int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
@@ -313,12 +325,11 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
     CUtensorMap m_xo{}, m_wo{}, m_xn{}, m_wn{};
     sq_status st;
     if (kn_pad > 0) {
-        if ((st = make_map(m_xn, X_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, M, kn_pad / 2, sqg::PROWB, 128,
-                           CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
-            return st;
-        if ((st = make_map(m_wn, W_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, N, kn_pad / 2, sqg::PROWB, 128,
-                           CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
-            return st;
+        const int64_t rb = FP8 ? kn_pad : kn_pad / 2;
+        const uint32_t box = FP8 ? sqg::KB_I8 : sqg::PROWB;
+        const CUtensorMapSwizzle swz = FP8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+        if ((st = make_map(m_xn, X_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, rb, M, rb, box, 128, swz)) != SQ_OK) return st;
+        if ((st = make_map(m_wn, W_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, rb, N, rb, box, 128, swz)) != SQ_OK) return st;
     }
     if (no_pad > 0) {
         if ((st = make_map(m_xo, X_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, M, no_pad * 2, sqg::KB_BF, 128,
@@ -345,7 +356,7 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
     const int64_t ntiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
     const int64_t clusters = std::min<int64_t>(ntiles, di.sms / 2);
     const bool dbg = dbg_i || dbg_f;
-    auto kern = dbg ? sqg::dual_gemm_pair_kernel<C, true> : sqg::dual_gemm_pair_kernel<C, false>;
+    auto kern = dbg ? sqg::dual_gemm_pair_kernel<C, true, FP8> : sqg::dual_gemm_pair_kernel<C, false, FP8>;
     int per_sm = 0;
     if ((st = kernel_setup(reinterpret_cast<const void *>(kern), sqg::PAIR_THREADS, C::SMEM_BYTES, per_sm, "gemm pair set-up")) != SQ_OK)
         return st;
@@ -358,7 +369,7 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
 
 // Swapped-operand split-K kernel for M <= 128: tiles of 128 W rows x MP
 // tokens; the K-blocks of each tile are spread over a cluster of S CTAs.
-template <class C>
+template <class C, bool FP8>
 sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O,
                                const void *W_N, const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K,
                                int64_t nO, void *Y, int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
@@ -367,11 +378,12 @@ sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *
     CUtensorMap m_xo{}, m_wo{}, m_xn{}, m_wn{};
     sq_status st;
     if (kn_pad > 0) {
-        // 128-byte boxes (two INT4 K-blocks) with the 128-byte swizzle.
-        if ((st = make_map(m_xn, X_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, M, kn_pad / 2, 2 * sqg::PROWB, C::MP,
+        // 128-byte boxes (two INT4 K-blocks, or one E4M3 K-block) with the 128-byte swizzle.
+        const int64_t rb = FP8 ? kn_pad : kn_pad / 2;
+        if ((st = make_map(m_xn, X_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, rb, M, rb, 128, C::MP,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
             return st;
-        if ((st = make_map(m_wn, W_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, kn_pad / 2, N, kn_pad / 2, 2 * sqg::PROWB, 128,
+        if ((st = make_map(m_wn, W_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, rb, N, rb, 128, 128,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
             return st;
     }
@@ -405,7 +417,7 @@ sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *
     S = std::max<int64_t>(S, 1);
     a.splits = static_cast<int>(S);
     const bool dbg = dbg_i || dbg_f;
-    auto kern = dbg ? sqg::dual_gemm_skinny_kernel<C, true> : sqg::dual_gemm_skinny_kernel<C, false>;
+    auto kern = dbg ? sqg::dual_gemm_skinny_kernel<C, true, FP8> : sqg::dual_gemm_skinny_kernel<C, false, FP8>;
     int per_sm = 0;
     if ((st = kernel_setup(reinterpret_cast<const void *>(kern), sqg::SK_THREADS, C::SMEM_BYTES, per_sm, "gemm skinny set-up")) != SQ_OK)
         return st;
@@ -417,29 +429,40 @@ sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *
 }
 
 using CfgPair = sqg::CfgPair<4, 4, 2>;
+using CfgPairF8 = sqg::CfgPair<6, 0, 2>;  // E4M3 tiles need no staging ring: a deeper operand ring instead
 using CfgSk16 = sqg::CfgSkinny<16, 8, 3>;
 using CfgSk32 = sqg::CfgSkinny<32, 7, 3>;
 using CfgSk64 = sqg::CfgSkinny<64, 6, 2>;
 using CfgSk128 = sqg::CfgSkinny<128, 4, 2>;
 
 
+template <bool FP8>
+sq_status gemm_dispatch(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O, const void *W_N,
+                        const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y,
+                        int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+{
+    using Pair = typename std::conditional<FP8, CfgPairF8, CfgPair>::type;
+    if (M > 128)
+        return launch_gemm_pair_t<Pair, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    if (M <= 16)
+        return launch_gemm_skinny_t<CfgSk16, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    if (M <= 32)
+        return launch_gemm_skinny_t<CfgSk32, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    if (M <= 64)
+        return launch_gemm_skinny_t<CfgSk64, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    return launch_gemm_skinny_t<CfgSk128, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+}
+
 sq_status gemm_impl(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
                     const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
-                    int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+                    int32_t *dbg_i, float *dbg_f, cudaStream_t stream, bool fp8)
 {
     if (M == 0 || N == 0) return SQ_OK;
     DevInfo di;
     sq_status st = device_info(di);
     if (st != SQ_OK) return st;
-    if (M > 128)
-        return launch_gemm_pair_t<CfgPair>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
-    if (M <= 16)
-        return launch_gemm_skinny_t<CfgSk16>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
-    if (M <= 32)
-        return launch_gemm_skinny_t<CfgSk32>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
-    if (M <= 64)
-        return launch_gemm_skinny_t<CfgSk64>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
-    return launch_gemm_skinny_t<CfgSk128>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    return fp8 ? gemm_dispatch<true>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream)
+               : gemm_dispatch<false>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
 }
 
 // ---------------------------------------------------------------- validation
@@ -466,7 +489,7 @@ sq_status check_ptr(const void *p, bool needed, const char *name)
     } while (0)
 
 sq_status quant_gather_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, int64_t nO,
-                            void *X_N, float *s_x, void *X_O, cudaStream_t stream)
+                            void *X_N, float *s_x, void *X_O, cudaStream_t stream, bool fp8 = false)
 {
     SQ_TRY(check_K_nO(K, nO));
     if (M < 0) return fail(SQ_ERR_INVALID_ARG, "M < 0");
@@ -479,13 +502,15 @@ sq_status quant_gather_impl(const void *X, int64_t M, int64_t K, int64_t ldx, co
     SQ_TRY(check_ptr(s_x, true, "s_x"));
     SQ_TRY(check_ptr(X_O, nO > 0, "X_O"));
     return launch_rowquant(static_cast<const uint16_t *>(X), M, K, ldx, chan_tab, nO, static_cast<uint8_t *>(X_N), s_x,
-                           static_cast<uint16_t *>(X_O), stream);
+                           static_cast<uint16_t *>(X_O), stream, fp8);
 }
 
 sq_status gemm_checked(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
                        const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
-                       int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+                       int32_t *dbg_i, float *dbg_f, cudaStream_t stream, bool fp8 = false)
 {
+    if (fp8 && K > sqq::kStreamMaxK)
+        return fail(SQ_ERR_UNSUPPORTED, "the FP8 low path supports K <= %d (K=%lld)", sqq::kStreamMaxK, (long long)K);
     SQ_TRY(check_K_nO(K, nO));
     if (M < 0 || M > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "M out of range");
     if (N < 0 || N % 8 != 0 || N > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "N must be a non-negative multiple of 8");
@@ -501,7 +526,7 @@ sq_status gemm_checked(const void *X_N, const float *s_x, const void *X_O, const
     SQ_TRY(check_ptr(Y, true, "Y"));
     if (dbg_i && !aligned16(dbg_i)) return fail(SQ_ERR_MISALIGNED, "dbg_acc_i32 is not 16-byte aligned");
     if (dbg_f && !aligned16(dbg_f)) return fail(SQ_ERR_MISALIGNED, "dbg_acc_f32 is not 16-byte aligned");
-    return gemm_impl(X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    return gemm_impl(X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream, fp8);
 }
 
 // Single-thread kernel that waits on a barrier nobody completes, with a
@@ -519,6 +544,81 @@ __global__ void watchdog_selftest_kernel(unsigned long long limit_ns)
             return;
         }
     }
+}
+
+// Low-path code bytes per row: kn_pad / 2 (packed INT4) or kn_pad (E4M3).
+int64_t code_row_bytes(int64_t K, int64_t nO, bool fp8) { return fp8 ? sq_kn_pad(K, nO) : sq_kn_pad(K, nO) / 2; }
+
+size_t linear_ws_bytes(int64_t M, int64_t K, int64_t nO, bool fp8)
+{
+    if (M <= 0) return 0;
+    const int64_t xn = round_up(M * code_row_bytes(K, nO, fp8), 256);
+    const int64_t sx = round_up(M * 4, 256);
+    const int64_t xo = round_up(M * sq_no_pad(nO) * 2, 256);
+    return static_cast<size_t>(xn + sx + xo);
+}
+
+sq_status prepare_impl(const void *W, int64_t N, int64_t K, int64_t ldw, const int32_t *O, int64_t nO, void *W_N,
+                       float *s_w, void *W_O, uint32_t *chan_tab, cudaStream_t s, bool fp8)
+{
+    SQ_TRY(check_K_nO(K, nO));
+    if (fp8 && K > sqq::kStreamMaxK)
+        return fail(SQ_ERR_UNSUPPORTED, "the FP8 low path supports K <= %d (K=%lld)", sqq::kStreamMaxK, (long long)K);
+    if (N < 0) return fail(SQ_ERR_INVALID_ARG, "N < 0");
+    if (ldw < K || ldw % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldw must be >= K and a multiple of 8");
+    if (nO > 0 && !O) return fail(SQ_ERR_INVALID_ARG, "O is NULL");
+    for (int64_t j = 0; j < nO; ++j) {
+        if (O[j] < 0 || O[j] >= K) return fail(SQ_ERR_INVALID_ARG, "O[%lld]=%d outside [0, K)", (long long)j, O[j]);
+        if (j > 0 && O[j] <= O[j - 1]) return fail(SQ_ERR_INVALID_ARG, "O must be strictly increasing (index %lld)", (long long)j);
+    }
+    SQ_TRY(check_ptr(chan_tab, true, "chan_tab"));
+    const int64_t kn_pad = sq_kn_pad(K, nO);
+    if (N > 0) {
+        SQ_TRY(check_ptr(W, true, "W"));
+        SQ_TRY(check_ptr(W_N, kn_pad > 0, "W_N"));
+        SQ_TRY(check_ptr(s_w, true, "s_w"));
+        SQ_TRY(check_ptr(W_O, nO > 0, "W_O"));
+    }
+    DevInfo di;
+    SQ_TRY(device_info(di));
+
+    // Static channel table: one word per 8 channels.
+    std::vector<uint32_t> tab(static_cast<size_t>(K / 8), 0u);
+    for (int64_t j = 0; j < nO; ++j) tab[O[j] / 8] |= 1u << (O[j] % 8);
+    uint32_t below = 0;
+    for (int64_t c = 0; c < K / 8; ++c) {
+        const uint32_t mask = tab[c];
+        tab[c] = (below << 8) | mask;
+        below += static_cast<uint32_t>(__builtin_popcount(mask));
+    }
+    cudaError_t e = cudaMemcpyAsync(chan_tab, tab.data(), tab.size() * sizeof(uint32_t), cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copy of the channel table");
+    SQ_TRY(launch_rowquant(static_cast<const uint16_t *>(W), N, K, ldw, chan_tab, nO, static_cast<uint8_t *>(W_N), s_w,
+                           static_cast<uint16_t *>(W_O), s, fp8));
+    if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "sq_prepare_weights");
+    return SQ_OK;
+}
+
+sq_status linear_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, const void *W_N,
+                      const float *s_w, const void *W_O, int64_t N, int64_t nO, void *Y, int64_t ldy, void *workspace,
+                      size_t ws_bytes, cudaStream_t s, bool fp8)
+{
+    SQ_TRY(check_K_nO(K, nO));
+    if (M < 0) return fail(SQ_ERR_INVALID_ARG, "M < 0");
+    if (M == 0) return SQ_OK;
+    const size_t need = linear_ws_bytes(M, K, nO, fp8);
+    if (ws_bytes < need) return fail(SQ_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+    SQ_TRY(check_ptr(workspace, true, "workspace"));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const int64_t kn_pad = sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
+    const int64_t xn_bytes = round_up(M * code_row_bytes(K, nO, fp8), 256);
+    uint8_t *X_N = ws;
+    float *s_x = reinterpret_cast<float *>(ws + xn_bytes);
+    uint16_t *X_O = reinterpret_cast<uint16_t *>(ws + xn_bytes + round_up(M * 4, 256));
+    SQ_TRY(quant_gather_impl(X, M, K, ldx, chan_tab, nO, kn_pad > 0 ? X_N : nullptr, s_x, no_pad > 0 ? X_O : nullptr, s,
+                             fp8));
+    return gemm_checked(kn_pad > 0 ? X_N : nullptr, s_x, no_pad > 0 ? X_O : nullptr, W_N, s_w, W_O, M, N, K, nO, Y, ldy,
+                        nullptr, nullptr, s, fp8);
 }
 
 }  // namespace
@@ -547,54 +647,22 @@ int64_t sq_no_pad(int64_t nO) { return round_up(nO, 64); }
 
 int64_t sq_chan_table_words(int64_t K) { return K / 8; }
 
-size_t sq_linear_workspace_bytes(int64_t M, int64_t K, int64_t nO)
-{
-    if (M <= 0) return 0;
-    const int64_t xn = round_up(M * (sq_kn_pad(K, nO) / 2), 256);
-    const int64_t sx = round_up(M * 4, 256);
-    const int64_t xo = round_up(M * sq_no_pad(nO) * 2, 256);
-    return static_cast<size_t>(xn + sx + xo);
-}
+size_t sq_linear_workspace_bytes(int64_t M, int64_t K, int64_t nO) { return linear_ws_bytes(M, K, nO, false); }
+
+size_t sq_linear_workspace_bytes_fp8(int64_t M, int64_t K, int64_t nO) { return linear_ws_bytes(M, K, nO, true); }
 
 sq_status sq_prepare_weights(const void *W, int64_t N, int64_t K, int64_t ldw, const int32_t *O, int64_t nO,
                              void *W_N, float *s_w, void *W_O, uint32_t *chan_tab, sq_stream_t stream)
 {
     g_detail.clear();
-    SQ_TRY(check_K_nO(K, nO));
-    if (N < 0) return fail(SQ_ERR_INVALID_ARG, "N < 0");
-    if (ldw < K || ldw % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldw must be >= K and a multiple of 8");
-    if (nO > 0 && !O) return fail(SQ_ERR_INVALID_ARG, "O is NULL");
-    for (int64_t j = 0; j < nO; ++j) {
-        if (O[j] < 0 || O[j] >= K) return fail(SQ_ERR_INVALID_ARG, "O[%lld]=%d outside [0, K)", (long long)j, O[j]);
-        if (j > 0 && O[j] <= O[j - 1]) return fail(SQ_ERR_INVALID_ARG, "O must be strictly increasing (index %lld)", (long long)j);
-    }
-    SQ_TRY(check_ptr(chan_tab, true, "chan_tab"));
-    const int64_t kn_pad = sq_kn_pad(K, nO);
-    if (N > 0) {
-        SQ_TRY(check_ptr(W, true, "W"));
-        SQ_TRY(check_ptr(W_N, kn_pad > 0, "W_N"));
-        SQ_TRY(check_ptr(s_w, true, "s_w"));
-        SQ_TRY(check_ptr(W_O, nO > 0, "W_O"));
-    }
-    DevInfo di;
-    SQ_TRY(device_info(di));
+    return prepare_impl(W, N, K, ldw, O, nO, W_N, s_w, W_O, chan_tab, reinterpret_cast<cudaStream_t>(stream), false);
+}
 
-    // Static channel table: one word per 8 channels.
-    std::vector<uint32_t> tab(static_cast<size_t>(K / 8), 0u);
-    for (int64_t j = 0; j < nO; ++j) tab[O[j] / 8] |= 1u << (O[j] % 8);
-    uint32_t below = 0;
-    for (int64_t c = 0; c < K / 8; ++c) {
-        const uint32_t mask = tab[c];
-        tab[c] = (below << 8) | mask;
-        below += static_cast<uint32_t>(__builtin_popcount(mask));
-    }
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = cudaMemcpyAsync(chan_tab, tab.data(), tab.size() * sizeof(uint32_t), cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return cuda_fail(e, "copy of the channel table");
-    SQ_TRY(launch_rowquant(static_cast<const uint16_t *>(W), N, K, ldw, chan_tab, nO, static_cast<uint8_t *>(W_N), s_w,
-                           static_cast<uint16_t *>(W_O), s));
-    if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "sq_prepare_weights");
-    return SQ_OK;
+sq_status sq_prepare_weights_fp8(const void *W, int64_t N, int64_t K, int64_t ldw, const int32_t *O, int64_t nO,
+                                 void *W_N8, float *s_w, void *W_O, uint32_t *chan_tab, sq_stream_t stream)
+{
+    g_detail.clear();
+    return prepare_impl(W, N, K, ldw, O, nO, W_N8, s_w, W_O, chan_tab, reinterpret_cast<cudaStream_t>(stream), true);
 }
 
 sq_status sq_quant_gather(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, int64_t nO,
@@ -602,6 +670,13 @@ sq_status sq_quant_gather(const void *X, int64_t M, int64_t K, int64_t ldx, cons
 {
     g_detail.clear();
     return quant_gather_impl(X, M, K, ldx, chan_tab, nO, X_N, s_x, X_O, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_quant_gather_fp8(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, int64_t nO,
+                              void *X_N8, float *s_x, void *X_O, sq_stream_t stream)
+{
+    g_detail.clear();
+    return quant_gather_impl(X, M, K, ldx, chan_tab, nO, X_N8, s_x, X_O, reinterpret_cast<cudaStream_t>(stream), true);
 }
 
 sq_status sq_gemm(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
@@ -613,26 +688,31 @@ sq_status sq_gemm(const void *X_N, const float *s_x, const void *X_O, const void
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
+sq_status sq_gemm_fp8(const void *X_N8, const float *s_x, const void *X_O, const void *W_N8, const float *s_w,
+                      const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
+                      float *dbg_acc_8, float *dbg_acc_f32, sq_stream_t stream)
+{
+    g_detail.clear();
+    return gemm_checked(X_N8, s_x, X_O, W_N8, s_w, W_O, M, N, K, nO, Y, ldy, reinterpret_cast<int32_t *>(dbg_acc_8),
+                        dbg_acc_f32, reinterpret_cast<cudaStream_t>(stream), true);
+}
+
 sq_status sq_linear(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, const void *W_N,
                     const float *s_w, const void *W_O, int64_t N, int64_t nO, void *Y, int64_t ldy, void *workspace,
                     size_t ws_bytes, sq_stream_t stream)
 {
     g_detail.clear();
-    SQ_TRY(check_K_nO(K, nO));
-    if (M < 0) return fail(SQ_ERR_INVALID_ARG, "M < 0");
-    if (M == 0) return SQ_OK;
-    const size_t need = sq_linear_workspace_bytes(M, K, nO);
-    if (ws_bytes < need) return fail(SQ_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", ws_bytes, need);
-    SQ_TRY(check_ptr(workspace, true, "workspace"));
-    uint8_t *ws = static_cast<uint8_t *>(workspace);
-    const int64_t kn_pad = sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
-    uint8_t *X_N = ws;
-    float *s_x = reinterpret_cast<float *>(ws + round_up(M * (kn_pad / 2), 256));
-    uint16_t *X_O = reinterpret_cast<uint16_t *>(ws + round_up(M * (kn_pad / 2), 256) + round_up(M * 4, 256));
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    SQ_TRY(quant_gather_impl(X, M, K, ldx, chan_tab, nO, kn_pad > 0 ? X_N : nullptr, s_x, no_pad > 0 ? X_O : nullptr, s));
-    return gemm_checked(kn_pad > 0 ? X_N : nullptr, s_x, no_pad > 0 ? X_O : nullptr, W_N, s_w, W_O, M, N, K, nO, Y, ldy,
-                        nullptr, nullptr, s);
+    return linear_impl(X, M, K, ldx, chan_tab, W_N, s_w, W_O, N, nO, Y, ldy, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+sq_status sq_linear_fp8(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, const void *W_N8,
+                        const float *s_w, const void *W_O, int64_t N, int64_t nO, void *Y, int64_t ldy, void *workspace,
+                        size_t ws_bytes, sq_stream_t stream)
+{
+    g_detail.clear();
+    return linear_impl(X, M, K, ldx, chan_tab, W_N8, s_w, W_O, N, nO, Y, ldy, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream), true);
 }
 
 sq_status sq_check(sq_stream_t stream)

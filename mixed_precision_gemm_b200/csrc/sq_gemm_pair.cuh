@@ -74,7 +74,11 @@ struct CfgPair {
                   "every ring slot must belong to one producer group");
 };
 
-template <class C, bool DBG>
+// FP8: the low path is E4M3 x E4M3 (kind::f8f6f4, OSC's FP8 fallback for the
+// inputs of W2): its tiles are plain bytes that TMA writes straight into the
+// operand ring, so the staging ring and the expansion are compiled out and the
+// normal accumulator is fp32.
+template <class C, bool DBG, bool FP8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
 dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_constant__ CUtensorMap tm_wo,
                       const __grid_constant__ CUtensorMap tm_xn, const __grid_constant__ CUtensorMap tm_wn,
@@ -152,7 +156,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         // ------------------------------------------------------------ staging producer (each CTA)
         // Packed INT4 tiles of this CTA's X rows and W rows, one K-block per
         // stage, in the order the expansion warps consume them.
-        if (lane == 0 && nkb_i > 0) {
+        if constexpr (!FP8) if (lane == 0 && nkb_i > 0) {
             const int F = my_tiles * nkb_i;
             const int r0 = static_cast<int>(rank) * 128;
             int last_armed = -1;
@@ -176,6 +180,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         if (leader && lane == 0) {
             constexpr uint32_t idesc_bf = sqd::make_idesc(false, PAIR_BM, PAIR_BN);
             constexpr uint32_t idesc_i8 = sqd::make_idesc(true, PAIR_BM, PAIR_BN);
+            constexpr uint32_t idesc_f8 = sqd::make_idesc_e4m3(PAIR_BM, PAIR_BN);
             bool ok = true;
             for (int lt = 0; lt < my_tiles && ok; ++lt) {
                 if (!sqd::mbar_wait(acc_empty, (lt & 1) ^ 1u, abort_flag, SITE_MMA_ACC)) { ok = false; break; }
@@ -194,6 +199,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t acc = (first && k == 0) ? 0u : 1u;
                         if (is_bf) sqd::mma_bf16_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_bf, acc);
+                        else if constexpr (FP8) sqd::mma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_f8, acc);
                         else sqd::mma_s8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_i8, acc);
                     }
                     sqd::mma_commit_pair_multicast(op_empty(e), 0x3);
@@ -214,6 +220,9 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         // INT4 block f: packed rows from staging stage f % STG -> int8 rows in
         // operand stage e (the tile's X rows, then its W rows).
         auto store = [&](int f) -> bool {
+          if constexpr (FP8) {
+            return false;  // FP8 tiles are never expanded
+          } else {
             const int lt = f / nkb_i;
             const int kb = f - lt * nkb_i;
             const int u = lt * per_tile + nkb_o + kb;
@@ -250,24 +259,24 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                 sqd::mbar_arrive_cluster(sqd::map_to_cta(op_full(e), 0));
             }
             return true;
+          }
         };
 
         const bool tma_thread = (et == 0);
         int last_armed = -1;
-        // bf16 block kb of tile lt: the group's first thread issues the two TMA
+        // Ring use u (tile lt) filled by TMA: the X and W tiles of map mx / mw
+        // at K offset x (elements).  The group's first thread issues the two
         // loads with their byte count; every other warp of the group arrives.
-        auto produce_bf16 = [&](int lt, int kb) -> bool {
+        auto produce_tma = [&](int lt, int u, const CUtensorMap *mx, const CUtensorMap *mw, int x) -> bool {
             int tmi, tni;
             tile_coords(args, pair + lt * num_pairs, tmi, tni);
-            const int u = lt * per_tile + kb;
             const int e = u % OPS;
             if (!sqd::mbar_wait(op_empty(e), ((u / OPS) & 1) ^ 1u, abort_flag, SITE_EXP_OP)) return false;
             const uint32_t full_leader = sqd::map_to_cta(op_full(e), 0);
             if (tma_thread) {
                 sqd::mbar_arrive_expect_tx_cluster(full_leader, C::OP_BYTES);
-                sqd::tma_load_2d_pair(op_a(e), &tm_xo, full_leader, kb * KB_BF, tmi * PAIR_BM + static_cast<int>(r0));
-                sqd::tma_load_2d_pair(op_a(e) + C::A_BYTES, &tm_wo, full_leader, kb * KB_BF,
-                                      tni * PAIR_BN + static_cast<int>(r0));
+                sqd::tma_load_2d_pair(op_a(e), mx, full_leader, x, tmi * PAIR_BM + static_cast<int>(r0));
+                sqd::tma_load_2d_pair(op_a(e) + C::A_BYTES, mw, full_leader, x, tni * PAIR_BN + static_cast<int>(r0));
                 last_armed = u;
             } else if (lane == 0) {
                 sqd::mbar_arrive_cluster(full_leader);
@@ -275,13 +284,16 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             return true;
         };
 
-        // Ring uses of this group, in order: u = gi, gi + NG, ...
+        // Ring uses of this group, in order: u = gi, gi + NG, ...  bf16 blocks
+        // first, then the low-path blocks (E4M3 by TMA, or INT4 expanded).
         bool ok = true;
         const int total = my_tiles * per_tile;
         for (int u = gi; u < total && ok; u += C::NG) {
             const int lt = u / per_tile;
             const int i = u - lt * per_tile;
-            ok = (i < nkb_o) ? produce_bf16(lt, i) : store(lt * nkb_i + (i - nkb_o));
+            if (i < nkb_o) ok = produce_tma(lt, u, &tm_xo, &tm_wo, i * KB_BF);
+            else if constexpr (FP8) ok = produce_tma(lt, u, &tm_xn, &tm_wn, (i - nkb_o) * KB_I8);
+            else ok = store(lt * nkb_i + (i - nkb_o));
         }
         if (!ok && tma_thread && last_armed >= 0 && leader) {
             // Let the last copies that were issued land before the CTA exits.
@@ -347,11 +359,21 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
                                 const int t = 8 * g + 2 * h + u;
-                                const int ai = has_i ? (static_cast<int>(vi[b][t]) >> 8) : 0;
+                                // low path: exact int32 sum (x256) for INT4, fp32 sum for E4M3
+                                float al;
+                                int32_t dbg_lo;
+                                if constexpr (FP8) {
+                                    al = has_i ? __uint_as_float(vi[b][t]) : 0.0f;
+                                    dbg_lo = __float_as_int(al);
+                                } else {
+                                    const int ai = has_i ? (static_cast<int>(vi[b][t]) >> 8) : 0;
+                                    al = static_cast<float>(ai);
+                                    dbg_lo = ai;
+                                }
                                 const float af = has_o ? __uint_as_float(vf[b][t]) : 0.0f;
-                                y2[u] = __fadd_rn(__fmul_rn(__fmul_rn(static_cast<float>(ai), sx), swv[2 * h + u]), af);
+                                y2[u] = __fadd_rn(__fmul_rn(__fmul_rn(al, sx), swv[2 * h + u]), af);
                                 if constexpr (DBG) {
-                                    if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + 2 * h + u] = ai;
+                                    if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + 2 * h + u] = dbg_lo;
                                     if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n + 2 * h + u] = af;
                                 }
                             }

@@ -110,7 +110,11 @@ __device__ __forceinline__ int skinny_first_block(int r, int S, int nkb_i, int n
     return c <= nkb_i ? c : nkb_i + (c - nkb_i + 1) / 2;
 }
 
-template <class C, bool DBG>
+// FP8: the low path is E4M3 x E4M3 (kind::f8f6f4, OSC's FP8 fallback for the
+// inputs of W2).  A stage then carries one K-block of bytes that the MMA reads
+// in place, as for bf16 stages; the expansion warps only run the epilogue, and
+// the low-path partials are fp32.
+template <class C, bool DBG, bool FP8>
 __global__ void __launch_bounds__(SK_THREADS, 1)
 dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_constant__ CUtensorMap tm_wo,
                         const __grid_constant__ CUtensorMap tm_xn, const __grid_constant__ CUtensorMap tm_wn,
@@ -150,7 +154,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
     const int n_i = min(b_hi, nkb_i) - i_lo;
     const int o_lo = max(b_lo, nkb_i) - nkb_i;
     const int n_o = max(b_hi, nkb_i) - nkb_i - o_lo;
-    const int ns_i = (n_i + 1) / 2;
+    const int ns_i = FP8 ? n_i : (n_i + 1) / 2;
     const int ns = ns_i + n_o;
 
     if (threadIdx.x == 0) {
@@ -199,7 +203,8 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
                 if (!sqd::mbar_wait(stg_empty(s), ((t / NST) & 1) ^ 1u, abort_flag, SITE_SK_STG)) { ok = false; break; }
                 sqd::mbar_arrive_expect_tx(stg_full(s), C::TILE_BYTES);
                 if (t < ns_i) {
-                    const int x = (i_lo + 2 * t) * PROWB;  // byte offset of the stage's first K-block
+                    // byte offset of the stage's first K-block (two INT4 blocks, or one E4M3 block)
+                    const int x = FP8 ? (i_lo + t) * KB_I8 : (i_lo + 2 * t) * PROWB;
                     sqd::tma_load_2d(stg_a(s), &tm_wn, stg_full(s), x, n0);
                     sqd::tma_load_2d(stg_a(s) + C::A_BYTES, &tm_xn, stg_full(s), x, 0);
                 } else {
@@ -216,8 +221,22 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
         if (lane == 0) {
             constexpr uint32_t idesc_bf = sqd::make_idesc(false, 128, MP);
             constexpr uint32_t idesc_i8 = sqd::make_idesc(true, 128, MP);
+            constexpr uint32_t idesc_f8 = sqd::make_idesc_e4m3(128, MP);
             bool ok = true;
-            for (int u = 0; u < n_i && ok; ++u) {  // INT4 blocks from the operand ring
+            if constexpr (FP8) {
+                for (int t = 0; t < ns_i && ok; ++t) {  // E4M3 blocks straight from the staging ring
+                    const int s = t % NST;
+                    if (!sqd::mbar_wait(stg_full(s), (t / NST) & 1, abort_flag, SITE_SK_MMA)) { ok = false; break; }
+                    sqd::tc_fence_after();
+                    const uint64_t adesc = sqd::make_sw128_desc(stg_a(s));
+                    const uint64_t bdesc = sqd::make_sw128_desc(stg_a(s) + C::A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        sqd::mma_f8(tmem, adesc + 2 * k, bdesc + 2 * k, idesc_f8, (t == 0 && k == 0) ? 0u : 1u);
+                    sqd::mma_commit(stg_empty(s));
+                }
+            }
+            for (int u = 0; u < (FP8 ? 0 : n_i) && ok; ++u) {  // INT4 blocks from the operand ring
                 const int e = u % OPS;
                 if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_SK_MMA)) { ok = false; break; }
                 sqd::tc_fence_after();
@@ -254,7 +273,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
         // threads read one whole row, so the loads are conflict-free.
         const int et = threadIdx.x - SK_PROD_WARP0 * 32;
         bool ok = true;
-        for (int t = 0; t < ns_i && ok; ++t) {
+        for (int t = 0; t < (FP8 ? 0 : ns_i) && ok; ++t) {
             const int s = t % NST;
             const int nblk = min(2, n_i - 2 * t);
             const int u0 = 2 * t;  // operand ring uses u0, u0 + 1
@@ -361,17 +380,19 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
             const int n = n0 + r0 + rl;
             if (m >= args.M || n >= args.N) continue;
             int32_t si = 0;
-            float sf = 0.0f;
+            float sl = 0.0f, sf = 0.0f;
             for (int s = 0; s < S; ++s) {
                 const int w = (s * RP + rl) * C::RSTRIDE + m;
-                si += red_i[w];
+                if constexpr (FP8) sl = __fadd_rn(sl, __int_as_float(red_i[w]));
+                else si += red_i[w];
                 sf = __fadd_rn(sf, red_f[w]);
             }
             const int ai = si >> 8;
-            const float y = __fadd_rn(__fmul_rn(__fmul_rn(static_cast<float>(ai), args.s_x[m]), args.s_w[n]), sf);
+            const float al = FP8 ? sl : static_cast<float>(ai);
+            const float y = __fadd_rn(__fmul_rn(__fmul_rn(al, args.s_x[m]), args.s_w[n]), sf);
             args.Y[static_cast<long long>(m) * args.ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
             if constexpr (DBG) {
-                if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n] = ai;
+                if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n] = FP8 ? __float_as_int(sl) : ai;
                 if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n] = sf;
             }
         }

@@ -29,6 +29,8 @@
 // kn_pad/2 + 2 no_pad + 4 written.
 #pragma once
 
+#include <cuda_fp8.h>
+
 #include "sq_device.cuh"
 
 namespace sqq {
@@ -169,6 +171,37 @@ __device__ __forceinline__ void quant8_pairs(const uint4 &v, const RowScale &rs,
     hi = low_bytes4(t[4], t[5], t[6], t[7]);
 }
 
+// E4M3 codes of the 8 channels of a chunk (lo: channels 0..3, hi: 4..7, one
+// byte each): the same correctly rounded fp32 quotient t = fl(x / s) as
+// quant8_pairs, then the hardware conversion to E4M3 (round to nearest even,
+// magnitudes above 448 saturate to 448, the sign of t kept).
+template <bool UP>
+__device__ __forceinline__ void quant8_fp8_pairs(const uint4 &v, const RowScale &rs, uint32_t &lo, uint32_t &hi)
+{
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t b[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        uint64_t x = f2_pack(w[p] << 16, w[p] & 0xFFFF0000u);
+        if constexpr (UP) x = f2_mul(x, rs.up2);
+        const uint64_t q0 = f2_mul(x, rs.inv2);
+        const uint64_t r = f2_fma(q0, rs.negs2, x);
+        const uint64_t q1 = f2_fma(r, rs.inv2, q0);
+        uint32_t t0, t1;
+        f2_unpack(q1, t0, t1);
+        b[p] = static_cast<uint32_t>(
+            __nv_cvt_float2_to_fp8x2(make_float2(__uint_as_float(t0), __uint_as_float(t1)), __NV_SATFINITE, __NV_E4M3));
+    }
+    // The correction step turns x = -0 into +0 (r = fma(-0, -s, -0) = +0 and
+    // +0 + -0 = +0), while fl(-0 / s) = -0.  For s > 0 the sign of every code
+    // is the sign of x, so it is copied from the bf16 inputs: byte i of the
+    // byte permutation holds the high byte (sign bit 7) of channel i.
+    lo = (b[0] | (b[1] << 16)) & 0x7F7F7F7Fu;
+    hi = (b[2] | (b[3] << 16)) & 0x7F7F7F7Fu;
+    lo |= __byte_perm(v.x, v.y, 0x7531) & 0x80808080u;
+    hi |= __byte_perm(v.z, v.w, 0x7531) & 0x80808080u;
+}
+
 // Group-wide maximum of a 32-bit value: warp shuffles, then (G > 1) the
 // warps' results through shared memory and one block barrier.
 template <int G>
@@ -187,15 +220,16 @@ __device__ __forceinline__ uint32_t group_max(uint32_t v, uint32_t *red)
 }
 
 
-// Scale of a row, s = fl(a / 7).  For a >= 2^-100 Markstein's correction (see
-// quant8_pairs) with y7 = fl(1/7) gives the correctly rounded quotient in
-// three operations; smaller a takes the division.
-__device__ __forceinline__ float row_scale(float a, float y7)
+// Scale of a row, s = fl(a / d) (d = 7 for INT4 codes, 448 for E4M3).  For
+// a >= 2^-100 Markstein's correction (see quant8_pairs) with yd = fl(1/d)
+// gives the correctly rounded quotient in three operations; smaller a takes
+// the division.
+__device__ __forceinline__ float row_scale(float a, float d, float yd)
 {
-    if (a < kTinyScale) return __fdiv_rn(a, 7.0f);
-    const float q0 = __fmul_rn(a, y7);
-    const float r = __fmaf_rn(-7.0f, q0, a);
-    return __fmaf_rn(r, y7, q0);
+    if (a < kTinyScale) return __fdiv_rn(a, d);
+    const float q0 = __fmul_rn(a, yd);
+    const float r = __fmaf_rn(-d, q0, a);
+    return __fmaf_rn(r, yd, q0);
 }
 
 // Row-invariant facts about one chunk, packed into a word: outlier mask in
@@ -311,7 +345,7 @@ __global__ void __launch_bounds__(32 * G, 512 / (32 * G)) rowquant_kernel(
 
         // 2. per-row scale and quantizer constants
         const bool zero = (amax == 0u);
-        const float s = zero ? 0.0f : row_scale(__uint_as_float(amax << 16), y7);
+        const float s = zero ? 0.0f : row_scale(__uint_as_float(amax << 16), 7.0f, y7);
         const bool up = !zero && s < kTinyScale;
         const float s1 = up ? s * kUpScale : s;
         const float inv_s = zero ? 0.0f : __frcp_rn(s1);

@@ -35,13 +35,13 @@ enum : unsigned { SITE_RQ_PROD = 0x601, SITE_RQ_CONS = 0x602 };
 // Shared-memory layout, computed identically on the host and the device.
 struct StreamLayout {
     int row_bytes;   // 2K, rounded up to 128
-    int pk_alloc;    // kn_pad / 2 + 16
+    int pk_alloc;    // code bytes per row (kn_pad / 2 INT4, kn_pad E4M3) + 16
     int off_pl, off_olist, off_pbuf, off_bar, off_misc, off_ring, bytes;
 
-    __host__ __device__ StreamLayout(int K, int kn_pad, int no_pad, int ngrp)
+    __host__ __device__ StreamLayout(int K, int kn_pad, int no_pad, int ngrp, bool fp8)
     {
         row_bytes = (2 * K + 127) & ~127;
-        pk_alloc = kn_pad / 2 + 16;
+        pk_alloc = (fp8 ? kn_pad : kn_pad / 2) + 16;
         off_pl = static_cast<int>(sizeof(QuantTables));
         off_olist = off_pl + ((4 * (K / 8) + 15) & ~15);
         off_pbuf = off_olist + ((2 * no_pad + 15) & ~15);
@@ -62,14 +62,16 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads)
 // without more shared memory).
 __host__ __device__ constexpr int stream_max_groups(int G) { return G <= 2 ? 10 : G == 4 ? 7 : 3; }
 
-template <int G>
+// FP8: E4M3 codes (one byte per normal channel, scale absmax / 448) in place
+// of INT4 codes (OSC's FP8 fallback for the inputs of W2).
+template <int G, bool FP8>
 __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowquant_stream_kernel(
     const uint16_t *__restrict__ src, int64_t rows, int K, int64_t ld,
     const uint32_t *__restrict__ chan_tab, int nO, int kn_pad, int no_pad,
     uint8_t *__restrict__ dst_n, float *__restrict__ dst_s, uint16_t *__restrict__ dst_o, int ngrp)
 {
     extern __shared__ __align__(128) uint8_t rs_smem[];
-    const StreamLayout L(K, kn_pad, no_pad, ngrp);
+    const StreamLayout L(K, kn_pad, no_pad, ngrp, FP8);
     QuantTables *tabs = reinterpret_cast<QuantTables *>(rs_smem);
     uint32_t *pl_tab = reinterpret_cast<uint32_t *>(rs_smem + L.off_pl);
     uint16_t *olist = reinterpret_cast<uint16_t *>(rs_smem + L.off_olist);
@@ -100,13 +102,15 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
     for (int i = tid; i < ngrp * ((L.pk_alloc + 15) / 16); i += nthr)
         reinterpret_cast<uint4 *>(rs_smem + L.off_pbuf)[i] = make_uint4(0, 0, 0, 0);
     for (int j = nO + tid; j < no_pad; j += nthr) olist[j] = kNoChannel;
-    // Per chunk: outlier mask, packed word and nibble shift of its first
-    // code (see rowquant_kernel); its outliers enter the list O.
+    // Per chunk: outlier mask, packed word and position inside it of its
+    // first code (a nibble for INT4, a byte for E4M3; see rowquant_kernel);
+    // its outliers enter the list O.
     for (int c = tid; c < nchunk; c += nthr) {
         const uint32_t tb = __ldg(chan_tab + c);
         const uint32_t below = tb >> 8;
         const uint32_t p = 8u * static_cast<uint32_t>(c) - below;
-        pl_tab[c] = (tb & 0xFFu) | ((p & 7u) << 8) | ((p >> 3) << 11);
+        pl_tab[c] = FP8 ? ((tb & 0xFFu) | ((p & 3u) << 8) | ((p >> 2) << 11))
+                        : ((tb & 0xFFu) | ((p & 7u) << 8) | ((p >> 3) << 11));
         for (uint32_t mm = tb & 0xFFu, j = below; mm; mm &= mm - 1, ++j)
             olist[j] = static_cast<uint16_t>(8 * c + __ffs(mm) - 1);
     }
@@ -145,8 +149,9 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
     const int bar_id = 1 + gi;
     uint32_t *pbuf = reinterpret_cast<uint32_t *>(rs_smem + L.off_pbuf + gi * L.pk_alloc);
     const uint32_t *ol2 = reinterpret_cast<const uint32_t *>(olist);
-    const int pk_bytes = kn_pad >> 1;
-    const float y7 = __frcp_rn(7.0f);
+    const int pk_bytes = FP8 ? kn_pad : (kn_pad >> 1);
+    constexpr float kDiv = FP8 ? 448.0f : 7.0f;  // largest code magnitude
+    const float ydiv = __frcp_rn(kDiv);
     const RowScale rs_const = [] {
         RowScale r{};
         r.magic2 = f2_pack(__float_as_uint(kMagic), __float_as_uint(kMagic));
@@ -186,7 +191,7 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
 
         // 2. scale and quantizer constants
         const bool zero = (amax == 0u);
-        const float sc = zero ? 0.0f : row_scale(__uint_as_float(amax << 16), y7);
+        const float sc = zero ? 0.0f : row_scale(__uint_as_float(amax << 16), kDiv, ydiv);
         const bool up = !zero && sc < kTinyScale;
         const float s1 = up ? sc * kUpScale : sc;
         const float inv_s = zero ? 0.0f : __frcp_rn(s1);
@@ -203,16 +208,39 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
             const uint4 v = *reinterpret_cast<const uint4 *>(rs_smem + L.off_ring + s * L.row_bytes + 16 * c);
             const uint32_t pl = pl_tab[c];
             uint32_t lo, hi;
-            if (!up) quant8_pairs<false>(v, rs, lo, hi);
-            else quant8_pairs<true>(v, rs, lo, hi);
             const uint4 pk = *reinterpret_cast<const uint4 *>(tabs->pack[chunk_mask(pl)]);
-            const uint32_t ev = __byte_perm(lo, hi, pk.x);  // normal codes 0, 2, 4, 6
-            const uint32_t od = __byte_perm(lo, hi, pk.y);  // normal codes 1, 3, 5, 7
-            const uint32_t V = ((ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u)) & pk.z;
-            const uint32_t sh = 4u * chunk_nib(pl);
-            uint32_t *dst = pbuf + chunk_word(pl);
-            atomicOr(dst, V << sh);
-            if (sh) atomicOr(dst + 1, V >> (32u - sh));
+            if constexpr (!FP8) {
+                if (!up) quant8_pairs<false>(v, rs, lo, hi);
+                else quant8_pairs<true>(v, rs, lo, hi);
+                const uint32_t ev = __byte_perm(lo, hi, pk.x);  // normal codes 0, 2, 4, 6
+                const uint32_t od = __byte_perm(lo, hi, pk.y);  // normal codes 1, 3, 5, 7
+                const uint32_t V = ((ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u)) & pk.z;
+                const uint32_t sh = 4u * chunk_nib(pl);
+                uint32_t *dst = pbuf + chunk_word(pl);
+                atomicOr(dst, V << sh);
+                if (sh) atomicOr(dst + 1, V >> (32u - sh));
+            } else {
+                if (zero) {
+                    lo = hi = 0u;  // a zero row has all-zero codes
+                } else if (!up) {
+                    quant8_fp8_pairs<false>(v, rs, lo, hi);
+                } else {
+                    quant8_fp8_pairs<true>(v, rs, lo, hi);
+                }
+                // normal codes in channel order: A = codes 0..3, B = 4..7, the
+                // bytes past the n normal channels cleared
+                const uint32_t ev = __byte_perm(lo, hi, pk.x);
+                const uint32_t od = __byte_perm(lo, hi, pk.y);
+                const uint32_t n = pk.w;
+                const uint32_t A = __byte_perm(ev, od, 0x5140) & (n >= 4 ? 0xFFFFFFFFu : (1u << (8 * n)) - 1u);
+                const uint32_t B = __byte_perm(ev, od, 0x7362) &
+                                   (n >= 8 ? 0xFFFFFFFFu : n > 4 ? (1u << (8 * (n - 4))) - 1u : 0u);
+                const uint32_t sh = 8u * chunk_nib(pl);
+                uint32_t *dst = pbuf + chunk_word(pl);
+                atomicOr(dst, A << sh);
+                atomicOr(dst + 1, __funnelshift_l(A, B, sh));
+                if (sh) atomicOr(dst + 2, __funnelshift_l(B, 0u, sh));
+            }
         }
 
         // 4. compact outlier row X_O[r, j] = X[r, O[j]], read from the slot

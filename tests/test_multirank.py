@@ -64,22 +64,23 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     import argparse
     import bench
     import workloads
-    args = argparse.Namespace(steps=1, warmup=0, ref_rows=1)
+    args = argparse.Namespace(steps=1, warmup=0, ref_rows=1, low="int4")
     assert bench.run_reference(args, workloads.TINY, rank=1, world=2) == 0
     assert capsys.readouterr().out == ""
 
 
-def test_reference_arm_json_line():
+@pytest.mark.parametrize("low", ["int4", "fp8"])
+def test_reference_arm_json_line(low):
     import json
     import subprocess
     import sys
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
     out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload",
-                          "tiny_64x256x256_o8", "--steps", "2", "--warmup", "3"],
+                          "tiny_64x256x256_o8", "--steps", "2", "--warmup", "3", "--low", low],
                          capture_output=True, text=True, timeout=300, env={**os.environ, "OMP_NUM_THREADS": "2"})
     assert out.returncode == 0, out.stderr
     line = json.loads(out.stdout.strip().splitlines()[-1])
     assert line["impl"] == "reference" and line["unit"] == "TOPS" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] == 2
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
-    assert line["config"]["workload"] == "tiny_64x256x256_o8"
+    assert line["config"]["workload"] == "tiny_64x256x256_o8" and line["config"]["low_path"] == low
