@@ -63,10 +63,11 @@ def _load():
             lib.orc_e4m3_decode_array.argtypes = [P, I, P]
             lib.orc_quantize_rows_fp8.argtypes = [P, I, I, I, P, I, P, P, P]
             lib.orc_dual_linear_rows_fp8.argtypes = [P, P, P, I, P, P, P, I, I, I, P, P, P]
+            lib.orc_select_outliers.argtypes = [P, I, I, I, P, I, I, I, I, P, P]
             for f in (lib.orc_validate_outliers, lib.orc_quantize_rows, lib.orc_pack_int4,
                       lib.orc_chan_table, lib.orc_dual_linear_rows, lib.orc_num_threads,
                       lib.orc_e4m3_encode_array, lib.orc_e4m3_decode_array, lib.orc_quantize_rows_fp8,
-                      lib.orc_dual_linear_rows_fp8):
+                      lib.orc_dual_linear_rows_fp8, lib.orc_select_outliers):
                 f.restype = ctypes.c_int
             _lib = lib
     return _lib
@@ -231,3 +232,29 @@ def linear_fp8(X_bits: np.ndarray, W_bits: np.ndarray, O, rows=None):
     qw, sw, wo = quantize_rows_fp8(W_bits, K, O)
     acc_8, acc_o, y = dual_linear_rows_fp8(qx, sx, xo, qw, sw, wo)
     return dict(qx=qx, sx=sx, xo=xo, qw=qw, sw=sw, wo=wo, acc_8=acc_8, acc_o=acc_o, y=y)
+
+
+# ---------------------------------------------------------------- static outlier selection
+SEL_BLOCK = 1024  # rows per partial sum in the score definition
+
+
+def select_outliers(X_bits: np.ndarray, W_bits: np.ndarray, nO: int, group: int = 1):
+    """Static outlier channels from calibration activations and the weights.
+
+    score[k] = mean_m |X[m,k]| * ||W[:,k]||_2 (fp64, row sums in blocks of
+    SEL_BLOCK rows); the nO/group groups of `group` consecutive channels with
+    the largest summed score (ties to the lower index).  Returns (O int32
+    ascending, score float64 [K]).
+    """
+    X = np.ascontiguousarray(X_bits, np.uint16)
+    W = np.ascontiguousarray(W_bits, np.uint16)
+    Mc, K = X.shape
+    N, K2 = W.shape
+    if K2 != K:
+        raise ValueError("X and W disagree on K")
+    O = np.zeros(nO, np.int32)
+    score = np.zeros(K, np.float64)
+    rc = _load().orc_select_outliers(_ptr(X), Mc, K, K, _ptr(W), N, K, nO, group, _ptr(O), _ptr(score))
+    if rc != 0:
+        raise ValueError("invalid sizes (group must divide K and nO)")
+    return O, score

@@ -328,6 +328,88 @@ int orc_dual_linear_rows_fp8(const uint8_t *qx, const float *sx, const uint16_t 
     return 0;
 }
 
+/* ------------------------------------------------------------------ static outlier selection
+ * SQ-format write-up of arXiv:2512.05409, section 5 (static strategy for
+ * activations) and section 9 (importance scores): the mean activation of each
+ * channel is collected on calibration data, and the importance of a channel
+ * is its activation times its contribution through the weights.  OSC
+ * (arXiv:2604.12782) selects the outlier channels offline, group-wise.
+ * Reading taken:
+ *   score[k] = mean_m |X[m,k]| * ||W[:,k]||_2                   (fp64)
+ *   group g (channels g*G .. g*G+G-1) scores sum_j score[g*G+j]  (G = 1: per channel)
+ *   O = the channels of the nO/G groups with the largest group score, ties to
+ *       the lower group index, in ascending channel order.
+ * Sums over rows are taken in consecutive blocks of ORC_SEL_BLOCK rows: each
+ * block summed in row order, then the block sums added in block order (fp64
+ * throughout; squares and absolute values of bf16 values are exact).  The
+ * order is part of the definition so that a parallel evaluation can match it
+ * bit for bit.
+ */
+#define ORC_SEL_BLOCK 1024
+
+static double orc_blocked_col_sum(const uint16_t *A, int64_t rows, int64_t ld, int64_t k, int square)
+{
+    double total = 0.0;
+    for (int64_t b = 0; b < rows; b += ORC_SEL_BLOCK) {
+        double part = 0.0;
+        const int64_t e = (b + ORC_SEL_BLOCK < rows) ? b + ORC_SEL_BLOCK : rows;
+        for (int64_t r = b; r < e; ++r) {
+            const double v = (double)orc_bf16_to_f32(A[r * ld + k]);
+            part += square ? v * v : fabs(v);
+        }
+        total += part;
+    }
+    return total;
+}
+
+static const double *orc_sort_keys;
+static int orc_group_cmp(const void *pa, const void *pb)
+{
+    const int64_t a = *(const int64_t *)pa, b = *(const int64_t *)pb;
+    if (orc_sort_keys[a] > orc_sort_keys[b]) return -1;
+    if (orc_sort_keys[a] < orc_sort_keys[b]) return 1;
+    return (a < b) ? -1 : (a > b) ? 1 : 0;
+}
+
+/* X: calibration activations bf16 [Mc, ldx]; W: weights bf16 [N, ldw].
+ * Outputs: O [nO] int32 (ascending), score [K] fp64 per channel.
+ * Returns 0, or -1 on invalid sizes. */
+int orc_select_outliers(const uint16_t *X, int64_t Mc, int64_t K, int64_t ldx,
+                        const uint16_t *W, int64_t N, int64_t ldw,
+                        int64_t nO, int64_t group, int32_t *O, double *score)
+{
+    if (Mc <= 0 || N <= 0 || K <= 0 || ldx < K || ldw < K || group < 1 || K % group != 0 || nO < 0 || nO > K ||
+        nO % group != 0)
+        return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t k = 0; k < K; ++k) {
+        const double mean_abs = orc_blocked_col_sum(X, Mc, ldx, k, 0) / (double)Mc;
+        score[k] = mean_abs * sqrt(orc_blocked_col_sum(W, N, ldw, k, 1));
+    }
+    const int64_t ng = K / group, pick = nO / group;
+    double *gs = (double *)malloc((size_t)ng * sizeof(double));
+    int64_t *idx = (int64_t *)malloc((size_t)ng * sizeof(int64_t));
+    char *chosen = (char *)calloc((size_t)ng, 1);
+    if (!gs || !idx || !chosen) { free(gs); free(idx); free(chosen); return -1; }
+    for (int64_t g = 0; g < ng; ++g) {
+        double t = 0.0;
+        for (int64_t j = 0; j < group; ++j) t += score[g * group + j];
+        gs[g] = t;
+        idx[g] = g;
+    }
+    orc_sort_keys = gs;
+    qsort(idx, (size_t)ng, sizeof(int64_t), orc_group_cmp);
+    for (int64_t i = 0; i < pick; ++i) chosen[idx[i]] = 1;
+    int64_t j = 0;
+    for (int64_t g = 0; g < ng; ++g)
+        if (chosen[g])
+            for (int64_t c = 0; c < group; ++c) O[j++] = (int32_t)(g * group + c);
+    free(gs);
+    free(idx);
+    free(chosen);
+    return 0;
+}
+
 #ifdef _OPENMP
 #include <omp.h>
 #endif

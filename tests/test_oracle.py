@@ -447,3 +447,89 @@ def test_fp8_path_tracks_the_exact_product():
     e8 = np.linalg.norm(oracle.linear_fp8(Xb, Wb, O.numpy())["y"] - exact) / np.linalg.norm(exact)
     e4 = np.linalg.norm(oracle.linear(Xb, Wb, O.numpy())["y"] - exact) / np.linalg.norm(exact)
     assert e8 < 0.05 and e8 < e4
+
+
+# ----------------------------------------------------------------- static outlier selection (write-up §5, §9; OSC)
+def _bf(t):
+    return workloads.bf16_bits(t.to(torch.bfloat16))
+
+
+def _f64(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _sel_case(Mc=300, K=256, N=96, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    X = torch.randn(Mc, K, generator=g)
+    W = torch.randn(N, K, generator=g) / 16
+    return X, W
+
+
+def test_selection_scores_match_library():
+    """score = mean |X| per column x L2 norm of the weight column (numpy, another summation order)."""
+    X, W = _sel_case(Mc=2500, N=1100)  # more than one 1024-row block on both sides
+    Xb, Wb = _bf(X), _bf(W)
+    O, sc = oracle.select_outliers(Xb, Wb, 16)
+    ref = np.mean(np.abs(_f64(Xb)), axis=0) * np.linalg.norm(_f64(Wb), axis=0)
+    assert np.allclose(sc, ref, rtol=1e-13, atol=0)
+    want = np.sort(np.argsort(-ref, kind="stable")[:16])
+    assert np.array_equal(O, want.astype(np.int32))
+
+
+def test_selection_finds_planted_channels():
+    """Channels amplified in the calibration activations, or whose weight column is
+    large, are selected; a large weight column with tiny activations is not."""
+    X, W = _sel_case(K=128, seed=1)
+    X[:, [7, 30, 101]] *= 40.0
+    W[:, 64] *= 50.0           # large weights, ordinary activations: contribution x50
+    W[:, 90] *= 50.0
+    X[:, 90] *= 1e-4           # ...but no activation: contribution tiny
+    O, _ = oracle.select_outliers(_bf(X), _bf(W), 4)
+    assert list(O) == [7, 30, 64, 101]
+
+
+def test_selection_ties_go_to_the_lower_index():
+    X, W = _sel_case(K=32, seed=2)
+    for c in (3, 9, 20):       # three identical, dominant columns
+        X[:, c] = X[:, 0] * 30.0
+        W[:, c] = W[:, 0]
+    O, sc = oracle.select_outliers(_bf(X), _bf(W), 2)
+    assert sc[3] == sc[9] == sc[20]
+    assert list(O) == [3, 9]
+
+
+def test_selection_group_aligned():
+    """Groups of G consecutive channels ranked by summed score; whole groups selected."""
+    X, W = _sel_case(K=256, seed=3)
+    X[:, 70] *= 50.0           # group 70 // 8 = 8
+    X[:, 200:203] *= 12.0      # group 25
+    Xb, Wb = _bf(X), _bf(W)
+    O, sc = oracle.select_outliers(Xb, Wb, 16, group=8)
+    gs = sc.reshape(-1, 8).sum(axis=1)
+    top = np.sort(np.argsort(-gs, kind="stable")[:2])
+    assert list(top) == [8, 25]
+    assert np.array_equal(O, np.concatenate([np.arange(64, 72), np.arange(200, 208)]).astype(np.int32))
+    with pytest.raises(ValueError):
+        oracle.select_outliers(Xb, Wb, 12, group=8)
+
+
+def test_selection_permutation_and_scaling_invariance():
+    X, W = _sel_case(K=192, seed=4)
+    Xb, Wb = _bf(X), _bf(W)
+    O, sc = oracle.select_outliers(Xb, Wb, 24)
+    perm = np.random.default_rng(5).permutation(192)
+    Op, scp = oracle.select_outliers(Xb[:, perm], Wb[:, perm], 24)
+    assert np.array_equal(scp, sc[perm])
+    assert np.array_equal(np.sort(perm[Op]), O)
+    # a power-of-two scale of X scales every score exactly and keeps the selection
+    O2, sc2 = oracle.select_outliers(_bf(X * 4.0), Wb, 24)
+    assert np.array_equal(sc2, 4.0 * sc) and np.array_equal(O2, O)
+
+
+def test_selection_edge_cases():
+    X, W = _sel_case(K=64, seed=6)
+    Xb, Wb = _bf(X), _bf(W)
+    O, _ = oracle.select_outliers(Xb, Wb, 0)
+    assert O.size == 0
+    O, _ = oracle.select_outliers(Xb, Wb, 64)
+    assert np.array_equal(O, np.arange(64, dtype=np.int32))
