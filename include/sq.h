@@ -230,6 +230,40 @@ sq_status sq_linear_fp8(const void *X, int64_t M, int64_t K, int64_t ldx,
                         int64_t N, int64_t nO, void *Y, int64_t ldy,
                         void *workspace, size_t ws_bytes, sq_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Static outlier-channel selection (the offline step that chooses O).
+ *
+ * SQ-format write-up of arXiv:2512.05409, section 5 (static strategy: mean
+ * activation per channel on calibration data) and section 9 (activation
+ * importance = activation times its contribution through the weights); OSC
+ * (arXiv:2604.12782) selects the outlier channels offline, group-wise.
+ *
+ *   score[k] = mean_m |Xc[m,k]| * ||W[:,k]||_2   (fp64)
+ *   O = the channels of the nO / group groups of `group` consecutive
+ *       channels with the largest summed score, ties to the lower index,
+ *       in ascending order.
+ *
+ * Row sums are taken in consecutive blocks of 1024 rows, each block summed in
+ * row order and the block sums added in block order; the result is therefore
+ * reproducible bit for bit.
+ *
+ *   Xc        calibration activations, bf16 [Mc, ldx] (dev), row-major
+ *   W         weights, bf16 [N, ldw] (dev), row-major
+ *   nO, group 0 <= nO <= K, group >= 1 divides K and nO
+ *   O         out: int32 [nO] (dev), ascending; feed it (copied to the host)
+ *             to sq_prepare_weights / sq_prepare_weights_fp8
+ *   scores    out (nullable): fp64 [K] (dev, 8-byte aligned)
+ *   workspace dev, ws_bytes >= sq_select_outliers_workspace_bytes(Mc, N, K, group)
+ * Asynchronous on `stream`; argument errors return SQ_ERR_INVALID_ARG before
+ * any launch.
+ * ------------------------------------------------------------------------ */
+size_t sq_select_outliers_workspace_bytes(int64_t Mc, int64_t N, int64_t K, int64_t group);
+
+sq_status sq_select_outliers(const void *Xc, int64_t Mc, int64_t K, int64_t ldx,
+                             const void *W, int64_t N, int64_t ldw,
+                             int64_t nO, int64_t group, int32_t *O, double *scores,
+                             void *workspace, size_t ws_bytes, sq_stream_t stream);
+
 /*
  * Waits for `stream`, then reports (and clears) the device error word of the
  * current device: SQ_ERR_TIMEOUT if a kernel's bounded wait ran out,

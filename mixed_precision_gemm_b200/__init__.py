@@ -35,7 +35,7 @@ __all__ = [
     "sq_status_string", "sq_kn_pad", "sq_no_pad", "sq_chan_table_words", "sq_linear_workspace_bytes",
     "sq_prepare_weights", "sq_quant_gather", "sq_gemm", "sq_linear", "sq_linear_noalloc", "sq_check",
     "sq_selftest_watchdog", "sq_linear_workspace_bytes_fp8", "sq_prepare_weights_fp8", "sq_quant_gather_fp8",
-    "sq_gemm_fp8", "sq_linear_fp8",
+    "sq_gemm_fp8", "sq_linear_fp8", "sq_select_outliers_workspace_bytes", "sq_select_outliers", "select_outliers",
     "PreparedWeights", "prepare_weights", "quant_gather", "gemm", "SQLinear",
 ]
 
@@ -102,9 +102,12 @@ def load():
     lib.sq_quant_gather_fp8.argtypes = [P, I, I, I, P, I, P, P, P, P]
     lib.sq_gemm_fp8.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P, P, P]
     lib.sq_linear_fp8.argtypes = [P, I, I, I, P, P, P, P, I, I, P, I, P, Z, P]
+    lib.sq_select_outliers_workspace_bytes.argtypes = [I, I, I, I]
+    lib.sq_select_outliers_workspace_bytes.restype = Z
+    lib.sq_select_outliers.argtypes = [P, I, I, I, P, I, I, I, I, P, P, P, Z, P]
     for f in (lib.sq_prepare_weights, lib.sq_quant_gather, lib.sq_gemm, lib.sq_linear, lib.sq_check,
               lib.sq_selftest_watchdog, lib.sq_linear_noalloc, lib.sq_prepare_weights_fp8, lib.sq_quant_gather_fp8,
-              lib.sq_gemm_fp8, lib.sq_linear_fp8):
+              lib.sq_gemm_fp8, lib.sq_linear_fp8, lib.sq_select_outliers):
         f.restype = F
     _lib = lib
     return lib
@@ -275,6 +278,25 @@ def sq_linear_fp8(X: torch.Tensor, chan_tab: torch.Tensor, W_N8, s_w, W_O, N: in
     _raise(st, "sq_linear_fp8")
 
 
+# Static outlier-channel selection (the offline step that chooses O).
+def sq_select_outliers_workspace_bytes(Mc: int, N: int, K: int, group: int = 1) -> int:
+    return int(load().sq_select_outliers_workspace_bytes(Mc, N, K, group))
+
+
+def sq_select_outliers(Xc: torch.Tensor, W: torch.Tensor, nO: int, group: int, O: Optional[torch.Tensor],
+                       scores: Optional[torch.Tensor], workspace: torch.Tensor, stream=None) -> None:
+    _rowmajor(Xc, "Xc", torch.bfloat16)
+    _rowmajor(W, "W", torch.bfloat16)
+    Mc, K = Xc.shape
+    N = W.shape[0]
+    if W.shape[1] != K:
+        raise ValueError("Xc and W disagree on K")
+    st = load().sq_select_outliers(_ptr(Xc), Mc, K, Xc.stride(0), _ptr(W), N, W.stride(0), nO, group, _ptr(O),
+                                   _ptr(scores), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _stream(stream))
+    _raise(st, "sq_select_outliers")
+
+
 def sq_check(stream=None) -> None:
     _raise(load().sq_check(_stream(stream)), "sq_check")
 
@@ -348,6 +370,19 @@ def gemm(X_N, s_x, X_O, pw: PreparedWeights, Y: Optional[torch.Tensor] = None, d
     (sq_gemm_fp8 if pw.fp8 else sq_gemm)(X_N, s_x, X_O, pw.W_N, pw.s_w, pw.W_O, M, pw.N, pw.K, pw.nO, Y, dbg_i, dbg_f,
                                          stream)
     return (Y, dbg_i, dbg_f) if debug else Y
+
+
+def select_outliers(Xc: torch.Tensor, W: torch.Tensor, nO: int, group: int = 1, stream=None):
+    """Static outlier channels from calibration activations Xc [Mc, K] and weights W [N, K]
+    (bf16, on the GPU): returns (O int32 [nO] ascending, scores float64 [K]), both on the device."""
+    dev = W.device
+    K = W.shape[1]
+    O = torch.zeros(nO, dtype=torch.int32, device=dev)
+    scores = torch.zeros(K, dtype=torch.float64, device=dev)
+    ws = torch.empty(max(256, sq_select_outliers_workspace_bytes(Xc.shape[0], W.shape[0], K, group)),
+                     dtype=torch.uint8, device=dev)
+    sq_select_outliers(Xc, W, nO, group, O, scores, ws, stream)
+    return O, scores
 
 
 class SQLinear:

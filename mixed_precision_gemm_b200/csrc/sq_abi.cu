@@ -21,6 +21,7 @@
 #include "sq_gemm_skinny.cuh"
 #include "sq_rowquant.cuh"
 #include "sq_rowquant_stream.cuh"
+#include "sq_select.cuh"
 
 namespace {
 
@@ -621,6 +622,69 @@ sq_status linear_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const ui
                         nullptr, nullptr, s, fp8);
 }
 
+// ---------------------------------------------------------------- static outlier selection
+struct SelectLayout {
+    int64_t nbx, nbw, off_px, off_pw, off_score, off_gs, bytes;
+    SelectLayout(int64_t Mc, int64_t N, int64_t K, int64_t group)
+    {
+        nbx = (Mc + sqs::kSelBlock - 1) / sqs::kSelBlock;
+        nbw = (N + sqs::kSelBlock - 1) / sqs::kSelBlock;
+        off_px = 0;
+        off_pw = round_up(nbx * K * 8, 256);
+        off_score = off_pw + round_up(nbw * K * 8, 256);
+        off_gs = off_score + round_up(K * 8, 256);
+        bytes = off_gs + round_up((group > 0 ? K / group : K) * 8, 256);
+    }
+};
+
+sq_status select_impl(const void *Xc, int64_t Mc, int64_t K, int64_t ldx, const void *W, int64_t N, int64_t ldw,
+                      int64_t nO, int64_t group, int32_t *O, double *scores, void *workspace, size_t ws_bytes,
+                      cudaStream_t s)
+{
+    if (K < 1 || K > SQ_MAX_K) return fail(SQ_ERR_INVALID_ARG, "K=%lld outside [1, %d]", (long long)K, SQ_MAX_K);
+    if (Mc < 1 || N < 1) return fail(SQ_ERR_INVALID_ARG, "Mc and N must be positive");
+    if ((Mc + sqs::kSelBlock - 1) / sqs::kSelBlock > 65535 || (N + sqs::kSelBlock - 1) / sqs::kSelBlock > 65535)
+        return fail(SQ_ERR_UNSUPPORTED, "more than 65535 blocks of %d rows", sqs::kSelBlock);
+    if (ldx < K || ldw < K) return fail(SQ_ERR_INVALID_ARG, "ldx and ldw must be >= K");
+    if (group < 1 || K % group != 0) return fail(SQ_ERR_INVALID_ARG, "group must divide K");
+    if (nO < 0 || nO > K || nO % group != 0) return fail(SQ_ERR_INVALID_ARG, "nO must lie in [0, K] and divide by group");
+    if (!Xc || !W) return fail(SQ_ERR_INVALID_ARG, "Xc or W is NULL");
+    if (nO > 0 && !O) return fail(SQ_ERR_INVALID_ARG, "O is NULL");
+    SQ_TRY(check_ptr(workspace, true, "workspace"));
+    if (scores && (reinterpret_cast<uintptr_t>(scores) & 7u)) return fail(SQ_ERR_MISALIGNED, "scores is not 8-byte aligned");
+    const SelectLayout L(Mc, N, K, group);
+    if (ws_bytes < static_cast<size_t>(L.bytes))
+        return fail(SQ_ERR_INVALID_ARG, "workspace of %zu bytes, %lld needed", ws_bytes, (long long)L.bytes);
+    DevInfo di;
+    SQ_TRY(device_info(di));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    double *px = reinterpret_cast<double *>(ws + L.off_px);
+    double *pw = reinterpret_cast<double *>(ws + L.off_pw);
+    double *sc = scores ? scores : reinterpret_cast<double *>(ws + L.off_score);
+    double *gs = reinterpret_cast<double *>(ws + L.off_gs);
+    const int k = static_cast<int>(K), ng = static_cast<int>(K / group);
+    const unsigned gk = static_cast<unsigned>((K + sqs::kColThreads - 1) / sqs::kColThreads);
+    cudaError_t e;
+    if ((e = launch_k(sqs::colsum_blocks_kernel, dim3(gk, static_cast<unsigned>(L.nbx)), dim3(sqs::kColThreads), 0, s,
+                      0u, static_cast<const uint16_t *>(Xc), Mc, k, ldx, 0, px)) != cudaSuccess)
+        return cuda_fail(e, "selection column sums (X)");
+    if ((e = launch_k(sqs::colsum_blocks_kernel, dim3(gk, static_cast<unsigned>(L.nbw)), dim3(sqs::kColThreads), 0, s,
+                      0u, static_cast<const uint16_t *>(W), N, k, ldw, 1, pw)) != cudaSuccess)
+        return cuda_fail(e, "selection column sums (W)");
+    if ((e = launch_k(sqs::score_kernel, dim3(gk), dim3(sqs::kColThreads), 0, s, 0u, static_cast<const double *>(px),
+                      static_cast<int>(L.nbx), Mc, static_cast<const double *>(pw), static_cast<int>(L.nbw), k, sc)) !=
+        cudaSuccess)
+        return cuda_fail(e, "selection scores");
+    if ((e = launch_k(sqs::group_score_kernel, dim3(static_cast<unsigned>((ng + sqs::kColThreads - 1) / sqs::kColThreads)),
+                      dim3(sqs::kColThreads), 0, s, 0u, static_cast<const double *>(sc), ng, static_cast<int>(group),
+                      gs)) != cudaSuccess)
+        return cuda_fail(e, "selection group scores");
+    if ((e = launch_k(sqs::select_top_kernel, dim3(1), dim3(sqs::kTopThreads), 0, s, 0u, static_cast<const double *>(gs),
+                      ng, static_cast<int>(nO / group), static_cast<int>(group), O)) != cudaSuccess)
+        return cuda_fail(e, "selection top-k");
+    return SQ_OK;
+}
+
 }  // namespace
 
 // ================================================================ C ABI
@@ -713,6 +777,21 @@ sq_status sq_linear_fp8(const void *X, int64_t M, int64_t K, int64_t ldx, const 
     g_detail.clear();
     return linear_impl(X, M, K, ldx, chan_tab, W_N8, s_w, W_O, N, nO, Y, ldy, workspace, ws_bytes,
                        reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+size_t sq_select_outliers_workspace_bytes(int64_t Mc, int64_t N, int64_t K, int64_t group)
+{
+    if (Mc < 1 || N < 1 || K < 1 || group < 1) return 0;
+    return static_cast<size_t>(SelectLayout(Mc, N, K, group).bytes);
+}
+
+sq_status sq_select_outliers(const void *Xc, int64_t Mc, int64_t K, int64_t ldx, const void *W, int64_t N, int64_t ldw,
+                             int64_t nO, int64_t group, int32_t *O, double *scores, void *workspace, size_t ws_bytes,
+                             sq_stream_t stream)
+{
+    g_detail.clear();
+    return select_impl(Xc, Mc, K, ldx, W, N, ldw, nO, group, O, scores, workspace, ws_bytes,
+                       reinterpret_cast<cudaStream_t>(stream));
 }
 
 sq_status sq_check(sq_stream_t stream)
