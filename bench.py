@@ -246,6 +246,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-rows", type=int, default=8, help="token rows per reference-arm step")
+    ap.add_argument("--select-calib-rows", type=int, default=0,
+                    help="also time the offline outlier selection on this many calibration rows (0: skip)")
     ap.add_argument("--low", default="int4", choices=["int4", "fp8"],
                     help="low path: INT4 (default) or FP8 E4M3 (the pages' fallback for the inputs of W2)")
     args = ap.parse_args()
@@ -416,6 +418,44 @@ def main():
     ms_e2e = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
     e2e_value = whole_job_tops(flops, ms_e2e, world)
 
+    # offline outlier selection (optional): each call after an L2 flush
+    select = None
+    if args.select_calib_rows > 0:
+        Rc = args.select_calib_rows
+        Xc = workloads.activations(Rc, K, O, w.x_kind, w.sigma, seed=workloads.SEED_X + 7).to(dev)
+        Wd = W.to(dev)
+        O_sel = torch.zeros(nO, dtype=torch.int32, device=dev)
+        sc_sel = torch.zeros(K, dtype=torch.float64, device=dev)
+        ws_sel = torch.empty(sq.sq_select_outliers_workspace_bytes(Rc, N, K, 1), dtype=torch.uint8, device=dev)
+        flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+        # one selection (five kernels) captured in a graph, replayed right
+        # behind an L2 flush so that no host launch gap enters the timing
+        sq.sq_select_outliers(Xc, Wd, nO, 1, O_sel, sc_sel, ws_sel, stream)
+        g_sel = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(g_sel, stream=cap):
+            sq.sq_select_outliers(Xc, Wd, nO, 1, O_sel, sc_sel, ws_sel, cap)
+        stream.wait_stream(cap)
+        times = []
+        for i in range(args.warmup + args.steps):
+            flush.fill_(i & 0xFF)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g_sel.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= args.warmup:
+                times.append(e0.elapsed_time(e1))
+        del g_sel
+        ms_sel = statistics.mean(times)
+        sel_bytes = 2.0 * Rc * K + 2.0 * N * K
+        select = {"bound": "hbm", "calib_rows": Rc, "ms": ms_sel, "algorithmic_bytes": sel_bytes,
+                  "achieved": sel_bytes / (ms_sel * 1e-3) / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                  "frac": sel_bytes / (ms_sel * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                  "l2": "flushed before each call", "timing": "one selection replayed from a CUDA graph"}
+        del flush, Wd, Xc
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tops, rows, secs, cores = time_oracle(w, O, X, W, args.cpu_seconds, fp8=fp8)
@@ -444,6 +484,8 @@ def main():
             "clocks": clocks,
             "gpu_launches": 2 * args.steps,
         }
+        if select is not None:
+            line["select_outliers"] = select
         print(json.dumps(line), flush=True)
 
     for s in sets:

@@ -243,7 +243,7 @@ sq_status sq_linear_fp8(const void *X, int64_t M, int64_t K, int64_t ldx,
  *       channels with the largest summed score, ties to the lower index,
  *       in ascending order.
  *
- * Row sums are taken in consecutive blocks of 1024 rows, each block summed in
+ * Row sums are taken in consecutive blocks of 256 rows, each block summed in
  * row order and the block sums added in block order; the result is therefore
  * reproducible bit for bit.
  *

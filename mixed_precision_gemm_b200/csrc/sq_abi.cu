@@ -665,12 +665,17 @@ sq_status select_impl(const void *Xc, int64_t Mc, int64_t K, int64_t ldx, const 
     const int k = static_cast<int>(K), ng = static_cast<int>(K / group);
     const unsigned gk = static_cast<unsigned>((K + sqs::kColThreads - 1) / sqs::kColThreads);
     cudaError_t e;
-    if ((e = launch_k(sqs::colsum_blocks_kernel, dim3(gk, static_cast<unsigned>(L.nbx)), dim3(sqs::kColThreads), 0, s,
-                      0u, static_cast<const uint16_t *>(Xc), Mc, k, ldx, 0, px)) != cudaSuccess)
-        return cuda_fail(e, "selection column sums (X)");
-    if ((e = launch_k(sqs::colsum_blocks_kernel, dim3(gk, static_cast<unsigned>(L.nbw)), dim3(sqs::kColThreads), 0, s,
-                      0u, static_cast<const uint16_t *>(W), N, k, ldw, 1, pw)) != cudaSuccess)
-        return cuda_fail(e, "selection column sums (W)");
+    auto colsums = [&](const void *A, int64_t rows, int64_t ld, int square, double *part, int64_t nb) {
+        const bool pair = K % 2 == 0 && ld % 2 == 0 && (reinterpret_cast<uintptr_t>(A) & 3u) == 0;
+        const unsigned g = static_cast<unsigned>((K / (pair ? 2 : 1) + sqs::kColThreads - 1) / sqs::kColThreads);
+        const dim3 grid(g, static_cast<unsigned>(nb));
+        return pair ? launch_k(sqs::colsum_blocks_kernel<true>, grid, dim3(sqs::kColThreads), 0, s, 0u,
+                               static_cast<const uint16_t *>(A), rows, k, ld, square, part)
+                    : launch_k(sqs::colsum_blocks_kernel<false>, grid, dim3(sqs::kColThreads), 0, s, 0u,
+                               static_cast<const uint16_t *>(A), rows, k, ld, square, part);
+    };
+    if ((e = colsums(Xc, Mc, ldx, 0, px, L.nbx)) != cudaSuccess) return cuda_fail(e, "selection column sums (X)");
+    if ((e = colsums(W, N, ldw, 1, pw, L.nbw)) != cudaSuccess) return cuda_fail(e, "selection column sums (W)");
     if ((e = launch_k(sqs::score_kernel, dim3(gk), dim3(sqs::kColThreads), 0, s, 0u, static_cast<const double *>(px),
                       static_cast<int>(L.nbx), Mc, static_cast<const double *>(pw), static_cast<int>(L.nbw), k, sc)) !=
         cudaSuccess)

@@ -12,7 +12,7 @@
 //
 // Row sums are defined block-wise: consecutive blocks of kSelBlock rows, each
 // summed in row order, then the block sums added in block order.  Kernel 1
-// computes one block sum per thread (one thread per channel and block, loads
+// computes the block sums (one thread per channel pair and block, loads
 // coalesced across channels), kernel 2 adds them in order and forms the score,
 // kernel 3 the group scores, kernel 4 (one CTA) selects by an 8-pass radix
 // select on the 64-bit score bits (non-negative doubles order like unsigned
@@ -25,36 +25,56 @@
 
 namespace sqs {
 
-constexpr int kSelBlock = 1024;   // rows per partial sum
+constexpr int kSelBlock = 256;    // rows per partial sum
 constexpr int kColThreads = 256;
 constexpr int kTopThreads = 1024;
+constexpr int kTopKeys = 16;      // keys per thread held in registers by the top-k kernel
 
 __device__ __forceinline__ double bf16_to_f64(uint16_t b) { return static_cast<double>(__uint_as_float(static_cast<uint32_t>(b) << 16)); }
 
 // part[b * K + k] = sum over rows [b*kSelBlock, ...) of |A[r,k]| (square = 0) or A[r,k]^2.
+// PAIR: each thread sums channels k and k+1 from one 4-byte load per row
+// (K and ld even, A 4-byte aligned), so more bytes are in flight per load.
+template <bool PAIR>
 __global__ void __launch_bounds__(kColThreads) colsum_blocks_kernel(const uint16_t *__restrict__ A, int64_t rows,
                                                                     int K, int64_t ld, int square,
                                                                     double *__restrict__ part)
 {
     sqd::pdl_launch_dependents();
     sqd::pdl_wait();
-    const int k = blockIdx.x * kColThreads + threadIdx.x;
+    constexpr int C = PAIR ? 2 : 1;
+    const int k = (blockIdx.x * kColThreads + threadIdx.x) * C;
     const int64_t r0 = static_cast<int64_t>(blockIdx.y) * kSelBlock;
     if (k >= K) return;
     const int64_t r1 = min(rows, r0 + kSelBlock);
-    const uint16_t *p = A + r0 * ld + k;
-    double acc = 0.0;
-    if (square) {
-#pragma unroll 8
-        for (int64_t r = r0; r < r1; ++r, p += ld) {
-            const double v = bf16_to_f64(__ldg(p));
-            acc = __dadd_rn(acc, __dmul_rn(v, v));
+    double a0 = 0.0, a1 = 0.0;
+    if constexpr (PAIR) {
+        const uint32_t *p = reinterpret_cast<const uint32_t *>(A + r0 * ld + k);
+        const int64_t step = ld / 2;
+#pragma unroll 32
+        for (int64_t r = r0; r < r1; ++r, p += step) {
+            const uint32_t w = __ldg(p);
+            const double v0 = static_cast<double>(__uint_as_float(w << 16));
+            const double v1 = static_cast<double>(__uint_as_float(w & 0xFFFF0000u));
+            if (square) {
+                a0 = __dadd_rn(a0, __dmul_rn(v0, v0));
+                a1 = __dadd_rn(a1, __dmul_rn(v1, v1));
+            } else {
+                a0 = __dadd_rn(a0, fabs(v0));
+                a1 = __dadd_rn(a1, fabs(v1));
+            }
         }
     } else {
-#pragma unroll 8
-        for (int64_t r = r0; r < r1; ++r, p += ld) acc = __dadd_rn(acc, fabs(bf16_to_f64(__ldg(p))));
+        const uint16_t *p = A + r0 * ld + k;
+#pragma unroll 16
+        for (int64_t r = r0; r < r1; ++r, p += ld) {
+            const double v = bf16_to_f64(__ldg(p));
+            a0 = __dadd_rn(a0, square ? __dmul_rn(v, v) : fabs(v));
+        }
     }
-    part[static_cast<int64_t>(blockIdx.y) * K + k] = acc;
+    double *out = part + static_cast<int64_t>(blockIdx.y) * K + k;
+    out[0] = a0;
+    if constexpr (PAIR) out[1] = a1;
 }
 
 // score[k] = (sum_b partX[b,k] / Mc) * sqrt(sum_b partW[b,k]), sums in block order.
@@ -130,25 +150,67 @@ __global__ void __launch_bounds__(kTopThreads) select_top_kernel(const double *_
 
     // 1. radix select, most significant byte first: the key T of the pick-th
     //    largest score, and how many keys equal to T are still to be taken.
+    //    Each thread keeps its keys (i = tid + j * kTopThreads) in registers
+    //    when they fit (ng <= kTopKeys * kTopThreads).
+    uint64_t kreg[kTopKeys];
+    const bool in_regs = ng <= kTopKeys * kTopThreads;
+#pragma unroll
+    for (int j = 0; j < kTopKeys; ++j) {
+        const int i = tid + j * kTopThreads;
+        kreg[j] = (in_regs && i < ng) ? __ldg(key + i) : 0ull;
+    }
     uint64_t prefix = 0, pmask = 0;
     int need = pick;
     if (pick > 0) {
         for (int d = 7; d >= 0; --d) {
             for (int i = tid; i < 256; i += kTopThreads) hist[i] = 0u;
             __syncthreads();
-            for (int i = tid; i < ng; i += kTopThreads) {
-                const uint64_t kv = __ldg(key + i);
-                if ((kv & pmask) == prefix) atomicAdd(&hist[(kv >> (8 * d)) & 255u], 1u);
+            // Neighbouring scores share their high bytes, so many keys fall in
+            // the same bin: lanes with equal bins add their count once.
+            auto count = [&](uint64_t kv, bool valid) {
+                const unsigned bin = (valid && (kv & pmask) == prefix) ? static_cast<unsigned>((kv >> (8 * d)) & 255u)
+                                                                        : 256u;
+                const unsigned same = __match_any_sync(0xFFFFFFFFu, bin);
+                if (bin < 256u && (tid & 31) == __ffs(same) - 1) atomicAdd(&hist[bin], static_cast<unsigned>(__popc(same)));
+            };
+            if (in_regs) {
+#pragma unroll
+                for (int j = 0; j < kTopKeys; ++j) count(kreg[j], tid + j * kTopThreads < ng);
+            } else {
+                for (int i0 = 0; i0 < ng; i0 += kTopThreads) {
+                    const int i = i0 + tid;
+                    count(i < ng ? __ldg(key + i) : 0ull, i < ng);
+                }
             }
             __syncthreads();
-            if (tid == 0) {
-                int cum = 0, v = 0;
-                for (v = 255; v > 0; --v) {
-                    if (cum + static_cast<int>(hist[v]) >= need) break;
-                    cum += static_cast<int>(hist[v]);
+            if (tid < 32) {
+                // Bins from the top: lane l holds bins 255-8l .. 248-8l.  The
+                // first bin v (from 255 down) whose count from 255 to v
+                // reaches `need` is the digit of T.
+                int c[8], sum = 0;
+#pragma unroll
+                for (int b = 0; b < 8; ++b) {
+                    c[b] = static_cast<int>(hist[255 - 8 * tid - b]);
+                    sum += c[b];
                 }
-                s_need = need - cum;
-                s_prefix = prefix | (static_cast<uint64_t>(v) << (8 * d));
+                int incl = sum;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+                    if (tid >= off) incl += y;
+                }
+                const int excl = incl - sum;
+                const unsigned hit = __ballot_sync(0xFFFFFFFFu, incl >= need);
+                const int owner = hit ? __ffs(hit) - 1 : 31;
+                if (tid == owner) {
+                    int cum = excl, b = 0;
+                    for (; b < 7; ++b) {
+                        if (cum + c[b] >= need) break;
+                        cum += c[b];
+                    }
+                    s_need = need - cum;
+                    s_prefix = prefix | (static_cast<uint64_t>(255 - 8 * tid - b) << (8 * d));
+                }
             }
             __syncthreads();
             need = s_need;

@@ -235,7 +235,7 @@ def linear_fp8(X_bits: np.ndarray, W_bits: np.ndarray, O, rows=None):
 
 
 # ---------------------------------------------------------------- static outlier selection
-SEL_BLOCK = 1024  # rows per partial sum in the score definition
+SEL_BLOCK = 256  # rows per partial sum in the score definition
 
 
 def select_outliers(X_bits: np.ndarray, W_bits: np.ndarray, nO: int, group: int = 1):

@@ -345,7 +345,7 @@ int orc_dual_linear_rows_fp8(const uint8_t *qx, const float *sx, const uint16_t 
  * order is part of the definition so that a parallel evaluation can match it
  * bit for bit.
  */
-#define ORC_SEL_BLOCK 1024
+#define ORC_SEL_BLOCK 256
 
 static double orc_blocked_col_sum(const uint16_t *A, int64_t rows, int64_t ld, int64_t k, int square)
 {

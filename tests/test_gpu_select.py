@@ -27,7 +27,7 @@ def run(X, W, nO, group=1):
 
 @pytest.mark.parametrize("Mc,K,N,nO,group", [
     (300, 256, 96, 16, 1),
-    (2500, 1024, 1100, 64, 1),      # several 1024-row blocks on both sides
+    (2500, 1024, 1100, 64, 1),      # several 256-row blocks on both sides
     (512, 4096, 6144, 256, 1),      # Llama-3-8B QKV weights, 512 calibration tokens
     (512, 14336, 1024, 1792, 8),    # down-projection width, group-aligned
     (64, 8192, 2048, 512, 64),

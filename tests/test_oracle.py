@@ -467,7 +467,7 @@ def _sel_case(Mc=300, K=256, N=96, seed=0):
 
 def test_selection_scores_match_library():
     """score = mean |X| per column x L2 norm of the weight column (numpy, another summation order)."""
-    X, W = _sel_case(Mc=2500, N=1100)  # more than one 1024-row block on both sides
+    X, W = _sel_case(Mc=2500, N=1100)  # several 256-row blocks on both sides
     Xb, Wb = _bf(X), _bf(W)
     O, sc = oracle.select_outliers(Xb, Wb, 16)
     ref = np.mean(np.abs(_f64(Xb)), axis=0) * np.linalg.norm(_f64(Wb), axis=0)
