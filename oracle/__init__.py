@@ -13,7 +13,10 @@ plus 16-bit branch GEMM, fused sum) and the SQ-format write-up of
 arXiv:2512.05409 (section 9: symmetric quantization, column reordering by the
 static mask).  The FP8 functions follow the same page's FP8 fallback for the
 inputs of W2 (E4M3 low path, scale = absolute maximum / 448; readings in the C
-file).
+file).  The MX functions follow the OSC abstract's fit with 4-bit
+micro-scaling hardware (and the SQ-format write-up, section 8, FP4 variant):
+the normal channels in MXFP4, blocks of 32 with an E8M0 scale each (readings
+in the C file).
 """
 from __future__ import annotations
 
@@ -64,6 +67,15 @@ def _load():
             lib.orc_quantize_rows_fp8.argtypes = [P, I, I, I, P, I, P, P, P]
             lib.orc_dual_linear_rows_fp8.argtypes = [P, P, P, I, P, P, P, I, I, I, P, P, P]
             lib.orc_select_outliers.argtypes = [P, I, I, I, P, I, I, I, I, P, P]
+            lib.orc_e2m1_encode_array.argtypes = [P, I, P]
+            lib.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+            lib.orc_e2m1_decode.restype = ctypes.c_double
+            lib.orc_mx_block_exponent.argtypes = [ctypes.c_double]
+            lib.orc_quantize_rows_mx.argtypes = [P, I, I, I, P, I, P, P, P]
+            lib.orc_dual_linear_rows_mx.argtypes = [P, P, P, I, P, P, P, I, I, I, P, P, P]
+            for f in (lib.orc_e2m1_encode_array, lib.orc_mx_block_exponent, lib.orc_quantize_rows_mx,
+                      lib.orc_dual_linear_rows_mx):
+                f.restype = ctypes.c_int
             for f in (lib.orc_validate_outliers, lib.orc_quantize_rows, lib.orc_pack_int4,
                       lib.orc_chan_table, lib.orc_dual_linear_rows, lib.orc_num_threads,
                       lib.orc_e4m3_encode_array, lib.orc_e4m3_decode_array, lib.orc_quantize_rows_fp8,
@@ -258,3 +270,116 @@ def select_outliers(X_bits: np.ndarray, W_bits: np.ndarray, nO: int, group: int 
     if rc != 0:
         raise ValueError("invalid sizes (group must divide K and nO)")
     return O, score
+
+
+# ---------------------------------------------------------------- micro-scaling FP4 (MXFP4) low path
+MX_BLOCK = 32      # entries per block scale
+E2M1_MAX = 6.0     # largest E2M1 magnitude
+
+
+def e2m1_encode(t) -> np.ndarray:
+    """E2M1 codes (uint8, sign bit 3) nearest to float64 values, ties to even, saturating at 6."""
+    t = np.ascontiguousarray(t, np.float64).reshape(-1)
+    out = np.zeros(t.size, np.uint8)
+    _load().orc_e2m1_encode_array(_ptr(t), t.size, _ptr(out))
+    return out
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    """float64 values of E2M1 codes (low 4 bits of each byte)."""
+    c = np.asarray(codes, np.uint8).reshape(-1)
+    lib = _load()
+    table = np.array([lib.orc_e2m1_decode(i) for i in range(16)], np.float64)
+    return table[c & 15]
+
+
+def mx_block_exponent(a: float) -> int:
+    """E of the block scale 2^E for a block with absolute maximum a (before the +127 bias)."""
+    return int(_load().orc_mx_block_exponent(float(a)))
+
+
+def quantize_rows_mx(src_bits: np.ndarray, K: int, O):
+    """MXFP4 quantize-and-gather of bf16 rows (uint16 bit patterns).
+
+    Returns (codes uint8 E2M1 [rows, K-nO] (one per byte), e8 uint8 [rows,
+    ceil((K-nO)/32)] E8M0 block scales, outl uint16 [rows, nO]).
+    """
+    src = np.ascontiguousarray(src_bits, dtype=np.uint16)
+    if src.ndim != 2 or src.shape[1] < K:
+        raise ValueError("src must be [rows, ld>=K]")
+    O = _as_O(O)
+    rows, ld = src.shape
+    KN = K - O.size
+    NB = (KN + MX_BLOCK - 1) // MX_BLOCK
+    codes = np.zeros((rows, KN), np.uint8)
+    e8 = np.zeros((rows, NB), np.uint8)
+    outl = np.zeros((rows, O.size), np.uint16)
+    rc = _load().orc_quantize_rows_mx(_ptr(src), rows, K, ld, _ptr(O), O.size,
+                                      _ptr(codes), _ptr(e8), _ptr(outl))
+    if rc != 0:
+        raise ValueError("invalid outlier channel set")
+    return codes, e8, outl
+
+
+def dual_linear_rows_mx(qx, ex, xo, qw, ew, wo):
+    """(acc_mx float64, acc_o float64, y float64), each [rows of qx, rows of qw]."""
+    qx = np.ascontiguousarray(qx, np.uint8)
+    qw = np.ascontiguousarray(qw, np.uint8)
+    ex = np.ascontiguousarray(ex, np.uint8)
+    ew = np.ascontiguousarray(ew, np.uint8)
+    xo = np.ascontiguousarray(xo, np.uint16)
+    wo = np.ascontiguousarray(wo, np.uint16)
+    Mr, KN = qx.shape
+    N = qw.shape[0]
+    nO = xo.shape[1]
+    NB = (KN + MX_BLOCK - 1) // MX_BLOCK
+    assert qw.shape[1] == KN and wo.shape == (N, nO) and xo.shape[0] == Mr
+    assert ex.shape == (Mr, NB) and ew.shape == (N, NB)
+    acc_mx = np.zeros((Mr, N), np.float64)
+    acc_o = np.zeros((Mr, N), np.float64)
+    y = np.zeros((Mr, N), np.float64)
+    _load().orc_dual_linear_rows_mx(_ptr(qx), _ptr(ex), _ptr(xo), Mr, _ptr(qw), _ptr(ew), _ptr(wo),
+                                    N, KN, nO, _ptr(acc_mx), _ptr(acc_o), _ptr(y))
+    return acc_mx, acc_o, y
+
+
+def linear_mx(X_bits: np.ndarray, W_bits: np.ndarray, O, rows=None):
+    """Whole layer with the MXFP4 low path for the selected activation rows (all when None)."""
+    K = W_bits.shape[1]
+    Xs = X_bits if rows is None else X_bits[np.asarray(rows)]
+    qx, ex, xo = quantize_rows_mx(Xs, K, O)
+    qw, ew, wo = quantize_rows_mx(W_bits, K, O)
+    acc_mx, acc_o, y = dual_linear_rows_mx(qx, ex, xo, qw, ew, wo)
+    return dict(qx=qx, ex=ex, xo=xo, qw=qw, ew=ew, wo=wo, acc_mx=acc_mx, acc_o=acc_o, y=y)
+
+
+def pack_fp4(codes: np.ndarray, row_bytes: int) -> np.ndarray:
+    """Packed storage of 4-bit codes: byte j = code 2j (low nibble) | code 2j+1 (high nibble), zero padded."""
+    codes = np.ascontiguousarray(codes, np.uint8)
+    rows, KN = codes.shape
+    if 2 * row_bytes < KN:
+        raise ValueError("row_bytes too small")
+    padded = np.zeros((rows, 2 * row_bytes), np.uint8)
+    padded[:, :KN] = codes & 15
+    return (padded[:, 0::2] | (padded[:, 1::2] << 4)).astype(np.uint8)
+
+
+def mx_scale_tiles(e8: np.ndarray, rows_pad: int, blocks_pad: int) -> np.ndarray:
+    """Block scales in the library's tiled storage order (format definition).
+
+    Rows are grouped by 128 and blocks by 4; each (row group, block group)
+    pair is a 512-byte tile in which row r and block b sit at byte
+    16*(r%32) + 4*((r%128)//32) + b%4.  Tiles are ordered by row group, then
+    block group.  Entries past the given rows and blocks are 0.
+    """
+    e8 = np.asarray(e8, np.uint8)
+    rows, nb = e8.shape
+    assert rows_pad % 128 == 0 and blocks_pad % 4 == 0 and rows <= rows_pad and nb <= blocks_pad
+    full = np.zeros((rows_pad, blocks_pad), np.uint8)
+    full[:rows, :nb] = e8
+    r = np.arange(rows_pad)[:, None]
+    b = np.arange(blocks_pad)[None, :]
+    off = ((r // 128) * (blocks_pad // 4) + b // 4) * 512 + 16 * (r % 32) + 4 * ((r % 128) // 32) + b % 4
+    out = np.zeros(rows_pad * blocks_pad, np.uint8)
+    out[off.reshape(-1)] = full.reshape(-1)
+    return out

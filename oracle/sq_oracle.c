@@ -328,6 +328,147 @@ int orc_dual_linear_rows_fp8(const uint8_t *qx, const float *sx, const uint16_t 
     return 0;
 }
 
+/* ------------------------------------------------------------------ micro-scaling FP4 low path
+ * OSC (arXiv:2604.12782), abstract: the channel split fits 4-bit
+ * micro-scaling hardware; SQ-format write-up of arXiv:2512.05409, section 8:
+ * the format also works with FP8/FP4 data types.  The pages name no block
+ * format, so the reading taken is the open MX definition of FP4 (MXFP4):
+ *   - the normal channels of a row, in ascending channel order, are cut into
+ *     blocks of 32 consecutive entries (j = 32b .. 32b+31; the last block may
+ *     be partial, the missing entries count as zero);
+ *   - every block has one power-of-two scale 2^E stored as an E8M0 byte
+ *     e8 = E + 127: E = floor(log2(a)) - 2 with a the block's absolute
+ *     maximum (2 is the largest exponent of E2M1), clamped to [-127, 127];
+ *     a == 0 gives E = -127 (byte 0);
+ *   - every entry becomes the E2M1 code (sign bit 3, exponent bits 2..1, bias
+ *     1, mantissa bit 0: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) nearest to
+ *     t = x / 2^E (exact), ties to the even code, magnitudes above 6
+ *     saturated to 6, the sign bit copied from x (so -0 and negative values
+ *     that round to zero give code 8);
+ *   - the outlier channels still run through the 16-bit branch, and
+ *     Y = sum_b 2^(Ex + Ew) * sum_{j in b} e(x_j) e(w_j) + sum_{k in O} X W.
+ * No per-row fp32 scale remains: both operands carry their block scales. */
+#define ORC_MX_BLOCK 32
+#define ORC_E2M1_MAX 6.0
+
+/* Value of an E2M1 code. */
+double orc_e2m1_decode(uint8_t code)
+{
+    const int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+    const double v = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return sign ? -v : v;
+}
+
+/* Nearest E2M1 code to t, ties to the even code (mantissa bit 0),
+ * saturating at 6; sign bit from t.  Codes 0..7 increase in value, so the
+ * neighbours of |t| are found by a linear scan. */
+uint8_t orc_e2m1_encode(double t)
+{
+    const uint8_t sign = signbit(t) ? 8 : 0;
+    const double v = fabs(t);
+    if (v >= ORC_E2M1_MAX) return (uint8_t)(sign | 7);
+    int lo = 0;
+    while (lo < 6 && orc_e2m1_decode((uint8_t)(lo + 1)) <= v) ++lo;
+    const int hi = lo + 1; /* decode(lo) <= v < decode(hi) */
+    const double dl = v - orc_e2m1_decode((uint8_t)lo), dh = orc_e2m1_decode((uint8_t)hi) - v;
+    const int code = (dl < dh) ? lo : (dh < dl) ? hi : ((lo % 2 == 0) ? lo : hi);
+    return (uint8_t)(sign | code);
+}
+
+int orc_e2m1_encode_array(const double *t, int64_t n, uint8_t *codes)
+{
+    for (int64_t i = 0; i < n; ++i) codes[i] = orc_e2m1_encode(t[i]);
+    return 0;
+}
+
+/* Block exponent E (before the E8M0 bias) of a block with absolute maximum a. */
+int orc_mx_block_exponent(double a)
+{
+    if (a == 0.0) return -127;
+    int e2;
+    frexp(a, &e2); /* a = f * 2^e2, f in [0.5, 1): floor(log2 a) = e2 - 1 */
+    int E = (e2 - 1) - 2;
+    if (E < -127) E = -127;
+    if (E > 127) E = 127;
+    return E;
+}
+
+/* Quantize-and-gather with the MXFP4 low path.
+ * Outputs (dense, caller-allocated):
+ *   codes [rows, K - nO]          one E2M1 code per byte (unpacked)
+ *   e8    [rows, ceil((K-nO)/32)] E8M0 block-scale bytes
+ *   outl  [rows, nO]              bf16 bit copies of the outlier channels */
+int orc_quantize_rows_mx(const uint16_t *src, int64_t rows, int64_t K, int64_t ld,
+                         const int32_t *O, int64_t nO,
+                         uint8_t *codes, uint8_t *e8, uint16_t *outl)
+{
+    if (orc_validate_outliers(O, nO, K) != 0 || ld < K) return -1;
+    const int64_t KN = K - nO, NB = (KN + ORC_MX_BLOCK - 1) / ORC_MX_BLOCK;
+    int64_t *normal = (int64_t *)malloc((size_t)(KN > 0 ? KN : 1) * sizeof(int64_t));
+    char *is_outlier = (char *)calloc((size_t)K, 1);
+    if (!normal || !is_outlier) { free(normal); free(is_outlier); return -1; }
+    for (int64_t j = 0; j < nO; ++j) is_outlier[O[j]] = 1;
+    for (int64_t k = 0, j = 0; k < K; ++k)
+        if (!is_outlier[k]) normal[j++] = k;
+
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *row = src + r * ld;
+        for (int64_t b = 0; b < NB; ++b) {
+            const int64_t j0 = b * ORC_MX_BLOCK;
+            const int64_t j1 = (j0 + ORC_MX_BLOCK < KN) ? j0 + ORC_MX_BLOCK : KN;
+            double a = 0.0;
+            for (int64_t j = j0; j < j1; ++j) {
+                const double v = fabs((double)orc_bf16_to_f32(row[normal[j]]));
+                if (v > a) a = v;
+            }
+            const int E = orc_mx_block_exponent(a);
+            e8[r * NB + b] = (uint8_t)(E + 127);
+            for (int64_t j = j0; j < j1; ++j) {
+                const double x = (double)orc_bf16_to_f32(row[normal[j]]);
+                codes[r * KN + j] = orc_e2m1_encode(ldexp(x, -E)); /* exact: a power-of-two rescale */
+            }
+        }
+        for (int64_t jo = 0; jo < nO; ++jo) outl[r * nO + jo] = row[O[jo]];
+    }
+    free(normal);
+    free(is_outlier);
+    return 0;
+}
+
+/* Dual-path products with the MXFP4 low path:
+ *   acc_mx [Mr, N]  sum over blocks of 2^(Ex+Ew) * (exact block sum of decoded
+ *                   E2M1 products), fp64, blocks in order
+ *   acc_o  [Mr, N]  16-bit branch, fp64
+ *   y      [Mr, N]  acc_mx + acc_o, fp64 */
+int orc_dual_linear_rows_mx(const uint8_t *qx, const uint8_t *ex, const uint16_t *xo, int64_t Mr,
+                            const uint8_t *qw, const uint8_t *ew, const uint16_t *wo, int64_t N,
+                            int64_t KN, int64_t nO,
+                            double *acc_mx, double *acc_o, double *y)
+{
+    const int64_t NB = (KN + ORC_MX_BLOCK - 1) / ORC_MX_BLOCK;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < Mr; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double amx = 0.0;
+            for (int64_t b = 0; b < NB; ++b) {
+                const int64_t j0 = b * ORC_MX_BLOCK;
+                const int64_t j1 = (j0 + ORC_MX_BLOCK < KN) ? j0 + ORC_MX_BLOCK : KN;
+                double s = 0.0;
+                for (int64_t j = j0; j < j1; ++j) s += orc_e2m1_decode(qx[m * KN + j]) * orc_e2m1_decode(qw[n * KN + j]);
+                amx += ldexp(s, ((int)ex[m * NB + b] - 127) + ((int)ew[n * NB + b] - 127));
+            }
+            double ao = 0.0;
+            for (int64_t j = 0; j < nO; ++j)
+                ao += (double)orc_bf16_to_f32(xo[m * nO + j]) * (double)orc_bf16_to_f32(wo[n * nO + j]);
+            acc_mx[m * N + n] = amx;
+            acc_o[m * N + n] = ao;
+            y[m * N + n] = amx + ao;
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------------ static outlier selection
  * SQ-format write-up of arXiv:2512.05409, section 5 (static strategy for
  * activations) and section 9 (importance scores): the mean activation of each
