@@ -44,6 +44,7 @@ import workloads  # noqa: E402
 DEFAULT_WORKLOAD = workloads.LLAMA8B_QKV.name
 METRIC = "dual-path W4A4+BF16 GEMM TOPS & % tensor peak; quant-gather HBM GB/s"
 INT8_PER_BF16 = 2.0   # nominal dense int8 (and fp8) : bf16 tensor rate on B200 (4.5 : 2.25 POPS)
+MXF4_PER_BF16 = 4.0   # nominal dense block-scaled fp4 : bf16 tensor rate on B200 (9 : 2.25 PFLOPS)
 
 
 # ----------------------------------------------------------------- helpers
@@ -78,15 +79,16 @@ def recorded_traffic(workload: str, kernel: str):
     return d.get("workloads", {}).get(workload, {}).get(kernel)
 
 
-def gemm_bytes(M, N, K, nO, cb=0.5):
-    """Algorithmic GEMM bytes; cb = bytes per low-path code (0.5 INT4, 1 E4M3)."""
+def gemm_bytes(M, N, K, nO, cb=0.5, rs=4):
+    """Algorithmic GEMM bytes; cb = bytes per low-path code (0.5 INT4, 1 E4M3,
+    0.5 + 1/32 E2M1 with its block scales), rs = row-scale bytes (4, or 0 for MX)."""
     KN = K - nO
-    return N * KN * cb + 2 * N * nO + 4 * N + M * KN * cb + 2 * M * nO + 4 * M + 2 * M * N
+    return N * KN * cb + 2 * N * nO + rs * N + M * KN * cb + 2 * M * nO + rs * M + 2 * M * N
 
 
-def quant_gather_bytes(M, K, nO, cb=0.5):
+def quant_gather_bytes(M, K, nO, cb=0.5, rs=4):
     KN = K - nO
-    return 2 * M * K + M * KN * cb + 2 * M * nO + 4 * M
+    return 2 * M * K + M * KN * cb + 2 * M * nO + rs * M
 
 
 class ClockSampler:
@@ -171,18 +173,20 @@ def whole_job_tops(ops_per_rank_step: float, ms_per_step_max: float, world: int)
 
 
 # ----------------------------------------------------------------- CPU oracle timing
-def oracle_fns(fp8: bool):
+def oracle_fns(low: str):
     import oracle
-    if fp8:
+    if low == "fp8":
         return oracle.quantize_rows_fp8, oracle.dual_linear_rows_fp8
+    if low == "mx":
+        return oracle.quantize_rows_mx, oracle.dual_linear_rows_mx
     return oracle.quantize_rows, oracle.dual_linear_rows
 
 
-def time_oracle(w, O, X, W, target_s: float, max_rows: int | None = None, fp8: bool = False):
+def time_oracle(w, O, X, W, target_s: float, max_rows: int | None = None, low: str = "int4"):
     """Time the oracle on a bounded sample of token rows (weights quantized beforehand,
     as the offline step is on the GPU side).  Returns (TOPS, rows, seconds, cores)."""
     import oracle
-    quantize, dual = oracle_fns(fp8)
+    quantize, dual = oracle_fns(low)
     Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
     O = O.numpy()
     qw, sw, wo = quantize(Wb, w.K, O)
@@ -206,7 +210,7 @@ def run_reference(args, w, rank, world):
         return 0
     O, X, W = workloads.make(w)
     import oracle
-    quantize, dual = oracle_fns(args.low == "fp8")
+    quantize, dual = oracle_fns(args.low)
     Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
     On = O.numpy()
     qw, sw, wo = quantize(Wb, w.K, On)
@@ -226,7 +230,7 @@ def run_reference(args, w, rank, world):
     sample = f"{rows} token rows of the workload per step (weights quantized before timing)"
     line = {"impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64" if args.low == "fp8" else "int64+f64",
+            "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64" if args.low == "int4" else "f64",
             "data": "synthetic", "config": {**w.describe(), "low_path": args.low},
             "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
@@ -248,8 +252,9 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=8, help="token rows per reference-arm step")
     ap.add_argument("--select-calib-rows", type=int, default=0,
                     help="also time the offline outlier selection on this many calibration rows (0: skip)")
-    ap.add_argument("--low", default="int4", choices=["int4", "fp8"],
-                    help="low path: INT4 (default) or FP8 E4M3 (the pages' fallback for the inputs of W2)")
+    ap.add_argument("--low", default="int4", choices=["int4", "fp8", "mx"],
+                    help="low path: INT4 (default), FP8 E4M3 (the pages' fallback for the inputs of W2) "
+                         "or MXFP4 (E2M1 with E8M0 block scales)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -278,28 +283,37 @@ def main():
     peaks = load_peaks()
     O, X, W = workloads.make(w)
     M, N, K, nO = w.M, w.N, w.K, w.nO
-    kn_pad, no_pad = sq.sq_kn_pad(K, nO), sq.sq_no_pad(nO)
+    no_pad = sq.sq_no_pad(nO)
 
     # Rotating input sets so that every step reads operands that are not L2-resident.
-    fp8 = args.low == "fp8"
-    cb = 1.0 if fp8 else 0.5  # bytes per low-path code
-    ws_bytes = sq.sq_linear_workspace_bytes_fp8 if fp8 else sq.sq_linear_workspace_bytes
-    quant_gather_fn = sq.sq_quant_gather_fp8 if fp8 else sq.sq_quant_gather
-    gemm_fn = sq.sq_gemm_fp8 if fp8 else sq.sq_gemm
-    linear_fn = sq.sq_linear_fp8 if fp8 else sq.sq_linear
+    fp8, mx = args.low == "fp8", args.low == "mx"
+    cb = 1.0 if fp8 else 0.5 + 1.0 / 32 if mx else 0.5  # bytes per low-path code (MX: with its block scale)
+    rs = 0 if mx else 4                                  # fp32 row-scale bytes per row
+    if mx:
+        ws_bytes = sq.sq_linear_workspace_bytes_mx
+        quant_gather_fn, linear_fn = sq.sq_quant_gather_mx, sq.sq_linear_mx
+
+        def gemm_fn(X_N, s_x, X_O, W_N, s_w, W_O, M_, N_, K_, nO_, Y, dbg_i, dbg_f, stream_):
+            sq.sq_gemm_mx(X_N, s_x, X_O, W_N, s_w, W_O, M_, N_, K_, nO_, Y, dbg_f, stream_)
+    else:
+        ws_bytes = sq.sq_linear_workspace_bytes_fp8 if fp8 else sq.sq_linear_workspace_bytes
+        quant_gather_fn = sq.sq_quant_gather_fp8 if fp8 else sq.sq_quant_gather
+        gemm_fn = sq.sq_gemm_fp8 if fp8 else sq.sq_gemm
+        linear_fn = sq.sq_linear_fp8 if fp8 else sq.sq_linear
     Xd = X.to(dev)
-    pw0 = sq.prepare_weights(W.to(dev), O, fp8=fp8)
+    pw0 = sq.prepare_weights(W.to(dev), O, fp8=fp8, mx=mx)
     foot = (2 * M * K + pw0.W_N.numel() + 2 * pw0.W_O.numel() + 4 * N + 2 * M * N + ws_bytes(M, K, nO))
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     n_sets = max(2, math.ceil(3 * l2 / foot))
     sets = []
     for i in range(n_sets):
         pw = pw0 if i == 0 else sq.PreparedWeights(N, K, nO, pw0.W_N.clone(), pw0.s_w.clone(), pw0.W_O.clone(),
-                                                      pw0.chan_tab.clone(), fp8)
+                                                      pw0.chan_tab.clone(), fp8, mx)
         sets.append({
             "X": Xd if i == 0 else Xd.clone(), "pw": pw,
             "X_N": torch.empty(M, pw0.code_bytes(K), dtype=torch.uint8, device=dev),
-            "s_x": torch.empty(M, dtype=torch.float32, device=dev),
+            "s_x": (torch.empty(max(16, sq.sq_mx_scale_bytes(M, K, nO)), dtype=torch.uint8, device=dev) if mx
+                    else torch.empty(M, dtype=torch.float32, device=dev)),
             "X_O": torch.empty(M, no_pad, dtype=torch.bfloat16, device=dev),
             "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
         })
@@ -369,13 +383,15 @@ def main():
     flops = 2.0 * M * N * K
     value = whole_job_tops(flops, ms_step, world)
 
-    # roofline of the GEMM: int8 path at 2x the bf16 peak, bf16 path at the bf16 peak (burst: timed alone)
+    # roofline of the GEMM: int8 / fp8 path at 2x the bf16 peak (block-scaled fp4 at 4x), bf16 path at
+    # the bf16 peak (burst: timed alone)
     p_bf = peaks["bf16_tflops"]
-    p_i8 = INT8_PER_BF16 * p_bf
+    low_ratio = MXF4_PER_BF16 if mx else INT8_PER_BF16
+    p_i8 = low_ratio * p_bf
     t_roof_s = (2.0 * M * N * (K - nO)) / (p_i8 * 1e12) + (2.0 * M * N * nO) / (p_bf * 1e12)
     peak_eff = flops / t_roof_s / 1e12
     gemm_tops = flops / (ms_gemm * 1e-3) / 1e12
-    g_bytes = gemm_bytes(M, N, K, nO, cb)
+    g_bytes = gemm_bytes(M, N, K, nO, cb, rs)
     t_hbm_s = g_bytes / (peaks["hbm_gbs"] * 1e9)
     if t_hbm_s > t_roof_s:
         # few tokens: the GEMM is bound by streaming the weights, not by the tensor cores
@@ -386,8 +402,8 @@ def main():
         gemm_roof = {"bound": "tensor", "achieved": gemm_tops, "peak": peak_eff, "unit": "TFLOP/s",
                      "frac": gemm_tops / peak_eff,
                      "peak_basis": f"{peaks['source']} bf16 {p_bf:.0f} TFLOP/s (burst), "
-                                   f"{'fp8' if fp8 else 'int8'} = {INT8_PER_BF16:g}x"}
-    qg_bytes = quant_gather_bytes(M, K, nO, cb)
+                                   f"{args.low if args.low != 'int4' else 'int8'} = {low_ratio:g}x"}
+    qg_bytes = quant_gather_bytes(M, K, nO, cb, rs)
     qg_gbs = qg_bytes / (ms_qg * 1e-3) / 1e9
 
     # end to end through sq_linear with pinned host buffers (copies inside the timed region)
@@ -458,7 +474,7 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tops, rows, secs, cores = time_oracle(w, O, X, W, args.cpu_seconds, fp8=fp8)
+        tops, rows, secs, cores = time_oracle(w, O, X, W, args.cpu_seconds, low=args.low)
         cpu = {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle",
                "sample": f"{rows} of {M} token rows x all {N} outputs ({secs:.1f} s; weights quantized beforehand)"}
 
@@ -467,7 +483,8 @@ def main():
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "e4m3*e4m3->f32 + bf16*bf16->f32" if fp8 else "s4*s4->s32 + bf16*bf16->f32",
+            "dtype": ("e4m3*e4m3->f32 + bf16*bf16->f32" if fp8 else
+                      "e2m1*e2m1 (e8m0 per 32)->f32 + bf16*bf16->f32" if mx else "s4*s4->s32 + bf16*bf16->f32"),
             "data": "synthetic",
             "config": {**w.describe(), "low_path": args.low, "parallelism": f"dp{world}" if world > 1 else "single",
                        "l2": f"{n_sets} rotating input sets of {foot / 1e6:.0f} MB (> L2 {l2 / 1e6:.0f} MB)",

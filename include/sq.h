@@ -231,6 +231,66 @@ sq_status sq_linear_fp8(const void *X, int64_t M, int64_t K, int64_t ldx,
                         void *workspace, size_t ws_bytes, sq_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Micro-scaling FP4 (MXFP4) low path.
+ *
+ * OSC (arXiv:2604.12782), abstract: the channel split fits 4-bit
+ * micro-scaling hardware; SQ-format write-up of arXiv:2512.05409, section 8:
+ * the format also works with FP4 data.  These calls run the normal channels
+ * as MXFP4 (the open MX block format: E2M1 codes, one E8M0 power-of-two scale
+ * per block of 32 normal channels) and keep the 16-bit branch:
+ *
+ *   Y[m,n] = sum_b 2^(Ex[m,b] + Ew[n,b]) * sum_{j in block b} e(X)[m,j] * e(W)[n,j]
+ *          + sum_{k in O} X[m,k] * W[n,k]
+ *
+ *   - Blocks: the normal channels of a row in ascending channel order, cut
+ *     into blocks of 32 (the last one may be partial).
+ *   - Scale: E = floor(log2 a) - 2 with a the block's absolute maximum,
+ *     clamped to [-127, 127] (a == 0 gives -127); stored as the byte E + 127.
+ *   - e(x) = the E2M1 code (sign bit 3; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6)
+ *     nearest to x / 2^E, ties to the even code, saturating at 6, the sign
+ *     kept (-0 and negative values that round to zero give code 8).
+ *   - Codes, [rows, kn_pad_mx / 2] bytes with kn_pad_mx = sq_kn_pad_mx(K, nO):
+ *     byte j = code 2j (low nibble) | code 2j+1 (high nibble); zero past K - nO.
+ *   - Scales, sq_mx_scale_bytes(rows, K, nO) bytes, in tiles of 128 rows x 4
+ *     blocks: row r, block b at byte ((r / 128) * (kn_pad_mx / 128) + b / 4)
+ *     * 512 + 16 * (r % 32) + 4 * ((r % 128) / 32) + b % 4; entries for rows
+ *     past the matrix and blocks past K - nO are 0.
+ *   - W_O, X_O and the channel table are as for INT4.
+ *   - The products run on the tensor cores (tcgen05 kind::mxf4, block
+ *     scales applied in hardware) and accumulate in fp32 together with the
+ *     16-bit branch; Y = bf16_rn(accumulator).
+ *   - dbg_acc (nullable, [M, N] fp32): that accumulator.
+ * Error behaviour, ownership and stream ordering are those of the INT4 calls.
+ * ------------------------------------------------------------------------ */
+int64_t sq_kn_pad_mx(int64_t K, int64_t nO);                   /* roundup(K - nO, 256) codes */
+size_t sq_mx_scale_bytes(int64_t rows, int64_t K, int64_t nO);  /* roundup(rows, 128) * kn_pad_mx / 32 */
+/* Workspace of sq_linear_mx: codes, scales and compact X_O, each 256-byte aligned. */
+size_t sq_linear_workspace_bytes_mx(int64_t M, int64_t K, int64_t nO);
+
+/* W_N4 dev u8 [N, kn_pad_mx / 2]; S_W dev u8 [sq_mx_scale_bytes(N, K, nO)];
+ * W_O and chan_tab as sq_prepare_weights.  Waits for its own work. */
+sq_status sq_prepare_weights_mx(const void *W, int64_t N, int64_t K, int64_t ldw,
+                                const int32_t *O, int64_t nO,
+                                void *W_N4, void *S_W, void *W_O, uint32_t *chan_tab,
+                                sq_stream_t stream);
+
+/* X_N4 dev u8 [M, kn_pad_mx / 2]; S_X dev u8 [sq_mx_scale_bytes(M, K, nO)]. */
+sq_status sq_quant_gather_mx(const void *X, int64_t M, int64_t K, int64_t ldx,
+                             const uint32_t *chan_tab, int64_t nO,
+                             void *X_N4, void *S_X, void *X_O, sq_stream_t stream);
+
+sq_status sq_gemm_mx(const void *X_N4, const void *S_X, const void *X_O,
+                     const void *W_N4, const void *S_W, const void *W_O,
+                     int64_t M, int64_t N, int64_t K, int64_t nO,
+                     void *Y, int64_t ldy, float *dbg_acc, sq_stream_t stream);
+
+sq_status sq_linear_mx(const void *X, int64_t M, int64_t K, int64_t ldx,
+                       const uint32_t *chan_tab,
+                       const void *W_N4, const void *S_W, const void *W_O,
+                       int64_t N, int64_t nO, void *Y, int64_t ldy,
+                       void *workspace, size_t ws_bytes, sq_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Static outlier-channel selection (the offline step that chooses O).
  *
  * SQ-format write-up of arXiv:2512.05409, section 5 (static strategy: mean

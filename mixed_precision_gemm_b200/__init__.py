@@ -16,7 +16,9 @@ Method: OSC (arXiv:2604.12782, abstract and technical framework) -- static
 outlier channels coalesced into a compact bf16 tensor for a 16-bit branch
 GEMM, all other channels through a 4-bit GEMM, results fused; SQ-format
 write-up of arXiv:2512.05409, sections 5 and 9 -- static mask chosen offline,
-symmetric quantization, weight columns reordered by the mask.
+symmetric quantization, weight columns reordered by the mask.  Two more low
+paths keep the same split: FP8 E4M3 (OSC's fallback for the inputs of W2)
+and MXFP4 (OSC abstract: the split fits 4-bit micro-scaling hardware).
 """
 from __future__ import annotations
 
@@ -35,7 +37,9 @@ __all__ = [
     "sq_status_string", "sq_kn_pad", "sq_no_pad", "sq_chan_table_words", "sq_linear_workspace_bytes",
     "sq_prepare_weights", "sq_quant_gather", "sq_gemm", "sq_linear", "sq_linear_noalloc", "sq_check",
     "sq_selftest_watchdog", "sq_linear_workspace_bytes_fp8", "sq_prepare_weights_fp8", "sq_quant_gather_fp8",
-    "sq_gemm_fp8", "sq_linear_fp8", "sq_select_outliers_workspace_bytes", "sq_select_outliers", "select_outliers",
+    "sq_gemm_fp8", "sq_linear_fp8", "sq_kn_pad_mx", "sq_mx_scale_bytes", "sq_linear_workspace_bytes_mx",
+    "sq_prepare_weights_mx", "sq_quant_gather_mx", "sq_gemm_mx", "sq_linear_mx",
+    "sq_select_outliers_workspace_bytes", "sq_select_outliers", "select_outliers",
     "PreparedWeights", "prepare_weights", "quant_gather", "gemm", "SQLinear",
 ]
 
@@ -102,12 +106,23 @@ def load():
     lib.sq_quant_gather_fp8.argtypes = [P, I, I, I, P, I, P, P, P, P]
     lib.sq_gemm_fp8.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P, P, P]
     lib.sq_linear_fp8.argtypes = [P, I, I, I, P, P, P, P, I, I, P, I, P, Z, P]
+    lib.sq_kn_pad_mx.argtypes = [I, I]
+    lib.sq_kn_pad_mx.restype = I
+    lib.sq_mx_scale_bytes.argtypes = [I, I, I]
+    lib.sq_mx_scale_bytes.restype = Z
+    lib.sq_linear_workspace_bytes_mx.argtypes = [I, I, I]
+    lib.sq_linear_workspace_bytes_mx.restype = Z
+    lib.sq_prepare_weights_mx.argtypes = [P, I, I, I, P, I, P, P, P, P, P]
+    lib.sq_quant_gather_mx.argtypes = [P, I, I, I, P, I, P, P, P, P]
+    lib.sq_gemm_mx.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P, P]
+    lib.sq_linear_mx.argtypes = [P, I, I, I, P, P, P, P, I, I, P, I, P, Z, P]
     lib.sq_select_outliers_workspace_bytes.argtypes = [I, I, I, I]
     lib.sq_select_outliers_workspace_bytes.restype = Z
     lib.sq_select_outliers.argtypes = [P, I, I, I, P, I, I, I, I, P, P, P, Z, P]
     for f in (lib.sq_prepare_weights, lib.sq_quant_gather, lib.sq_gemm, lib.sq_linear, lib.sq_check,
               lib.sq_selftest_watchdog, lib.sq_linear_noalloc, lib.sq_prepare_weights_fp8, lib.sq_quant_gather_fp8,
-              lib.sq_gemm_fp8, lib.sq_linear_fp8, lib.sq_select_outliers):
+              lib.sq_gemm_fp8, lib.sq_linear_fp8, lib.sq_select_outliers, lib.sq_prepare_weights_mx,
+              lib.sq_quant_gather_mx, lib.sq_gemm_mx, lib.sq_linear_mx):
         f.restype = F
     _lib = lib
     return lib
@@ -278,6 +293,61 @@ def sq_linear_fp8(X: torch.Tensor, chan_tab: torch.Tensor, W_N8, s_w, W_O, N: in
     _raise(st, "sq_linear_fp8")
 
 
+# MXFP4 low path (OSC abstract: 4-bit micro-scaling hardware): packed E2M1
+# codes (u8 [rows, kn_pad_mx / 2]) with tiled E8M0 block scales (u8
+# [sq_mx_scale_bytes(rows, K, nO)]) in place of the fp32 row scales.
+def sq_kn_pad_mx(K: int, nO: int) -> int:
+    return int(load().sq_kn_pad_mx(K, nO))
+
+
+def sq_mx_scale_bytes(rows: int, K: int, nO: int) -> int:
+    return int(load().sq_mx_scale_bytes(rows, K, nO))
+
+
+def sq_linear_workspace_bytes_mx(M: int, K: int, nO: int) -> int:
+    return int(load().sq_linear_workspace_bytes_mx(M, K, nO))
+
+
+def sq_prepare_weights_mx(W: torch.Tensor, O, W_N4: torch.Tensor, S_W: torch.Tensor, W_O: Optional[torch.Tensor],
+                          chan_tab: torch.Tensor, stream=None) -> None:
+    _rowmajor(W, "W", torch.bfloat16)
+    N, K = W.shape
+    O_host = torch.as_tensor(O, dtype=torch.int32).reshape(-1).contiguous().cpu()
+    nO = O_host.numel()
+    st = load().sq_prepare_weights_mx(_ptr(W), N, K, W.stride(0),
+                                      ctypes.c_void_p(O_host.data_ptr()) if nO else None, nO,
+                                      _ptr(W_N4), _ptr(S_W), _ptr(W_O), _ptr(chan_tab), _stream(stream))
+    _raise(st, "sq_prepare_weights_mx")
+
+
+def sq_quant_gather_mx(X: torch.Tensor, chan_tab: torch.Tensor, nO: int, X_N4: Optional[torch.Tensor],
+                       S_X: Optional[torch.Tensor], X_O: Optional[torch.Tensor], stream=None) -> None:
+    _rowmajor(X, "X", torch.bfloat16)
+    M, K = X.shape
+    st = load().sq_quant_gather_mx(_ptr(X), M, K, X.stride(0), _ptr(chan_tab), nO, _ptr(X_N4), _ptr(S_X),
+                                   _ptr(X_O), _stream(stream))
+    _raise(st, "sq_quant_gather_mx")
+
+
+def sq_gemm_mx(X_N4, S_X, X_O, W_N4, S_W, W_O, M: int, N: int, K: int, nO: int, Y: torch.Tensor,
+               dbg_acc: Optional[torch.Tensor] = None, stream=None) -> None:
+    _rowmajor(Y, "Y", torch.bfloat16)
+    st = load().sq_gemm_mx(_ptr(X_N4), _ptr(S_X), _ptr(X_O), _ptr(W_N4), _ptr(S_W), _ptr(W_O), M, N, K, nO,
+                           _ptr(Y), Y.stride(0), _ptr(dbg_acc), _stream(stream))
+    _raise(st, "sq_gemm_mx")
+
+
+def sq_linear_mx(X: torch.Tensor, chan_tab: torch.Tensor, W_N4, S_W, W_O, N: int, nO: int, Y: torch.Tensor,
+                 workspace: torch.Tensor, stream=None) -> None:
+    _rowmajor(X, "X", torch.bfloat16)
+    _rowmajor(Y, "Y", torch.bfloat16)
+    M, K = X.shape
+    st = load().sq_linear_mx(_ptr(X), M, K, X.stride(0), _ptr(chan_tab), _ptr(W_N4), _ptr(S_W), _ptr(W_O), N, nO,
+                             _ptr(Y), Y.stride(0), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream(stream))
+    _raise(st, "sq_linear_mx")
+
+
 # Static outlier-channel selection (the offline step that chooses O).
 def sq_select_outliers_workspace_bytes(Mc: int, N: int, K: int, group: int = 1) -> int:
     return int(load().sq_select_outliers_workspace_bytes(Mc, N, K, group))
@@ -312,57 +382,80 @@ class PreparedWeights:
     N: int
     K: int
     nO: int
-    W_N: torch.Tensor        # uint8 [N, kn_pad/2] packed INT4, or [N, kn_pad] E4M3 when fp8
-    s_w: torch.Tensor        # float32 [N]
+    W_N: torch.Tensor        # uint8 [N, kn_pad/2] packed INT4, [N, kn_pad] E4M3 (fp8), [N, kn_pad_mx/2] E2M1 (mx)
+    s_w: torch.Tensor        # float32 [N]; mx: uint8 [sq_mx_scale_bytes(N, K, nO)] tiled E8M0 block scales
     W_O: torch.Tensor        # bf16 [N, no_pad]
     chan_tab: torch.Tensor   # int32 view of uint32 [K/8]
     fp8: bool = False        # low path in FP8 E4M3 (the W2 fallback) instead of INT4
+    mx: bool = False         # low path in MXFP4 (E2M1 + E8M0 block scales) instead of INT4
 
     def state_dict(self) -> dict:
         return {"N": self.N, "K": self.K, "nO": self.nO, "W_N": self.W_N, "s_w": self.s_w,
-                "W_O": self.W_O, "chan_tab": self.chan_tab, "fp8": self.fp8}
+                "W_O": self.W_O, "chan_tab": self.chan_tab, "fp8": self.fp8, "mx": self.mx}
 
     @classmethod
     def from_state_dict(cls, d: dict, device=None) -> "PreparedWeights":
         mv = (lambda t: t.to(device)) if device is not None else (lambda t: t)
         return cls(int(d["N"]), int(d["K"]), int(d["nO"]), mv(d["W_N"]), mv(d["s_w"]), mv(d["W_O"]),
-                   mv(d["chan_tab"]), bool(d.get("fp8", False)))
+                   mv(d["chan_tab"]), bool(d.get("fp8", False)), bool(d.get("mx", False)))
 
     def code_bytes(self, K: int) -> int:
+        if self.mx:
+            return sq_kn_pad_mx(K, self.nO) // 2
         kn = sq_kn_pad(K, self.nO)
         return kn if self.fp8 else kn // 2
 
 
-def prepare_weights(W: torch.Tensor, O: Sequence[int], stream=None, fp8: bool = False) -> PreparedWeights:
-    """Offline weight step; fp8=True prepares the FP8 (E4M3) low path instead of INT4."""
+def prepare_weights(W: torch.Tensor, O: Sequence[int], stream=None, fp8: bool = False,
+                    mx: bool = False) -> PreparedWeights:
+    """Offline weight step; fp8=True prepares the FP8 (E4M3) low path, mx=True
+    the MXFP4 one, instead of INT4."""
+    if fp8 and mx:
+        raise ValueError("choose one low path")
     N, K = W.shape
     nO = len(torch.as_tensor(O).reshape(-1))
     dev = W.device
+    W_O = torch.zeros(N, sq_no_pad(nO), dtype=torch.bfloat16, device=dev)
+    tab = torch.zeros(sq_chan_table_words(K), dtype=torch.int32, device=dev)
+    if mx:
+        W_N = torch.zeros(N, sq_kn_pad_mx(K, nO) // 2, dtype=torch.uint8, device=dev)
+        S_W = torch.zeros(max(sq_mx_scale_bytes(N, K, nO), 16), dtype=torch.uint8, device=dev)
+        sq_prepare_weights_mx(W, O, W_N, S_W, W_O, tab, stream)
+        return PreparedWeights(N, K, nO, W_N, S_W, W_O, tab, False, True)
     kn = sq_kn_pad(K, nO)
     W_N = torch.zeros(N, kn if fp8 else kn // 2, dtype=torch.uint8, device=dev)
     s_w = torch.zeros(N, dtype=torch.float32, device=dev)
-    W_O = torch.zeros(N, sq_no_pad(nO), dtype=torch.bfloat16, device=dev)
-    tab = torch.zeros(sq_chan_table_words(K), dtype=torch.int32, device=dev)
     (sq_prepare_weights_fp8 if fp8 else sq_prepare_weights)(W, O, W_N, s_w, W_O, tab, stream)
     return PreparedWeights(N, K, nO, W_N, s_w, W_O, tab, fp8)
 
 
 def quant_gather(X: torch.Tensor, pw: PreparedWeights, stream=None):
+    """Online step: (X_N, s_x, X_O).  For the MX path s_x is the tiled E8M0
+    block-scale buffer (uint8)."""
     M, K = X.shape
     dev = X.device
     X_N = torch.empty(M, pw.code_bytes(K), dtype=torch.uint8, device=dev)
-    s_x = torch.empty(M, dtype=torch.float32, device=dev)
     X_O = torch.empty(M, sq_no_pad(pw.nO), dtype=torch.bfloat16, device=dev)
+    if pw.mx:
+        S_X = torch.empty(max(sq_mx_scale_bytes(M, K, pw.nO), 16), dtype=torch.uint8, device=dev)
+        sq_quant_gather_mx(X, pw.chan_tab, pw.nO, X_N, S_X, X_O, stream)
+        return X_N, S_X, X_O
+    s_x = torch.empty(M, dtype=torch.float32, device=dev)
     (sq_quant_gather_fp8 if pw.fp8 else sq_quant_gather)(X, pw.chan_tab, pw.nO, X_N, s_x, X_O, stream)
     return X_N, s_x, X_O
 
 
 def gemm(X_N, s_x, X_O, pw: PreparedWeights, Y: Optional[torch.Tensor] = None, debug: bool = False, stream=None):
     """Dual GEMM.  With debug=True also returns the two accumulators: the low
-    path's (int32 for INT4, fp32 for FP8) and the bf16 branch's (fp32)."""
-    M = s_x.shape[0]
+    path's (int32 for INT4, fp32 for FP8) and the bf16 branch's (fp32).  For
+    the MX path the two share one fp32 accumulator, returned as (Y, None, acc)."""
+    M = X_N.shape[0]
     if Y is None:
-        Y = torch.empty(M, pw.N, dtype=torch.bfloat16, device=s_x.device)
+        Y = torch.empty(M, pw.N, dtype=torch.bfloat16, device=X_N.device)
+    if pw.mx:
+        acc = torch.empty(M, pw.N, dtype=torch.float32, device=X_N.device) if debug else None
+        sq_gemm_mx(X_N, s_x, X_O, pw.W_N, pw.s_w, pw.W_O, M, pw.N, pw.K, pw.nO, Y, acc, stream)
+        return (Y, None, acc) if debug else Y
     dbg_i = dbg_f = None
     if debug:
         dbg_i = torch.empty(M, pw.N, dtype=torch.float32 if pw.fp8 else torch.int32, device=s_x.device)
@@ -388,14 +481,17 @@ def select_outliers(Xc: torch.Tensor, W: torch.Tensor, nO: int, group: int = 1, 
 class SQLinear:
     """A prepared dual-path linear layer: ``y = layer(x)`` for bf16 x [M, K] on the GPU.
 
-    fp8=True runs the low path in FP8 E4M3 (OSC's fallback for the inputs of W2)."""
+    fp8=True runs the low path in FP8 E4M3 (OSC's fallback for the inputs of W2);
+    mx=True runs it in MXFP4 (E2M1 codes, E8M0 scales per 32 channels)."""
 
-    def __init__(self, W: torch.Tensor, O: Sequence[int], stream=None, fp8: bool = False):
-        self.weights = prepare_weights(W, O, stream, fp8)
+    def __init__(self, W: torch.Tensor, O: Sequence[int], stream=None, fp8: bool = False, mx: bool = False):
+        self.weights = prepare_weights(W, O, stream, fp8, mx)
         self._ws = None
 
     def workspace(self, M: int, device) -> torch.Tensor:
-        ws_fn = sq_linear_workspace_bytes_fp8 if self.weights.fp8 else sq_linear_workspace_bytes
+        pw = self.weights
+        ws_fn = (sq_linear_workspace_bytes_mx if pw.mx else
+                 sq_linear_workspace_bytes_fp8 if pw.fp8 else sq_linear_workspace_bytes)
         need = ws_fn(M, self.weights.K, self.weights.nO)
         if self._ws is None or self._ws.numel() < need or self._ws.device != torch.device(device):
             self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
@@ -406,6 +502,6 @@ class SQLinear:
         M = X.shape[0]
         if out is None:
             out = torch.empty(M, pw.N, dtype=torch.bfloat16, device=X.device)
-        (sq_linear_fp8 if pw.fp8 else sq_linear)(X, pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, pw.N, pw.nO, out,
-                                                 self.workspace(M, X.device), stream)
+        fn = sq_linear_mx if pw.mx else sq_linear_fp8 if pw.fp8 else sq_linear
+        fn(X, pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, pw.N, pw.nO, out, self.workspace(M, X.device), stream)
         return out

@@ -19,6 +19,7 @@
 #include "sq_gemm_common.cuh"
 #include "sq_gemm_pair.cuh"
 #include "sq_gemm_skinny.cuh"
+#include "sq_mxquant.cuh"
 #include "sq_rowquant.cuh"
 #include "sq_rowquant_stream.cuh"
 #include "sq_select.cuh"
@@ -314,23 +315,37 @@ int raster_group(int tiles_m, int tile_rows, int64_t kn_pad, int64_t no_pad)
 }
 
 // Pair (cta_group::2) kernel: 256 x 256 tiles over clusters of two CTAs.
-// FP8: E4M3 low path (kn_pad bytes per row, tiles loaded straight into the
-// operand ring with the 128-byte swizzle); otherwise packed INT4 (kn_pad / 2
-// bytes per row, 64-byte staging boxes).
-template <class C, bool FP8>
+// kLowFp8: E4M3 low path (kn_pad bytes per row, tiles loaded straight into
+// the operand ring with the 128-byte swizzle).  kLowMx: packed E2M1 (kn_pad /
+// 2 bytes per row, kn_pad = sq_kn_pad_mx, 128-byte boxes of 256 codes, also
+// straight into the ring) plus the tiled E8M0 scales S_X / S_W (passed in
+// place of s_x / s_w), read as rows of 128 bytes, 8 rows (two tiles) per box.
+// kLowInt4: packed INT4 (kn_pad / 2 bytes per row, 64-byte staging boxes).
+template <class C, int LOW>
 sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O, const void *W_N,
                              const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y,
                              int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
 {
-    const int64_t kn_pad = sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
-    CUtensorMap m_xo{}, m_wo{}, m_xn{}, m_wn{};
+    constexpr bool FP8 = LOW == sqg::kLowFp8, MX = LOW == sqg::kLowMx;
+    const int64_t kn_pad = MX ? sq_kn_pad_mx(K, nO) : sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
+    CUtensorMap m_xo{}, m_wo{}, m_xn{}, m_wn{}, m_sx{}, m_sw{};
     sq_status st;
     if (kn_pad > 0) {
         const int64_t rb = FP8 ? kn_pad : kn_pad / 2;
-        const uint32_t box = FP8 ? sqg::KB_I8 : sqg::PROWB;
-        const CUtensorMapSwizzle swz = FP8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
+        const uint32_t box = (FP8 || MX) ? 128u : static_cast<uint32_t>(sqg::PROWB);
+        const CUtensorMapSwizzle swz = (FP8 || MX) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE;
         if ((st = make_map(m_xn, X_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, rb, M, rb, box, 128, swz)) != SQ_OK) return st;
         if ((st = make_map(m_wn, W_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, rb, N, rb, box, 128, swz)) != SQ_OK) return st;
+        if (MX) {
+            const uint64_t sx_rows = static_cast<uint64_t>(sq_mx_scale_bytes(M, K, nO) / 128);
+            const uint64_t sw_rows = static_cast<uint64_t>(sq_mx_scale_bytes(N, K, nO) / 128);
+            if ((st = make_map(m_sx, s_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, sx_rows, 128, 128, 8,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
+                return st;
+            if ((st = make_map(m_sw, s_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, sw_rows, 128, 128, 8,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
+                return st;
+        }
     }
     if (no_pad > 0) {
         if ((st = make_map(m_xo, X_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, M, no_pad * 2, sqg::KB_BF, 128,
@@ -349,21 +364,22 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
     a.M = static_cast<int>(M);
     a.N = static_cast<int>(N);
     a.ldy = ldy;
-    a.nkb_i = static_cast<int>(kn_pad / sqg::KB_I8);
+    a.nkb_i = static_cast<int>(kn_pad / (MX ? sqg::KB_MX : sqg::KB_I8));
     a.nkb_o = static_cast<int>(no_pad / sqg::KB_BF);
+    if (MX) a.s_x = a.s_w = nullptr;
     a.tiles_m = static_cast<int>((M + sqg::PAIR_BM - 1) / sqg::PAIR_BM);
     a.tiles_n = static_cast<int>((N + sqg::PAIR_BN - 1) / sqg::PAIR_BN);
     a.group_m = raster_group(a.tiles_m, sqg::PAIR_BM, kn_pad, no_pad);
     const int64_t ntiles = static_cast<int64_t>(a.tiles_m) * a.tiles_n;
     const int64_t clusters = std::min<int64_t>(ntiles, di.sms / 2);
     const bool dbg = dbg_i || dbg_f;
-    auto kern = dbg ? sqg::dual_gemm_pair_kernel<C, true, FP8> : sqg::dual_gemm_pair_kernel<C, false, FP8>;
+    auto kern = dbg ? sqg::dual_gemm_pair_kernel<C, true, LOW> : sqg::dual_gemm_pair_kernel<C, false, LOW>;
     int per_sm = 0;
     if ((st = kernel_setup(reinterpret_cast<const void *>(kern), sqg::PAIR_THREADS, C::SMEM_BYTES, per_sm, "gemm pair set-up")) != SQ_OK)
         return st;
     cudaError_t e;
     if ((e = launch_k(kern, dim3(static_cast<unsigned>(2 * clusters)), dim3(sqg::PAIR_THREADS), C::SMEM_BYTES, stream, 0u,
-                      m_xo, m_wo, m_xn, m_wn, a)) != cudaSuccess)
+                      m_xo, m_wo, m_xn, m_wn, m_sx, m_sw, a)) != cudaSuccess)
         return cuda_fail(e, "gemm pair launch");
     return SQ_OK;
 }
@@ -431,6 +447,7 @@ sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *
 
 using CfgPair = sqg::CfgPair<4, 4, 2>;
 using CfgPairF8 = sqg::CfgPair<6, 0, 2>;  // E4M3 tiles need no staging ring: a deeper operand ring instead
+using CfgPairMx = sqg::CfgPair<6, 0, 2, sqg::MX_SF_BYTES>;  // E2M1 tiles plus their block scales
 using CfgSk16 = sqg::CfgSkinny<16, 8, 3>;
 using CfgSk32 = sqg::CfgSkinny<32, 7, 3>;
 using CfgSk64 = sqg::CfgSkinny<64, 6, 2>;
@@ -444,7 +461,7 @@ sq_status gemm_dispatch(const DevInfo &di, const void *X_N, const float *s_x, co
 {
     using Pair = typename std::conditional<FP8, CfgPairF8, CfgPair>::type;
     if (M > 128)
-        return launch_gemm_pair_t<Pair, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+        return launch_gemm_pair_t<Pair, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (M <= 16)
         return launch_gemm_skinny_t<CfgSk16, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (M <= 32)
@@ -559,6 +576,35 @@ size_t linear_ws_bytes(int64_t M, int64_t K, int64_t nO, bool fp8)
     return static_cast<size_t>(xn + sx + xo);
 }
 
+// O: host list, already validated.  Static channel table: one word per 8
+// channels, (outliers below) << 8 | outlier bits; copied on stream s from a
+// host vector that lives until the caller synchronizes.
+sq_status upload_chan_table(const int32_t *O, int64_t nO, int64_t K, uint32_t *chan_tab, cudaStream_t s)
+{
+    static thread_local std::vector<uint32_t> tab;
+    tab.assign(static_cast<size_t>(K / 8), 0u);
+    for (int64_t j = 0; j < nO; ++j) tab[O[j] / 8] |= 1u << (O[j] % 8);
+    uint32_t below = 0;
+    for (int64_t c = 0; c < K / 8; ++c) {
+        const uint32_t mask = tab[c];
+        tab[c] = (below << 8) | mask;
+        below += static_cast<uint32_t>(__builtin_popcount(mask));
+    }
+    cudaError_t e = cudaMemcpyAsync(chan_tab, tab.data(), tab.size() * sizeof(uint32_t), cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "copy of the channel table");
+    return SQ_OK;
+}
+
+sq_status check_outlier_list(const int32_t *O, int64_t nO, int64_t K)
+{
+    if (nO > 0 && !O) return fail(SQ_ERR_INVALID_ARG, "O is NULL");
+    for (int64_t j = 0; j < nO; ++j) {
+        if (O[j] < 0 || O[j] >= K) return fail(SQ_ERR_INVALID_ARG, "O[%lld]=%d outside [0, K)", (long long)j, O[j]);
+        if (j > 0 && O[j] <= O[j - 1]) return fail(SQ_ERR_INVALID_ARG, "O must be strictly increasing (index %lld)", (long long)j);
+    }
+    return SQ_OK;
+}
+
 sq_status prepare_impl(const void *W, int64_t N, int64_t K, int64_t ldw, const int32_t *O, int64_t nO, void *W_N,
                        float *s_w, void *W_O, uint32_t *chan_tab, cudaStream_t s, bool fp8)
 {
@@ -567,11 +613,7 @@ sq_status prepare_impl(const void *W, int64_t N, int64_t K, int64_t ldw, const i
         return fail(SQ_ERR_UNSUPPORTED, "the FP8 low path supports K <= %d (K=%lld)", sqq::kStreamMaxK, (long long)K);
     if (N < 0) return fail(SQ_ERR_INVALID_ARG, "N < 0");
     if (ldw < K || ldw % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldw must be >= K and a multiple of 8");
-    if (nO > 0 && !O) return fail(SQ_ERR_INVALID_ARG, "O is NULL");
-    for (int64_t j = 0; j < nO; ++j) {
-        if (O[j] < 0 || O[j] >= K) return fail(SQ_ERR_INVALID_ARG, "O[%lld]=%d outside [0, K)", (long long)j, O[j]);
-        if (j > 0 && O[j] <= O[j - 1]) return fail(SQ_ERR_INVALID_ARG, "O must be strictly increasing (index %lld)", (long long)j);
-    }
+    SQ_TRY(check_outlier_list(O, nO, K));
     SQ_TRY(check_ptr(chan_tab, true, "chan_tab"));
     const int64_t kn_pad = sq_kn_pad(K, nO);
     if (N > 0) {
@@ -582,18 +624,8 @@ sq_status prepare_impl(const void *W, int64_t N, int64_t K, int64_t ldw, const i
     }
     DevInfo di;
     SQ_TRY(device_info(di));
-
-    // Static channel table: one word per 8 channels.
-    std::vector<uint32_t> tab(static_cast<size_t>(K / 8), 0u);
-    for (int64_t j = 0; j < nO; ++j) tab[O[j] / 8] |= 1u << (O[j] % 8);
-    uint32_t below = 0;
-    for (int64_t c = 0; c < K / 8; ++c) {
-        const uint32_t mask = tab[c];
-        tab[c] = (below << 8) | mask;
-        below += static_cast<uint32_t>(__builtin_popcount(mask));
-    }
-    cudaError_t e = cudaMemcpyAsync(chan_tab, tab.data(), tab.size() * sizeof(uint32_t), cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return cuda_fail(e, "copy of the channel table");
+    SQ_TRY(upload_chan_table(O, nO, K, chan_tab, s));
+    cudaError_t e;
     SQ_TRY(launch_rowquant(static_cast<const uint16_t *>(W), N, K, ldw, chan_tab, nO, static_cast<uint8_t *>(W_N), s_w,
                            static_cast<uint16_t *>(W_O), s, fp8));
     if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "sq_prepare_weights");
@@ -620,6 +652,130 @@ sq_status linear_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const ui
                              fp8));
     return gemm_checked(kn_pad > 0 ? X_N : nullptr, s_x, no_pad > 0 ? X_O : nullptr, W_N, s_w, W_O, M, N, K, nO, Y, ldy,
                         nullptr, nullptr, s, fp8);
+}
+
+// ---------------------------------------------------------------- MXFP4 low path
+// Quantize-and-gather of `rows` rows into packed E2M1 codes (dn), tiled
+// E8M0 block scales (ds, rows padded to 128) and the compact outlier part.
+sq_status launch_mxquant(const uint16_t *src, int64_t rows, int64_t K, int64_t ld, const uint32_t *tab, int64_t nO,
+                         uint8_t *dn, uint8_t *ds, uint16_t *dout, cudaStream_t stream)
+{
+    if (rows == 0) return SQ_OK;
+    DevInfo di;
+    SQ_TRY(device_info(di));
+    const int64_t kn_pad = sq_kn_pad_mx(K, nO), no_pad = sq_no_pad(nO);
+    const int64_t rows_pad = round_up(rows, 128);
+    const size_t smem = static_cast<size_t>(2 * (kn_pad + no_pad));
+    int per_sm = 0;
+    SQ_TRY(kernel_setup(reinterpret_cast<const void *>(sqq::mx_quant_kernel), sqq::kMxThreads, smem, per_sm,
+                        "MX quantize set-up"));
+    const int64_t grid = std::min<int64_t>(rows_pad, static_cast<int64_t>(di.sms) * per_sm);
+    cudaError_t e = launch_k(sqq::mx_quant_kernel, dim3(static_cast<unsigned>(grid)), dim3(sqq::kMxThreads), smem,
+                             stream, 0u, src, static_cast<int>(rows), static_cast<int>(rows_pad), static_cast<int>(K),
+                             ld, tab, static_cast<int>(nO), static_cast<int>(K - nO), static_cast<int>(kn_pad),
+                             static_cast<int>(no_pad), dn, ds, dout);
+    if (e != cudaSuccess) return cuda_fail(e, "MX quantize launch");
+    return SQ_OK;
+}
+
+sq_status quant_gather_mx_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, int64_t nO,
+                               void *X_N4, void *S_X, void *X_O, cudaStream_t stream)
+{
+    SQ_TRY(check_K_nO(K, nO));
+    if (M < 0 || M > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "M out of range");
+    if (ldx < K || ldx % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldx must be >= K and a multiple of 8");
+    if (M == 0) return SQ_OK;
+    const int64_t kn_pad = sq_kn_pad_mx(K, nO);
+    SQ_TRY(check_ptr(X, true, "X"));
+    SQ_TRY(check_ptr(chan_tab, true, "chan_tab"));
+    SQ_TRY(check_ptr(X_N4, kn_pad > 0, "X_N4"));
+    SQ_TRY(check_ptr(S_X, kn_pad > 0, "S_X"));
+    SQ_TRY(check_ptr(X_O, nO > 0, "X_O"));
+    return launch_mxquant(static_cast<const uint16_t *>(X), M, K, ldx, chan_tab, nO, static_cast<uint8_t *>(X_N4),
+                          static_cast<uint8_t *>(S_X), static_cast<uint16_t *>(X_O), stream);
+}
+
+sq_status gemm_mx_checked(const void *X_N4, const void *S_X, const void *X_O, const void *W_N4, const void *S_W,
+                          const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
+                          float *dbg, cudaStream_t stream)
+{
+    SQ_TRY(check_K_nO(K, nO));
+    if (M < 0 || M > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "M out of range");
+    if (N < 0 || N % 8 != 0 || N > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "N must be a non-negative multiple of 8");
+    if (ldy < N || ldy % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldy must be >= N and a multiple of 8");
+    if (M == 0 || N == 0) return SQ_OK;
+    const int64_t kn_pad = sq_kn_pad_mx(K, nO);
+    SQ_TRY(check_ptr(X_N4, kn_pad > 0, "X_N4"));
+    SQ_TRY(check_ptr(W_N4, kn_pad > 0, "W_N4"));
+    SQ_TRY(check_ptr(S_X, kn_pad > 0, "S_X"));
+    SQ_TRY(check_ptr(S_W, kn_pad > 0, "S_W"));
+    SQ_TRY(check_ptr(X_O, nO > 0, "X_O"));
+    SQ_TRY(check_ptr(W_O, nO > 0, "W_O"));
+    SQ_TRY(check_ptr(Y, true, "Y"));
+    if (dbg && !aligned16(dbg)) return fail(SQ_ERR_MISALIGNED, "dbg_acc is not 16-byte aligned");
+    DevInfo di;
+    SQ_TRY(device_info(di));
+    // The scale operands travel in place of the fp32 scale pointers.
+    return launch_gemm_pair_t<CfgPairMx, sqg::kLowMx>(di, X_N4, static_cast<const float *>(S_X), X_O, W_N4,
+                                                      static_cast<const float *>(S_W), W_O, M, N, K, nO, Y, ldy,
+                                                      nullptr, dbg, stream);
+}
+
+size_t linear_ws_bytes_mx(int64_t M, int64_t K, int64_t nO)
+{
+    if (M <= 0) return 0;
+    const int64_t xn = round_up(M * (sq_kn_pad_mx(K, nO) / 2), 256);
+    const int64_t sx = round_up(static_cast<int64_t>(sq_mx_scale_bytes(M, K, nO)), 256);
+    const int64_t xo = round_up(M * sq_no_pad(nO) * 2, 256);
+    return static_cast<size_t>(xn + sx + xo);
+}
+
+sq_status prepare_mx_impl(const void *W, int64_t N, int64_t K, int64_t ldw, const int32_t *O, int64_t nO, void *W_N4,
+                          void *S_W, void *W_O, uint32_t *chan_tab, cudaStream_t s)
+{
+    SQ_TRY(check_K_nO(K, nO));
+    if (N < 0 || N > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "N out of range");
+    if (ldw < K || ldw % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldw must be >= K and a multiple of 8");
+    SQ_TRY(check_outlier_list(O, nO, K));
+    SQ_TRY(check_ptr(chan_tab, true, "chan_tab"));
+    const int64_t kn_pad = sq_kn_pad_mx(K, nO);
+    if (N > 0) {
+        SQ_TRY(check_ptr(W, true, "W"));
+        SQ_TRY(check_ptr(W_N4, kn_pad > 0, "W_N4"));
+        SQ_TRY(check_ptr(S_W, kn_pad > 0, "S_W"));
+        SQ_TRY(check_ptr(W_O, nO > 0, "W_O"));
+    }
+    DevInfo di;
+    SQ_TRY(device_info(di));
+    SQ_TRY(upload_chan_table(O, nO, K, chan_tab, s));
+    SQ_TRY(launch_mxquant(static_cast<const uint16_t *>(W), N, K, ldw, chan_tab, nO, static_cast<uint8_t *>(W_N4),
+                          static_cast<uint8_t *>(S_W), static_cast<uint16_t *>(W_O), s));
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "sq_prepare_weights_mx");
+    return SQ_OK;
+}
+
+sq_status linear_mx_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, const void *W_N4,
+                         const void *S_W, const void *W_O, int64_t N, int64_t nO, void *Y, int64_t ldy,
+                         void *workspace, size_t ws_bytes, cudaStream_t s)
+{
+    SQ_TRY(check_K_nO(K, nO));
+    if (M < 0) return fail(SQ_ERR_INVALID_ARG, "M < 0");
+    if (M == 0) return SQ_OK;
+    const size_t need = linear_ws_bytes_mx(M, K, nO);
+    if (ws_bytes < need) return fail(SQ_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+    SQ_TRY(check_ptr(workspace, true, "workspace"));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    const int64_t kn_pad = sq_kn_pad_mx(K, nO), no_pad = sq_no_pad(nO);
+    const int64_t xn_bytes = round_up(M * (kn_pad / 2), 256);
+    const int64_t sx_bytes = round_up(static_cast<int64_t>(sq_mx_scale_bytes(M, K, nO)), 256);
+    uint8_t *X_N4 = ws;
+    uint8_t *S_X = ws + xn_bytes;
+    uint16_t *X_O = reinterpret_cast<uint16_t *>(ws + xn_bytes + sx_bytes);
+    SQ_TRY(quant_gather_mx_impl(X, M, K, ldx, chan_tab, nO, kn_pad > 0 ? X_N4 : nullptr, kn_pad > 0 ? S_X : nullptr,
+                                no_pad > 0 ? X_O : nullptr, s));
+    return gemm_mx_checked(kn_pad > 0 ? X_N4 : nullptr, kn_pad > 0 ? S_X : nullptr, no_pad > 0 ? X_O : nullptr, W_N4,
+                           S_W, W_O, M, N, K, nO, Y, ldy, nullptr, s);
 }
 
 // ---------------------------------------------------------------- static outlier selection
@@ -719,6 +875,48 @@ int64_t sq_chan_table_words(int64_t K) { return K / 8; }
 size_t sq_linear_workspace_bytes(int64_t M, int64_t K, int64_t nO) { return linear_ws_bytes(M, K, nO, false); }
 
 size_t sq_linear_workspace_bytes_fp8(int64_t M, int64_t K, int64_t nO) { return linear_ws_bytes(M, K, nO, true); }
+
+int64_t sq_kn_pad_mx(int64_t K, int64_t nO) { return round_up(K - nO, 256); }
+
+size_t sq_mx_scale_bytes(int64_t rows, int64_t K, int64_t nO)
+{
+    if (rows <= 0) return 0;
+    return static_cast<size_t>(round_up(rows, 128) * (sq_kn_pad_mx(K, nO) / 32));
+}
+
+size_t sq_linear_workspace_bytes_mx(int64_t M, int64_t K, int64_t nO) { return linear_ws_bytes_mx(M, K, nO); }
+
+sq_status sq_prepare_weights_mx(const void *W, int64_t N, int64_t K, int64_t ldw, const int32_t *O, int64_t nO,
+                                void *W_N4, void *S_W, void *W_O, uint32_t *chan_tab, sq_stream_t stream)
+{
+    g_detail.clear();
+    return prepare_mx_impl(W, N, K, ldw, O, nO, W_N4, S_W, W_O, chan_tab, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_quant_gather_mx(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, int64_t nO,
+                             void *X_N4, void *S_X, void *X_O, sq_stream_t stream)
+{
+    g_detail.clear();
+    return quant_gather_mx_impl(X, M, K, ldx, chan_tab, nO, X_N4, S_X, X_O, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_gemm_mx(const void *X_N4, const void *S_X, const void *X_O, const void *W_N4, const void *S_W,
+                     const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y, int64_t ldy,
+                     float *dbg_acc, sq_stream_t stream)
+{
+    g_detail.clear();
+    return gemm_mx_checked(X_N4, S_X, X_O, W_N4, S_W, W_O, M, N, K, nO, Y, ldy, dbg_acc,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_linear_mx(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, const void *W_N4,
+                       const void *S_W, const void *W_O, int64_t N, int64_t nO, void *Y, int64_t ldy, void *workspace,
+                       size_t ws_bytes, sq_stream_t stream)
+{
+    g_detail.clear();
+    return linear_mx_impl(X, M, K, ldx, chan_tab, W_N4, S_W, W_O, N, nO, Y, ldy, workspace, ws_bytes,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
 
 sq_status sq_prepare_weights(const void *W, int64_t N, int64_t K, int64_t ldw, const int32_t *O, int64_t nO,
                              void *W_N, float *s_w, void *W_O, uint32_t *chan_tab, sq_stream_t stream)

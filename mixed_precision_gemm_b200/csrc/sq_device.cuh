@@ -187,6 +187,54 @@ __host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N)
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor for kind::mxf4 (block-scaled, dense): E2M1 A and B
+// (format 1 in bits [7,10) and [10,13)), K-major, N >> 3 in [17,23), E8M0
+// scale factors (bit 23), M >> 4 in [24,29), K = 64 per instruction (bit 31
+// clear).  The scale-factor byte selectors (bits [29,31) for A, [4,6) for B)
+// are added per instruction.
+__host__ __device__ constexpr uint32_t make_idesc_mxf4(int M, int N)
+{
+    return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+           (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// Shared-memory descriptor of one 512-byte scale-factor tile for tcgen05.cp
+// (32 rows of 16 bytes, no swizzle): 8-row core matrices 128 bytes apart
+// (stride byte offset), a single core matrix along the row (leading byte
+// offset unused, set to 16).
+__device__ __forceinline__ uint64_t make_sf_desc(uint32_t smem_addr)
+{
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1u) << 16;
+    d |= static_cast<uint64_t>(128u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    return d;
+}
+
+// Copy of a 512-byte scale-factor tile into 4 TMEM columns: byte 16r + 4c + j
+// of the tile lands in lane r (and r + 32, r + 64, r + 96) of column c, byte
+// j.  Issued by the pair's first CTA; each CTA of the pair copies from its
+// own shared memory into its own tensor memory.  Ordered with the MMAs the
+// same thread issues.
+__device__ __forceinline__ void sf_copy_pair(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Block-scaled pair MMA, kind::mxf4 with one E8M0 scale per 32 K-elements of
+// every A row (scale_a, TMEM) and every B row (scale_b, TMEM).
+__device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate, uint32_t scale_a, uint32_t scale_b)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(scale_a), "r"(scale_b)
+        : "memory");
+}
+
 __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                        uint32_t accumulate)
 {

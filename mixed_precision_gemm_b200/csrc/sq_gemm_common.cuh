@@ -38,6 +38,17 @@ constexpr int KB_I8 = 128;      // int8 K elements per block
 constexpr int KB_BF = 64;       // bf16 K elements per block
 constexpr int NUM_EXP_WARPS = 8;  // operand-producer warps of the pair kernel
 
+// Low-path formats.  INT4: packed codes expanded to int8 (kind::i8), one
+// fp32 scale per row.  FP8: E4M3 bytes (kind::f8f6f4), one fp32 scale per
+// row.  MX: packed E2M1 codes (kind::mxf4) with one E8M0 scale per 32
+// K-elements of each row; the tensor core applies the scales, so the low path
+// and the 16-bit branch accumulate into one fp32 accumulator.
+enum : int { kLowInt4 = 0, kLowFp8 = 1, kLowMx = 2 };
+constexpr int KB_MX = 256;        // E2M1 K elements per block (128 packed bytes per row)
+constexpr int MX_SF_BYTES = 3072; // scale bytes per ring slot: 2 tiles of X rows, 4 of W rows
+constexpr int MX_SFA_COL = 256;   // TMEM columns of the X-row scales (2 K-tiles x 4)
+constexpr int MX_SFB_COL = 264;   // TMEM columns of the W-row scales (2 K-tiles x 8)
+
 // Site codes stored in the device error word by a bounded wait that ran out.
 enum : unsigned {
     SITE_EXP_OP = 0x202, SITE_MMA_FULL = 0x301, SITE_MMA_ACC = 0x302, SITE_EPI = 0x401
@@ -51,7 +62,7 @@ struct GemmArgs {
     float *dbg_f;
     int M, N;
     long long ldy;
-    int nkb_i;    // INT4 K-blocks per tile (kn_pad / 128)
+    int nkb_i;    // low-path K-blocks per tile (kn_pad / 128; MX: kn_pad / 256)
     int nkb_o;    // bf16 K-blocks per tile (no_pad / 64)
     int tiles_m, tiles_n, group_m;
 };

@@ -29,6 +29,14 @@
 // K-blocks deep) and are expanded from shared memory, so no producer thread
 // has long global loads outstanding when it publishes a tile.
 // TMEM per CTA: acc_f in columns [0, 256), acc_i in [256, 512).
+//
+// MX low path (kLowMx): the packed E2M1 tiles travel by TMA straight into
+// the operand ring, together with their E8M0 scales (tiles of 128 rows x 4
+// blocks, see sq_mxquant.cuh); the MMA thread copies the scales into tensor
+// memory (tcgen05.cp, columns MX_SFA_COL / MX_SFB_COL) just before the
+// K-block's four kind::mxf4 MMAs.  The block-scaled products and the 16-bit
+// branch accumulate into the one fp32 accumulator in columns [0, 256), and
+// the epilogue only rounds it to bf16.
 #pragma once
 
 #include "sq_gemm_common.cuh"
@@ -42,7 +50,7 @@ constexpr int PAIR_EPI_WARPS = 8;  // two per TMEM lane quarter, each half of th
 constexpr int PAIR_EXP_WARP0 = PAIR_EPI_WARP0 + PAIR_EPI_WARPS;
 constexpr int PAIR_THREADS = 32 * (PAIR_EXP_WARP0 + NUM_EXP_WARPS);
 
-template <int OPS_, int STG_, int NG_>
+template <int OPS_, int STG_, int NG_, int SF_ = 0>
 struct CfgPair {
     static constexpr int OPS = OPS_;                  // operand ring stages (expanded int8 or bf16 tiles)
     static constexpr int STG = STG_;                  // staging ring stages (packed INT4 tiles)
@@ -54,8 +62,10 @@ struct CfgPair {
     static constexpr int OP_BYTES = A_BYTES + B_BYTES;
     static constexpr int PA_BYTES = 128 * PROWB;      // packed X rows of one K-block
     static constexpr int STG_BYTES = 256 * PROWB;     // packed X + W rows of one K-block
+    static constexpr int SF_BYTES = SF_;              // block scales per operand stage (MX only)
     static constexpr int OFF_OP = 0;
-    static constexpr int OFF_STG = OPS * OP_BYTES;
+    static constexpr int OFF_SF = OPS * OP_BYTES;
+    static constexpr int OFF_STG = OFF_SF + OPS * SF_BYTES;
     static constexpr int OFF_BAR = OFF_STG + STG * STG_BYTES;
     // barriers: op_full[OPS] op_empty[OPS] stg_full[STG] stg_empty[STG] acc_full acc_empty drain
     static constexpr int NBAR = 2 * OPS + 2 * STG + 3;
@@ -74,16 +84,21 @@ struct CfgPair {
                   "every ring slot must belong to one producer group");
 };
 
-// FP8: the low path is E4M3 x E4M3 (kind::f8f6f4, OSC's FP8 fallback for the
-// inputs of W2): its tiles are plain bytes that TMA writes straight into the
-// operand ring, so the staging ring and the expansion are compiled out and the
-// normal accumulator is fp32.
-template <class C, bool DBG, bool FP8>
+// LOW selects the low path.  kLowFp8: E4M3 x E4M3 (kind::f8f6f4, OSC's FP8
+// fallback for the inputs of W2) and kLowMx: block-scaled E2M1 (kind::mxf4):
+// their tiles are plain bytes that TMA writes straight into the operand ring,
+// so the staging ring and the expansion are compiled out and the low-path
+// accumulator is fp32.  tm_sx / tm_sw (block scales) are used by kLowMx only.
+template <class C, bool DBG, int LOW>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
 dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_constant__ CUtensorMap tm_wo,
                       const __grid_constant__ CUtensorMap tm_xn, const __grid_constant__ CUtensorMap tm_wn,
+                      const __grid_constant__ CUtensorMap tm_sx, const __grid_constant__ CUtensorMap tm_sw,
                       const GemmArgs args)
 {
+    constexpr bool FP8 = LOW == kLowFp8;
+    constexpr bool MX = LOW == kLowMx;
+    constexpr bool EXPAND = LOW == kLowInt4;
     constexpr int OPS = C::OPS, EC = C::EXP_CHUNKS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -133,6 +148,10 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         if (args.nkb_i > 0) {
             sqd::prefetch_tensormap(&tm_xn);
             sqd::prefetch_tensormap(&tm_wn);
+            if constexpr (MX) {
+                sqd::prefetch_tensormap(&tm_sx);
+                sqd::prefetch_tensormap(&tm_sw);
+            }
         }
     }
     if (warp == 1) {
@@ -156,7 +175,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         // ------------------------------------------------------------ staging producer (each CTA)
         // Packed INT4 tiles of this CTA's X rows and W rows, one K-block per
         // stage, in the order the expansion warps consume them.
-        if constexpr (!FP8) if (lane == 0 && nkb_i > 0) {
+        if constexpr (EXPAND) if (lane == 0 && nkb_i > 0) {
             const int F = my_tiles * nkb_i;
             const int r0 = static_cast<int>(rank) * 128;
             int last_armed = -1;
@@ -181,6 +200,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             constexpr uint32_t idesc_bf = sqd::make_idesc(false, PAIR_BM, PAIR_BN);
             constexpr uint32_t idesc_i8 = sqd::make_idesc(true, PAIR_BM, PAIR_BN);
             constexpr uint32_t idesc_f8 = sqd::make_idesc_e4m3(PAIR_BM, PAIR_BN);
+            constexpr uint32_t idesc_mx = sqd::make_idesc_mxf4(PAIR_BM, PAIR_BN);
             bool ok = true;
             for (int lt = 0; lt < my_tiles && ok; ++lt) {
                 if (!sqd::mbar_wait(acc_empty, (lt & 1) ^ 1u, abort_flag, SITE_MMA_ACC)) { ok = false; break; }
@@ -193,13 +213,34 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                     const bool is_bf = i < nkb_o;
                     const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
                     const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
-                    const uint32_t d = tmem + (is_bf ? 0u : static_cast<uint32_t>(PAIR_BN));
-                    const bool first = (i == 0) || (i == nkb_o);
+                    // MX: one accumulator for both paths; otherwise the low path has its own.
+                    const uint32_t d = tmem + ((is_bf || MX) ? 0u : static_cast<uint32_t>(PAIR_BN));
+                    const bool first = MX ? (i == 0) : ((i == 0) || (i == nkb_o));
+                    if constexpr (MX) {
+                        if (!is_bf) {
+                            // Scales of this K-block: X-row tiles (K-tiles 0, 1) at sf, sf + 512; W-row
+                            // tiles of rows 0-127 at sf + 1024 (+512 for K-tile 1), rows 128-255 at sf + 2048.
+                            const uint32_t sf = sbase + C::OFF_SF + e * C::SF_BYTES;
+                            sqd::sf_copy_pair(tmem + MX_SFA_COL, sqd::make_sf_desc(sf));
+                            sqd::sf_copy_pair(tmem + MX_SFA_COL + 4, sqd::make_sf_desc(sf + 512));
+                            sqd::sf_copy_pair(tmem + MX_SFB_COL, sqd::make_sf_desc(sf + 1024));
+                            sqd::sf_copy_pair(tmem + MX_SFB_COL + 4, sqd::make_sf_desc(sf + 2048));
+                            sqd::sf_copy_pair(tmem + MX_SFB_COL + 8, sqd::make_sf_desc(sf + 1536));
+                            sqd::sf_copy_pair(tmem + MX_SFB_COL + 12, sqd::make_sf_desc(sf + 2560));
+                        }
+                    }
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const uint32_t acc = (first && k == 0) ? 0u : 1u;
                         if (is_bf) sqd::mma_bf16_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_bf, acc);
-                        else if constexpr (FP8) sqd::mma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_f8, acc);
+                        else if constexpr (MX) {
+                            // MMA k covers scale blocks 2k, 2k+1: K-tile k / 2, bytes 2 (k % 2) and up.
+                            const uint32_t id = 2u * static_cast<uint32_t>(k & 1);
+                            const uint32_t sfa = (tmem + MX_SFA_COL + 4 * (k >> 1)) | (id << 30);
+                            const uint32_t sfb = (tmem + MX_SFB_COL + 8 * (k >> 1)) | (id << 30);
+                            sqd::mma_mxf4_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_mx | (id << 29) | (id << 4), acc,
+                                               sfa, sfb);
+                        } else if constexpr (FP8) sqd::mma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_f8, acc);
                         else sqd::mma_s8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_i8, acc);
                     }
                     sqd::mma_commit_pair_multicast(op_empty(e), 0x3);
@@ -220,8 +261,8 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         // INT4 block f: packed rows from staging stage f % STG -> int8 rows in
         // operand stage e (the tile's X rows, then its W rows).
         auto store = [&](int f) -> bool {
-          if constexpr (FP8) {
-            return false;  // FP8 tiles are never expanded
+          if constexpr (!EXPAND) {
+            return false;  // E4M3 and E2M1 tiles are never expanded
           } else {
             const int lt = f / nkb_i;
             const int kb = f - lt * nkb_i;
@@ -284,8 +325,40 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             return true;
         };
 
+        // MX ring use u (tile lt, low K-block kb): the packed E2M1 tiles plus
+        // the block scales of this CTA's 128 X rows (one box: K-tiles 2kb,
+        // 2kb+1) and of all 256 W rows of the tile (two boxes, one per
+        // 128-row band).  Both CTAs of the pair need every W-row scale.
+        auto produce_mx = [&](int lt, int u, int kb) -> bool {
+            if constexpr (MX) {
+                int tmi, tni;
+                tile_coords(args, pair + lt * num_pairs, tmi, tni);
+                const int e = u % OPS;
+                if (!sqd::mbar_wait(op_empty(e), ((u / OPS) & 1) ^ 1u, abort_flag, SITE_EXP_OP)) return false;
+                const uint32_t full_leader = sqd::map_to_cta(op_full(e), 0);
+                if (tma_thread) {
+                    const int na = 2 * nkb_i;  // scale tiles per 128-row band
+                    const uint32_t sf = sbase + C::OFF_SF + e * C::SF_BYTES;
+                    sqd::mbar_arrive_expect_tx_cluster(full_leader, C::OP_BYTES + C::SF_BYTES);
+                    sqd::tma_load_2d_pair(op_a(e), &tm_xn, full_leader, kb * (KB_MX / 2),
+                                          tmi * PAIR_BM + static_cast<int>(r0));
+                    sqd::tma_load_2d_pair(op_a(e) + C::A_BYTES, &tm_wn, full_leader, kb * (KB_MX / 2),
+                                          tni * PAIR_BN + static_cast<int>(r0));
+                    sqd::tma_load_2d_pair(sf, &tm_sx, full_leader, 0, ((2 * tmi + static_cast<int>(rank)) * na + 2 * kb) * 4);
+                    sqd::tma_load_2d_pair(sf + 1024, &tm_sw, full_leader, 0, ((2 * tni) * na + 2 * kb) * 4);
+                    sqd::tma_load_2d_pair(sf + 2048, &tm_sw, full_leader, 0, ((2 * tni + 1) * na + 2 * kb) * 4);
+                    last_armed = u;
+                } else if (lane == 0) {
+                    sqd::mbar_arrive_cluster(full_leader);
+                }
+                return true;
+            } else {
+                return false;
+            }
+        };
+
         // Ring uses of this group, in order: u = gi, gi + NG, ...  bf16 blocks
-        // first, then the low-path blocks (E4M3 by TMA, or INT4 expanded).
+        // first, then the low-path blocks (E4M3 or E2M1 by TMA, or INT4 expanded).
         bool ok = true;
         const int total = my_tiles * per_tile;
         for (int u = gi; u < total && ok; u += C::NG) {
@@ -293,6 +366,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             const int i = u - lt * per_tile;
             if (i < nkb_o) ok = produce_tma(lt, u, &tm_xo, &tm_wo, i * KB_BF);
             else if constexpr (FP8) ok = produce_tma(lt, u, &tm_xn, &tm_wn, (i - nkb_o) * KB_I8);
+            else if constexpr (MX) ok = produce_mx(lt, u, i - nkb_o);
             else ok = store(lt * nkb_i + (i - nkb_o));
         }
         if (!ok && tma_thread && last_armed >= 0 && leader) {
@@ -320,9 +394,9 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             // Scales of this warp's 128 columns and of this lane's row, fetched
             // while the tile's MMAs still run.
             const int ncol = tni * PAIR_BN + c_base + 4 * lane;
-            const float4 swp = ncol < args.N ? __ldg(reinterpret_cast<const float4 *>(args.s_w + ncol))
-                                             : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float sx = row_ok ? args.s_x[m] : 0.0f;
+            const float4 swp = (!MX && ncol < args.N) ? __ldg(reinterpret_cast<const float4 *>(args.s_w + ncol))
+                                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float sx = (!MX && row_ok) ? args.s_x[m] : 0.0f;
             uint16_t *yrow = args.Y + static_cast<long long>(row_ok ? m : 0) * args.ldy;
             if (!sqd::mbar_wait(acc_full, lt & 1, abort_flag, SITE_EPI)) break;
             sqd::tc_fence_after();
@@ -332,8 +406,12 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             __syncwarp();
             uint32_t vi[2][CW] = {}, vf[2][CW] = {};
             auto issue = [&](int ch, int b) {
-                if (has_i) sqd::tmem_ld_32x32b_x16(tl + PAIR_BN + c_base + ch * CW, vi[b]);
-                if (has_o) sqd::tmem_ld_32x32b_x16(tl + c_base + ch * CW, vf[b]);
+                if constexpr (MX) {
+                    sqd::tmem_ld_32x32b_x16(tl + c_base + ch * CW, vf[b]);  // the one accumulator
+                } else {
+                    if (has_i) sqd::tmem_ld_32x32b_x16(tl + PAIR_BN + c_base + ch * CW, vi[b]);
+                    if (has_o) sqd::tmem_ld_32x32b_x16(tl + c_base + ch * CW, vf[b]);
+                }
             };
             issue(0, 0);
             sqd::tmem_wait_ld_dep(vi[0], vf[0]);
@@ -359,10 +437,14 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
                                 const int t = 8 * g + 2 * h + u;
-                                // low path: exact int32 sum (x256) for INT4, fp32 sum for E4M3
+                                // low path: exact int32 sum (x256) for INT4, fp32 sum for E4M3;
+                                // MX: the accumulator already holds the whole sum
                                 float al;
                                 int32_t dbg_lo;
-                                if constexpr (FP8) {
+                                if constexpr (MX) {
+                                    al = 0.0f;
+                                    dbg_lo = 0;
+                                } else if constexpr (FP8) {
                                     al = has_i ? __uint_as_float(vi[b][t]) : 0.0f;
                                     dbg_lo = __float_as_int(al);
                                 } else {
@@ -370,8 +452,8 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                                     al = static_cast<float>(ai);
                                     dbg_lo = ai;
                                 }
-                                const float af = has_o ? __uint_as_float(vf[b][t]) : 0.0f;
-                                y2[u] = __fadd_rn(__fmul_rn(__fmul_rn(al, sx), swv[2 * h + u]), af);
+                                const float af = (MX || has_o) ? __uint_as_float(vf[b][t]) : 0.0f;
+                                y2[u] = MX ? af : __fadd_rn(__fmul_rn(__fmul_rn(al, sx), swv[2 * h + u]), af);
                                 if constexpr (DBG) {
                                     if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + 2 * h + u] = dbg_lo;
                                     if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n + 2 * h + u] = af;

@@ -100,3 +100,35 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_build, "LIB_PATH", str(tmp_path / "nope.so"))
     with pytest.raises(RuntimeError, match="missing"):
         sq.load()
+
+
+def test_mx_layout_queries(lib):
+    assert sq.sq_kn_pad_mx(4096, 256) == 3840
+    assert sq.sq_kn_pad_mx(1040, 24) == 1024
+    assert sq.sq_kn_pad_mx(200, 3) == 256
+    assert sq.sq_kn_pad_mx(64, 64) == 0
+    # 128-row bands of one byte per 32 codes
+    assert sq.sq_mx_scale_bytes(300, 4096, 256) == 384 * 3840 // 32
+    assert sq.sq_mx_scale_bytes(128, 4096, 0) == 128 * 4096 // 32
+    assert sq.sq_mx_scale_bytes(0, 4096, 0) == 0
+    assert sq.sq_mx_scale_bytes(5, 64, 64) == 0
+    M, K, nO = 2048, 4096, 256
+    ws = sq.sq_linear_workspace_bytes_mx(M, K, nO)
+    assert ws >= M * 3840 // 2 + sq.sq_mx_scale_bytes(M, K, nO) + 2 * M * 256 and ws % 256 == 0
+    assert sq.sq_linear_workspace_bytes_mx(0, K, nO) == 0
+
+
+def test_mx_argument_errors_before_device(lib):
+    assert lib.sq_quant_gather_mx(None, 4, 12, 16, None, 0, None, None, None, None) == sq.SQ_ERR_INVALID_ARG
+    assert lib.sq_quant_gather_mx(None, 4, 64, 60, None, 0, None, None, None, None) == sq.SQ_ERR_INVALID_ARG
+    assert lib.sq_gemm_mx(None, None, None, None, None, None, 4, 12, 64, 0, None, 16, None, None) == \
+        sq.SQ_ERR_INVALID_ARG
+    assert lib.sq_gemm_mx(None, None, None, None, None, None, 4, 16, 64, 0, None, 16, None, None) == \
+        sq.SQ_ERR_INVALID_ARG   # NULL operands
+    buf = ctypes.create_string_buffer(64)
+    mis = ctypes.c_void_p(ctypes.addressof(buf) + 1)
+    assert lib.sq_gemm_mx(mis, mis, None, mis, mis, None, 4, 16, 64, 0, mis, 16, None, None) == sq.SQ_ERR_MISALIGNED
+    assert lib.sq_linear_mx(None, 4, 64, 64, None, None, None, None, 16, 0, None, 16, None, 0, None) == \
+        sq.SQ_ERR_INVALID_ARG   # workspace too small
+    O = (ctypes.c_int32 * 2)(5, 3)
+    assert lib.sq_prepare_weights_mx(None, 4, 64, 64, O, 2, None, None, None, None, None) == sq.SQ_ERR_INVALID_ARG

@@ -69,7 +69,7 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     assert capsys.readouterr().out == ""
 
 
-@pytest.mark.parametrize("low", ["int4", "fp8"])
+@pytest.mark.parametrize("low", ["int4", "fp8", "mx"])
 def test_reference_arm_json_line(low):
     import json
     import subprocess
