@@ -386,16 +386,18 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
 
 // Swapped-operand split-K kernel for M <= 128: tiles of 128 W rows x MP
 // tokens; the K-blocks of each tile are spread over a cluster of S CTAs.
-template <class C, bool FP8>
+// kLowMx passes the tiled block scales S_X / S_W in place of s_x / s_w.
+template <class C, int LOW>
 sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O,
                                const void *W_N, const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K,
                                int64_t nO, void *Y, int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
 {
-    const int64_t kn_pad = sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
-    CUtensorMap m_xo{}, m_wo{}, m_xn{}, m_wn{};
+    constexpr bool FP8 = LOW == sqg::kLowFp8, MX = LOW == sqg::kLowMx;
+    const int64_t kn_pad = MX ? sq_kn_pad_mx(K, nO) : sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
+    CUtensorMap m_xo{}, m_wo{}, m_xn{}, m_wn{}, m_sx{}, m_sw{};
     sq_status st;
     if (kn_pad > 0) {
-        // 128-byte boxes (two INT4 K-blocks, or one E4M3 K-block) with the 128-byte swizzle.
+        // 128-byte boxes (two INT4 K-blocks, one E4M3 K-block or one E2M1 K-block) with the 128-byte swizzle.
         const int64_t rb = FP8 ? kn_pad : kn_pad / 2;
         if ((st = make_map(m_xn, X_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, rb, M, rb, 128, C::MP,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
@@ -403,6 +405,16 @@ sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *
         if ((st = make_map(m_wn, W_N, CU_TENSOR_MAP_DATA_TYPE_UINT8, rb, N, rb, 128, 128,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != SQ_OK)
             return st;
+        if (MX) {
+            const uint64_t sx_rows = static_cast<uint64_t>(sq_mx_scale_bytes(M, K, nO) / 128);
+            const uint64_t sw_rows = static_cast<uint64_t>(sq_mx_scale_bytes(N, K, nO) / 128);
+            if ((st = make_map(m_sx, s_x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, sx_rows, 128, 128, 8,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
+                return st;
+            if ((st = make_map(m_sw, s_w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, sw_rows, 128, 128, 8,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != SQ_OK)
+                return st;
+        }
     }
     if (no_pad > 0) {
         if ((st = make_map(m_xo, X_O, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, no_pad, M, no_pad * 2, sqg::KB_BF, C::MP,
@@ -421,26 +433,27 @@ sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *
     a.M = static_cast<int>(M);
     a.N = static_cast<int>(N);
     a.ldy = ldy;
-    a.nkb_i = static_cast<int>(kn_pad / sqg::KB_I8);
+    a.nkb_i = static_cast<int>(kn_pad / (MX ? sqg::KB_MX : sqg::KB_I8));
     a.nkb_o = static_cast<int>(no_pad / sqg::KB_BF);
+    if (MX) a.s_x = a.s_w = nullptr;
     const int64_t tiles_n = (N + 127) / 128;
     // As many K ranges per W tile as fill the SMs once, at most 8 (portable
     // cluster size) and at most half the tile's byte count in 64-byte units,
     // so that every range holds at least one K-block.
-    const int cost = a.nkb_i + 2 * a.nkb_o;
+    const int cost = (MX ? 2 : 1) * a.nkb_i + 2 * a.nkb_o;
     int64_t S = tiles_n >= di.sms ? 1 : di.sms / tiles_n;
     S = std::min<int64_t>(S, sqg::SK_MAX_SPLITS);
     S = std::min<int64_t>(S, std::max(1, cost / 2));
     S = std::max<int64_t>(S, 1);
     a.splits = static_cast<int>(S);
     const bool dbg = dbg_i || dbg_f;
-    auto kern = dbg ? sqg::dual_gemm_skinny_kernel<C, true, FP8> : sqg::dual_gemm_skinny_kernel<C, false, FP8>;
+    auto kern = dbg ? sqg::dual_gemm_skinny_kernel<C, true, LOW> : sqg::dual_gemm_skinny_kernel<C, false, LOW>;
     int per_sm = 0;
     if ((st = kernel_setup(reinterpret_cast<const void *>(kern), sqg::SK_THREADS, C::SMEM_BYTES, per_sm, "gemm skinny set-up")) != SQ_OK)
         return st;
     cudaError_t e;
     if ((e = launch_k(kern, dim3(static_cast<unsigned>(tiles_n * S)), dim3(sqg::SK_THREADS), C::SMEM_BYTES, stream,
-                      static_cast<unsigned>(S), m_xo, m_wo, m_xn, m_wn, a)) != cudaSuccess)
+                      static_cast<unsigned>(S), m_xo, m_wo, m_xn, m_wn, m_sx, m_sw, a)) != cudaSuccess)
         return cuda_fail(e, "gemm skinny launch");
     return SQ_OK;
 }
@@ -452,6 +465,11 @@ using CfgSk16 = sqg::CfgSkinny<16, 8, 3>;
 using CfgSk32 = sqg::CfgSkinny<32, 7, 3>;
 using CfgSk64 = sqg::CfgSkinny<64, 6, 2>;
 using CfgSk128 = sqg::CfgSkinny<128, 4, 2>;
+// MX: no operand ring (stages are read in place), a deeper staging ring with 2 KB of scales per stage.
+using CfgSk16Mx = sqg::CfgSkinny<16, 10, 0, 2048>;
+using CfgSk32Mx = sqg::CfgSkinny<32, 9, 0, 2048>;
+using CfgSk64Mx = sqg::CfgSkinny<64, 8, 0, 2048>;
+using CfgSk128Mx = sqg::CfgSkinny<128, 6, 0, 2048>;
 
 
 template <bool FP8>
@@ -463,12 +481,12 @@ sq_status gemm_dispatch(const DevInfo &di, const void *X_N, const float *s_x, co
     if (M > 128)
         return launch_gemm_pair_t<Pair, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (M <= 16)
-        return launch_gemm_skinny_t<CfgSk16, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+        return launch_gemm_skinny_t<CfgSk16, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (M <= 32)
-        return launch_gemm_skinny_t<CfgSk32, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+        return launch_gemm_skinny_t<CfgSk32, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (M <= 64)
-        return launch_gemm_skinny_t<CfgSk64, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
-    return launch_gemm_skinny_t<CfgSk128, FP8>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+        return launch_gemm_skinny_t<CfgSk64, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    return launch_gemm_skinny_t<CfgSk128, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
 }
 
 sq_status gemm_impl(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
@@ -716,9 +734,21 @@ sq_status gemm_mx_checked(const void *X_N4, const void *S_X, const void *X_O, co
     DevInfo di;
     SQ_TRY(device_info(di));
     // The scale operands travel in place of the fp32 scale pointers.
-    return launch_gemm_pair_t<CfgPairMx, sqg::kLowMx>(di, X_N4, static_cast<const float *>(S_X), X_O, W_N4,
-                                                      static_cast<const float *>(S_W), W_O, M, N, K, nO, Y, ldy,
-                                                      nullptr, dbg, stream);
+    const float *sx = static_cast<const float *>(S_X), *sw = static_cast<const float *>(S_W);
+    if (M > 128)
+        return launch_gemm_pair_t<CfgPairMx, sqg::kLowMx>(di, X_N4, sx, X_O, W_N4, sw, W_O, M, N, K, nO, Y, ldy,
+                                                          nullptr, dbg, stream);
+    if (M <= 16)
+        return launch_gemm_skinny_t<CfgSk16Mx, sqg::kLowMx>(di, X_N4, sx, X_O, W_N4, sw, W_O, M, N, K, nO, Y, ldy,
+                                                            nullptr, dbg, stream);
+    if (M <= 32)
+        return launch_gemm_skinny_t<CfgSk32Mx, sqg::kLowMx>(di, X_N4, sx, X_O, W_N4, sw, W_O, M, N, K, nO, Y, ldy,
+                                                            nullptr, dbg, stream);
+    if (M <= 64)
+        return launch_gemm_skinny_t<CfgSk64Mx, sqg::kLowMx>(di, X_N4, sx, X_O, W_N4, sw, W_O, M, N, K, nO, Y, ldy,
+                                                            nullptr, dbg, stream);
+    return launch_gemm_skinny_t<CfgSk128Mx, sqg::kLowMx>(di, X_N4, sx, X_O, W_N4, sw, W_O, M, N, K, nO, Y, ldy,
+                                                         nullptr, dbg, stream);
 }
 
 size_t linear_ws_bytes_mx(int64_t M, int64_t K, int64_t nO)

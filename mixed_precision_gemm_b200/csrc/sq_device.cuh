@@ -222,6 +222,23 @@ __device__ __forceinline__ void sf_copy_pair(uint32_t taddr, uint64_t sdesc)
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// Single-CTA forms of the two above (cta_group::1).
+__device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate, uint32_t scale_a, uint32_t scale_b)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(scale_a), "r"(scale_b)
+        : "memory");
+}
+
 // Block-scaled pair MMA, kind::mxf4 with one E8M0 scale per 32 K-elements of
 // every A row (scale_a, TMEM) and every B row (scale_b, TMEM).
 __device__ __forceinline__ void mma_mxf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,

@@ -41,6 +41,14 @@
 // were its own or were consumed before it reached the slot, so the
 // phase-parity waits cannot alias.
 // TMEM: acc_i (int32) in columns [0, MP), acc_f (fp32) in [MP, 2 MP).
+//
+// MX low path (kLowMx): a stage is one K-block of 256 E2M1 codes (128 bytes
+// per row) read by the MMA in place, plus two 1 KB scale boxes: the W rows'
+// (two K-tiles of the tile's 128-row band) and the tokens' (band 0).  The MMA
+// thread copies them into TMEM (columns MP .. MP+7 for W, MP+8 .. MP+15 for
+// the tokens) before the K-block's four kind::mxf4 MMAs; the 16-bit branch
+// adds into the same fp32 accumulator in [0, MP), and only that accumulator
+// is reduced over the cluster.
 #pragma once
 
 #include "sq_gemm_common.cuh"
@@ -55,23 +63,27 @@ constexpr int SK_MAX_SPLITS = 8;
 
 enum : unsigned { SITE_SK_STG = 0x501, SITE_SK_OP = 0x502, SITE_SK_MMA = 0x503, SITE_SK_EPI = 0x504 };
 
-template <int MP_, int NST_, int OPS_>
+template <int MP_, int NST_, int OPS_, int SF_ = 0>
 struct CfgSkinny {
     static constexpr int MP = MP_;                    // token columns of D (MMA N)
     static constexpr int NST = NST_;                  // staging ring stages
     static constexpr int OPS = OPS_;                  // expanded int8 operand ring stages
+    static constexpr int SF_BYTES = SF_;              // block scales per staging stage (MX only)
     static constexpr int ROWS = 128 + MP;             // W rows, then token rows, in every tile
     static constexpr int A_BYTES = 128 * ROWB;
     static constexpr int TILE_BYTES = ROWS * ROWB;    // one stage = one operand tile (128-byte rows)
     static constexpr int OFF_STG = 0;
     static constexpr int OFF_OP = NST * TILE_BYTES;
-    static constexpr int OFF_BAR = OFF_OP + OPS * TILE_BYTES;
+    static constexpr int OFF_SF = OFF_OP + OPS * TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_SF + NST * SF_BYTES;
     // barriers: stg_full[NST] stg_empty[NST] op_full[OPS] op_empty[OPS] acc_full drain
     static constexpr int NBAR = 2 * NST + 2 * OPS + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_CNT = OFF_MISC + 16;           // per staging slot: expansion warps done
     static constexpr int SMEM_BYTES = OFF_CNT + NST * 4 + 1024;
-    static constexpr int TMEM_COLS = 2 * MP < 32 ? 32 : 2 * MP;
+    // MX: the accumulator [0, MP) and 16 scale columns; otherwise two accumulators.
+    static constexpr int TMEM_NEED = SF_ > 0 ? MP + 16 : 2 * MP;
+    static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : 256;
     static constexpr int EXP_CHUNKS = ROWS * 8 / SK_PT;   // 16-byte packed chunks per thread per stage
     // Reduction buffer (aliases the rings): int32 and fp32 regions of
     // S * RP <= 128 + S - 1 partial rows, RSTRIDE words apart.
@@ -82,7 +94,7 @@ struct CfgSkinny {
     static_assert(MP == 16 || MP == 32 || MP == 64 || MP == 128, "MP");
     static_assert(TILE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned");
     static_assert(ROWS * 8 % SK_PT == 0, "expansion work split");
-    static_assert(OPS >= 2, "an INT4 stage fills two operand tiles");
+    static_assert(OPS >= 2 || SF_ > 0, "an INT4 stage fills two operand tiles");
     static_assert(2 * RED_ROWS * RSTRIDE * 4 <= OFF_BAR, "reduction buffer must fit in the rings");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -100,26 +112,32 @@ struct SkinnyArgs {
     int splits;  // CTAs per cluster = K ranges per W tile
 };
 
-// First K-block of split r of S: blocks 0..nkb_i-1 are INT4 (64 bytes per W
-// row), then nkb_o bf16 blocks (128 bytes per W row); the split points are
-// the block boundaries at or after r/S of the total bytes.
-__device__ __forceinline__ int skinny_first_block(int r, int S, int nkb_i, int nkb_o)
+// First K-block of split r of S: blocks 0..nkb_i-1 are low-path blocks of
+// lw 64-byte units per W row (INT4: 1; MX: 2), then nkb_o bf16 blocks (2
+// units); the split points are the block boundaries at or after r/S of the
+// total bytes.
+__device__ __forceinline__ int skinny_first_block(int r, int S, int nkb_i, int nkb_o, int lw)
 {
-    const int cost = nkb_i + 2 * nkb_o;
+    const int cost = lw * nkb_i + 2 * nkb_o;
     const int c = static_cast<int>(static_cast<long long>(cost) * r / S);
-    return c <= nkb_i ? c : nkb_i + (c - nkb_i + 1) / 2;
+    return c <= lw * nkb_i ? (c + lw - 1) / lw : nkb_i + (c - lw * nkb_i + 1) / 2;
 }
 
-// FP8: the low path is E4M3 x E4M3 (kind::f8f6f4, OSC's FP8 fallback for the
-// inputs of W2).  A stage then carries one K-block of bytes that the MMA reads
-// in place, as for bf16 stages; the expansion warps only run the epilogue, and
-// the low-path partials are fp32.
-template <class C, bool DBG, bool FP8>
+// LOW selects the low path.  kLowFp8 (E4M3 x E4M3, kind::f8f6f4, OSC's FP8
+// fallback for the inputs of W2) and kLowMx (block-scaled E2M1, kind::mxf4):
+// a stage carries one K-block of bytes that the MMA reads in place, as for
+// bf16 stages; the expansion warps only run the epilogue, and the low-path
+// partials are fp32.  tm_sx / tm_sw (block scales) are used by kLowMx only.
+template <class C, bool DBG, int LOW>
 __global__ void __launch_bounds__(SK_THREADS, 1)
 dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_constant__ CUtensorMap tm_wo,
                         const __grid_constant__ CUtensorMap tm_xn, const __grid_constant__ CUtensorMap tm_wn,
+                        const __grid_constant__ CUtensorMap tm_sx, const __grid_constant__ CUtensorMap tm_sw,
                         const SkinnyArgs args)
 {
+    constexpr bool FP8 = LOW == kLowFp8;
+    constexpr bool MX = LOW == kLowMx;
+    constexpr bool DIRECT = FP8 || MX;   // low-path stages read by the MMA in place
     constexpr int MP = C::MP, NST = C::NST, OPS = C::OPS, EC = C::EXP_CHUNKS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -148,13 +166,14 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
     // This CTA's K range: INT4 blocks [i_lo, i_lo + n_i) in ns_i stages of
     // two, then bf16 blocks [o_lo, o_lo + n_o), one stage each.
     const int nkb_i = args.nkb_i, nkb_o = args.nkb_o;
-    const int b_lo = skinny_first_block(rank, S, nkb_i, nkb_o);
-    const int b_hi = skinny_first_block(rank + 1, S, nkb_i, nkb_o);
+    const int lw = MX ? 2 : 1;
+    const int b_lo = skinny_first_block(rank, S, nkb_i, nkb_o, lw);
+    const int b_hi = skinny_first_block(rank + 1, S, nkb_i, nkb_o, lw);
     const int i_lo = min(b_lo, nkb_i);
     const int n_i = min(b_hi, nkb_i) - i_lo;
     const int o_lo = max(b_lo, nkb_i) - nkb_i;
     const int n_o = max(b_hi, nkb_i) - nkb_i - o_lo;
-    const int ns_i = FP8 ? n_i : (n_i + 1) / 2;
+    const int ns_i = DIRECT ? n_i : (n_i + 1) / 2;
     const int ns = ns_i + n_o;
 
     if (threadIdx.x == 0) {
@@ -181,6 +200,10 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
         if (n_i > 0) {
             sqd::prefetch_tensormap(&tm_xn);
             sqd::prefetch_tensormap(&tm_wn);
+            if constexpr (MX) {
+                sqd::prefetch_tensormap(&tm_sx);
+                sqd::prefetch_tensormap(&tm_sw);
+            }
         }
     }
     if (warp == 1) {
@@ -201,6 +224,21 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
             for (int t = 0; t < ns; ++t) {
                 const int s = t % NST;
                 if (!sqd::mbar_wait(stg_empty(s), ((t / NST) & 1) ^ 1u, abort_flag, SITE_SK_STG)) { ok = false; break; }
+                if constexpr (MX) {
+                    if (t < ns_i) {
+                        // codes of K-block kb (128 bytes per row), and the scale tiles 2kb, 2kb+1 of
+                        // the W rows' band and of the tokens' band 0
+                        const int kb = i_lo + t;
+                        const uint32_t sf = sbase + C::OFF_SF + s * C::SF_BYTES;
+                        sqd::mbar_arrive_expect_tx(stg_full(s), C::TILE_BYTES + C::SF_BYTES);
+                        sqd::tma_load_2d(stg_a(s), &tm_wn, stg_full(s), kb * (KB_MX / 2), n0);
+                        sqd::tma_load_2d(stg_a(s) + C::A_BYTES, &tm_xn, stg_full(s), kb * (KB_MX / 2), 0);
+                        sqd::tma_load_2d(sf, &tm_sw, stg_full(s), 0, ((n0 / 128) * 2 * nkb_i + 2 * kb) * 4);
+                        sqd::tma_load_2d(sf + 1024, &tm_sx, stg_full(s), 0, (2 * kb) * 4);
+                        last_armed = t;
+                        continue;
+                    }
+                }
                 sqd::mbar_arrive_expect_tx(stg_full(s), C::TILE_BYTES);
                 if (t < ns_i) {
                     // byte offset of the stage's first K-block (two INT4 blocks, or one E4M3 block)
@@ -222,7 +260,31 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
             constexpr uint32_t idesc_bf = sqd::make_idesc(false, 128, MP);
             constexpr uint32_t idesc_i8 = sqd::make_idesc(true, 128, MP);
             constexpr uint32_t idesc_f8 = sqd::make_idesc_e4m3(128, MP);
+            constexpr uint32_t idesc_mx = sqd::make_idesc_mxf4(128, MP);
             bool ok = true;
+            if constexpr (MX) {
+                for (int t = 0; t < ns_i && ok; ++t) {  // E2M1 blocks and their scales from the staging ring
+                    const int s = t % NST;
+                    if (!sqd::mbar_wait(stg_full(s), (t / NST) & 1, abort_flag, SITE_SK_MMA)) { ok = false; break; }
+                    sqd::tc_fence_after();
+                    const uint32_t sf = sbase + C::OFF_SF + s * C::SF_BYTES;
+                    sqd::sf_copy(tmem + MP, sqd::make_sf_desc(sf));                // W rows, K-tile 0
+                    sqd::sf_copy(tmem + MP + 4, sqd::make_sf_desc(sf + 512));      // W rows, K-tile 1
+                    sqd::sf_copy(tmem + MP + 8, sqd::make_sf_desc(sf + 1024));     // tokens, K-tile 0
+                    sqd::sf_copy(tmem + MP + 12, sqd::make_sf_desc(sf + 1536));    // tokens, K-tile 1
+                    const uint64_t adesc = sqd::make_sw128_desc(stg_a(s));
+                    const uint64_t bdesc = sqd::make_sw128_desc(stg_a(s) + C::A_BYTES);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const uint32_t id = 2u * static_cast<uint32_t>(k & 1);
+                        const uint32_t sfa = (tmem + MP + 4 * (k >> 1)) | (id << 30);
+                        const uint32_t sfb = (tmem + MP + 8 + 4 * (k >> 1)) | (id << 30);
+                        sqd::mma_mxf4(tmem, adesc + 2 * k, bdesc + 2 * k, idesc_mx | (id << 29) | (id << 4),
+                                      (t == 0 && k == 0) ? 0u : 1u, sfa, sfb);
+                    }
+                    sqd::mma_commit(stg_empty(s));
+                }
+            }
             if constexpr (FP8) {
                 for (int t = 0; t < ns_i && ok; ++t) {  // E4M3 blocks straight from the staging ring
                     const int s = t % NST;
@@ -236,7 +298,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
                     sqd::mma_commit(stg_empty(s));
                 }
             }
-            for (int u = 0; u < (FP8 ? 0 : n_i) && ok; ++u) {  // INT4 blocks from the operand ring
+            for (int u = 0; u < (DIRECT ? 0 : n_i) && ok; ++u) {  // INT4 blocks from the operand ring
                 const int e = u % OPS;
                 if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_SK_MMA)) { ok = false; break; }
                 sqd::tc_fence_after();
@@ -254,8 +316,11 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
                 const uint64_t adesc = sqd::make_sw128_desc(stg_a(s));
                 const uint64_t bdesc = sqd::make_sw128_desc(stg_a(s) + C::A_BYTES);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    sqd::mma_bf16(tmem + MP, adesc + 2 * k, bdesc + 2 * k, idesc_bf, (t == ns_i && k == 0) ? 0u : 1u);
+                for (int k = 0; k < 4; ++k) {
+                    // MX: the branch adds into the one accumulator (cleared by whichever MMA comes first)
+                    const uint32_t acc = MX ? ((t == 0 && k == 0) ? 0u : 1u) : ((t == ns_i && k == 0) ? 0u : 1u);
+                    sqd::mma_bf16(MX ? tmem : tmem + MP, adesc + 2 * k, bdesc + 2 * k, idesc_bf, acc);
+                }
                 sqd::mma_commit(stg_empty(s));
             }
             if (ok) {
@@ -273,7 +338,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
         // threads read one whole row, so the loads are conflict-free.
         const int et = threadIdx.x - SK_PROD_WARP0 * 32;
         bool ok = true;
-        for (int t = 0; t < (FP8 ? 0 : ns_i) && ok; ++t) {
+        for (int t = 0; t < (DIRECT ? 0 : ns_i) && ok; ++t) {
             const int s = t % NST;
             const int nblk = min(2, n_i - 2 * t);
             const int u0 = 2 * t;  // operand ring uses u0, u0 + 1
@@ -350,12 +415,15 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
         const uint32_t off = static_cast<uint32_t>(((rank * RP + rl) * C::RSTRIDE) * 4);
         const uint32_t dst_i = sqd::map_to_cta(sbase + C::OFF_RED_I + off, static_cast<uint32_t>(owner));
         const uint32_t dst_f = sqd::map_to_cta(sbase + C::OFF_RED_F + off, static_cast<uint32_t>(owner));
-        const bool has_i = n_i > 0 && !*abort_flag, has_f = n_o > 0 && !*abort_flag;
+        // MX: one accumulator in [0, MP), sent as the "fp32" partial.
+        const bool has_i = !MX && n_i > 0 && !*abort_flag;
+        const bool has_f = (MX ? (n_i + n_o > 0) : n_o > 0) && !*abort_flag;
+        const uint32_t col_f = MX ? 0u : static_cast<uint32_t>(MP);
 #pragma unroll 1
         for (int ch = 0; ch < MP / 16; ++ch) {
             uint32_t vi[16] = {}, vf[16] = {};
             if (has_i) sqd::tmem_ld_32x32b_x16(tl + ch * 16, vi);
-            if (has_f) sqd::tmem_ld_32x32b_x16(tl + MP + ch * 16, vf);
+            if (has_f) sqd::tmem_ld_32x32b_x16(tl + col_f + ch * 16, vf);
             sqd::tmem_wait_ld_dep(vi, vf);
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
@@ -389,7 +457,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
             }
             const int ai = si >> 8;
             const float al = FP8 ? sl : static_cast<float>(ai);
-            const float y = __fadd_rn(__fmul_rn(__fmul_rn(al, args.s_x[m]), args.s_w[n]), sf);
+            const float y = MX ? sf : __fadd_rn(__fmul_rn(__fmul_rn(al, args.s_x[m]), args.s_w[n]), sf);
             args.Y[static_cast<long long>(m) * args.ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
             if constexpr (DBG) {
                 if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n] = FP8 ? __float_as_int(sl) : ai;

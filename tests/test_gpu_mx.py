@@ -109,6 +109,11 @@ SHAPES = [
     (40, 2048, 384, 0),
     (100, 3072, 1152, 320),
     (128, 14336, 512, 1792),
+    # few tokens: the split-K kernel (one W tile -> 8 K ranges crossing the E2M1 / bf16 boundary)
+    (16, 4096, 128, 256),
+    (64, 8192, 256, 512),
+    (1, 1024, 64, 8),
+    (33, 2048, 1032, 0),
 ]
 
 
@@ -143,6 +148,13 @@ def test_mx_ties_signed_zero_and_zero_blocks():
     W = workloads.weights(N, K, seed=33).float()
     W[5] = 0.0
     check_layer_mx(O.numpy(), X.to(torch.bfloat16), W.to(torch.bfloat16))
+
+
+def test_mx_decode_sweep_point():
+    """M = 16 tokens against an 8192 x 8192 layer with nO = K/16 (a sweep point), every row."""
+    w = workloads.CONFIGS["sweep_M16_o1/16"]
+    O, X, W = workloads.make(w)
+    check_layer_mx(O.numpy(), X, W)
 
 
 def test_mx_qkv_sampled():
