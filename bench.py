@@ -67,8 +67,9 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str, kernel: str):
-    """DRAM bytes per launch from the committed ncu summary, if the kernels are unchanged since."""
+def recorded_traffic(workload: str, kernel: str, low: str = "int4"):
+    """DRAM bytes per launch from the committed ncu summary, if the kernels are unchanged since.
+    Entries of the FP8 and MX low paths are keyed "<workload>|<low>"."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -76,7 +77,8 @@ def recorded_traffic(workload: str, kernel: str):
         d = json.load(f)
     if d.get("source_hash") != source_hash():
         return None
-    return d.get("workloads", {}).get(workload, {}).get(kernel)
+    key = workload if low == "int4" else f"{workload}|{low}"
+    return d.get("workloads", {}).get(key, {}).get(kernel)
 
 
 def gemm_bytes(M, N, K, nO, cb=0.5, rs=4):
@@ -489,12 +491,12 @@ def main():
             "config": {**w.describe(), "low_path": args.low, "parallelism": f"dp{world}" if world > 1 else "single",
                        "l2": f"{n_sets} rotating input sets of {foot / 1e6:.0f} MB (> L2 {l2 / 1e6:.0f} MB)",
                        "timing": "K steps replayed from one CUDA graph; per-kernel times from graphs of K launches"},
-            "roofline": {**gemm_roof, "traffic": recorded_traffic(w.name, "dual_gemm"),
+            "roofline": {**gemm_roof, "traffic": recorded_traffic(w.name, "dual_gemm", args.low),
                          "kernel": "dual_gemm", "ms": ms_gemm, "algorithmic_bytes": g_bytes,
                          "algorithmic_ops": flops},
             "quant_gather": {"bound": "hbm", "achieved": qg_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                              "frac": qg_gbs / peaks["hbm_gbs"], "ms": ms_qg, "algorithmic_bytes": qg_bytes,
-                             "traffic": recorded_traffic(w.name, "rowquant")},
+                             "traffic": recorded_traffic(w.name, "rowquant", args.low)},
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": 2 * M * K,
                     "d2h_bytes_per_step": 2 * M * N, "ms_per_step": ms_e2e},
             "cpu_baseline": cpu,
