@@ -16,7 +16,10 @@ inputs of W2 (E4M3 low path, scale = absolute maximum / 448; readings in the C
 file).  The MX functions follow the OSC abstract's fit with 4-bit
 micro-scaling hardware (and the SQ-format write-up, section 8, FP4 variant):
 the normal channels in MXFP4, blocks of 32 with an E8M0 scale each (readings
-in the C file).
+in the C file).  The SQF functions follow the SQ-format write-up's element-level
+format for weights (banks with a fixed number of high-precision entries chosen
+by magnitude, INT4 low part with the mask code -8, E4M3 high part; readings in
+the C file).
 """
 from __future__ import annotations
 
@@ -73,8 +76,11 @@ def _load():
             lib.orc_mx_block_exponent.argtypes = [ctypes.c_double]
             lib.orc_quantize_rows_mx.argtypes = [P, I, I, I, P, I, P, P, P]
             lib.orc_dual_linear_rows_mx.argtypes = [P, P, P, I, P, P, P, I, I, I, P, P, P]
+            C = ctypes.c_int
+            lib.orc_sqf_weights.argtypes = [P, I, I, I, C, C, P, P, P, P, P]
+            lib.orc_sqf_linear_rows.argtypes = [P, P, P, P, I, P, P, P, P, P, I, I, P, P, P]
             for f in (lib.orc_e2m1_encode_array, lib.orc_mx_block_exponent, lib.orc_quantize_rows_mx,
-                      lib.orc_dual_linear_rows_mx):
+                      lib.orc_dual_linear_rows_mx, lib.orc_sqf_weights, lib.orc_sqf_linear_rows):
                 f.restype = ctypes.c_int
             for f in (lib.orc_validate_outliers, lib.orc_quantize_rows, lib.orc_pack_int4,
                       lib.orc_chan_table, lib.orc_dual_linear_rows, lib.orc_num_threads,
@@ -383,3 +389,77 @@ def mx_scale_tiles(e8: np.ndarray, rows_pad: int, blocks_pad: int) -> np.ndarray
     out = np.zeros(rows_pad * blocks_pad, np.uint8)
     out[off.reshape(-1)] = full.reshape(-1)
     return out
+
+
+# ---------------------------------------------------------------- element-level SQ-format (weights)
+SQF_BANKS = [(4, 1), (4, 2), (8, 1), (8, 2), (16, 1), (16, 2)]   # (bank, high entries per bank)
+
+
+def sqf_weights(W_bits: np.ndarray, bank: int, h: int):
+    """Element-level SQ-format of bf16 weight rows: dict with lo (int8 [N, K], -8 at high
+    positions), s_lo (fp32 [N]), hi_mask (uint8 [N, K]), hi (uint8 E4M3 [N, K], 0 at low
+    positions), s_hi (fp32 [N])."""
+    src = np.ascontiguousarray(W_bits, np.uint16)
+    rows, K = src.shape
+    lo = np.zeros((rows, K), np.int8)
+    s_lo = np.zeros(rows, np.float32)
+    mask = np.zeros((rows, K), np.uint8)
+    hi = np.zeros((rows, K), np.uint8)
+    s_hi = np.zeros(rows, np.float32)
+    if _load().orc_sqf_weights(_ptr(src), rows, K, K, bank, h, _ptr(lo), _ptr(s_lo), _ptr(mask), _ptr(hi),
+                               _ptr(s_hi)) != 0:
+        raise ValueError("need 1 <= h < bank and K % bank == 0")
+    return dict(lo=lo, s_lo=s_lo, hi_mask=mask, hi=hi, s_hi=s_hi)
+
+
+def sqf_linear(X_bits: np.ndarray, W_bits: np.ndarray, bank: int, h: int, rows=None):
+    """Whole layer with element-level SQ-format weights for the selected token rows (all when None):
+    the weight format (sqf_weights), the tokens' INT4 and E4M3 codes over all channels, and
+    acc_lo (int64), acc_hi (fp64), y (fp64), each [rows, N]."""
+    K = W_bits.shape[1]
+    Xs = np.ascontiguousarray(X_bits if rows is None else X_bits[np.asarray(rows)], np.uint16)
+    none = np.zeros(0, np.int32)
+    qx4, sx4, _ = quantize_rows(Xs, K, none)
+    qx8, sx8, _ = quantize_rows_fp8(Xs, K, none)
+    w = sqf_weights(W_bits, bank, h)
+    Mr, N = Xs.shape[0], W_bits.shape[0]
+    acc_lo = np.zeros((Mr, N), np.int64)
+    acc_hi = np.zeros((Mr, N), np.float64)
+    y = np.zeros((Mr, N), np.float64)
+    _load().orc_sqf_linear_rows(_ptr(qx4), _ptr(sx4), _ptr(qx8), _ptr(sx8), Mr, _ptr(w["lo"]), _ptr(w["s_lo"]),
+                                _ptr(w["hi_mask"]), _ptr(w["hi"]), _ptr(w["s_hi"]), N, K,
+                                _ptr(acc_lo), _ptr(acc_hi), _ptr(y))
+    return dict(w, qx4=qx4, sx4=sx4, qx8=qx8, sx8=sx8, acc_lo=acc_lo, acc_hi=acc_hi, y=y)
+
+
+def compress_24(hi_mask: np.ndarray, hi_codes: np.ndarray):
+    """2:4 storage of the high part (format definition): for every aligned group of 4
+    channels, 2 value bytes (the group's high codes in channel order; a group with fewer
+    than two high channels stores zeros in the free slots) and one metadata nibble (group i
+    in byte i // 2, low nibble for even i) whose bits [1:0] and [3:2] give the in-group
+    indices of the two stored values, first < second.  One high channel at index p uses
+    indices (p, p + 1) with the zero second, or (2, 3) with the zero first when p = 3; no
+    high channel uses (0, 1).  Returns (values uint8 [rows, K/2], meta uint8 [rows, K/8])."""
+    mask = np.asarray(hi_mask, np.uint8)
+    codes = np.asarray(hi_codes, np.uint8)
+    rows, K = mask.shape
+    vals = np.zeros((rows, K // 2), np.uint8)
+    meta = np.zeros((rows, K // 8), np.uint8)
+    for r in range(rows):
+        for g in range(K // 4):
+            idx = [i for i in range(4) if mask[r, 4 * g + i]]
+            assert len(idx) <= 2, "more than two high channels in a group of four"
+            if len(idx) == 2:
+                i0, i1 = idx
+                v0, v1 = codes[r, 4 * g + i0], codes[r, 4 * g + i1]
+            elif len(idx) == 1:
+                p = idx[0]
+                if p < 3:
+                    i0, i1, v0, v1 = p, p + 1, codes[r, 4 * g + p], 0
+                else:
+                    i0, i1, v0, v1 = 2, 3, 0, codes[r, 4 * g + 3]
+            else:
+                i0, i1, v0, v1 = 0, 1, 0, 0
+            vals[r, 2 * g], vals[r, 2 * g + 1] = v0, v1
+            meta[r, g // 2] |= (i0 | (i1 << 2)) << (4 * (g % 2))
+    return vals, meta

@@ -469,6 +469,119 @@ int orc_dual_linear_rows_mx(const uint8_t *qx, const uint8_t *ex, const uint16_t
     return 0;
 }
 
+/* ------------------------------------------------------------------ element-level SQ-format weights
+ * SQ-format write-up of arXiv:2512.05409: section 3 (the low-precision part
+ * keeps its storage format with a mask value marking the positions that need
+ * high precision, which a gather unit handles as sparse data), section 7
+ * (banks with a fixed sparsity pattern each), section 9 (symmetric
+ * quantization, the unused top code is the mask; in each bank the top (1-s)
+ * fraction by importance is high precision), section 8 (FP8/FP4 combination);
+ * the abstract (the sparse part is accelerated in high precision).  Readings
+ * taken where the pages leave it open:
+ *   - a bank is `bank` consecutive input channels of one weight row; its `h`
+ *     channels with the largest |w| are high precision (importance without
+ *     calibration Hessians reduces to the magnitude), ties to the lower index;
+ *   - low part: symmetric INT4 over the row's low channels, s_lo = a/7 (fp32),
+ *     code = clamp(rint(fl(w/s_lo)), -7, 7), and the mask code -8 at every
+ *     high position; a == 0 gives s_lo = 0 and zero codes (the mask stays);
+ *   - high part: FP8 E4M3 with s_hi = (absmax over the row's high channels) /
+ *     448, code = E4M3 nearest to fl(w/s_hi) as for the FP8 path;
+ *   - activations: per token, INT4 over all K channels for the low part and
+ *     E4M3 over all K channels for the high part (the two row quantizers of
+ *     this file with an empty outlier set);
+ *   - Y = s_x4 s_lo sum_{k low} qx4 qw + s_x8 s_hi sum_{k high} e(x) e(w).
+ */
+
+/* One weight row: in each bank, mark the h channels with the largest |w|
+ * (ties to the lower index) in hi[k] (1 high, 0 low). */
+static void orc_bank_select(const uint16_t *row, int64_t K, int bank, int h, char *hi)
+{
+    for (int64_t g = 0; g < K / bank; ++g) {
+        for (int i = 0; i < bank; ++i) {
+            const int64_t k = g * bank + i;
+            const float vi = fabsf(orc_bf16_to_f32(row[k]));
+            int rank = 0; /* channels of the bank ranked above channel k */
+            for (int j = 0; j < bank; ++j) {
+                const float vj = fabsf(orc_bf16_to_f32(row[g * bank + j]));
+                if (vj > vi || (vj == vi && j < i)) ++rank;
+            }
+            hi[k] = (char)(rank < h);
+        }
+    }
+}
+
+/* Element-level SQ-format of weight rows (bf16 [rows, ld]).
+ * Outputs: lo [rows, K] int8 codes (-8 at high positions), s_lo [rows],
+ * hi_mask [rows, K] (1 at high positions), hi_codes [rows, K] E4M3 (0 at low
+ * positions), s_hi [rows].  K % bank == 0, 1 <= h < bank. */
+int orc_sqf_weights(const uint16_t *src, int64_t rows, int64_t K, int64_t ld, int bank, int h,
+                    int8_t *lo, float *s_lo, uint8_t *hi_mask, uint8_t *hi_codes, float *s_hi)
+{
+    if (bank < 2 || h < 1 || h >= bank || K % bank != 0 || ld < K) return -1;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *row = src + r * ld;
+        char *hi = (char *)(hi_mask + r * K);
+        orc_bank_select(row, K, bank, h, hi);
+        float a = 0.0f, ah = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            const float v = fabsf(orc_bf16_to_f32(row[k]));
+            if (hi[k]) { if (v > ah) ah = v; }
+            else if (v > a) a = v;
+        }
+        const float s = (a == 0.0f) ? 0.0f : a / 7.0f;
+        const float sh = (ah == 0.0f) ? 0.0f : ah / 448.0f;
+        s_lo[r] = s;
+        s_hi[r] = sh;
+        for (int64_t k = 0; k < K; ++k) {
+            const float x = orc_bf16_to_f32(row[k]);
+            if (hi[k]) {
+                lo[r * K + k] = -8;
+                hi_codes[r * K + k] = (ah == 0.0f) ? 0 : orc_e4m3_encode(x / sh);
+            } else {
+                int q = 0;
+                if (a != 0.0f) {
+                    q = (int)nearbyintf(x / s);
+                    if (q > ORC_QMAX) q = ORC_QMAX;
+                    if (q < -ORC_QMAX) q = -ORC_QMAX;
+                }
+                lo[r * K + k] = (int8_t)q;
+                hi_codes[r * K + k] = 0;
+            }
+        }
+    }
+    return 0;
+}
+
+/* Products of the element-level format for Mr token rows against N weight
+ * rows.  qx4 / sx4: INT4 codes and scales of the tokens over all K channels;
+ * qx8 / sx8: their E4M3 codes and scales.
+ *   acc_lo [Mr, N]  exact integer sum over the low positions (int64)
+ *   acc_hi [Mr, N]  sum of decoded E4M3 products over the high positions (fp64)
+ *   y      [Mr, N]  acc_lo sx4 s_lo + acc_hi sx8 s_hi (fp64) */
+int orc_sqf_linear_rows(const int8_t *qx4, const float *sx4, const uint8_t *qx8, const float *sx8, int64_t Mr,
+                        const int8_t *lo, const float *s_lo, const uint8_t *hi_mask, const uint8_t *hi_codes,
+                        const float *s_hi, int64_t N, int64_t K, int64_t *acc_lo, double *acc_hi, double *y)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < Mr; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t al = 0;
+            double ahs = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                if (hi_mask[n * K + k])
+                    ahs += orc_e4m3_decode(qx8[m * K + k]) * orc_e4m3_decode(hi_codes[n * K + k]);
+                else
+                    al += (int64_t)qx4[m * K + k] * (int64_t)lo[n * K + k];
+            }
+            acc_lo[m * N + n] = al;
+            acc_hi[m * N + n] = ahs;
+            y[m * N + n] = (double)al * (double)sx4[m] * (double)s_lo[n] + ahs * (double)sx8[m] * (double)s_hi[n];
+        }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------------ static outlier selection
  * SQ-format write-up of arXiv:2512.05409, section 5 (static strategy for
  * activations) and section 9 (importance scores): the mean activation of each
