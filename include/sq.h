@@ -291,6 +291,63 @@ sq_status sq_linear_mx(const void *X, int64_t M, int64_t K, int64_t ldx,
                        void *workspace, size_t ws_bytes, sq_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Element-level SQ-format weights (no outlier channels).
+ *
+ * SQ-format (arXiv:2512.05409): abstract (the sparse part is accelerated in
+ * high precision, the dense low-precision part as a low-precision GEMM);
+ * write-up sections 3, 7, 8, 9 (a mask value in the low-precision format
+ * marks the high-precision positions; banks with a fixed sparsity; the top
+ * (1-s) of every bank by importance; FP8/FP4 combinations).
+ *
+ *   Y[m,n] = s_x4[m] s_lo[n] sum_{k low(n)}  q4(X)[m,k] q4(W)[n,k]
+ *          + s_x8[m] s_hi[n] sum_{k high(n)} e(X)[m,k]  e(W)[n,k]
+ *
+ *   - Banks: `bank` (4, 8 or 16) consecutive channels of a weight row; in each
+ *     the `h` (1 or 2) entries of largest |w| are high, ties to the lower
+ *     index (sparsity 1 - h/bank: 50 % to 93.75 %).
+ *   - Low part W_N [N, K/2]: packed INT4 as for sq_prepare_weights, s_lo =
+ *     (absmax over the row's low entries) / 7, mask code -8 at high positions
+ *     (the GEMM reads it as 0).
+ *   - High part: E4M3 codes of w / s_hi, s_hi = (absmax over the row's high
+ *     entries) / 448, stored 2:4: W_H [N, K/2] (two value bytes per aligned
+ *     group of 4 channels, the group's high codes in channel order, 0 in free
+ *     slots) and W_E [N, K/8] metadata (group i in byte i/2, low nibble for
+ *     even i; bits [1:0] and [3:2] = in-group indices of the two stored values,
+ *     first < second; one high entry at p < 3 uses (p, p+1), at 3 uses (2, 3);
+ *     none uses (0, 1)).
+ *   - Tokens: INT4 codes over all K channels (X_N [M, K/2], s_x4 = absmax/7)
+ *     and E4M3 codes over all K channels (X_8 [M, K], s_x8 = absmax/448).
+ *   - GEMM: the high part runs on the 2:4 sparse tensor cores (tcgen05.mma.sp,
+ *     kind::f8f6f4) into P [M, N] fp32 = s_x8 s_hi (e(X) e(W_hi)^T); the low
+ *     part is the INT4 GEMM with P added before the bf16 rounding:
+ *     Y = bf16_rn((float)acc_lo s_x4 s_lo + P).  dbg_acc_lo (nullable,
+ *     [M, N] int32): the exact low-part sums.
+ *   - Limits: K a multiple of 256 in [256, 16384]; N % 8 == 0.
+ * Error behaviour, ownership and stream ordering are those of the INT4 calls.
+ * ------------------------------------------------------------------------ */
+/* Workspace of sq_linear_sqf: X_N, s_x4, X_8, s_x8 and P, each 256-byte aligned. */
+size_t sq_linear_workspace_bytes_sqf(int64_t M, int64_t N, int64_t K);
+
+/* W: dev bf16 [N, ldw].  Writes W_N, s_lo, W_H, W_E, s_hi and chan_tab (K/8
+ * words, all zero: no outlier channels).  Waits for its own work. */
+sq_status sq_prepare_weights_sqf(const void *W, int64_t N, int64_t K, int64_t ldw, int bank, int h,
+                                 void *W_N, float *s_lo, void *W_H, void *W_E, float *s_hi,
+                                 uint32_t *chan_tab, sq_stream_t stream);
+
+sq_status sq_quant_gather_sqf(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab,
+                              void *X_N, float *s_x4, void *X_8, float *s_x8, sq_stream_t stream);
+
+/* P: dev fp32 [M, N] scratch (the high part). */
+sq_status sq_gemm_sqf(const void *X_N, const float *s_x4, const void *X_8, const float *s_x8,
+                      const void *W_N, const float *s_lo, const void *W_H, const void *W_E, const float *s_hi,
+                      int64_t M, int64_t N, int64_t K, void *Y, int64_t ldy, float *P,
+                      int32_t *dbg_acc_lo, sq_stream_t stream);
+
+sq_status sq_linear_sqf(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab,
+                        const void *W_N, const float *s_lo, const void *W_H, const void *W_E, const float *s_hi,
+                        int64_t N, void *Y, int64_t ldy, void *workspace, size_t ws_bytes, sq_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Static outlier-channel selection (the offline step that chooses O).
  *
  * SQ-format write-up of arXiv:2512.05409, section 5 (static strategy: mean

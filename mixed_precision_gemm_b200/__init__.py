@@ -39,6 +39,8 @@ __all__ = [
     "sq_selftest_watchdog", "sq_linear_workspace_bytes_fp8", "sq_prepare_weights_fp8", "sq_quant_gather_fp8",
     "sq_gemm_fp8", "sq_linear_fp8", "sq_kn_pad_mx", "sq_mx_scale_bytes", "sq_linear_workspace_bytes_mx",
     "sq_prepare_weights_mx", "sq_quant_gather_mx", "sq_gemm_mx", "sq_linear_mx",
+    "sq_linear_workspace_bytes_sqf", "sq_prepare_weights_sqf", "sq_quant_gather_sqf", "sq_gemm_sqf", "sq_linear_sqf",
+    "PreparedSQF", "prepare_weights_sqf", "quant_gather_sqf", "gemm_sqf",
     "sq_select_outliers_workspace_bytes", "sq_select_outliers", "select_outliers",
     "PreparedWeights", "prepare_weights", "quant_gather", "gemm", "SQLinear",
 ]
@@ -116,13 +118,21 @@ def load():
     lib.sq_quant_gather_mx.argtypes = [P, I, I, I, P, I, P, P, P, P]
     lib.sq_gemm_mx.argtypes = [P, P, P, P, P, P, I, I, I, I, P, I, P, P]
     lib.sq_linear_mx.argtypes = [P, I, I, I, P, P, P, P, I, I, P, I, P, Z, P]
+    C = ctypes.c_int
+    lib.sq_linear_workspace_bytes_sqf.argtypes = [I, I, I]
+    lib.sq_linear_workspace_bytes_sqf.restype = Z
+    lib.sq_prepare_weights_sqf.argtypes = [P, I, I, I, C, C, P, P, P, P, P, P, P]
+    lib.sq_quant_gather_sqf.argtypes = [P, I, I, I, P, P, P, P, P, P]
+    lib.sq_gemm_sqf.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, P, I, P, P, P]
+    lib.sq_linear_sqf.argtypes = [P, I, I, I, P, P, P, P, P, P, I, P, I, P, Z, P]
     lib.sq_select_outliers_workspace_bytes.argtypes = [I, I, I, I]
     lib.sq_select_outliers_workspace_bytes.restype = Z
     lib.sq_select_outliers.argtypes = [P, I, I, I, P, I, I, I, I, P, P, P, Z, P]
     for f in (lib.sq_prepare_weights, lib.sq_quant_gather, lib.sq_gemm, lib.sq_linear, lib.sq_check,
               lib.sq_selftest_watchdog, lib.sq_linear_noalloc, lib.sq_prepare_weights_fp8, lib.sq_quant_gather_fp8,
               lib.sq_gemm_fp8, lib.sq_linear_fp8, lib.sq_select_outliers, lib.sq_prepare_weights_mx,
-              lib.sq_quant_gather_mx, lib.sq_gemm_mx, lib.sq_linear_mx):
+              lib.sq_quant_gather_mx, lib.sq_gemm_mx, lib.sq_linear_mx, lib.sq_prepare_weights_sqf,
+              lib.sq_quant_gather_sqf, lib.sq_gemm_sqf, lib.sq_linear_sqf):
         f.restype = F
     _lib = lib
     return lib
@@ -348,6 +358,50 @@ def sq_linear_mx(X: torch.Tensor, chan_tab: torch.Tensor, W_N4, S_W, W_O, N: int
     _raise(st, "sq_linear_mx")
 
 
+# Element-level SQ-format weights (SQ-format write-up sections 3, 7, 8, 9): banks
+# of 4/8/16 channels with 1 or 2 E4M3 high entries (2:4 sparse tensor cores) and
+# an INT4 low part carrying the mask code -8.
+def sq_linear_workspace_bytes_sqf(M: int, N: int, K: int) -> int:
+    return int(load().sq_linear_workspace_bytes_sqf(M, N, K))
+
+
+def sq_prepare_weights_sqf(W: torch.Tensor, bank: int, h: int, W_N, s_lo, W_H, W_E, s_hi, chan_tab,
+                           stream=None) -> None:
+    _rowmajor(W, "W", torch.bfloat16)
+    N, K = W.shape
+    st = load().sq_prepare_weights_sqf(_ptr(W), N, K, W.stride(0), bank, h, _ptr(W_N), _ptr(s_lo), _ptr(W_H),
+                                       _ptr(W_E), _ptr(s_hi), _ptr(chan_tab), _stream(stream))
+    _raise(st, "sq_prepare_weights_sqf")
+
+
+def sq_quant_gather_sqf(X: torch.Tensor, chan_tab, X_N, s_x4, X_8, s_x8, stream=None) -> None:
+    _rowmajor(X, "X", torch.bfloat16)
+    M, K = X.shape
+    st = load().sq_quant_gather_sqf(_ptr(X), M, K, X.stride(0), _ptr(chan_tab), _ptr(X_N), _ptr(s_x4), _ptr(X_8),
+                                    _ptr(s_x8), _stream(stream))
+    _raise(st, "sq_quant_gather_sqf")
+
+
+def sq_gemm_sqf(X_N, s_x4, X_8, s_x8, W_N, s_lo, W_H, W_E, s_hi, M: int, N: int, K: int, Y: torch.Tensor,
+                P: torch.Tensor, dbg_acc_lo: Optional[torch.Tensor] = None, stream=None) -> None:
+    _rowmajor(Y, "Y", torch.bfloat16)
+    st = load().sq_gemm_sqf(_ptr(X_N), _ptr(s_x4), _ptr(X_8), _ptr(s_x8), _ptr(W_N), _ptr(s_lo), _ptr(W_H),
+                            _ptr(W_E), _ptr(s_hi), M, N, K, _ptr(Y), Y.stride(0), _ptr(P), _ptr(dbg_acc_lo),
+                            _stream(stream))
+    _raise(st, "sq_gemm_sqf")
+
+
+def sq_linear_sqf(X: torch.Tensor, chan_tab, W_N, s_lo, W_H, W_E, s_hi, N: int, Y: torch.Tensor,
+                  workspace: torch.Tensor, stream=None) -> None:
+    _rowmajor(X, "X", torch.bfloat16)
+    _rowmajor(Y, "Y", torch.bfloat16)
+    M, K = X.shape
+    st = load().sq_linear_sqf(_ptr(X), M, K, X.stride(0), _ptr(chan_tab), _ptr(W_N), _ptr(s_lo), _ptr(W_H),
+                              _ptr(W_E), _ptr(s_hi), N, _ptr(Y), Y.stride(0), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
+    _raise(st, "sq_linear_sqf")
+
+
 # Static outlier-channel selection (the offline step that chooses O).
 def sq_select_outliers_workspace_bytes(Mc: int, N: int, K: int, group: int = 1) -> int:
     return int(load().sq_select_outliers_workspace_bytes(Mc, N, K, group))
@@ -505,3 +559,55 @@ class SQLinear:
         fn = sq_linear_mx if pw.mx else sq_linear_fp8 if pw.fp8 else sq_linear
         fn(X, pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, pw.N, pw.nO, out, self.workspace(M, X.device), stream)
         return out
+
+
+@dataclasses.dataclass
+class PreparedSQF:
+    """Element-level SQ-format weights of one layer (see sq_prepare_weights_sqf)."""
+    N: int
+    K: int
+    bank: int
+    h: int
+    W_N: torch.Tensor       # uint8 [N, K/2] packed INT4, mask code -8 at high positions
+    s_lo: torch.Tensor      # float32 [N]
+    W_H: torch.Tensor       # uint8 [N, K/2] 2:4-compressed E4M3 high entries
+    W_E: torch.Tensor       # uint8 [N, K/8] 2:4 metadata
+    s_hi: torch.Tensor      # float32 [N]
+    chan_tab: torch.Tensor  # int32 [K/8], all zero (no outlier channels)
+
+
+def prepare_weights_sqf(W: torch.Tensor, bank: int, h: int, stream=None) -> PreparedSQF:
+    N, K = W.shape
+    dev = W.device
+    u8 = dict(dtype=torch.uint8, device=dev)
+    pw = PreparedSQF(N, K, bank, h, torch.zeros(N, K // 2, **u8), torch.zeros(N, dtype=torch.float32, device=dev),
+                     torch.zeros(N, K // 2, **u8), torch.zeros(N, K // 8, **u8),
+                     torch.zeros(N, dtype=torch.float32, device=dev),
+                     torch.zeros(K // 8, dtype=torch.int32, device=dev))
+    sq_prepare_weights_sqf(W, bank, h, pw.W_N, pw.s_lo, pw.W_H, pw.W_E, pw.s_hi, pw.chan_tab, stream)
+    return pw
+
+
+def quant_gather_sqf(X: torch.Tensor, pw: PreparedSQF, stream=None):
+    """(X_N int4 [M, K/2], s_x4 [M], X_8 e4m3 [M, K], s_x8 [M])."""
+    M, K = X.shape
+    dev = X.device
+    X_N = torch.empty(M, K // 2, dtype=torch.uint8, device=dev)
+    X_8 = torch.empty(M, K, dtype=torch.uint8, device=dev)
+    s_x4 = torch.empty(M, dtype=torch.float32, device=dev)
+    s_x8 = torch.empty(M, dtype=torch.float32, device=dev)
+    sq_quant_gather_sqf(X, pw.chan_tab, X_N, s_x4, X_8, s_x8, stream)
+    return X_N, s_x4, X_8, s_x8
+
+
+def gemm_sqf(X_N, s_x4, X_8, s_x8, pw: PreparedSQF, Y: Optional[torch.Tensor] = None, debug: bool = False,
+             stream=None):
+    """Y (bf16).  With debug=True returns (Y, acc_lo int32, P fp32 high part)."""
+    M = X_N.shape[0]
+    dev = X_N.device
+    if Y is None:
+        Y = torch.empty(M, pw.N, dtype=torch.bfloat16, device=dev)
+    P = torch.empty(M, pw.N, dtype=torch.float32, device=dev)
+    acc = torch.empty(M, pw.N, dtype=torch.int32, device=dev) if debug else None
+    sq_gemm_sqf(X_N, s_x4, X_8, s_x8, pw.W_N, pw.s_lo, pw.W_H, pw.W_E, pw.s_hi, M, pw.N, pw.K, Y, P, acc, stream)
+    return (Y, acc, P) if debug else Y

@@ -14,7 +14,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB_NAME = "libsq_b200.so"
 LIB_PATH = os.path.join(HERE, LIB_NAME)
 SOURCES = ["sq_abi.cu"]
-DEPS = ["sq_abi.cu", "sq_device.cuh", "sq_gemm_common.cuh", "sq_gemm_pair.cuh", "sq_gemm_skinny.cuh", "sq_mxquant.cuh", "sq_rowquant.cuh", "sq_rowquant_stream.cuh", "sq_select.cuh"]
+DEPS = ["sq_abi.cu", "sq_device.cuh", "sq_gemm_common.cuh", "sq_gemm_pair.cuh", "sq_gemm_skinny.cuh", "sq_mxquant.cuh", "sq_rowquant.cuh", "sq_rowquant_stream.cuh", "sq_select.cuh", "sq_sqf.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

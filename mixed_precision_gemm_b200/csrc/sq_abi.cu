@@ -23,6 +23,7 @@
 #include "sq_rowquant.cuh"
 #include "sq_rowquant_stream.cuh"
 #include "sq_select.cuh"
+#include "sq_sqf.cuh"
 
 namespace {
 
@@ -324,7 +325,8 @@ int raster_group(int tiles_m, int tile_rows, int64_t kn_pad, int64_t no_pad)
 template <class C, int LOW>
 sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O, const void *W_N,
                              const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K, int64_t nO, void *Y,
-                             int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+                             int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream,
+                             const float *addend = nullptr)
 {
     constexpr bool FP8 = LOW == sqg::kLowFp8, MX = LOW == sqg::kLowMx;
     const int64_t kn_pad = MX ? sq_kn_pad_mx(K, nO) : sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
@@ -361,6 +363,7 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
     a.Y = static_cast<uint16_t *>(Y);
     a.dbg_i = dbg_i;
     a.dbg_f = dbg_f;
+    a.addend = addend;
     a.M = static_cast<int>(M);
     a.N = static_cast<int>(N);
     a.ldy = ldy;
@@ -390,7 +393,8 @@ sq_status launch_gemm_pair_t(const DevInfo &di, const void *X_N, const float *s_
 template <class C, int LOW>
 sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *s_x, const void *X_O,
                                const void *W_N, const float *s_w, const void *W_O, int64_t M, int64_t N, int64_t K,
-                               int64_t nO, void *Y, int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream)
+                               int64_t nO, void *Y, int64_t ldy, int32_t *dbg_i, float *dbg_f, cudaStream_t stream,
+                               const float *addend = nullptr)
 {
     constexpr bool FP8 = LOW == sqg::kLowFp8, MX = LOW == sqg::kLowMx;
     const int64_t kn_pad = MX ? sq_kn_pad_mx(K, nO) : sq_kn_pad(K, nO), no_pad = sq_no_pad(nO);
@@ -430,6 +434,7 @@ sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *
     a.Y = static_cast<uint16_t *>(Y);
     a.dbg_i = dbg_i;
     a.dbg_f = dbg_f;
+    a.addend = addend;
     a.M = static_cast<int>(M);
     a.N = static_cast<int>(N);
     a.ldy = ldy;
@@ -808,6 +813,161 @@ sq_status linear_mx_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const
                            S_W, W_O, M, N, K, nO, Y, ldy, nullptr, s);
 }
 
+// ---------------------------------------------------------------- element-level SQ-format
+using CfgHigh32 = sqf::CfgHigh<32, 6>;
+using CfgHigh128 = sqf::CfgHigh<128, 4>;
+
+bool sqf_bank_ok(int bank, int h) { return (bank == 4 || bank == 8 || bank == 16) && (h == 1 || h == 2); }
+
+sq_status check_sqf_K(int64_t K)
+{
+    if (K < 256 || K > sqq::kStreamMaxK || K % 256 != 0)
+        return fail(SQ_ERR_INVALID_ARG, "the SQ-format path needs K a multiple of 256 in [256, %d] (K=%lld)",
+                    sqq::kStreamMaxK, (long long)K);
+    return SQ_OK;
+}
+
+size_t sqf_ws_bytes(int64_t M, int64_t N, int64_t K)
+{
+    if (M <= 0) return 0;
+    return static_cast<size_t>(round_up(M * K / 2, 256) + round_up(M * 4, 256) + round_up(M * K, 256) +
+                               round_up(M * 4, 256) + round_up(M * N * 4, 256));
+}
+
+sq_status prepare_sqf_impl(const void *W, int64_t N, int64_t K, int64_t ldw, int bank, int h, void *W_N, float *s_lo,
+                           void *W_H, void *W_E, float *s_hi, uint32_t *chan_tab, cudaStream_t s)
+{
+    SQ_TRY(check_sqf_K(K));
+    if (!sqf_bank_ok(bank, h)) return fail(SQ_ERR_INVALID_ARG, "bank must be 4, 8 or 16 and h 1 or 2 (bank=%d h=%d)", bank, h);
+    if (N < 0 || N > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "N out of range");
+    if (ldw < K || ldw % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldw must be >= K and a multiple of 8");
+    SQ_TRY(check_ptr(chan_tab, true, "chan_tab"));
+    if (N > 0) {
+        SQ_TRY(check_ptr(W, true, "W"));
+        SQ_TRY(check_ptr(W_N, true, "W_N"));
+        SQ_TRY(check_ptr(s_lo, true, "s_lo"));
+        SQ_TRY(check_ptr(W_H, true, "W_H"));
+        SQ_TRY(check_ptr(W_E, true, "W_E"));
+        SQ_TRY(check_ptr(s_hi, true, "s_hi"));
+    }
+    DevInfo di;
+    SQ_TRY(device_info(di));
+    // no outlier channels: the channel table is all zeros
+    cudaError_t e = cudaMemsetAsync(chan_tab, 0, static_cast<size_t>(K / 8) * 4, s);
+    if (e != cudaSuccess) return cuda_fail(e, "channel table");
+    if (N > 0) {
+        const int64_t grid = std::min<int64_t>((N + 7) / 8, static_cast<int64_t>(di.sms) * 8);
+        if ((e = launch_k(sqf::sqf_prep_kernel, dim3(static_cast<unsigned>(grid)), dim3(sqf::kPrepThreads), 0, s, 0u,
+                          static_cast<const uint16_t *>(W), static_cast<int>(N), static_cast<int>(K), ldw, bank, h,
+                          static_cast<uint8_t *>(W_N), s_lo, static_cast<uint8_t *>(W_H), static_cast<uint8_t *>(W_E),
+                          s_hi)) != cudaSuccess)
+            return cuda_fail(e, "SQ-format weight preparation");
+    }
+    if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_fail(e, "sq_prepare_weights_sqf");
+    return SQ_OK;
+}
+
+sq_status quant_sqf_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, void *X_N,
+                         float *s_x4, void *X_8, float *s_x8, cudaStream_t s)
+{
+    SQ_TRY(check_sqf_K(K));
+    if (M < 0 || M > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "M out of range");
+    if (ldx < K || ldx % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldx must be >= K and a multiple of 8");
+    if (M == 0) return SQ_OK;
+    SQ_TRY(check_ptr(X, true, "X"));
+    SQ_TRY(check_ptr(chan_tab, true, "chan_tab"));
+    SQ_TRY(check_ptr(X_N, true, "X_N"));
+    SQ_TRY(check_ptr(s_x4, true, "s_x4"));
+    SQ_TRY(check_ptr(X_8, true, "X_8"));
+    SQ_TRY(check_ptr(s_x8, true, "s_x8"));
+    const uint16_t *x = static_cast<const uint16_t *>(X);
+    SQ_TRY(launch_rowquant(x, M, K, ldx, chan_tab, 0, static_cast<uint8_t *>(X_N), s_x4, nullptr, s, false));
+    return launch_rowquant(x, M, K, ldx, chan_tab, 0, static_cast<uint8_t *>(X_8), s_x8, nullptr, s, true);
+}
+
+sq_status gemm_sqf_impl(const void *X_N, const float *s_x4, const void *X_8, const float *s_x8, const void *W_N,
+                        const float *s_lo, const void *W_H, const void *W_E, const float *s_hi, int64_t M, int64_t N,
+                        int64_t K, void *Y, int64_t ldy, float *P, int32_t *dbg_lo, cudaStream_t s)
+{
+    SQ_TRY(check_sqf_K(K));
+    if (M < 0 || M > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "M out of range");
+    if (N < 0 || N % 8 != 0 || N > (1ll << 30)) return fail(SQ_ERR_INVALID_ARG, "N must be a non-negative multiple of 8");
+    if (ldy < N || ldy % 8 != 0) return fail(SQ_ERR_INVALID_ARG, "ldy must be >= N and a multiple of 8");
+    if (M == 0 || N == 0) return SQ_OK;
+    SQ_TRY(check_ptr(X_N, true, "X_N"));
+    SQ_TRY(check_ptr(s_x4, true, "s_x4"));
+    SQ_TRY(check_ptr(X_8, true, "X_8"));
+    SQ_TRY(check_ptr(s_x8, true, "s_x8"));
+    SQ_TRY(check_ptr(W_N, true, "W_N"));
+    SQ_TRY(check_ptr(s_lo, true, "s_lo"));
+    SQ_TRY(check_ptr(W_H, true, "W_H"));
+    SQ_TRY(check_ptr(W_E, true, "W_E"));
+    SQ_TRY(check_ptr(s_hi, true, "s_hi"));
+    SQ_TRY(check_ptr(Y, true, "Y"));
+    SQ_TRY(check_ptr(P, true, "P"));
+    if (dbg_lo && !aligned16(dbg_lo)) return fail(SQ_ERR_MISALIGNED, "dbg_acc_lo is not 16-byte aligned");
+    DevInfo di;
+    SQ_TRY(device_info(di));
+    // 1. high part on the sparse tensor cores: P = s_x8 s_hi (e(X) . e(W_hi)^T)
+    CUtensorMap m_wh{}, m_we{}, m_x8{};
+    const bool small = M <= 32;
+    const int mt = small ? CfgHigh32::MT : CfgHigh128::MT;
+    SQ_TRY(make_map(m_wh, W_H, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B));
+    SQ_TRY(make_map(m_we, W_E, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 8, N, K / 8, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE));
+    SQ_TRY(make_map(m_x8, X_8, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, static_cast<uint32_t>(mt),
+                    CU_TENSOR_MAP_SWIZZLE_128B));
+    sqf::HighArgs ha;
+    ha.s_x8 = s_x8;
+    ha.s_hi = s_hi;
+    ha.P = P;
+    ha.M = static_cast<int>(M);
+    ha.N = static_cast<int>(N);
+    ha.K = static_cast<int>(K);
+    const dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((M + mt - 1) / mt));
+    auto kern = small ? sqf::sqf_high_kernel<CfgHigh32> : sqf::sqf_high_kernel<CfgHigh128>;
+    const size_t smem = small ? CfgHigh32::SMEM_BYTES : CfgHigh128::SMEM_BYTES;
+    int per_sm = 0;
+    SQ_TRY(kernel_setup(reinterpret_cast<const void *>(kern), sqf::kHiThreads, smem, per_sm, "SQ-format high part set-up"));
+    cudaError_t e = launch_k(kern, grid, dim3(sqf::kHiThreads), smem, s, 0u, m_wh, m_we, m_x8, ha);
+    if (e != cudaSuccess) return cuda_fail(e, "SQ-format high part launch");
+    // 2. low part (INT4, mask code cleared) with P added before the bf16 rounding
+    const float *sx = s_x4, *sw = s_lo;
+    if (M > 128)
+        return launch_gemm_pair_t<CfgPair, sqg::kLowSqf>(di, X_N, sx, nullptr, W_N, sw, nullptr, M, N, K, 0, Y, ldy,
+                                                         dbg_lo, nullptr, s, P);
+    if (M <= 16)
+        return launch_gemm_skinny_t<CfgSk16, sqg::kLowSqf>(di, X_N, sx, nullptr, W_N, sw, nullptr, M, N, K, 0, Y, ldy,
+                                                           dbg_lo, nullptr, s, P);
+    if (M <= 32)
+        return launch_gemm_skinny_t<CfgSk32, sqg::kLowSqf>(di, X_N, sx, nullptr, W_N, sw, nullptr, M, N, K, 0, Y, ldy,
+                                                           dbg_lo, nullptr, s, P);
+    if (M <= 64)
+        return launch_gemm_skinny_t<CfgSk64, sqg::kLowSqf>(di, X_N, sx, nullptr, W_N, sw, nullptr, M, N, K, 0, Y, ldy,
+                                                           dbg_lo, nullptr, s, P);
+    return launch_gemm_skinny_t<CfgSk128, sqg::kLowSqf>(di, X_N, sx, nullptr, W_N, sw, nullptr, M, N, K, 0, Y, ldy,
+                                                        dbg_lo, nullptr, s, P);
+}
+
+sq_status linear_sqf_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, const void *W_N,
+                          const float *s_lo, const void *W_H, const void *W_E, const float *s_hi, int64_t N, void *Y,
+                          int64_t ldy, void *workspace, size_t ws_bytes, cudaStream_t s)
+{
+    SQ_TRY(check_sqf_K(K));
+    if (M < 0 || N < 0) return fail(SQ_ERR_INVALID_ARG, "M and N must be non-negative");
+    if (M == 0 || N == 0) return SQ_OK;
+    const size_t need = sqf_ws_bytes(M, N, K);
+    if (ws_bytes < need) return fail(SQ_ERR_INVALID_ARG, "workspace of %zu bytes, %zu needed", ws_bytes, need);
+    SQ_TRY(check_ptr(workspace, true, "workspace"));
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint8_t *X_N = ws;
+    float *s_x4 = reinterpret_cast<float *>(ws + round_up(M * K / 2, 256));
+    uint8_t *X_8 = reinterpret_cast<uint8_t *>(s_x4) + round_up(M * 4, 256);
+    float *s_x8 = reinterpret_cast<float *>(X_8 + round_up(M * K, 256));
+    float *P = reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(s_x8) + round_up(M * 4, 256));
+    SQ_TRY(quant_sqf_impl(X, M, K, ldx, chan_tab, X_N, s_x4, X_8, s_x8, s));
+    return gemm_sqf_impl(X_N, s_x4, X_8, s_x8, W_N, s_lo, W_H, W_E, s_hi, M, N, K, Y, ldy, P, nullptr, s);
+}
+
 // ---------------------------------------------------------------- static outlier selection
 struct SelectLayout {
     int64_t nbx, nbw, off_px, off_pw, off_score, off_gs, bytes;
@@ -907,6 +1067,42 @@ size_t sq_linear_workspace_bytes(int64_t M, int64_t K, int64_t nO) { return line
 size_t sq_linear_workspace_bytes_fp8(int64_t M, int64_t K, int64_t nO) { return linear_ws_bytes(M, K, nO, true); }
 
 int64_t sq_kn_pad_mx(int64_t K, int64_t nO) { return round_up(K - nO, 256); }
+
+size_t sq_linear_workspace_bytes_sqf(int64_t M, int64_t N, int64_t K) { return sqf_ws_bytes(M, N, K); }
+
+sq_status sq_prepare_weights_sqf(const void *W, int64_t N, int64_t K, int64_t ldw, int bank, int h, void *W_N,
+                                 float *s_lo, void *W_H, void *W_E, float *s_hi, uint32_t *chan_tab,
+                                 sq_stream_t stream)
+{
+    g_detail.clear();
+    return prepare_sqf_impl(W, N, K, ldw, bank, h, W_N, s_lo, W_H, W_E, s_hi, chan_tab,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_quant_gather_sqf(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, void *X_N,
+                              float *s_x4, void *X_8, float *s_x8, sq_stream_t stream)
+{
+    g_detail.clear();
+    return quant_sqf_impl(X, M, K, ldx, chan_tab, X_N, s_x4, X_8, s_x8, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_gemm_sqf(const void *X_N, const float *s_x4, const void *X_8, const float *s_x8, const void *W_N,
+                      const float *s_lo, const void *W_H, const void *W_E, const float *s_hi, int64_t M, int64_t N,
+                      int64_t K, void *Y, int64_t ldy, float *P, int32_t *dbg_acc_lo, sq_stream_t stream)
+{
+    g_detail.clear();
+    return gemm_sqf_impl(X_N, s_x4, X_8, s_x8, W_N, s_lo, W_H, W_E, s_hi, M, N, K, Y, ldy, P, dbg_acc_lo,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
+sq_status sq_linear_sqf(const void *X, int64_t M, int64_t K, int64_t ldx, const uint32_t *chan_tab, const void *W_N,
+                        const float *s_lo, const void *W_H, const void *W_E, const float *s_hi, int64_t N, void *Y,
+                        int64_t ldy, void *workspace, size_t ws_bytes, sq_stream_t stream)
+{
+    g_detail.clear();
+    return linear_sqf_impl(X, M, K, ldx, chan_tab, W_N, s_lo, W_H, W_E, s_hi, N, Y, ldy, workspace, ws_bytes,
+                           reinterpret_cast<cudaStream_t>(stream));
+}
 
 size_t sq_mx_scale_bytes(int64_t rows, int64_t K, int64_t nO)
 {

@@ -43,7 +43,18 @@ constexpr int NUM_EXP_WARPS = 8;  // operand-producer warps of the pair kernel
 // row.  MX: packed E2M1 codes (kind::mxf4) with one E8M0 scale per 32
 // K-elements of each row; the tensor core applies the scales, so the low path
 // and the 16-bit branch accumulate into one fp32 accumulator.
-enum : int { kLowInt4 = 0, kLowFp8 = 1, kLowMx = 2 };
+// SQF: the element-level SQ-format (sq_sqf.cuh): INT4 low part whose mask code
+// -8 the expansion turns into 0, plus a precomputed fp32 high part added in
+// the epilogue (GemmArgs::addend).
+enum : int { kLowInt4 = 0, kLowFp8 = 1, kLowMx = 2, kLowSqf = 3 };
+
+// Expanded INT4 word (bytes 16*c) with the bytes of code -8 (0x80) cleared:
+// a byte is 0x80 exactly when bit 7 is set and bits 6..4 are clear.
+__device__ __forceinline__ uint32_t clear_mask_code(uint32_t x)
+{
+    const uint32_t nz = ((x & 0x70707070u) + 0x70707070u) & 0x80808080u;  // bit 7: bits 6..4 not all clear
+    return x ^ (x & ~nz & 0x80808080u);
+}
 constexpr int KB_MX = 256;        // E2M1 K elements per block (128 packed bytes per row)
 constexpr int MX_SF_BYTES = 3072; // scale bytes per ring slot: 2 tiles of X rows, 4 of W rows
 constexpr int MX_SFA_COL = 256;   // TMEM columns of the X-row scales (2 K-tiles x 4)
@@ -65,6 +76,7 @@ struct GemmArgs {
     int nkb_i;    // low-path K-blocks per tile (kn_pad / 128; MX: kn_pad / 256)
     int nkb_o;    // bf16 K-blocks per tile (no_pad / 64)
     int tiles_m, tiles_n, group_m;
+    const float *addend;   // SQF: fp32 [M, N] added to the low part in place of the 16-bit branch
 };
 
 // Tile t -> (M-tile, N-tile): groups of `group_m` M-tiles sweep all N-tiles,

@@ -98,7 +98,8 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
 {
     constexpr bool FP8 = LOW == kLowFp8;
     constexpr bool MX = LOW == kLowMx;
-    constexpr bool EXPAND = LOW == kLowInt4;
+    constexpr bool SQF = LOW == kLowSqf;
+    constexpr bool EXPAND = LOW == kLowInt4 || SQF;
     constexpr int OPS = C::OPS, EC = C::EXP_CHUNKS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -286,12 +287,13 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                 const uint32_t j = static_cast<uint32_t>(q & 3);
                 const uint32_t sw = static_cast<uint32_t>(r & 7);
                 const uint32_t row = dst + r * ROWB;
+                auto ex = [&](uint32_t v) { return SQF ? clear_mask_code(v) : v; };
                 sqd::sts128(row + (((2u * j) ^ sw) << 4),
-                            (w[c].x << 4) & 0xF0F0F0F0u, w[c].x & 0xF0F0F0F0u,
-                            (w[c].y << 4) & 0xF0F0F0F0u, w[c].y & 0xF0F0F0F0u);
+                            ex((w[c].x << 4) & 0xF0F0F0F0u), ex(w[c].x & 0xF0F0F0F0u),
+                            ex((w[c].y << 4) & 0xF0F0F0F0u), ex(w[c].y & 0xF0F0F0F0u));
                 sqd::sts128(row + (((2u * j + 1u) ^ sw) << 4),
-                            (w[c].z << 4) & 0xF0F0F0F0u, w[c].z & 0xF0F0F0F0u,
-                            (w[c].w << 4) & 0xF0F0F0F0u, w[c].w & 0xF0F0F0F0u);
+                            ex((w[c].z << 4) & 0xF0F0F0F0u), ex(w[c].z & 0xF0F0F0F0u),
+                            ex((w[c].w << 4) & 0xF0F0F0F0u), ex(w[c].w & 0xF0F0F0F0u));
             }
             sqd::fence_proxy_async_smem();
             __syncwarp();
@@ -427,6 +429,14 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                         if (n >= args.N) break;
                         const uint4 sw0 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g));
                         const uint4 sw1 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g + 4));
+                        // SQF: the precomputed high part of these 8 outputs
+                        float4 ad0 = make_float4(0.f, 0.f, 0.f, 0.f), ad1 = ad0;
+                        if constexpr (SQF) {
+                            const float4 *ap = reinterpret_cast<const float4 *>(args.addend + static_cast<long long>(m) * args.N + n);
+                            ad0 = ap[0];
+                            ad1 = ap[1];
+                        }
+                        const float adv[8] = {ad0.x, ad0.y, ad0.z, ad0.w, ad1.x, ad1.y, ad1.z, ad1.w};
                         const float swv[8] = {__uint_as_float(sw0.x), __uint_as_float(sw0.y), __uint_as_float(sw0.z),
                                               __uint_as_float(sw0.w), __uint_as_float(sw1.x), __uint_as_float(sw1.y),
                                               __uint_as_float(sw1.z), __uint_as_float(sw1.w)};
@@ -452,7 +462,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                                     al = static_cast<float>(ai);
                                     dbg_lo = ai;
                                 }
-                                const float af = (MX || has_o) ? __uint_as_float(vf[b][t]) : 0.0f;
+                                const float af = SQF ? adv[2 * h + u] : (MX || has_o) ? __uint_as_float(vf[b][t]) : 0.0f;
                                 y2[u] = MX ? af : __fadd_rn(__fmul_rn(__fmul_rn(al, sx), swv[2 * h + u]), af);
                                 if constexpr (DBG) {
                                     if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + 2 * h + u] = dbg_lo;

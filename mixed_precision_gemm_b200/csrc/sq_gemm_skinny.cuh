@@ -100,6 +100,7 @@ struct CfgSkinny {
 };
 
 struct SkinnyArgs {
+    const float *addend;   // SQF: fp32 [M, N] added in place of the 16-bit branch
     const float *s_x;
     const float *s_w;
     uint16_t *Y;
@@ -138,6 +139,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
     constexpr bool FP8 = LOW == kLowFp8;
     constexpr bool MX = LOW == kLowMx;
     constexpr bool DIRECT = FP8 || MX;   // low-path stages read by the MMA in place
+    constexpr bool SQF = LOW == kLowSqf;  // INT4 stages with the mask code -8 cleared, fp32 addend
     constexpr int MP = C::MP, NST = C::NST, OPS = C::OPS, EC = C::EXP_CHUNKS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -369,10 +371,11 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
                     const uint32_t row = op_a((u0 + j) % OPS) + r * ROWB;
                     const uint32_t a0 = row + (((2u * jj) ^ sw) << 4);
                     const uint32_t a1 = row + (((2u * jj + 1u) ^ sw) << 4);
-                    const uint32_t lo0 = (w[c].x << 4) & 0xF0F0F0F0u, hi0 = w[c].x & 0xF0F0F0F0u;
-                    const uint32_t lo1 = (w[c].y << 4) & 0xF0F0F0F0u, hi1 = w[c].y & 0xF0F0F0F0u;
-                    const uint32_t lo2 = (w[c].z << 4) & 0xF0F0F0F0u, hi2 = w[c].z & 0xF0F0F0F0u;
-                    const uint32_t lo3 = (w[c].w << 4) & 0xF0F0F0F0u, hi3 = w[c].w & 0xF0F0F0F0u;
+                    auto ex = [&](uint32_t v) { return SQF ? clear_mask_code(v) : v; };
+                    const uint32_t lo0 = ex((w[c].x << 4) & 0xF0F0F0F0u), hi0 = ex(w[c].x & 0xF0F0F0F0u);
+                    const uint32_t lo1 = ex((w[c].y << 4) & 0xF0F0F0F0u), hi1 = ex(w[c].y & 0xF0F0F0F0u);
+                    const uint32_t lo2 = ex((w[c].z << 4) & 0xF0F0F0F0u), hi2 = ex(w[c].z & 0xF0F0F0F0u);
+                    const uint32_t lo3 = ex((w[c].w << 4) & 0xF0F0F0F0u), hi3 = ex(w[c].w & 0xF0F0F0F0u);
                     // The two K-blocks' threads of a row store in opposite
                     // order, so the eight stores of a phase hit distinct banks.
                     if (j == 0) {
@@ -457,7 +460,8 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
             }
             const int ai = si >> 8;
             const float al = FP8 ? sl : static_cast<float>(ai);
-            const float y = MX ? sf : __fadd_rn(__fmul_rn(__fmul_rn(al, args.s_x[m]), args.s_w[n]), sf);
+            const float add = SQF ? args.addend[static_cast<long long>(m) * args.N + n] : sf;
+            const float y = MX ? sf : __fadd_rn(__fmul_rn(__fmul_rn(al, args.s_x[m]), args.s_w[n]), add);
             args.Y[static_cast<long long>(m) * args.ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
             if constexpr (DBG) {
                 if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n] = FP8 ? __float_as_int(sl) : ai;

@@ -1,0 +1,346 @@
+// Element-level SQ-format weights on the sparse tensor cores.
+//
+// SQ-format (arXiv:2512.05409): the abstract (a sparse matrix is accelerated
+// in high precision while the dense low-precision product is accelerated as
+// usual); write-up section 3 (the low-precision part keeps its format with a
+// mask value at the positions handled in high precision by a gather of
+// sparse data), section 7 (banks with a fixed sparsity pattern), section 9
+// (the unused top code of symmetric quantization is the mask; the top (1-s)
+// of every bank by importance is high precision), section 8 (FP8/FP4).
+//
+// Format of a weight row (K channels, banks of `bank` = 4, 8 or 16 channels,
+// `h` = 1 or 2 high entries per bank -- sparsity 50 % to 93.75 %):
+//   - high set: per bank the h entries of largest |w|, ties to the lower index;
+//   - low part W_N: packed INT4 (byte j = code 2j | code 2j+1 << 4), symmetric
+//     codes clamp(rint(w / s_lo), -7, 7) with s_lo = (absmax over the low
+//     entries) / 7, and the mask code -8 at every high position;
+//   - high part: E4M3 codes of w / s_hi, s_hi = (absmax over the high
+//     entries) / 448, stored 2:4-compressed: W_H [N, K/2] bytes, two per
+//     aligned group of 4 channels (the group's high codes in channel order,
+//     zero in free slots), and W_E [N, K/8] metadata bytes, group i in byte
+//     i/2 (low nibble for even i), bits [1:0] / [3:2] = in-group index of the
+//     first / second stored value (first < second; one high entry at p uses
+//     (p, p+1), or (2, 3) with the zero first when p = 3; none uses (0, 1)).
+// With h <= 2 per bank and banks of 4, 8 or 16, no aligned group of 4 holds
+// more than two high entries, so the high part is exactly a 2:4 sparse matrix
+// for tcgen05.mma.sp (kind::f8f6f4).  The metadata layout was confirmed on the
+// device: a row-major [128 rows x 16 bytes] tile per 128 channels lands in
+// TMEM lanes 0..127, 4 columns, by tcgen05.cp.128x128b, and an MMA of 64
+// channels reads 2 of those columns.
+#pragma once
+
+#include <cuda_fp8.h>
+
+#include "sq_gemm_common.cuh"
+
+namespace sqf {
+
+constexpr int kPrepThreads = 256;        // 8 warps, one weight row per warp at a time
+constexpr int kChunk = 16;               // channels per lane per step (covers a bank of 16)
+
+__device__ __forceinline__ float bf16f(uint32_t b) { return __uint_as_float(b << 16); }
+
+// High mask (bit i = channel i is high) of 16 consecutive channels, banks of
+// `bank` channels, h per bank, by rank: entry i is high when fewer than h
+// entries of its bank are larger, or equal with a lower index.
+__device__ __forceinline__ uint32_t chunk_high_mask(const float (&a)[kChunk], int bank, int h)
+{
+    uint32_t mask = 0;
+#pragma unroll
+    for (int i = 0; i < kChunk; ++i) {
+        const int g0 = (i / bank) * bank;
+        int rank = 0;
+#pragma unroll
+        for (int j = 0; j < kChunk; ++j) {
+            const bool same_bank = j >= g0 && j < g0 + bank;
+            rank += (same_bank && (a[j] > a[i] || (a[j] == a[i] && j < i))) ? 1 : 0;
+        }
+        mask |= (rank < h ? 1u : 0u) << i;
+    }
+    return mask;
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, off));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t e4m3_of(float t)
+{
+    return static_cast<uint32_t>(__nv_cvt_float_to_fp8(t, __NV_SATFINITE, __NV_E4M3));
+}
+
+// Offline weight preparation: one warp per row (rows strided over the grid);
+// each lane takes 16 consecutive channels per step.  Pass 1 finds the row's
+// low and high absolute maxima, pass 2 writes the codes.  K % 16 == 0.
+__global__ void __launch_bounds__(kPrepThreads) sqf_prep_kernel(const uint16_t *__restrict__ W, int N, int K,
+                                                                 int64_t ldw, int bank, int h,
+                                                                 uint8_t *__restrict__ W_N, float *__restrict__ s_lo,
+                                                                 uint8_t *__restrict__ W_H, uint8_t *__restrict__ W_E,
+                                                                 float *__restrict__ s_hi)
+{
+    const int lane = threadIdx.x & 31;
+    const int warps = kPrepThreads / 32;
+    const int nchunk = K / kChunk;
+    for (int row = blockIdx.x * warps + (threadIdx.x >> 5); row < N; row += gridDim.x * warps) {
+        const uint16_t *wr = W + static_cast<int64_t>(row) * ldw;
+        auto load = [&](int c, float (&v)[kChunk]) {
+            const uint4 p0 = *reinterpret_cast<const uint4 *>(wr + kChunk * c);
+            const uint4 p1 = *reinterpret_cast<const uint4 *>(wr + kChunk * c + 8);
+            const uint32_t w[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                v[2 * i] = bf16f(w[i] & 0xFFFFu);
+                v[2 * i + 1] = bf16f(w[i] >> 16);
+            }
+        };
+        // pass 1: maxima of the low and the high entries
+        float amax_lo = 0.0f, amax_hi = 0.0f;
+        for (int c = lane; c < nchunk; c += 32) {
+            float v[kChunk], a[kChunk];
+            load(c, v);
+#pragma unroll
+            for (int i = 0; i < kChunk; ++i) a[i] = fabsf(v[i]);
+            const uint32_t hm = chunk_high_mask(a, bank, h);
+#pragma unroll
+            for (int i = 0; i < kChunk; ++i) {
+                if ((hm >> i) & 1u) amax_hi = fmaxf(amax_hi, a[i]);
+                else amax_lo = fmaxf(amax_lo, a[i]);
+            }
+        }
+        amax_lo = warp_max(amax_lo);
+        amax_hi = warp_max(amax_hi);
+        const float sl = amax_lo == 0.0f ? 0.0f : __fdiv_rn(amax_lo, 7.0f);
+        const float sh = amax_hi == 0.0f ? 0.0f : __fdiv_rn(amax_hi, 448.0f);
+        if (lane == 0) {
+            s_lo[row] = sl;
+            s_hi[row] = sh;
+        }
+        // pass 2: codes, 2:4 values and metadata
+        for (int c = lane; c < nchunk; c += 32) {
+            float v[kChunk], a[kChunk];
+            load(c, v);
+#pragma unroll
+            for (int i = 0; i < kChunk; ++i) a[i] = fabsf(v[i]);
+            const uint32_t hm = chunk_high_mask(a, bank, h);
+            uint32_t lo_w[2] = {0u, 0u};   // 16 nibbles
+            uint32_t hv[2] = {0u, 0u};     // 8 value bytes (4 groups x 2)
+            uint32_t meta = 0u;            // 4 nibbles
+#pragma unroll
+            for (int i = 0; i < kChunk; ++i) {
+                uint32_t q;
+                if ((hm >> i) & 1u) {
+                    q = 8u;   // mask code -8
+                } else if (amax_lo == 0.0f) {
+                    q = 0u;
+                } else {
+                    const float t = rintf(__fdiv_rn(v[i], sl));
+                    q = static_cast<uint32_t>(static_cast<int>(fminf(fmaxf(t, -7.0f), 7.0f))) & 15u;
+                }
+                lo_w[i >> 3] |= q << (4 * (i & 7));
+            }
+#pragma unroll
+            for (int g = 0; g < kChunk / 4; ++g) {
+                const uint32_t gm = (hm >> (4 * g)) & 15u;
+                uint32_t i0, i1, c0 = 0u, c1 = 0u;
+                const int n = __popc(gm);
+                if (n == 2) {
+                    i0 = __ffs(gm) - 1;
+                    i1 = 31 - __clz(gm);
+                } else if (n == 1) {
+                    const uint32_t p = __ffs(gm) - 1;
+                    i0 = p < 3 ? p : 2u;
+                    i1 = p < 3 ? p + 1 : 3u;
+                } else {
+                    i0 = 0u;
+                    i1 = 1u;
+                }
+                if (amax_hi != 0.0f) {
+                    if ((gm >> i0) & 1u) c0 = e4m3_of(__fdiv_rn(v[4 * g + i0], sh));
+                    if ((gm >> i1) & 1u) c1 = e4m3_of(__fdiv_rn(v[4 * g + i1], sh));
+                }
+                hv[g >> 1] |= (c0 | (c1 << 8)) << (16 * (g & 1));
+                meta |= (i0 | (i1 << 2)) << (4 * g);
+            }
+            const int64_t rb = static_cast<int64_t>(row) * (K / 2) + 8 * c;
+            *reinterpret_cast<uint2 *>(W_N + rb) = make_uint2(lo_w[0], lo_w[1]);
+            *reinterpret_cast<uint2 *>(W_H + rb) = make_uint2(hv[0], hv[1]);
+            *reinterpret_cast<uint16_t *>(W_E + static_cast<int64_t>(row) * (K / 8) + 2 * c) =
+                static_cast<uint16_t>(meta);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- high part
+// P[m, n] = s_x8[m] * s_hi[n] * sum over the 2:4 structure of e(X)[m, k] e(W)[n, k]
+// Swapped operands: the 128 W rows of a tile are the MMA's A side (the
+// sparse operand), MT tokens its N side.  A stage holds 256 channels: the
+// compressed W tile (128 bytes per row), two 128-channel boxes of E4M3
+// tokens and two 16-byte metadata boxes.  TMEM: accumulator in [0, MT), the
+// stage's metadata in [MT, MT + 8).
+constexpr int kHiWarps = 6;                 // 0 TMA, 1 MMA, 2..5 epilogue
+constexpr int kHiThreads = 32 * kHiWarps;
+enum : unsigned { SITE_HI_STG = 0x601, SITE_HI_MMA = 0x602, SITE_HI_EPI = 0x603 };
+
+template <int MT_, int NST_>
+struct CfgHigh {
+    static constexpr int MT = MT_;
+    static constexpr int NST = NST_;
+    static constexpr int A_BYTES = 128 * 128;
+    static constexpr int B_BYTES = MT * 128;          // one 128-channel box of tokens
+    static constexpr int E_BYTES = 128 * 16;          // one 128-channel metadata box
+    static constexpr int STAGE = A_BYTES + 2 * B_BYTES + 2 * E_BYTES;
+    static constexpr int OFF_BAR = NST * STAGE;
+    static constexpr int SMEM_BYTES = OFF_BAR + (2 * NST + 2) * 8 + 16 + 1024;
+    static constexpr int TMEM_COLS = MT + 8 <= 32 ? 32 : MT + 8 <= 64 ? 64 : MT + 8 <= 128 ? 128 : 256;
+    static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+struct HighArgs {
+    const float *s_x8;
+    const float *s_hi;
+    float *P;
+    int M, N, K;
+};
+
+template <class C>
+__global__ void __launch_bounds__(kHiThreads, 1)
+sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant__ CUtensorMap tm_we,
+                const __grid_constant__ CUtensorMap tm_x8, const HighArgs args)
+{
+    constexpr int MT = C::MT, NST = C::NST;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = sqd::smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n0 = static_cast<int>(blockIdx.x) * 128;
+    const int m0 = static_cast<int>(blockIdx.y) * MT;
+    sqd::pdl_launch_dependents();
+
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (NST + s); };
+    const uint32_t acc_full = bar0 + 8u * (2 * NST);
+    const uint32_t drain = acc_full + 8u;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + (2 * NST + 2) * 8);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(tmem_slot + 1);
+    auto stage = [&](int s) { return sbase + s * C::STAGE; };
+    const int nst_k = args.K / 256;   // stages
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            sqd::mbar_init(full(s), 1);
+            sqd::mbar_init(empty(s), 1);
+        }
+        sqd::mbar_init(acc_full, 1);
+        sqd::mbar_init(drain, 1);
+        *abort_flag = 0u;
+        sqd::fence_barrier_init();
+        sqd::fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        sqd::prefetch_tensormap(&tm_wh);
+        sqd::prefetch_tensormap(&tm_we);
+        sqd::prefetch_tensormap(&tm_x8);
+    }
+    if (warp == 1) {
+        sqd::tmem_alloc(sqd::smem_u32(tmem_slot), C::TMEM_COLS);
+        sqd::tmem_relinquish();
+    }
+    sqd::tc_fence_before();
+    __syncthreads();
+    sqd::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    sqd::pdl_wait();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int last = -1;
+            bool ok = true;
+            for (int t = 0; t < nst_k; ++t) {
+                const int s = t % NST;
+                if (!sqd::mbar_wait(empty(s), ((t / NST) & 1) ^ 1u, abort_flag, SITE_HI_STG)) { ok = false; break; }
+                const uint32_t st = stage(s);
+                sqd::mbar_arrive_expect_tx(full(s), C::STAGE);
+                sqd::tma_load_2d(st, &tm_wh, full(s), t * 128, n0);
+                sqd::tma_load_2d(st + C::A_BYTES, &tm_x8, full(s), t * 256, m0);
+                sqd::tma_load_2d(st + C::A_BYTES + C::B_BYTES, &tm_x8, full(s), t * 256 + 128, m0);
+                sqd::tma_load_2d(st + C::A_BYTES + 2 * C::B_BYTES, &tm_we, full(s), t * 32, n0);
+                sqd::tma_load_2d(st + C::A_BYTES + 2 * C::B_BYTES + C::E_BYTES, &tm_we, full(s), t * 32 + 16, n0);
+                last = t;
+            }
+            if (!ok && last >= 0) sqd::mbar_drain(full(last % NST), (last / NST) & 1);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // kind::f8f6f4, E4M3 x E4M3, fp32 D, sparse A (bit 2), M = 128, N = MT
+            constexpr uint32_t idesc = (1u << 2) | (1u << 4) | (static_cast<uint32_t>(MT >> 3) << 17) |
+                                       (static_cast<uint32_t>(128 >> 4) << 24);
+            const uint32_t ecol = tmem + MT;
+            bool ok = true;
+            for (int t = 0; t < nst_k && ok; ++t) {
+                const int s = t % NST;
+                if (!sqd::mbar_wait(full(s), (t / NST) & 1, abort_flag, SITE_HI_MMA)) { ok = false; break; }
+                sqd::tc_fence_after();
+                const uint32_t st = stage(s);
+                const uint32_t e0 = st + C::A_BYTES + 2 * C::B_BYTES;
+                asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(ecol), "l"(sqd::make_sf_desc(e0))
+                             : "memory");
+                asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(ecol + 4),
+                             "l"(sqd::make_sf_desc(e0 + C::E_BYTES))
+                             : "memory");
+                const uint64_t adesc = sqd::make_sw128_desc(st);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint64_t bdesc = sqd::make_sw128_desc(st + C::A_BYTES + (j >> 1) * C::B_BYTES) + 4 * (j & 1);
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                        "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%5], %3, p;\n\t}\n" ::"r"(tmem),
+                        "l"(adesc + 2 * j), "l"(bdesc), "r"(idesc), "r"((t == 0 && j == 0) ? 0u : 1u),
+                        "r"(ecol + 2 * j)
+                        : "memory");
+                }
+                sqd::mma_commit(empty(s));
+            }
+            if (ok) {
+                sqd::mma_commit(acc_full);
+            } else {
+                sqd::mma_commit(drain);
+                sqd::mbar_drain(drain, 0);
+            }
+        }
+    } else {
+        // epilogue: TMEM lane quarter warp % 4 = W rows n0 + 32 (warp % 4) + lane
+        const int q = warp & 3;
+        const int n = n0 + 32 * q + lane;
+        const bool n_ok = n < args.N;
+        const float sh = n_ok ? args.s_hi[n] : 0.0f;
+        if (sqd::mbar_wait(acc_full, 0, abort_flag, SITE_HI_EPI)) {
+            sqd::tc_fence_after();
+            const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
+            for (int c = 0; c < MT; c += 16) {
+                uint32_t v[16];
+                sqd::tmem_ld_32x32b_x16(tl + c, v);
+                sqd::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int m = m0 + c + i;
+                    if (n_ok && m < args.M)
+                        args.P[static_cast<int64_t>(m) * args.N + n] =
+                            __fmul_rn(__fmul_rn(__uint_as_float(v[i]), args.s_x8[m]), sh);
+                }
+            }
+        }
+    }
+    sqd::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        sqd::tc_fence_after();
+        sqd::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace sqf
