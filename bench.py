@@ -24,6 +24,7 @@ collective on the data path); value = all ranks' work / max-over-ranks time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import glob
 import hashlib
 import json
@@ -184,19 +185,34 @@ def oracle_fns(low: str):
     return oracle.quantize_rows, oracle.dual_linear_rows
 
 
-def time_oracle(w, O, X, W, target_s: float, max_rows: int | None = None, low: str = "int4"):
+def oracle_step_fn(low: str, w, O, Wb, bank: int = 16, high: int = 1):
+    """f(X_bits rows) running the oracle's online part for one batch of token rows; the
+    weights are prepared here, beforehand, as the offline step is on the GPU side."""
+    import oracle
+    if low == "sqf":
+        wf = oracle.sqf_weights(Wb, bank, high)
+        return lambda Xs: oracle.sqf_products(Xs, wf)
+    quantize, dual = oracle_fns(low)
+    On = O.numpy()
+    qw, sw, wo = quantize(Wb, w.K, On)
+
+    def f(Xs):
+        qx, sx, xo = quantize(Xs, w.K, On)
+        dual(qx, sx, xo, qw, sw, wo)
+    return f
+
+
+def time_oracle(w, O, X, W, target_s: float, max_rows: int | None = None, low: str = "int4",
+                bank: int = 16, high: int = 1):
     """Time the oracle on a bounded sample of token rows (weights quantized beforehand,
     as the offline step is on the GPU side).  Returns (TOPS, rows, seconds, cores)."""
     import oracle
-    quantize, dual = oracle_fns(low)
     Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
-    O = O.numpy()
-    qw, sw, wo = quantize(Wb, w.K, O)
+    step = oracle_step_fn(low, w, O, Wb, bank, high)
 
     def run(rows):
         t0 = time.perf_counter()
-        qx, sx, xo = quantize(Xb[:rows], w.K, O)
-        dual(qx, sx, xo, qw, sw, wo)
+        step(Xb[:rows])
         return time.perf_counter() - t0
 
     probe = min(8, w.M)
@@ -212,15 +228,12 @@ def run_reference(args, w, rank, world):
         return 0
     O, X, W = workloads.make(w)
     import oracle
-    quantize, dual = oracle_fns(args.low)
     Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
-    On = O.numpy()
-    qw, sw, wo = quantize(Wb, w.K, On)
     rows = args.ref_rows
+    f = oracle_step_fn(args.low, w, O, Wb, args.bank, args.high)
 
     def step():
-        qx, sx, xo = quantize(Xb[:rows], w.K, On)
-        dual(qx, sx, xo, qw, sw, wo)
+        f(Xb[:rows])
 
     for _ in range(args.warmup):
         step()
@@ -233,12 +246,19 @@ def run_reference(args, w, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64" if args.low == "int4" else "f64",
-            "data": "synthetic", "config": {**w.describe(), "low_path": args.low},
+            "data": "synthetic", "config": {**w.describe(), **low_config(args)},
             "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def low_config(args) -> dict:
+    if args.low == "sqf":
+        return {"low_path": "sqf", "nO": 0, "outlier_channels": "none (element-level format)",
+                "bank": args.bank, "high_per_bank": args.high, "sparsity": 1.0 - args.high / args.bank}
+    return {"low_path": args.low}
 
 
 # ----------------------------------------------------------------- GPU arm
@@ -254,9 +274,12 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=8, help="token rows per reference-arm step")
     ap.add_argument("--select-calib-rows", type=int, default=0,
                     help="also time the offline outlier selection on this many calibration rows (0: skip)")
-    ap.add_argument("--low", default="int4", choices=["int4", "fp8", "mx"],
-                    help="low path: INT4 (default), FP8 E4M3 (the pages' fallback for the inputs of W2) "
-                         "or MXFP4 (E2M1 with E8M0 block scales)")
+    ap.add_argument("--low", default="int4", choices=["int4", "fp8", "mx", "sqf"],
+                    help="low path: INT4 (default), FP8 E4M3 (the pages' fallback for the inputs of W2), "
+                         "MXFP4 (E2M1 with E8M0 block scales), or sqf: the element-level SQ-format "
+                         "(no outlier channels; banked E4M3 high entries on the 2:4 sparse tensor cores)")
+    ap.add_argument("--bank", type=int, default=16, help="sqf: channels per bank (4, 8, 16)")
+    ap.add_argument("--high", type=int, default=1, help="sqf: high-precision entries per bank (1, 2)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -288,7 +311,10 @@ def main():
     no_pad = sq.sq_no_pad(nO)
 
     # Rotating input sets so that every step reads operands that are not L2-resident.
-    fp8, mx = args.low == "fp8", args.low == "mx"
+    fp8, mx, sqf = args.low == "fp8", args.low == "mx", args.low == "sqf"
+    if sqf:
+        nO = 0
+        no_pad = 0
     cb = 1.0 if fp8 else 0.5 + 1.0 / 32 if mx else 0.5  # bytes per low-path code (MX: with its block scale)
     rs = 0 if mx else 4                                  # fp32 row-scale bytes per row
     if mx:
@@ -303,12 +329,32 @@ def main():
         gemm_fn = sq.sq_gemm_fp8 if fp8 else sq.sq_gemm
         linear_fn = sq.sq_linear_fp8 if fp8 else sq.sq_linear
     Xd = X.to(dev)
-    pw0 = sq.prepare_weights(W.to(dev), O, fp8=fp8, mx=mx)
-    foot = (2 * M * K + pw0.W_N.numel() + 2 * pw0.W_O.numel() + 4 * N + 2 * M * N + ws_bytes(M, K, nO))
+    if sqf:
+        def ws_bytes(M_, K_, nO_):
+            return sq.sq_linear_workspace_bytes_sqf(M_, N, K_)
+        pw0 = sq.prepare_weights_sqf(W.to(dev), args.bank, args.high)
+        foot = 2 * M * K + pw0.W_N.numel() + pw0.W_H.numel() + pw0.W_E.numel() + 8 * N + 2 * M * N + \
+            ws_bytes(M, K, 0)
+    else:
+        pw0 = sq.prepare_weights(W.to(dev), O, fp8=fp8, mx=mx)
+        foot = (2 * M * K + pw0.W_N.numel() + 2 * pw0.W_O.numel() + 4 * N + 2 * M * N + ws_bytes(M, K, nO))
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     n_sets = max(2, math.ceil(3 * l2 / foot))
     sets = []
-    for i in range(n_sets):
+    for i in range(n_sets if sqf else 0):
+        pw = pw0 if i == 0 else dataclasses.replace(
+            pw0, W_N=pw0.W_N.clone(), s_lo=pw0.s_lo.clone(), W_H=pw0.W_H.clone(), W_E=pw0.W_E.clone(),
+            s_hi=pw0.s_hi.clone())
+        sets.append({
+            "X": Xd if i == 0 else Xd.clone(), "pw": pw,
+            "X_N": torch.empty(M, K // 2, dtype=torch.uint8, device=dev),
+            "s_x4": torch.empty(M, dtype=torch.float32, device=dev),
+            "X_8": torch.empty(M, K, dtype=torch.uint8, device=dev),
+            "s_x8": torch.empty(M, dtype=torch.float32, device=dev),
+            "P": torch.empty(M, N, dtype=torch.float32, device=dev),
+            "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
+        })
+    for i in range(0 if sqf else n_sets):
         pw = pw0 if i == 0 else sq.PreparedWeights(N, K, nO, pw0.W_N.clone(), pw0.s_w.clone(), pw0.W_O.clone(),
                                                       pw0.chan_tab.clone(), fp8, mx)
         sets.append({
@@ -320,11 +366,18 @@ def main():
             "Y": torch.empty(M, N, dtype=torch.bfloat16, device=dev),
         })
     def quant(s, stream):
-        quant_gather_fn(s["X"], s["pw"].chan_tab, nO, s["X_N"], s["s_x"], s["X_O"], stream)
+        if sqf:
+            sq.sq_quant_gather_sqf(s["X"], s["pw"].chan_tab, s["X_N"], s["s_x4"], s["X_8"], s["s_x8"], stream)
+        else:
+            quant_gather_fn(s["X"], s["pw"].chan_tab, nO, s["X_N"], s["s_x"], s["X_O"], stream)
 
     def gemm(s, stream):
         pw = s["pw"]
-        gemm_fn(s["X_N"], s["s_x"], s["X_O"], pw.W_N, pw.s_w, pw.W_O, M, N, K, nO, s["Y"], None, None, stream)
+        if sqf:
+            sq.sq_gemm_sqf(s["X_N"], s["s_x4"], s["X_8"], s["s_x8"], pw.W_N, pw.s_lo, pw.W_H, pw.W_E, pw.s_hi,
+                           M, N, K, s["Y"], s["P"], None, stream)
+        else:
+            gemm_fn(s["X_N"], s["s_x"], s["X_O"], pw.W_N, pw.s_w, pw.W_O, M, N, K, nO, s["Y"], None, None, stream)
 
     def step(s, stream):
         quant(s, stream)
@@ -391,9 +444,14 @@ def main():
     low_ratio = MXF4_PER_BF16 if mx else INT8_PER_BF16
     p_i8 = low_ratio * p_bf
     t_roof_s = (2.0 * M * N * (K - nO)) / (p_i8 * 1e12) + (2.0 * M * N * nO) / (p_bf * 1e12)
+    if sqf:
+        # dense int8 over all K (low part) + 2:4 sparse e4m3 over all K at twice the dense e4m3 rate
+        t_roof_s = (2.0 * M * N * K) / (p_i8 * 1e12) + (2.0 * M * N * K) / (2 * INT8_PER_BF16 * p_bf * 1e12)
     peak_eff = flops / t_roof_s / 1e12
     gemm_tops = flops / (ms_gemm * 1e-3) / 1e12
     g_bytes = gemm_bytes(M, N, K, nO, cb, rs)
+    if sqf:   # W_N + W_H + W_E + 2 row scales, X_N + X_8 + 2 token scales, Y (the fp32 partial P excluded)
+        g_bytes = N * K / 2 + N * K / 2 + N * K / 8 + 8 * N + M * K / 2 + M * K + 8 * M + 2 * M * N
     t_hbm_s = g_bytes / (peaks["hbm_gbs"] * 1e9)
     if t_hbm_s > t_roof_s:
         # few tokens: the GEMM is bound by streaming the weights, not by the tensor cores
@@ -404,8 +462,11 @@ def main():
         gemm_roof = {"bound": "tensor", "achieved": gemm_tops, "peak": peak_eff, "unit": "TFLOP/s",
                      "frac": gemm_tops / peak_eff,
                      "peak_basis": f"{peaks['source']} bf16 {p_bf:.0f} TFLOP/s (burst), "
-                                   f"{args.low if args.low != 'int4' else 'int8'} = {low_ratio:g}x"}
+                                   f"{args.low if args.low not in ('int4', 'sqf') else 'int8'} = {low_ratio:g}x"
+                                   + ("; 2:4 sparse e4m3 = 2 x int8" if sqf else "")}
     qg_bytes = quant_gather_bytes(M, K, nO, cb, rs)
+    if sqf:   # X read once; INT4 and E4M3 codes plus two scales written
+        qg_bytes = 2 * M * K + M * K / 2 + M * K + 8 * M
     qg_gbs = qg_bytes / (ms_qg * 1e-3) / 1e9
 
     # end to end through sq_linear with pinned host buffers (copies inside the timed region)
@@ -418,7 +479,11 @@ def main():
         s = e2e_sets[i % len(e2e_sets)]
         s["X"].copy_(X_host, non_blocking=True)
         pw = s["pw"]
-        linear_fn(s["X"], pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, N, nO, s["Y"], ws[i % len(ws)], stream)
+        if sqf:
+            sq.sq_linear_sqf(s["X"], pw.chan_tab, pw.W_N, pw.s_lo, pw.W_H, pw.W_E, pw.s_hi, N, s["Y"],
+                             ws[i % len(ws)], stream)
+        else:
+            linear_fn(s["X"], pw.chan_tab, pw.W_N, pw.s_w, pw.W_O, N, nO, s["Y"], ws[i % len(ws)], stream)
         Y_host.copy_(s["Y"], non_blocking=True)
 
     for i in range(args.warmup):
@@ -476,7 +541,8 @@ def main():
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tops, rows, secs, cores = time_oracle(w, O, X, W, args.cpu_seconds, low=args.low)
+        tops, rows, secs, cores = time_oracle(w, O, X, W, args.cpu_seconds, low=args.low, bank=args.bank,
+                                              high=args.high)
         cpu = {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle",
                "sample": f"{rows} of {M} token rows x all {N} outputs ({secs:.1f} s; weights quantized beforehand)"}
 
@@ -486,9 +552,10 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None,
             "dtype": ("e4m3*e4m3->f32 + bf16*bf16->f32" if fp8 else
-                      "e2m1*e2m1 (e8m0 per 32)->f32 + bf16*bf16->f32" if mx else "s4*s4->s32 + bf16*bf16->f32"),
+                      "e2m1*e2m1 (e8m0 per 32)->f32 + bf16*bf16->f32" if mx else
+                      "s4*s4->s32 + e4m3 (2:4 sparse)*e4m3->f32" if sqf else "s4*s4->s32 + bf16*bf16->f32"),
             "data": "synthetic",
-            "config": {**w.describe(), "low_path": args.low, "parallelism": f"dp{world}" if world > 1 else "single",
+            "config": {**w.describe(), **low_config(args), "parallelism": f"dp{world}" if world > 1 else "single",
                        "l2": f"{n_sets} rotating input sets of {foot / 1e6:.0f} MB (> L2 {l2 / 1e6:.0f} MB)",
                        "timing": "K steps replayed from one CUDA graph; per-kernel times from graphs of K launches"},
             "roofline": {**gemm_roof, "traffic": recorded_traffic(w.name, "dual_gemm", args.low),
@@ -501,7 +568,7 @@ def main():
                     "d2h_bytes_per_step": 2 * M * N, "ms_per_step": ms_e2e},
             "cpu_baseline": cpu,
             "clocks": clocks,
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": (4 if sqf else 2) * args.steps,
         }
         if select is not None:
             line["select_outliers"] = select

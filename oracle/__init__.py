@@ -416,13 +416,18 @@ def sqf_linear(X_bits: np.ndarray, W_bits: np.ndarray, bank: int, h: int, rows=N
     """Whole layer with element-level SQ-format weights for the selected token rows (all when None):
     the weight format (sqf_weights), the tokens' INT4 and E4M3 codes over all channels, and
     acc_lo (int64), acc_hi (fp64), y (fp64), each [rows, N]."""
-    K = W_bits.shape[1]
-    Xs = np.ascontiguousarray(X_bits if rows is None else X_bits[np.asarray(rows)], np.uint16)
+    Xs = X_bits if rows is None else X_bits[np.asarray(rows)]
+    return sqf_products(Xs, sqf_weights(W_bits, bank, h))
+
+
+def sqf_products(X_bits: np.ndarray, w: dict):
+    """The layer for token rows X_bits against a weight format w from sqf_weights."""
+    Xs = np.ascontiguousarray(X_bits, np.uint16)
+    K = w["lo"].shape[1]
     none = np.zeros(0, np.int32)
     qx4, sx4, _ = quantize_rows(Xs, K, none)
     qx8, sx8, _ = quantize_rows_fp8(Xs, K, none)
-    w = sqf_weights(W_bits, bank, h)
-    Mr, N = Xs.shape[0], W_bits.shape[0]
+    Mr, N = Xs.shape[0], w["lo"].shape[0]
     acc_lo = np.zeros((Mr, N), np.int64)
     acc_hi = np.zeros((Mr, N), np.float64)
     y = np.zeros((Mr, N), np.float64)

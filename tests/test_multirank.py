@@ -64,12 +64,12 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
     import argparse
     import bench
     import workloads
-    args = argparse.Namespace(steps=1, warmup=0, ref_rows=1, low="int4")
+    args = argparse.Namespace(steps=1, warmup=0, ref_rows=1, low="int4", bank=16, high=1)
     assert bench.run_reference(args, workloads.TINY, rank=1, world=2) == 0
     assert capsys.readouterr().out == ""
 
 
-@pytest.mark.parametrize("low", ["int4", "fp8", "mx"])
+@pytest.mark.parametrize("low", ["int4", "fp8", "mx", "sqf"])
 def test_reference_arm_json_line(low):
     import json
     import subprocess
