@@ -466,10 +466,18 @@ sq_status launch_gemm_skinny_t(const DevInfo &di, const void *X_N, const float *
 using CfgPair = sqg::CfgPair<4, 4, 2>;
 using CfgPairF8 = sqg::CfgPair<6, 0, 2>;  // E4M3 tiles need no staging ring: a deeper operand ring instead
 using CfgPairMx = sqg::CfgPair<6, 0, 2, sqg::MX_SF_BYTES>;  // E2M1 tiles plus their block scales
-using CfgSk16 = sqg::CfgSkinny<16, 8, 3>;
-using CfgSk32 = sqg::CfgSkinny<32, 7, 3>;
-using CfgSk64 = sqg::CfgSkinny<64, 6, 2>;
-using CfgSk128 = sqg::CfgSkinny<128, 4, 2>;
+// INT4 stages carry two K-blocks; an operand ring of four slots lets the
+// expansion of one stage overlap the MMAs of the previous one (with fewer, the
+// expansion waits for the MMAs of its predecessor's own blocks).
+using CfgSk16 = sqg::CfgSkinny<16, 7, 4>;
+using CfgSk32 = sqg::CfgSkinny<32, 6, 4>;
+using CfgSk64 = sqg::CfgSkinny<64, 4, 4>;
+using CfgSk128 = sqg::CfgSkinny<128, 3, 4>;
+// E4M3 stages are read by the MMA in place: a deeper staging ring instead.
+using CfgSk16F8 = sqg::CfgSkinny<16, 8, 3>;
+using CfgSk32F8 = sqg::CfgSkinny<32, 7, 3>;
+using CfgSk64F8 = sqg::CfgSkinny<64, 6, 2>;
+using CfgSk128F8 = sqg::CfgSkinny<128, 4, 2>;
 // MX: no operand ring (stages are read in place), a deeper staging ring with 2 KB of scales per stage.
 using CfgSk16Mx = sqg::CfgSkinny<16, 10, 0, 2048>;
 using CfgSk32Mx = sqg::CfgSkinny<32, 9, 0, 2048>;
@@ -486,12 +494,12 @@ sq_status gemm_dispatch(const DevInfo &di, const void *X_N, const float *s_x, co
     if (M > 128)
         return launch_gemm_pair_t<Pair, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (M <= 16)
-        return launch_gemm_skinny_t<CfgSk16, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+        return launch_gemm_skinny_t<typename std::conditional<FP8, CfgSk16F8, CfgSk16>::type, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (M <= 32)
-        return launch_gemm_skinny_t<CfgSk32, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+        return launch_gemm_skinny_t<typename std::conditional<FP8, CfgSk32F8, CfgSk32>::type, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
     if (M <= 64)
-        return launch_gemm_skinny_t<CfgSk64, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
-    return launch_gemm_skinny_t<CfgSk128, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+        return launch_gemm_skinny_t<typename std::conditional<FP8, CfgSk64F8, CfgSk64>::type, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
+    return launch_gemm_skinny_t<typename std::conditional<FP8, CfgSk128F8, CfgSk128>::type, FP8 ? sqg::kLowFp8 : sqg::kLowInt4>(di, X_N, s_x, X_O, W_N, s_w, W_O, M, N, K, nO, Y, ldy, dbg_i, dbg_f, stream);
 }
 
 sq_status gemm_impl(const void *X_N, const float *s_x, const void *X_O, const void *W_N, const float *s_w,
