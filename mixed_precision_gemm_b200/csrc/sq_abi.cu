@@ -824,6 +824,7 @@ sq_status linear_mx_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const
 // ---------------------------------------------------------------- element-level SQ-format
 using CfgHigh32 = sqf::CfgHigh<32, 6>;
 using CfgHigh128 = sqf::CfgHigh<128, 4>;
+using CfgHighPair = sqf::CfgHighPair<4>;
 
 bool sqf_bank_ok(int bank, int h) { return (bank == 4 || bank == 8 || bank == 16) && (h == 1 || h == 2); }
 
@@ -916,10 +917,12 @@ sq_status gemm_sqf_impl(const void *X_N, const float *s_x4, const void *X_8, con
     if (dbg_lo && !aligned16(dbg_lo)) return fail(SQ_ERR_MISALIGNED, "dbg_acc_lo is not 16-byte aligned");
     DevInfo di;
     SQ_TRY(device_info(di));
-    // 1. high part on the sparse tensor cores: P = s_x8 s_hi (e(X) . e(W_hi)^T)
+    // 1. high part on the sparse tensor cores: P = s_x8 s_hi (e(X) . e(W_hi)^T); CTA pairs of
+    //    256 W rows x 256 tokens for M > 128, single CTAs of 128 W rows x 32 or 128 tokens otherwise
     CUtensorMap m_wh{}, m_we{}, m_x8{};
+    const bool pair = M > 128;
     const bool small = M <= 32;
-    const int mt = small ? CfgHigh32::MT : CfgHigh128::MT;
+    const int mt = small ? CfgHigh32::MT : CfgHigh128::MT;   // token rows per TMA box (128 for the pair kernel)
     SQ_TRY(make_map(m_wh, W_H, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B));
     SQ_TRY(make_map(m_we, W_E, CU_TENSOR_MAP_DATA_TYPE_UINT8, K / 8, N, K / 8, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE));
     SQ_TRY(make_map(m_x8, X_8, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, 128, static_cast<uint32_t>(mt),
@@ -931,16 +934,28 @@ sq_status gemm_sqf_impl(const void *X_N, const float *s_x4, const void *X_8, con
     ha.M = static_cast<int>(M);
     ha.N = static_cast<int>(N);
     ha.K = static_cast<int>(K);
-    const dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((M + mt - 1) / mt));
-    auto kern = small ? sqf::sqf_high_kernel<CfgHigh32> : sqf::sqf_high_kernel<CfgHigh128>;
-    const size_t smem = small ? CfgHigh32::SMEM_BYTES : CfgHigh128::SMEM_BYTES;
-    int per_sm = 0;
-    SQ_TRY(kernel_setup(reinterpret_cast<const void *>(kern), sqf::kHiThreads, smem, per_sm, "SQ-format high part set-up"));
-    cudaError_t e = launch_k(kern, grid, dim3(sqf::kHiThreads), smem, s, 0u, m_wh, m_we, m_x8, ha);
+    cudaError_t e;
+    if (pair) {
+        auto kern = sqf::sqf_high_pair_kernel<CfgHighPair>;
+        const int64_t pairs = ((N + 255) / 256) * ((M + 255) / 256);
+        int per_sm = 0;
+        SQ_TRY(kernel_setup(reinterpret_cast<const void *>(kern), sqf::kHiThreads, CfgHighPair::SMEM_BYTES, per_sm,
+                            "SQ-format high part set-up"));
+        e = launch_k(kern, dim3(static_cast<unsigned>(2 * pairs)), dim3(sqf::kHiThreads), CfgHighPair::SMEM_BYTES, s,
+                     0u, m_wh, m_we, m_x8, ha);
+    } else {
+        const dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((M + mt - 1) / mt));
+        auto kern = small ? sqf::sqf_high_kernel<CfgHigh32> : sqf::sqf_high_kernel<CfgHigh128>;
+        const size_t smem = small ? CfgHigh32::SMEM_BYTES : CfgHigh128::SMEM_BYTES;
+        int per_sm = 0;
+        SQ_TRY(kernel_setup(reinterpret_cast<const void *>(kern), sqf::kHiThreads, smem, per_sm,
+                            "SQ-format high part set-up"));
+        e = launch_k(kern, grid, dim3(sqf::kHiThreads), smem, s, 0u, m_wh, m_we, m_x8, ha);
+    }
     if (e != cudaSuccess) return cuda_fail(e, "SQ-format high part launch");
     // 2. low part (INT4, mask code cleared) with P added before the bf16 rounding
     const float *sx = s_x4, *sw = s_lo;
-    if (M > 128)
+    if (pair)
         return launch_gemm_pair_t<CfgPair, sqg::kLowSqf>(di, X_N, sx, nullptr, W_N, sw, nullptr, M, N, K, 0, Y, ldy,
                                                          dbg_lo, nullptr, s, P);
     if (M <= 16)

@@ -343,4 +343,169 @@ sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant
     }
 }
 
+// ---------------------------------------------------------------- high part, CTA pairs
+// The same product on 256 W rows x 256 tokens per cluster of two CTAs
+// (tcgen05 cta_group::2): each CTA supplies its 128 W rows (the sparse A
+// operand), their metadata and 128 of the 256 token rows (half of B), and
+// receives its 128 W rows x 256 tokens of D.  Per CTA a stage carries the same
+// 52 KB as the single-CTA kernel for twice the products, which halves the L2
+// traffic per product.  The metadata copy of a pair moves each CTA's own
+// shared memory into its own tensor memory.
+template <int NST_>
+struct CfgHighPair {
+    static constexpr int NST = NST_;
+    static constexpr int A_BYTES = 128 * 128;   // this CTA's 128 W rows, 256 channels (2:4)
+    static constexpr int B_BYTES = 128 * 128;   // this CTA's 128 tokens, one 128-channel box
+    static constexpr int E_BYTES = 128 * 16;    // metadata of this CTA's W rows, 128 channels
+    static constexpr int STAGE = A_BYTES + 2 * B_BYTES + 2 * E_BYTES;
+    static constexpr int OFF_BAR = NST * STAGE;
+    static constexpr int SMEM_BYTES = OFF_BAR + (2 * NST + 2) * 8 + 16 + 1024;
+    static constexpr int TMEM_COLS = 512;       // 256 accumulator columns + 8 metadata columns
+    static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
+    static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+template <class C>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kHiThreads, 1)
+sqf_high_pair_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant__ CUtensorMap tm_we,
+                     const __grid_constant__ CUtensorMap tm_x8, const HighArgs args)
+{
+    constexpr int NST = C::NST;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t sbase = sqd::smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = sqd::cluster_ctarank();
+    const bool leader = rank == 0;
+    const int tiles_n = (args.N + 255) / 256;
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int n0 = (pair % tiles_n) * 256 + static_cast<int>(rank) * 128;   // this CTA's W rows
+    const int m0 = (pair / tiles_n) * 256;                                   // the pair's tokens
+    sqd::pdl_launch_dependents();
+
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto full = [&](int s) { return bar0 + 8u * s; };
+    auto empty = [&](int s) { return bar0 + 8u * (NST + s); };
+    const uint32_t acc_full = bar0 + 8u * (2 * NST);
+    const uint32_t drain = acc_full + 8u;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + (2 * NST + 2) * 8);
+    volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(tmem_slot + 1);
+    auto stage = [&](int s) { return sbase + s * C::STAGE; };
+    const int nst_k = args.K / 256;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NST; ++s) {
+            sqd::mbar_init(full(s), 2);    // both CTAs' producers (the first CTA's copy is used)
+            sqd::mbar_init(empty(s), 1);   // multicast commit
+        }
+        sqd::mbar_init(acc_full, 1);       // multicast commit
+        sqd::mbar_init(drain, 1);
+        *abort_flag = 0u;
+        sqd::fence_barrier_init();
+        sqd::fence_proxy_async_smem();
+    }
+    if (warp == 0 && lane == 0) {
+        sqd::prefetch_tensormap(&tm_wh);
+        sqd::prefetch_tensormap(&tm_we);
+        sqd::prefetch_tensormap(&tm_x8);
+    }
+    if (warp == 1) {
+        sqd::tmem_alloc_pair(sqd::smem_u32(tmem_slot), C::TMEM_COLS);
+        sqd::tmem_relinquish_pair();
+    }
+    sqd::tc_fence_before();
+    sqd::cluster_sync();
+    sqd::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    sqd::pdl_wait();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int last = -1;
+            bool ok = true;
+            for (int t = 0; t < nst_k; ++t) {
+                const int s = t % NST;
+                if (!sqd::mbar_wait(empty(s), ((t / NST) & 1) ^ 1u, abort_flag, SITE_HI_STG)) { ok = false; break; }
+                const uint32_t st = stage(s);
+                const uint32_t fl = sqd::map_to_cta(full(s), 0);
+                const int mt = m0 + static_cast<int>(rank) * 128;
+                sqd::mbar_arrive_expect_tx_cluster(fl, C::STAGE);
+                sqd::tma_load_2d_pair(st, &tm_wh, fl, t * 128, n0);
+                sqd::tma_load_2d_pair(st + C::A_BYTES, &tm_x8, fl, t * 256, mt);
+                sqd::tma_load_2d_pair(st + C::A_BYTES + C::B_BYTES, &tm_x8, fl, t * 256 + 128, mt);
+                sqd::tma_load_2d_pair(st + C::A_BYTES + 2 * C::B_BYTES, &tm_we, fl, t * 32, n0);
+                sqd::tma_load_2d_pair(st + C::A_BYTES + 2 * C::B_BYTES + C::E_BYTES, &tm_we, fl, t * 32 + 16, n0);
+                last = t;
+            }
+            if (!ok && last >= 0 && leader) sqd::mbar_drain(full(last % NST), (last / NST) & 1);
+        }
+    } else if (warp == 1) {
+        if (leader && lane == 0) {
+            // kind::f8f6f4, E4M3 x E4M3, fp32 D, sparse A (bit 2), M = 256 (pair), N = 256
+            constexpr uint32_t idesc = (1u << 2) | (1u << 4) | (static_cast<uint32_t>(256 >> 3) << 17) |
+                                       (static_cast<uint32_t>(256 >> 4) << 24);
+            const uint32_t ecol = tmem + 256;
+            bool ok = true;
+            for (int t = 0; t < nst_k && ok; ++t) {
+                const int s = t % NST;
+                if (!sqd::mbar_wait(full(s), (t / NST) & 1, abort_flag, SITE_HI_MMA)) { ok = false; break; }
+                sqd::tc_fence_after();
+                const uint32_t st = stage(s);
+                const uint32_t e0 = st + C::A_BYTES + 2 * C::B_BYTES;
+                asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(ecol), "l"(sqd::make_sf_desc(e0))
+                             : "memory");
+                asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(ecol + 4),
+                             "l"(sqd::make_sf_desc(e0 + C::E_BYTES))
+                             : "memory");
+                const uint64_t adesc = sqd::make_sw128_desc(st);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint64_t bdesc = sqd::make_sw128_desc(st + C::A_BYTES + (j >> 1) * C::B_BYTES) + 4 * (j & 1);
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                        "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %1, %2, [%5], %3, p;\n\t}\n" ::"r"(tmem),
+                        "l"(adesc + 2 * j), "l"(bdesc), "r"(idesc), "r"((t == 0 && j == 0) ? 0u : 1u),
+                        "r"(ecol + 2 * j)
+                        : "memory");
+                }
+                sqd::mma_commit_pair_multicast(empty(s), 0x3);
+            }
+            if (ok) {
+                sqd::mma_commit_pair_multicast(acc_full, 0x3);
+            } else {
+                sqd::mma_commit_pair(drain);
+                sqd::mbar_drain(drain, 0);
+            }
+        }
+    } else {
+        // epilogue (each CTA): TMEM lane quarter warp % 4 = W rows n0 + 32 (warp % 4) + lane
+        const int q = warp & 3;
+        const int n = n0 + 32 * q + lane;
+        const bool n_ok = n < args.N;
+        const float sh = n_ok ? args.s_hi[n] : 0.0f;
+        if (sqd::mbar_wait(acc_full, 0, abort_flag, SITE_HI_EPI)) {
+            sqd::tc_fence_after();
+            const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
+            for (int c = 0; c < 256; c += 16) {
+                uint32_t v[16];
+                sqd::tmem_ld_32x32b_x16(tl + c, v);
+                sqd::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int m = m0 + c + i;
+                    if (n_ok && m < args.M)
+                        args.P[static_cast<int64_t>(m) * args.N + n] =
+                            __fmul_rn(__fmul_rn(__uint_as_float(v[i]), args.s_x8[m]), sh);
+                }
+            }
+        }
+    }
+    sqd::tc_fence_before();
+    sqd::cluster_sync();   // every pair MMA and TMEM read of both CTAs is done
+    if (warp == 1) {
+        sqd::tc_fence_after();
+        sqd::tmem_dealloc_pair(tmem, C::TMEM_COLS);
+    }
+}
+
 }  // namespace sqf
