@@ -445,26 +445,24 @@ def compress_24(hi_mask: np.ndarray, hi_codes: np.ndarray):
     indices of the two stored values, first < second.  One high channel at index p uses
     indices (p, p + 1) with the zero second, or (2, 3) with the zero first when p = 3; no
     high channel uses (0, 1).  Returns (values uint8 [rows, K/2], meta uint8 [rows, K/8])."""
-    mask = np.asarray(hi_mask, np.uint8)
+    mask = np.asarray(hi_mask, np.uint8).astype(bool)
     codes = np.asarray(hi_codes, np.uint8)
     rows, K = mask.shape
-    vals = np.zeros((rows, K // 2), np.uint8)
-    meta = np.zeros((rows, K // 8), np.uint8)
-    for r in range(rows):
-        for g in range(K // 4):
-            idx = [i for i in range(4) if mask[r, 4 * g + i]]
-            assert len(idx) <= 2, "more than two high channels in a group of four"
-            if len(idx) == 2:
-                i0, i1 = idx
-                v0, v1 = codes[r, 4 * g + i0], codes[r, 4 * g + i1]
-            elif len(idx) == 1:
-                p = idx[0]
-                if p < 3:
-                    i0, i1, v0, v1 = p, p + 1, codes[r, 4 * g + p], 0
-                else:
-                    i0, i1, v0, v1 = 2, 3, 0, codes[r, 4 * g + 3]
-            else:
-                i0, i1, v0, v1 = 0, 1, 0, 0
-            vals[r, 2 * g], vals[r, 2 * g + 1] = v0, v1
-            meta[r, g // 2] |= (i0 | (i1 << 2)) << (4 * (g % 2))
+    m4 = mask.reshape(rows, K // 4, 4)
+    c4 = codes.reshape(rows, K // 4, 4)
+    cnt = m4.sum(axis=2)
+    if np.any(cnt > 2):
+        raise ValueError("more than two high channels in a group of four")
+    first = np.argmax(m4, axis=2)                    # lowest high index (0 when none)
+    last = 3 - np.argmax(m4[:, :, ::-1], axis=2)     # highest high index
+    one_lo = (cnt == 1) & (first < 3)                # (p, p + 1), value first
+    one_hi = (cnt == 1) & (first == 3)               # (2, 3), value second
+    i0 = np.where(cnt == 2, first, np.where(one_lo, first, np.where(one_hi, 2, 0)))
+    i1 = np.where(cnt == 2, last, np.where(one_lo, first + 1, np.where(one_hi, 3, 1)))
+    take = lambda idx: np.take_along_axis(c4, idx[:, :, None], axis=2)[:, :, 0]
+    v0 = np.where((cnt == 2) | one_lo, take(first), 0).astype(np.uint8)
+    v1 = np.where(cnt == 2, take(last), np.where(one_hi, take(np.full_like(first, 3)), 0)).astype(np.uint8)
+    vals = np.stack([v0, v1], axis=2).reshape(rows, K // 2)
+    nib = (i0 | (i1 << 2)).astype(np.uint8)
+    meta = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
     return vals, meta

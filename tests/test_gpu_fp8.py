@@ -157,3 +157,10 @@ def test_fp8_wide_rows_rejected():
     with pytest.raises(sq.SQError) as e:
         sq.prepare_weights(W, [1, 2], fp8=True)
     assert e.value.status == sq.SQ_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_qkv_2048x4096x6144_o256", "sweep_M8192_o1/16"])
+def test_fp8_full_size_sampled(name):
+    w = workloads.CONFIGS[name]
+    O, X, W = workloads.make(w)
+    check_layer_fp8(O.numpy(), X, W, rows=sampled_rows(w.M, 8))

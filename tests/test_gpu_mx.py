@@ -29,8 +29,10 @@ def bits(t: torch.Tensor) -> np.ndarray:
 
 
 def dequant_abs(codes: np.ndarray, e8: np.ndarray) -> np.ndarray:
+    """|code value| * 2^E, float32 (exact: E2M1 magnitudes times a power of two in range); only bounds use it."""
     R, KN = codes.shape
-    return E2M1[codes & 7] * np.exp2(np.repeat(e8.astype(np.float64) - 127, 32, axis=1)[:, :KN])
+    return E2M1.astype(np.float32)[codes & 7] * np.exp2(
+        np.repeat(e8.astype(np.float32) - 127, 32, axis=1)[:, :KN])
 
 
 def check_quant_mx(O, src: torch.Tensor, codes_dev, S_dev, XO_dev, K):
@@ -78,7 +80,7 @@ def check_layer_mx(O, X, W, rows=None, ldy_extra=0):
     Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
     sel = np.arange(M) if rows is None else np.asarray(rows)
     ref = oracle.linear_mx(Xb, Wb, O, rows=sel)
-    absum = dequant_abs(ref["qx"], ref["ex"]) @ dequant_abs(ref["qw"], ref["ew"]).T
+    absum = (dequant_abs(ref["qx"], ref["ex"]) @ dequant_abs(ref["qw"], ref["ew"]).T).astype(np.float64)
     if len(O):
         xo = (ref["xo"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
         wo = (ref["wo"].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
@@ -208,3 +210,12 @@ def test_mx_argument_errors():
         sq.sq_gemm_mx(X_N4, S_X, X_O, pw.W_N, pw.s_w, pw.W_O, 4, 12, 256, 2,
                       torch.zeros(4, 16, dtype=torch.bfloat16, device=dev))
     assert e.value.status == sq.SQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_down_4096x14336x4096_o1792", "llama3_70b_gateup_8192x8192x57344_o512",
+                                  "sweep_M8192_o1/16"])
+def test_mx_full_size_sampled(name):
+    """The remaining full-size configurations with the MX low path, every quantizer row, sampled GEMM rows."""
+    w = workloads.CONFIGS[name]
+    O, X, W = workloads.make(w)
+    check_layer_mx(O.numpy(), X, W, rows=sampled_rows(w.M, 8))

@@ -63,11 +63,13 @@ def check_sqf(X, W, bank, h, rows=None, ldy_extra=0):
     sel = np.arange(M) if rows is None else np.asarray(rows)
     ref = oracle.sqf_linear(Xb, Wb, bank, h, rows=sel)
     assert np.array_equal(acc_lo.cpu().numpy()[sel].astype(np.int64), ref["acc_lo"]), "low-part sums differ"
-    dx = np.abs(oracle.e4m3_decode(ref["qx8"]).reshape(ref["qx8"].shape))
-    dw = np.where(ref["hi_mask"] == 1, np.abs(oracle.e4m3_decode(ref["hi"]).reshape(ref["hi"].shape)), 0.0)
+    # |decoded codes| in float32 (E4M3 values are exact in fp32); only the bound uses them
+    e4 = np.abs(oracle.e4m3_decode(np.arange(256, dtype=np.uint8))).astype(np.float32)
+    dx = e4[ref["qx8"]]
+    dw = np.where(ref["hi_mask"] == 1, e4[ref["hi"]], np.float32(0))
     scale = ref["sx8"][:, None].astype(np.float64) * ref["s_hi"][None, :].astype(np.float64)
     p_ref = ref["acc_hi"] * scale
-    bound = ACC_REL * (dx @ dw.T) * scale + 2.0 ** -20 * np.abs(p_ref) + 1e-30
+    bound = ACC_REL * (dx @ dw.T).astype(np.float64) * scale + 2.0 ** -20 * np.abs(p_ref) + 1e-30
     err = np.abs(P.cpu().numpy()[sel].astype(np.float64) - p_ref)
     assert np.all(err <= bound), f"high part off: worst {float((err / bound).max()):.3g} of the bound"
     y = Y.float().cpu().numpy().astype(np.float64)[sel]
@@ -145,3 +147,16 @@ def test_sqf_argument_errors():
     with pytest.raises(sq.SQError) as e:
         sq.prepare_weights_sqf(torch.zeros(16, 384, dtype=torch.bfloat16, device=dev), 8, 1)
     assert e.value.status == sq.SQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("name,bank,h", [("llama3_8b_down_4096x14336x4096_o1792", 8, 2),
+                                         ("llama3_70b_gateup_8192x8192x57344_o512", 16, 1),
+                                         ("sweep_M8192_o0", 4, 1)])
+def test_sqf_full_size_sampled(name, bank, h):
+    """Full-size configurations with element-level SQ-format weights, sampled GEMM rows."""
+    w = workloads.CONFIGS[name]
+    X = workloads.activations(w.M, w.K, workloads.outlier_channels(w.K, w.nO), kind=w.x_kind, sigma=w.sigma, seed=91)
+    W = workloads.weights(w.N, w.K, seed=92)
+    rng = np.random.default_rng(7)
+    rows = np.unique(np.concatenate([rng.choice(w.M, 6, replace=False), [0, w.M - 1]]))
+    check_sqf(X, W, bank, h, rows=rows)
