@@ -221,13 +221,16 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                         if (!is_bf) {
                             // Scales of this K-block: X-row tiles (K-tiles 0, 1) at sf, sf + 512; W-row
                             // tiles of rows 0-127 at sf + 1024 (+512 for K-tile 1), rows 128-255 at sf + 2048.
+                            // Two TMEM scale buffers alternate by K-block, so the copies of one
+                            // block need not wait for the MMAs that read the previous one.
                             const uint32_t sf = sbase + C::OFF_SF + e * C::SF_BYTES;
-                            sqd::sf_copy_pair(tmem + MX_SFA_COL, sqd::make_sf_desc(sf));
-                            sqd::sf_copy_pair(tmem + MX_SFA_COL + 4, sqd::make_sf_desc(sf + 512));
-                            sqd::sf_copy_pair(tmem + MX_SFB_COL, sqd::make_sf_desc(sf + 1024));
-                            sqd::sf_copy_pair(tmem + MX_SFB_COL + 4, sqd::make_sf_desc(sf + 2048));
-                            sqd::sf_copy_pair(tmem + MX_SFB_COL + 8, sqd::make_sf_desc(sf + 1536));
-                            sqd::sf_copy_pair(tmem + MX_SFB_COL + 12, sqd::make_sf_desc(sf + 2560));
+                            const uint32_t sb = tmem + MX_SF_BUF * static_cast<uint32_t>((i - nkb_o) & 1);
+                            sqd::sf_copy_pair(sb + MX_SFA_COL, sqd::make_sf_desc(sf));
+                            sqd::sf_copy_pair(sb + MX_SFA_COL + 4, sqd::make_sf_desc(sf + 512));
+                            sqd::sf_copy_pair(sb + MX_SFB_COL, sqd::make_sf_desc(sf + 1024));
+                            sqd::sf_copy_pair(sb + MX_SFB_COL + 4, sqd::make_sf_desc(sf + 2048));
+                            sqd::sf_copy_pair(sb + MX_SFB_COL + 8, sqd::make_sf_desc(sf + 1536));
+                            sqd::sf_copy_pair(sb + MX_SFB_COL + 12, sqd::make_sf_desc(sf + 2560));
                         }
                     }
 #pragma unroll
@@ -237,8 +240,9 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                         else if constexpr (MX) {
                             // MMA k covers scale blocks 2k, 2k+1: K-tile k / 2, bytes 2 (k % 2) and up.
                             const uint32_t id = 2u * static_cast<uint32_t>(k & 1);
-                            const uint32_t sfa = (tmem + MX_SFA_COL + 4 * (k >> 1)) | (id << 30);
-                            const uint32_t sfb = (tmem + MX_SFB_COL + 8 * (k >> 1)) | (id << 30);
+                            const uint32_t sb = tmem + MX_SF_BUF * static_cast<uint32_t>((i - nkb_o) & 1);
+                            const uint32_t sfa = (sb + MX_SFA_COL + 4 * (k >> 1)) | (id << 30);
+                            const uint32_t sfb = (sb + MX_SFB_COL + 8 * (k >> 1)) | (id << 30);
                             sqd::mma_mxf4_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_mx | (id << 29) | (id << 4), acc,
                                                sfa, sfb);
                         } else if constexpr (FP8) sqd::mma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_f8, acc);
