@@ -78,6 +78,7 @@ struct GemmArgs {
     int nkb_o;    // bf16 K-blocks per tile (no_pad / 64)
     int tiles_m, tiles_n, group_m;
     const float *addend;   // SQF: fp32 [M, N] added to the low part in place of the 16-bit branch
+    int y_tma = 0;         // pair kernel: Y written by bulk tensor stores (tm_y) instead of per-lane stores
 };
 
 // Tile t -> (M-tile, N-tile): groups of `group_m` M-tiles sweep all N-tiles,

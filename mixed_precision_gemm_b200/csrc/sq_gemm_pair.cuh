@@ -50,7 +50,7 @@ constexpr int PAIR_EPI_WARPS = 8;  // two per TMEM lane quarter, each half of th
 constexpr int PAIR_EXP_WARP0 = PAIR_EPI_WARP0 + PAIR_EPI_WARPS;
 constexpr int PAIR_THREADS = 32 * (PAIR_EXP_WARP0 + NUM_EXP_WARPS);
 
-template <int OPS_, int STG_, int NG_, int SF_ = 0>
+template <int OPS_, int STG_, int NG_, int SF_ = 0, int YB_ = 0>
 struct CfgPair {
     static constexpr int OPS = OPS_;                  // operand ring stages (expanded int8 or bf16 tiles)
     static constexpr int STG = STG_;                  // staging ring stages (packed INT4 tiles)
@@ -63,6 +63,7 @@ struct CfgPair {
     static constexpr int PA_BYTES = 128 * PROWB;      // packed X rows of one K-block
     static constexpr int STG_BYTES = 256 * PROWB;     // packed X + W rows of one K-block
     static constexpr int SF_BYTES = SF_;              // block scales per operand stage (MX only)
+    static constexpr int YB = YB_;                    // Y staging boxes per epilogue warp (1 KB each); 0: per-lane stores
     static constexpr int OFF_OP = 0;
     static constexpr int OFF_SF = OPS * OP_BYTES;
     static constexpr int OFF_STG = OFF_SF + OPS * SF_BYTES;
@@ -71,10 +72,16 @@ struct CfgPair {
     static constexpr int NBAR = 2 * OPS + 2 * STG + 3;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SW = (OFF_MISC + 16 + 15) / 16 * 16;   // per epilogue warp: its 128 s_w values
-    static constexpr int SMEM_BYTES = OFF_SW + PAIR_EPI_WARPS * 128 * 4 + 1024;
+    // Per epilogue warp: YB boxes of 32 x 16 bf16, the source of bulk tensor
+    // stores, whose shared-memory address must be 128-byte aligned.
+    static constexpr int OFF_YST = (OFF_SW + PAIR_EPI_WARPS * 128 * 4 + 127) / 128 * 128;
+    static constexpr int SMEM_BYTES = OFF_YST + PAIR_EPI_WARPS * YB * 1024 + 1024;
     static constexpr int TMEM_COLS = 512;
     static constexpr int EXP_CHUNKS = 256 * (PROWB / 16) / GT;  // packed 16-byte chunks per thread per K-block
     static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(YB >= 0 && YB <= 2, "Y staging boxes");
+    static_assert(OFF_YST % 128 == 0 && OFF_OP % 1024 == 0 && OFF_STG % 1024 == 0 && OFF_SF % 128 == 0,
+                  "bulk tensor copies need 128-byte aligned shared memory (1024 for the 128-byte swizzle)");
     // Each slot of both rings must be used by a single producer group: a group
     // waiting on a slot only knows that its own earlier blocks have landed, and
     // bulk copies may complete out of order, so a slot shared by two groups
@@ -94,7 +101,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PAIR_THREADS, 1)
 dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_constant__ CUtensorMap tm_wo,
                       const __grid_constant__ CUtensorMap tm_xn, const __grid_constant__ CUtensorMap tm_wn,
                       const __grid_constant__ CUtensorMap tm_sx, const __grid_constant__ CUtensorMap tm_sw,
-                      const GemmArgs args)
+                      const __grid_constant__ CUtensorMap tm_y, const GemmArgs args)
 {
     constexpr bool FP8 = LOW == kLowFp8;
     constexpr bool MX = LOW == kLowMx;
@@ -154,6 +161,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                 sqd::prefetch_tensormap(&tm_sw);
             }
         }
+        if (args.y_tma) sqd::prefetch_tensormap(&tm_y);
     }
     if (warp == 1) {
         sqd::tmem_alloc_pair(sqd::smem_u32(tmem_slot), C::TMEM_COLS);
@@ -391,6 +399,10 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         const uint32_t empty_leader = sqd::map_to_cta(acc_empty, 0);
         constexpr int CW = 16;                   // columns per TMEM load
         constexpr int NCH = (PAIR_BN / 2) / CW;  // 8 loads per accumulator per warp
+        static_assert(CW == 16, "one staging box is 16 columns");
+        const bool y_tma = C::YB > 0 && args.y_tma != 0;
+        const uint32_t yst = sbase + C::OFF_YST + (warp - PAIR_EPI_WARP0) * C::YB * 1024;
+        int last_box = -1;  // staging box of this warp's latest bulk store
         for (int lt = 0; lt < my_tiles; ++lt) {
             int tmi, tni;
             tile_coords(args, pair + lt * num_pairs, tmi, tni);
@@ -421,24 +433,41 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             };
             issue(0, 0);
             sqd::tmem_wait_ld_dep(vi[0], vf[0]);
+            const int m0 = tmi * PAIR_BM + static_cast<int>(rank) * 128 + sub * 32;  // this warp's first row
 #pragma unroll
             for (int ch = 0; ch < NCH; ++ch) {
                 const int b = ch & 1;
                 if (ch + 1 < NCH) issue(ch + 1, b ^ 1);
                 const int n0 = tni * PAIR_BN + c_base + ch * CW;
-                if (row_ok && n0 < args.N) {
+                // Bulk-store form: all 32 lanes fill the 32 x 16 box (the store
+                // drops rows past M and columns past N); otherwise each lane
+                // stores its own row.
+                if (y_tma ? (m0 < args.M && n0 < args.N) : (row_ok && n0 < args.N)) {
+                    // Staging box (two alternate when YB == 2): wait until the bulk
+                    // store that last read it is done.
+                    const int bb = C::YB == 2 ? b : 0;
+                    const uint32_t box = yst + 1024u * static_cast<uint32_t>(bb);
+                    if (y_tma) {
+                        if (lane == 0) {
+                            if (C::YB == 2 && last_box == (bb ^ 1)) sqd::bulk_wait_read<1>();
+                            else sqd::bulk_wait_read<0>();
+                        }
+                        __syncwarp();
+                    }
 #pragma unroll
                     for (int g = 0; g < CW / 8; ++g) {
                         const int n = n0 + 8 * g;
-                        if (n >= args.N) break;
+                        const bool ok8 = row_ok && n < args.N;  // N is a multiple of 8
                         const uint4 sw0 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g));
                         const uint4 sw1 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g + 4));
                         // SQF: the precomputed high part of these 8 outputs
                         float4 ad0 = make_float4(0.f, 0.f, 0.f, 0.f), ad1 = ad0;
                         if constexpr (SQF) {
-                            const float4 *ap = reinterpret_cast<const float4 *>(args.addend + static_cast<long long>(m) * args.N + n);
-                            ad0 = ap[0];
-                            ad1 = ap[1];
+                            if (ok8) {
+                                const float4 *ap = reinterpret_cast<const float4 *>(args.addend + static_cast<long long>(m) * args.N + n);
+                                ad0 = ap[0];
+                                ad1 = ap[1];
+                            }
                         }
                         const float adv[8] = {ad0.x, ad0.y, ad0.z, ad0.w, ad1.x, ad1.y, ad1.z, ad1.w};
                         const float swv[8] = {__uint_as_float(sw0.x), __uint_as_float(sw0.y), __uint_as_float(sw0.z),
@@ -469,14 +498,26 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                                 const float af = SQF ? adv[2 * h + u] : (MX || has_o) ? __uint_as_float(vf[b][t]) : 0.0f;
                                 y2[u] = MX ? af : __fadd_rn(__fmul_rn(__fmul_rn(al, sx), swv[2 * h + u]), af);
                                 if constexpr (DBG) {
-                                    if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + 2 * h + u] = dbg_lo;
-                                    if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n + 2 * h + u] = af;
+                                    if (ok8) {
+                                        if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + 2 * h + u] = dbg_lo;
+                                        if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n + 2 * h + u] = af;
+                                    }
                                 }
                             }
                             const __nv_bfloat162 b2 = __floats2bfloat162_rn(y2[0], y2[1]);
                             out[h] = *reinterpret_cast<const uint32_t *>(&b2);
                         }
-                        *reinterpret_cast<uint4 *>(yrow + n) = make_uint4(out[0], out[1], out[2], out[3]);
+                        if (y_tma) sqd::sts128(box + 32 * lane + 16 * g, out[0], out[1], out[2], out[3]);
+                        else if (n < args.N) *reinterpret_cast<uint4 *>(yrow + n) = make_uint4(out[0], out[1], out[2], out[3]);
+                    }
+                    if (y_tma) {
+                        sqd::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            sqd::tma_store_2d(&tm_y, box, n0, m0);
+                            sqd::bulk_commit();
+                        }
+                        last_box = bb;
                     }
                 }
                 if (ch + 1 < NCH) {
@@ -490,6 +531,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                 }
             }
         }
+        if (y_tma && lane == 0) sqd::bulk_wait_all();  // the staging boxes stay valid until stored
     }
 
     sqd::tc_fence_before();
