@@ -476,13 +476,13 @@ using CfgPair = sqg::CfgPair<4, 4, 2>;     // INT4: per-lane Y stores (bulk stor
 using CfgPairSqf = sqg::CfgPair<4, 4, 2, 0, 2>;  // SQ-format low part: Y by bulk tensor stores
 using CfgPairF8 = sqg::CfgPair<6, 0, 2, 0, 2>;  // E4M3 tiles need no staging ring: a deeper operand ring instead
 using CfgPairMx = sqg::CfgPair<6, 0, 2, sqg::MX_SF_BYTES, 1>;  // E2M1 tiles plus their block scales; one Y box per warp
-// INT4 stages carry two K-blocks; an operand ring of four slots lets the
-// expansion of one stage overlap the MMAs of the previous one (with fewer, the
-// expansion waits for the MMAs of its predecessor's own blocks).
-using CfgSk16 = sqg::CfgSkinny<16, 7, 4>;
-using CfgSk32 = sqg::CfgSkinny<32, 6, 4>;
-using CfgSk64 = sqg::CfgSkinny<64, 4, 4>;
-using CfgSk128 = sqg::CfgSkinny<128, 3, 4>;
+// INT4 stages carry two K-blocks.  The W codes go to tensor memory; the
+// operand ring (six slots: the expansion runs up to three stages ahead of the
+// MMAs) holds only the token rows, which leaves room for deeper staging rings.
+using CfgSk16 = sqg::CfgSkinny<16, 10, 6, 0, true>;
+using CfgSk32 = sqg::CfgSkinny<32, 9, 6, 0, true>;
+using CfgSk64 = sqg::CfgSkinny<64, 7, 6, 0, true>;
+using CfgSk128 = sqg::CfgSkinny<128, 3, 6, 0, true>;
 // E4M3 stages are read by the MMA in place: a deeper staging ring instead.
 using CfgSk16F8 = sqg::CfgSkinny<16, 8, 3>;
 using CfgSk32F8 = sqg::CfgSkinny<32, 7, 3>;

@@ -63,27 +63,40 @@ constexpr int SK_MAX_SPLITS = 8;
 
 enum : unsigned { SITE_SK_STG = 0x501, SITE_SK_OP = 0x502, SITE_SK_MMA = 0x503, SITE_SK_EPI = 0x504 };
 
-template <int MP_, int NST_, int OPS_, int SF_ = 0>
+template <int MP_, int NST_, int OPS_, int SF_ = 0, bool TA_ = false>
 struct CfgSkinny {
     static constexpr int MP = MP_;                    // token columns of D (MMA N)
     static constexpr int NST = NST_;                  // staging ring stages
     static constexpr int OPS = OPS_;                  // expanded int8 operand ring stages
     static constexpr int SF_BYTES = SF_;              // block scales per staging stage (MX only)
+    // INT4 with the W operand in tensor memory: each expansion thread writes
+    // its W row's int8 codes straight into TMEM (the MMA's A operand), and only
+    // the token rows go through a shared-memory operand tile.
+    static constexpr bool TA = TA_;
     static constexpr int ROWS = 128 + MP;             // W rows, then token rows, in every tile
     static constexpr int A_BYTES = 128 * ROWB;
     static constexpr int TILE_BYTES = ROWS * ROWB;    // one stage = one operand tile (128-byte rows)
+    static constexpr int OP_BYTES = TA ? MP * ROWB : TILE_BYTES;  // one operand ring slot
     static constexpr int OFF_STG = 0;
     static constexpr int OFF_OP = NST * TILE_BYTES;
-    static constexpr int OFF_SF = OFF_OP + OPS * TILE_BYTES;
+    static constexpr int OFF_SF = OFF_OP + OPS * OP_BYTES;
     static constexpr int OFF_BAR = OFF_SF + NST * SF_BYTES;
     // barriers: stg_full[NST] stg_empty[NST] op_full[OPS] op_empty[OPS] acc_full drain
     static constexpr int NBAR = 2 * NST + 2 * OPS + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_CNT = OFF_MISC + 16;           // per staging slot: expansion warps done
-    static constexpr int SMEM_BYTES = OFF_CNT + NST * 4 + 1024;
-    // MX: the accumulator [0, MP) and 16 scale columns; otherwise two accumulators.
-    static constexpr int TMEM_NEED = SF_ > 0 ? MP + 16 : 2 * MP;
-    static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128 : 256;
+    // Row scales for the epilogue, fetched at the start: s_w of the tile's 128
+    // W rows, then s_x of the MP token columns (0 past N or M).
+    static constexpr int OFF_SCL = (OFF_CNT + NST * 4 + 15) / 16 * 16;
+    static constexpr int SMEM_BYTES = OFF_SCL + (128 + MP) * 4 + 1024;
+    // MX: the accumulator [0, MP) and 16 scale columns; otherwise two
+    // accumulators, and with TA the OPS W-operand slots (32 columns = 128 int8
+    // K-elements per lane each) from column TA_COL.
+    static constexpr int COL_F = SF_ > 0 ? 0 : MP;   // fp32 accumulator of the 16-bit branch
+    static constexpr int TA_COL = 2 * MP < 32 ? 32 : 2 * MP;
+    static constexpr int TMEM_NEED = SF_ > 0 ? MP + 16 : TA ? TA_COL + 32 * OPS : 2 * MP;
+    static constexpr int TMEM_COLS = TMEM_NEED <= 32 ? 32 : TMEM_NEED <= 64 ? 64 : TMEM_NEED <= 128 ? 128
+                                   : TMEM_NEED <= 256 ? 256 : 512;
     static constexpr int EXP_CHUNKS = ROWS * 8 / SK_PT;   // 16-byte packed chunks per thread per stage
     // Reduction buffer (aliases the rings): int32 and fp32 regions of
     // S * RP <= 128 + S - 1 partial rows, RSTRIDE words apart.
@@ -92,7 +105,9 @@ struct CfgSkinny {
     static constexpr int OFF_RED_I = 0;
     static constexpr int OFF_RED_F = RED_ROWS * RSTRIDE * 4;
     static_assert(MP == 16 || MP == 32 || MP == 64 || MP == 128, "MP");
-    static_assert(TILE_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned");
+    static_assert(TILE_BYTES % 1024 == 0 && OP_BYTES % 1024 == 0, "tiles must stay 1024-byte aligned");
+    static_assert(TMEM_NEED <= 512, "tensor memory");
+    static_assert(!TA || SF_ == 0, "TA is an INT4 layout");
     static_assert(ROWS * 8 % SK_PT == 0, "expansion work split");
     static_assert(OPS >= 2 || SF_ > 0, "an INT4 stage fills two operand tiles");
     static_assert(2 * RED_ROWS * RSTRIDE * 4 <= OFF_BAR, "reduction buffer must fit in the rings");
@@ -163,7 +178,9 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC + 4);
     uint32_t *stg_done = reinterpret_cast<uint32_t *>(smem + C::OFF_CNT);
     auto stg_a = [&](int s) { return sbase + C::OFF_STG + s * C::TILE_BYTES; };
-    auto op_a = [&](int e) { return sbase + C::OFF_OP + e * C::TILE_BYTES; };
+    auto op_a = [&](int e) { return sbase + C::OFF_OP + e * C::OP_BYTES; };
+    // token rows of operand slot e (with TA the slot holds nothing else)
+    auto op_b = [&](int e) { return op_a(e) + (C::TA ? 0 : C::A_BYTES); };
 
     // This CTA's K range: INT4 blocks [i_lo, i_lo + n_i) in ns_i stages of
     // two, then bf16 blocks [o_lo, o_lo + n_o), one stage each.
@@ -217,6 +234,16 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
     sqd::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     sqd::pdl_wait();  // operands and Y may belong to the previous kernel
+
+    // The epilogue's row scales, loaded now so that their latency is hidden
+    // behind the main loop (read after the cluster barriers below).
+    float *scl_w = reinterpret_cast<float *>(smem + C::OFF_SCL);
+    float *scl_x = scl_w + 128;
+    if (!MX && warp >= SK_PROD_WARP0) {
+        const int et = threadIdx.x - SK_PROD_WARP0 * 32;
+        scl_w[et] = n0 + et < args.N ? __ldg(args.s_w + n0 + et) : 0.0f;
+        if (et < MP) scl_x[et] = et < args.M ? __ldg(args.s_x + et) : 0.0f;
+    }
 
     if (warp == 0) {
         // ------------------------------------------------------------ staging producer
@@ -304,11 +331,19 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
                 const int e = u % OPS;
                 if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_SK_MMA)) { ok = false; break; }
                 sqd::tc_fence_after();
-                const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
-                const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
+                const uint64_t bdesc = sqd::make_sw128_desc(op_b(e));
+                if constexpr (C::TA) {
+                    // A: 32 TMEM columns of slot e, 8 columns (32 int8 K-elements) per MMA
+                    const uint32_t at = tmem + static_cast<uint32_t>(C::TA_COL + 32 * e);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    sqd::mma_s8(tmem, adesc + 2 * k, bdesc + 2 * k, idesc_i8, (u == 0 && k == 0) ? 0u : 1u);
+                    for (int k = 0; k < 4; ++k)
+                        sqd::mma_s8_ta(tmem, at + 8 * k, bdesc + 2 * k, idesc_i8, (u == 0 && k == 0) ? 0u : 1u);
+                } else {
+                    const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        sqd::mma_s8(tmem, adesc + 2 * k, bdesc + 2 * k, idesc_i8, (u == 0 && k == 0) ? 0u : 1u);
+                }
                 sqd::mma_commit(op_empty(e));
             }
             for (int t = ns_i; t < ns && ok; ++t) {  // bf16 blocks straight from the staging ring
@@ -321,7 +356,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
                 for (int k = 0; k < 4; ++k) {
                     // MX: the branch adds into the one accumulator (cleared by whichever MMA comes first)
                     const uint32_t acc = MX ? ((t == 0 && k == 0) ? 0u : 1u) : ((t == ns_i && k == 0) ? 0u : 1u);
-                    sqd::mma_bf16(MX ? tmem : tmem + MP, adesc + 2 * k, bdesc + 2 * k, idesc_bf, acc);
+                    sqd::mma_bf16(tmem + C::COL_F, adesc + 2 * k, bdesc + 2 * k, idesc_bf, acc);
                 }
                 sqd::mma_commit(stg_empty(s));
             }
@@ -353,37 +388,90 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
             }
             if (!ok) break;
             const uint32_t src = stg_a(s);
-            uint4 w[EC];
+            auto ex = [&](uint32_t v) { return SQF ? clear_mask_code(v) : v; };
+            if constexpr (C::TA) {
+                // W row of this thread = its TMEM lane (warp quarter): its 128
+                // packed bytes (both K-blocks) expanded into one 32-column slot
+                // per K-block.  Eight consecutive rows read eight different
+                // 16-byte positions (swizzle), so the loads are conflict-free.
+                const int quarter = warp & 3;
+                const int wr = quarter * 32 + lane;
+                const uint32_t srow = src + wr * ROWB;
+                const uint32_t tl = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + C::TA_COL;
 #pragma unroll
-            for (int c = 0; c < EC; ++c) {
-                const int q = et + c * SK_PT;
-                const int r = q >> 3;
-                w[c] = sqd::lds128(src + r * ROWB + (((q & 7) ^ (r & 7)) << 4));
-            }
+                for (int j = 0; j < 2; ++j) {
+                    if (j < nblk) {
+                        uint4 c4[4];
 #pragma unroll
-            for (int c = 0; c < EC; ++c) {
-                const int q = et + c * SK_PT;
-                const int r = q >> 3;
-                const int j = (q >> 2) & 1;  // K-block of the stage
-                if (j < nblk) {
-                    const uint32_t sw = static_cast<uint32_t>(r & 7);
-                    const uint32_t jj = static_cast<uint32_t>(q & 3);
-                    const uint32_t row = op_a((u0 + j) % OPS) + r * ROWB;
-                    const uint32_t a0 = row + (((2u * jj) ^ sw) << 4);
-                    const uint32_t a1 = row + (((2u * jj + 1u) ^ sw) << 4);
-                    auto ex = [&](uint32_t v) { return SQF ? clear_mask_code(v) : v; };
-                    const uint32_t lo0 = ex((w[c].x << 4) & 0xF0F0F0F0u), hi0 = ex(w[c].x & 0xF0F0F0F0u);
-                    const uint32_t lo1 = ex((w[c].y << 4) & 0xF0F0F0F0u), hi1 = ex(w[c].y & 0xF0F0F0F0u);
-                    const uint32_t lo2 = ex((w[c].z << 4) & 0xF0F0F0F0u), hi2 = ex(w[c].z & 0xF0F0F0F0u);
-                    const uint32_t lo3 = ex((w[c].w << 4) & 0xF0F0F0F0u), hi3 = ex(w[c].w & 0xF0F0F0F0u);
-                    // The two K-blocks' threads of a row store in opposite
-                    // order, so the eight stores of a phase hit distinct banks.
-                    if (j == 0) {
-                        sqd::sts128(a0, lo0, hi0, lo1, hi1);
-                        sqd::sts128(a1, lo2, hi2, lo3, hi3);
-                    } else {
-                        sqd::sts128(a1, lo2, hi2, lo3, hi3);
-                        sqd::sts128(a0, lo0, hi0, lo1, hi1);
+                        for (int q = 0; q < 4; ++q) c4[q] = sqd::lds128(srow + (((4 * j + q) ^ (wr & 7)) << 4));
+                        uint32_t v[32];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            v[8 * q + 0] = ex((c4[q].x << 4) & 0xF0F0F0F0u);
+                            v[8 * q + 1] = ex(c4[q].x & 0xF0F0F0F0u);
+                            v[8 * q + 2] = ex((c4[q].y << 4) & 0xF0F0F0F0u);
+                            v[8 * q + 3] = ex(c4[q].y & 0xF0F0F0F0u);
+                            v[8 * q + 4] = ex((c4[q].z << 4) & 0xF0F0F0F0u);
+                            v[8 * q + 5] = ex(c4[q].z & 0xF0F0F0F0u);
+                            v[8 * q + 6] = ex((c4[q].w << 4) & 0xF0F0F0F0u);
+                            v[8 * q + 7] = ex(c4[q].w & 0xF0F0F0F0u);
+                        }
+                        sqd::tmem_st_32x32b_x32(tl + 32u * static_cast<uint32_t>((u0 + j) % OPS), v);
+                    }
+                }
+                // Token rows (staging rows 128 .. 128 + MP - 1): 16-byte chunk q
+                // of the MP x 8 chunks, into the slot's swizzled token tile.
+#pragma unroll
+                for (int c = 0; c < C::MP * 8 / SK_PT; ++c) {
+                    const int q = et + c * SK_PT;
+                    const int tr = q >> 3;
+                    const int ck = q & 7;
+                    const int j = ck >> 2;
+                    if (j < nblk) {
+                        const uint4 w4 = sqd::lds128(src + (128 + tr) * ROWB + ((ck ^ (tr & 7)) << 4));
+                        const uint32_t sw = static_cast<uint32_t>(tr & 7);
+                        const uint32_t jj = static_cast<uint32_t>(ck & 3);
+                        const uint32_t row = op_b((u0 + j) % OPS) + tr * ROWB;
+                        sqd::sts128(row + (((2u * jj) ^ sw) << 4), ex((w4.x << 4) & 0xF0F0F0F0u), ex(w4.x & 0xF0F0F0F0u),
+                                    ex((w4.y << 4) & 0xF0F0F0F0u), ex(w4.y & 0xF0F0F0F0u));
+                        sqd::sts128(row + (((2u * jj + 1u) ^ sw) << 4), ex((w4.z << 4) & 0xF0F0F0F0u), ex(w4.z & 0xF0F0F0F0u),
+                                    ex((w4.w << 4) & 0xF0F0F0F0u), ex(w4.w & 0xF0F0F0F0u));
+                    }
+                }
+                sqd::tmem_wait_st();
+                sqd::tc_fence_before();
+            } else {
+                uint4 w[EC];
+#pragma unroll
+                for (int c = 0; c < EC; ++c) {
+                    const int q = et + c * SK_PT;
+                    const int r = q >> 3;
+                    w[c] = sqd::lds128(src + r * ROWB + (((q & 7) ^ (r & 7)) << 4));
+                }
+#pragma unroll
+                for (int c = 0; c < EC; ++c) {
+                    const int q = et + c * SK_PT;
+                    const int r = q >> 3;
+                    const int j = (q >> 2) & 1;  // K-block of the stage
+                    if (j < nblk) {
+                        const uint32_t sw = static_cast<uint32_t>(r & 7);
+                        const uint32_t jj = static_cast<uint32_t>(q & 3);
+                        const uint32_t row = op_a((u0 + j) % OPS) + r * ROWB;
+                        const uint32_t a0 = row + (((2u * jj) ^ sw) << 4);
+                        const uint32_t a1 = row + (((2u * jj + 1u) ^ sw) << 4);
+                        const uint32_t lo0 = ex((w[c].x << 4) & 0xF0F0F0F0u), hi0 = ex(w[c].x & 0xF0F0F0F0u);
+                        const uint32_t lo1 = ex((w[c].y << 4) & 0xF0F0F0F0u), hi1 = ex(w[c].y & 0xF0F0F0F0u);
+                        const uint32_t lo2 = ex((w[c].z << 4) & 0xF0F0F0F0u), hi2 = ex(w[c].z & 0xF0F0F0F0u);
+                        const uint32_t lo3 = ex((w[c].w << 4) & 0xF0F0F0F0u), hi3 = ex(w[c].w & 0xF0F0F0F0u);
+                        // The two K-blocks' threads of a row store in opposite
+                        // order, so the eight stores of a phase hit distinct banks.
+                        if (j == 0) {
+                            sqd::sts128(a0, lo0, hi0, lo1, hi1);
+                            sqd::sts128(a1, lo2, hi2, lo3, hi3);
+                        } else {
+                            sqd::sts128(a1, lo2, hi2, lo3, hi3);
+                            sqd::sts128(a0, lo0, hi0, lo1, hi1);
+                        }
                     }
                 }
             }
@@ -421,7 +509,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
         // MX: one accumulator in [0, MP), sent as the "fp32" partial.
         const bool has_i = !MX && n_i > 0 && !*abort_flag;
         const bool has_f = (MX ? (n_i + n_o > 0) : n_o > 0) && !*abort_flag;
-        const uint32_t col_f = MX ? 0u : static_cast<uint32_t>(MP);
+        const uint32_t col_f = static_cast<uint32_t>(C::COL_F);
 #pragma unroll 1
         for (int ch = 0; ch < MP / 16; ++ch) {
             uint32_t vi[16] = {}, vf[16] = {};
@@ -445,27 +533,42 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
         const int R = max(0, min(128 - r0, RP));
         const int32_t *red_i = reinterpret_cast<const int32_t *>(smem + C::OFF_RED_I);
         const float *red_f = reinterpret_cast<const float *>(smem + C::OFF_RED_F);
-        for (int idx = et; idx < R * MP; idx += SK_PT) {
-            const int rl = idx % R;
-            const int m = idx / R;
+        // Thread et sums row rl = et % R for tokens m = et / R, + G, + 2G, ...
+        // (one division per thread; rows of a warp are consecutive, so the Y
+        // stores of one token coalesce).
+        if (R > 0) {
+            const int G = SK_PT / R;
+            const int rl = et % R;
+            const int mg = et / R;
             const int n = n0 + r0 + rl;
-            if (m >= args.M || n >= args.N) continue;
-            int32_t si = 0;
-            float sl = 0.0f, sf = 0.0f;
-            for (int s = 0; s < S; ++s) {
-                const int w = (s * RP + rl) * C::RSTRIDE + m;
-                if constexpr (FP8) sl = __fadd_rn(sl, __int_as_float(red_i[w]));
-                else si += red_i[w];
-                sf = __fadd_rn(sf, red_f[w]);
-            }
-            const int ai = si >> 8;
-            const float al = FP8 ? sl : static_cast<float>(ai);
-            const float add = SQF ? args.addend[static_cast<long long>(m) * args.N + n] : sf;
-            const float y = MX ? sf : __fadd_rn(__fmul_rn(__fmul_rn(al, args.s_x[m]), args.s_w[n]), add);
-            args.Y[static_cast<long long>(m) * args.ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
-            if constexpr (DBG) {
-                if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n] = FP8 ? __float_as_int(sl) : ai;
-                if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n] = sf;
+            const int mlim = min(args.M, MP);
+            if (mg < G && n < args.N) {
+                const float swn = scl_w[r0 + rl];
+                const int wb = rl * C::RSTRIDE;
+                const int sstep = RP * C::RSTRIDE;
+#pragma unroll 4
+                for (int m = mg; m < mlim; m += G) {
+                    int32_t si = 0;
+                    float sl = 0.0f, sf = 0.0f;
+#pragma unroll
+                    for (int s = 0; s < SK_MAX_SPLITS; ++s) {
+                        if (s < S) {
+                            const int w = wb + s * sstep + m;
+                            if constexpr (FP8) sl = __fadd_rn(sl, __int_as_float(red_i[w]));
+                            else si += red_i[w];
+                            sf = __fadd_rn(sf, red_f[w]);
+                        }
+                    }
+                    const int ai = si >> 8;
+                    const float al = FP8 ? sl : static_cast<float>(ai);
+                    const float add = SQF ? args.addend[static_cast<long long>(m) * args.N + n] : sf;
+                    const float y = MX ? sf : __fadd_rn(__fmul_rn(__fmul_rn(al, scl_x[m]), swn), add);
+                    args.Y[static_cast<long long>(m) * args.ldy + n] = __bfloat16_as_ushort(__float2bfloat16_rn(y));
+                    if constexpr (DBG) {
+                        if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n] = FP8 ? __float_as_int(sl) : ai;
+                        if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n] = sf;
+                    }
+                }
             }
         }
     }
