@@ -60,11 +60,38 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without comments and with whitespace runs collapsed, so that the
+    hash below changes with the code and not with its comments."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_hash() -> str:
+    """Hash of the CUDA sources' code (comments excluded): recorded ncu traffic is used only
+    while it matches."""
     h = hashlib.sha256()
     for p in sorted(glob.glob(os.path.join(ROOT, "mixed_precision_gemm_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
-            h.update(f.read())
+        with open(p, encoding="utf-8") as f:
+            h.update(os.path.basename(p).encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -17,7 +17,10 @@
 //                            barriers of both CTAs (multicast commit).
 //   warps 2..9 (each CTA)    epilogue of the CTA's 128 rows (two warps per TMEM
 //                            lane quarter); they report to the first CTA's
-//                            acc_empty barrier when TMEM is read.
+//                            acc_empty barrier when TMEM is read.  Y goes out
+//                            per lane (16-byte stores), or with C::YB > 0
+//                            through 32 x 16 staging boxes and bulk tensor
+//                            stores.
 //   warps 10..17 (each CTA)  operand producers for the CTA's halves, in ring
 //                            order: bf16 blocks by TMA (.cta_group::2 form, no
 //                            multicast, completion bytes counted on the first
@@ -25,7 +28,7 @@
 //                            staging ring into int8 operand tiles (see
 //                            sq_gemm_common.cuh).  Every producer warp of both CTAs
 //                            arrives on the first CTA's op_full.
-// The packed tiles travel by TMA into a staging ring (asynchronous, six
+// The packed tiles travel by TMA into a staging ring (asynchronous, C::STG
 // K-blocks deep) and are expanded from shared memory, so no producer thread
 // has long global loads outstanding when it publishes a tile.
 // TMEM per CTA: acc_f in columns [0, 256), acc_i in [256, 512).

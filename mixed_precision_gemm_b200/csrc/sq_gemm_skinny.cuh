@@ -24,23 +24,27 @@
 //
 // Wide loads, deep ring.  Weight rows are fetched 128 bytes at a time (two
 // packed INT4 K-blocks, or one bf16 K-block) with the 128-byte swizzle, into
-// a staging ring of about 144 KB, which keeps enough bytes in flight per SM
-// to stream HBM.  bf16 stages are read by the MMA where they land; INT4
-// stages are expanded into a small ring of int8 operand tiles.
+// a staging ring of 96-180 KB, which keeps enough bytes in flight per SM to
+// stream HBM.  bf16 stages are read by the MMA where they land; INT4 stages
+// are expanded into a small ring of int8 operand slots (with C::TA: the W
+// rows into tensor memory, the token rows into shared memory).
 //
 // Roles (6 warps, one tile-split per CTA):
 //   warp 0      TMA producer of the staging ring: for each stage, 128 W rows
 //               and MP token rows of 128 bytes.
 //   warp 1      allocates TMEM; one lane issues every MMA and commits.
-//   warps 2..5  expand INT4 stages (both K-blocks at once, eight threads per
-//               128-byte row) into the operand ring, in order; afterwards
-//               they run the epilogue.
+//   warps 2..5  expand INT4 stages (both K-blocks at once) into the operand
+//               ring, in order: with C::TA one thread per W row (its TMEM
+//               lane), writing the row's int8 codes with tcgen05.st, and the
+//               token rows spread over all threads; otherwise eight threads
+//               per 128-byte row.  Afterwards they run the epilogue.
 // Stage order is every INT4 stage, then every bf16 stage.  The INT4 stages
 // are consumed by the expansion warps and the bf16 stages by the MMA issuer;
 // because all INT4 stages come first, each consumer's earlier uses of a slot
 // were its own or were consumed before it reached the slot, so the
 // phase-parity waits cannot alias.
-// TMEM: acc_i (int32) in columns [0, MP), acc_f (fp32) in [MP, 2 MP).
+// TMEM: acc_i (int32) in columns [0, MP), acc_f (fp32) in [MP, 2 MP); with
+// C::TA the W-operand slots follow from column C::TA_COL, 32 columns each.
 //
 // MX low path (kLowMx): a stage is one K-block of 256 E2M1 codes (128 bytes
 // per row) read by the MMA in place, plus two 1 KB scale boxes: the W rows'
