@@ -160,6 +160,9 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
     constexpr bool DIRECT = FP8 || MX;   // low-path stages read by the MMA in place
     constexpr bool SQF = LOW == kLowSqf;  // INT4 stages with the mask code -8 cleared, fp32 addend
     constexpr int MP = C::MP, NST = C::NST, OPS = C::OPS, EC = C::EXP_CHUNKS;
+    // Modulus of the INT4 operand ring.  The direct-read configurations have no
+    // ring (OPS = 0) and never run the code that uses it.
+    constexpr int OPR = OPS > 0 ? OPS : 1;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = sqd::smem_u32(smem);
@@ -332,8 +335,8 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
                 }
             }
             for (int u = 0; u < (DIRECT ? 0 : n_i) && ok; ++u) {  // INT4 blocks from the operand ring
-                const int e = u % OPS;
-                if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_SK_MMA)) { ok = false; break; }
+                const int e = u % OPR;
+                if (!sqd::mbar_wait(op_full(e), (u / OPR) & 1, abort_flag, SITE_SK_MMA)) { ok = false; break; }
                 sqd::tc_fence_after();
                 const uint64_t bdesc = sqd::make_sw128_desc(op_b(e));
                 if constexpr (C::TA) {
@@ -385,7 +388,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
             const int u0 = 2 * t;  // operand ring uses u0, u0 + 1
             if (!sqd::mbar_wait(stg_full(s), (t / NST) & 1, abort_flag, SITE_SK_OP)) { ok = false; break; }
             for (int j = 0; j < nblk; ++j) {
-                if (!sqd::mbar_wait(op_empty((u0 + j) % OPS), (((u0 + j) / OPS) & 1) ^ 1u, abort_flag, SITE_SK_OP)) {
+                if (!sqd::mbar_wait(op_empty((u0 + j) % OPR), (((u0 + j) / OPR) & 1) ^ 1u, abort_flag, SITE_SK_OP)) {
                     ok = false;
                     break;
                 }
@@ -420,7 +423,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
                             v[8 * q + 6] = ex((c4[q].w << 4) & 0xF0F0F0F0u);
                             v[8 * q + 7] = ex(c4[q].w & 0xF0F0F0F0u);
                         }
-                        sqd::tmem_st_32x32b_x32(tl + 32u * static_cast<uint32_t>((u0 + j) % OPS), v);
+                        sqd::tmem_st_32x32b_x32(tl + 32u * static_cast<uint32_t>((u0 + j) % OPR), v);
                     }
                 }
                 // Token rows (staging rows 128 .. 128 + MP - 1): 16-byte chunk q
@@ -435,7 +438,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
                         const uint4 w4 = sqd::lds128(src + (128 + tr) * ROWB + ((ck ^ (tr & 7)) << 4));
                         const uint32_t sw = static_cast<uint32_t>(tr & 7);
                         const uint32_t jj = static_cast<uint32_t>(ck & 3);
-                        const uint32_t row = op_b((u0 + j) % OPS) + tr * ROWB;
+                        const uint32_t row = op_b((u0 + j) % OPR) + tr * ROWB;
                         sqd::sts128(row + (((2u * jj) ^ sw) << 4), ex((w4.x << 4) & 0xF0F0F0F0u), ex(w4.x & 0xF0F0F0F0u),
                                     ex((w4.y << 4) & 0xF0F0F0F0u), ex(w4.y & 0xF0F0F0F0u));
                         sqd::sts128(row + (((2u * jj + 1u) ^ sw) << 4), ex((w4.z << 4) & 0xF0F0F0F0u), ex(w4.z & 0xF0F0F0F0u),
@@ -460,7 +463,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
                     if (j < nblk) {
                         const uint32_t sw = static_cast<uint32_t>(r & 7);
                         const uint32_t jj = static_cast<uint32_t>(q & 3);
-                        const uint32_t row = op_a((u0 + j) % OPS) + r * ROWB;
+                        const uint32_t row = op_a((u0 + j) % OPR) + r * ROWB;
                         const uint32_t a0 = row + (((2u * jj) ^ sw) << 4);
                         const uint32_t a1 = row + (((2u * jj + 1u) ^ sw) << 4);
                         const uint32_t lo0 = ex((w[c].x << 4) & 0xF0F0F0F0u), hi0 = ex(w[c].x & 0xF0F0F0F0u);
@@ -482,7 +485,7 @@ dual_gemm_skinny_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_
             sqd::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                for (int j = 0; j < nblk; ++j) sqd::mbar_arrive(op_full((u0 + j) % OPS));
+                for (int j = 0; j < nblk; ++j) sqd::mbar_arrive(op_full((u0 + j) % OPR));
                 // The stage is released by the last of the four warps to have
                 // read it (a running count per slot, never reset).
                 if ((atomicAdd(&stg_done[s], 1u) + 1u) % SK_PROD_WARPS == 0u) sqd::mbar_arrive(stg_empty(s));
