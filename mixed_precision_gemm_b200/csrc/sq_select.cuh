@@ -10,8 +10,12 @@
 //   O        = the channels of the nO/G best groups (ties to the lower index),
 //              ascending.
 //
-// Row sums are defined block-wise: consecutive blocks of kSelBlock rows, each
-// summed in row order, then the block sums added in block order.  Kernel 1
+// Each column sum is taken here in consecutive blocks of kSelBlock rows, each
+// block summed in row order and the block sums added in block order, for
+// parallelism.  The plain statement sums in row order; any order of adding n
+// nonnegative fp64 terms lies within (n-1)*2^-53 of the exact sum, relative,
+// so the scores agree with it to that bound and the selection can differ
+// only between channels whose scores tie within it.  Kernel 1
 // computes the block sums (one thread per channel pair and block, loads
 // coalesced across channels), kernel 2 adds them in order and forms the score,
 // kernel 3 the group scores, kernel 4 (one CTA) selects by an 8-pass radix

@@ -253,14 +253,11 @@ def linear_fp8(X_bits: np.ndarray, W_bits: np.ndarray, O, rows=None):
 
 
 # ---------------------------------------------------------------- static outlier selection
-SEL_BLOCK = 256  # rows per partial sum in the score definition
-
-
 def select_outliers(X_bits: np.ndarray, W_bits: np.ndarray, nO: int, group: int = 1):
     """Static outlier channels from calibration activations and the weights.
 
-    score[k] = mean_m |X[m,k]| * ||W[:,k]||_2 (fp64, row sums in blocks of
-    SEL_BLOCK rows); the nO/group groups of `group` consecutive channels with
+    score[k] = mean_m |X[m,k]| * ||W[:,k]||_2 (fp64, each column summed in row
+    order); the nO/group groups of `group` consecutive channels with
     the largest summed score (ties to the lower index).  Returns (O int32
     ascending, score float64 [K]).
     """

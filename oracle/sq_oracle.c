@@ -593,25 +593,19 @@ int orc_sqf_linear_rows(const int8_t *qx4, const float *sx4, const uint8_t *qx8,
  *   group g (channels g*G .. g*G+G-1) scores sum_j score[g*G+j]  (G = 1: per channel)
  *   O = the channels of the nO/G groups with the largest group score, ties to
  *       the lower group index, in ascending channel order.
- * Sums over rows are taken in consecutive blocks of ORC_SEL_BLOCK rows: each
- * block summed in row order, then the block sums added in block order (fp64
- * throughout; squares and absolute values of bf16 values are exact).  The
- * order is part of the definition so that a parallel evaluation can match it
- * bit for bit.
+ * Each column sum runs over the rows in order, 0 to rows-1, in fp64 (|x| and
+ * x*x of a bf16 value are exact in fp64, so the only rounding is that of the
+ * additions).  This is the plain statement of the two sums.  Any order of
+ * adding n nonnegative terms in fp64 lands within (n-1)*2^-53 of the exact
+ * sum, relative, so another evaluation order differs from this one by at
+ * most twice that.
  */
-#define ORC_SEL_BLOCK 256
-
-static double orc_blocked_col_sum(const uint16_t *A, int64_t rows, int64_t ld, int64_t k, int square)
+static double orc_col_sum(const uint16_t *A, int64_t rows, int64_t ld, int64_t k, int square)
 {
     double total = 0.0;
-    for (int64_t b = 0; b < rows; b += ORC_SEL_BLOCK) {
-        double part = 0.0;
-        const int64_t e = (b + ORC_SEL_BLOCK < rows) ? b + ORC_SEL_BLOCK : rows;
-        for (int64_t r = b; r < e; ++r) {
-            const double v = (double)orc_bf16_to_f32(A[r * ld + k]);
-            part += square ? v * v : fabs(v);
-        }
-        total += part;
+    for (int64_t r = 0; r < rows; ++r) {
+        const double v = (double)orc_bf16_to_f32(A[r * ld + k]);
+        total += square ? v * v : fabs(v);
     }
     return total;
 }
@@ -637,8 +631,8 @@ int orc_select_outliers(const uint16_t *X, int64_t Mc, int64_t K, int64_t ldx,
         return -1;
 #pragma omp parallel for schedule(static)
     for (int64_t k = 0; k < K; ++k) {
-        const double mean_abs = orc_blocked_col_sum(X, Mc, ldx, k, 0) / (double)Mc;
-        score[k] = mean_abs * sqrt(orc_blocked_col_sum(W, N, ldw, k, 1));
+        const double mean_abs = orc_col_sum(X, Mc, ldx, k, 0) / (double)Mc;
+        score[k] = mean_abs * sqrt(orc_col_sum(W, N, ldw, k, 1));
     }
     const int64_t ng = K / group, pick = nO / group;
     double *gs = (double *)malloc((size_t)ng * sizeof(double));

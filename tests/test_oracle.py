@@ -291,6 +291,30 @@ def test_chan_table_definition():
         assert int(tab[c]) == (below << 8) | mask
 
 
+def decode_chan_map(tab: np.ndarray, K: int) -> np.ndarray:
+    """The per-channel map the channel table stands for: >= 0 is the channel's rank among
+    the normal channels, -(1+j) marks outlier j (its rank in O)."""
+    out = np.zeros(K, np.int64)
+    for k in range(K):
+        word = int(tab[k // 8])
+        below, mask = word >> 8, word & 0xFF
+        before = below + bin(mask & ((1 << (k % 8)) - 1)).count("1")   # outliers below k
+        out[k] = -(1 + before) if mask >> (k % 8) & 1 else k - before
+    return out
+
+
+@pytest.mark.parametrize("K,nO,seed", [(64, 7, 0), (4096, 256, 1), (2048, 0, 2), (1024, 1024, 3), (14336, 1792, 4)])
+def test_chan_table_decodes_to_rank_and_outlier_map(K, nO, seed):
+    """The compact table (one word per 8 channels) holds exactly the per-channel
+    map chan_map[k] = normal rank, or -(1+j) for outlier j, for a random O."""
+    O = np.sort(np.random.default_rng(seed).choice(K, nO, replace=False)).astype(np.int32)
+    want = np.zeros(K, np.int64)
+    normal = np.setdiff1d(np.arange(K), O)
+    want[normal] = np.arange(normal.size)
+    want[O] = -(1 + np.arange(nO))
+    assert np.array_equal(decode_chan_map(oracle.chan_table(O, K), K), want)
+
+
 def test_outlier_set_validation():
     assert oracle.validate_outliers([1, 4, 9], 10)
     assert oracle.validate_outliers([], 10)
@@ -467,13 +491,39 @@ def _sel_case(Mc=300, K=256, N=96, seed=0):
 
 def test_selection_scores_match_library():
     """score = mean |X| per column x L2 norm of the weight column (numpy, another summation order)."""
-    X, W = _sel_case(Mc=2500, N=1100)  # several 256-row blocks on both sides
+    X, W = _sel_case(Mc=2500, N=1100)
     Xb, Wb = _bf(X), _bf(W)
     O, sc = oracle.select_outliers(Xb, Wb, 16)
     ref = np.mean(np.abs(_f64(Xb)), axis=0) * np.linalg.norm(_f64(Wb), axis=0)
     assert np.allclose(sc, ref, rtol=1e-13, atol=0)
     want = np.sort(np.argsort(-ref, kind="stable")[:16])
     assert np.array_equal(O, want.astype(np.int32))
+
+
+def test_selection_scores_within_the_bound_of_the_exact_score():
+    """Against exact rationals: S1 = sum |x| and S2 = sum w^2 over each column, summed
+    exactly; score = (S1 / Mc) * sqrt(S2) evaluated to 40 digits.  fp64 sums of n
+    nonnegative terms are within (n-1)*2^-53 of the exact sum, relative; the square
+    root halves that, and the division, root and product add one rounding each."""
+    from decimal import Decimal, getcontext
+    from fractions import Fraction
+    getcontext().prec = 40
+    X, W = _sel_case(Mc=97, K=24, N=53, seed=12)
+    X[5] *= 2.0 ** 30        # rows of very different size: the sums round
+    X[6] *= 2.0 ** -30
+    W[7] *= 2.0 ** 20
+    Xb, Wb = _bf(X), _bf(W)
+    _, sc = oracle.select_outliers(Xb, Wb, 4)
+    xf, wf = _f64(Xb), _f64(Wb)
+    Mc, N = xf.shape[0], wf.shape[0]
+    bound = ((Mc - 1) + (N - 1) / 2 + 4) * 2.0 ** -53
+    for k in range(xf.shape[1]):
+        s1 = sum((Fraction(abs(float(v))) for v in xf[:, k]), Fraction(0))
+        s2 = sum((Fraction(float(v)) ** 2 for v in wf[:, k]), Fraction(0))
+        exact = (Decimal(s1.numerator) / Decimal(s1.denominator) / Mc) * \
+            (Decimal(s2.numerator) / Decimal(s2.denominator)).sqrt()
+        rel = abs(Decimal(float(sc[k])) - exact) / exact
+        assert rel <= Decimal(bound), (k, float(rel), bound)
 
 
 def test_selection_finds_planted_channels():
