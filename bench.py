@@ -6,8 +6,9 @@ quantize-and-gather of X (per-token scales, packed INT4 codes, compact bf16
 outlier channels) followed by the dual-path GEMM with its fused epilogue.
 The offline weight preparation is done once before timing.
 
-Default workload: the Llama-3-8B fused QKV projection shape
-(M=2048 tokens, K=4096, N=6144, |O|=256 outlier channels).
+Default workload: the Llama-3-70B fused gate+up projection shape
+(M=8192 tokens, K=8192, N=57344, |O|=512 outlier channels), the largest
+single-GPU configuration and one of the 8192-token shapes.
 
 Output: one JSON line on rank 0 (see the keys written in ``main``).
   value        whole-job TOPS = 2*M*N*K per step (all MACs of both paths), device-timed
@@ -42,7 +43,7 @@ import torch  # noqa: E402
 
 import workloads  # noqa: E402
 
-DEFAULT_WORKLOAD = workloads.LLAMA8B_QKV.name
+DEFAULT_WORKLOAD = workloads.LLAMA70B_GATEUP.name
 METRIC = "dual-path W4A4+BF16 GEMM TOPS & % tensor peak; quant-gather HBM GB/s"
 INT8_PER_BF16 = 2.0   # nominal dense int8 (and fp8) : bf16 tensor rate on B200 (4.5 : 2.25 POPS)
 MXF4_PER_BF16 = 4.0   # nominal dense block-scaled fp4 : bf16 tensor rate on B200 (9 : 2.25 PFLOPS)
@@ -273,12 +274,17 @@ def run_reference(args, w, rank, world):
     line = {"impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int64+f64" if args.low == "int4" else "f64",
-            "data": "synthetic", "config": {**w.describe(), **low_config(args)},
+            "data": "synthetic", "config": run_config(w, args, world),
             "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def run_config(w, args, world: int) -> dict:
+    """The workload's description, the same on both arms."""
+    return {**w.describe(), **low_config(args), "parallelism": f"dp{world}" if world > 1 else "single"}
 
 
 def low_config(args) -> dict:
@@ -609,9 +615,9 @@ def main():
                       "e2m1*e2m1 (e8m0 per 32)->f32 + bf16*bf16->f32" if mx else
                       "s4*s4->s32 + e4m3 (2:4 sparse)*e4m3->f32" if sqf else "s4*s4->s32 + bf16*bf16->f32"),
             "data": "synthetic",
-            "config": {**w.describe(), **low_config(args), "parallelism": f"dp{world}" if world > 1 else "single",
-                       "l2": f"{n_sets} rotating input sets of {foot / 1e6:.0f} MB (> L2 {l2 / 1e6:.0f} MB)",
-                       "timing": "K steps replayed from one CUDA graph; per-kernel times from graphs of K launches"},
+            "config": run_config(w, args, world),
+            "timing": {"l2": f"{n_sets} rotating input sets of {foot / 1e6:.0f} MB (> L2 {l2 / 1e6:.0f} MB)",
+                       "method": "K steps replayed from one CUDA graph; per-kernel times from graphs of K launches"},
             "roofline": {**gemm_roof, "traffic": recorded_traffic(w.name, "dual_gemm", args.low),
                          "kernel": "dual_gemm", "ms": ms_gemm, "algorithmic_bytes": g_bytes,
                          "algorithmic_ops": flops},
