@@ -130,13 +130,6 @@ def test_fp8_ties_signed_zero_and_zero_rows():
     check_layer_fp8(O.numpy(), X.to(torch.bfloat16), W.to(torch.bfloat16))
 
 
-def test_fp8_down_projection_sampled():
-    """The layer the pages' FP8 fallback is for: Llama-3-8B down projection, full size."""
-    w = workloads.LLAMA8B_DOWN
-    O, X, W = workloads.make(w)
-    check_layer_fp8(O.numpy(), X, W, rows=sampled_rows(w.M, 16))
-
-
 def test_fp8_linear_matches_two_calls():
     w = workloads.Workload("t", 257, 2048, 640, 96, x_kind="swiglu", sigma=40.0)
     O, X, W = workloads.make(w)
@@ -157,10 +150,3 @@ def test_fp8_wide_rows_rejected():
     with pytest.raises(sq.SQError) as e:
         sq.prepare_weights(W, [1, 2], fp8=True)
     assert e.value.status == sq.SQ_ERR_UNSUPPORTED
-
-
-@pytest.mark.parametrize("name", ["llama3_8b_qkv_2048x4096x6144_o256", "sweep_M8192_o1/16"])
-def test_fp8_full_size_sampled(name):
-    w = workloads.CONFIGS[name]
-    O, X, W = workloads.make(w)
-    check_layer_fp8(O.numpy(), X, W, rows=sampled_rows(w.M, 8))

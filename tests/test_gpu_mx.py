@@ -159,13 +159,6 @@ def test_mx_decode_sweep_point():
     check_layer_mx(O.numpy(), X, W)
 
 
-def test_mx_qkv_sampled():
-    """Llama-3-8B QKV projection at full size with the MX low path, sampled rows."""
-    w = workloads.LLAMA8B_QKV
-    O, X, W = workloads.make(w)
-    check_layer_mx(O.numpy(), X, W, rows=sampled_rows(w.M, 16))
-
-
 def test_mx_quant_padded_ld_and_wide_rows():
     """X with a row stride above K, and rows wider than any configuration."""
     dev = torch.device("cuda")
@@ -210,12 +203,3 @@ def test_mx_argument_errors():
         sq.sq_gemm_mx(X_N4, S_X, X_O, pw.W_N, pw.s_w, pw.W_O, 4, 12, 256, 2,
                       torch.zeros(4, 16, dtype=torch.bfloat16, device=dev))
     assert e.value.status == sq.SQ_ERR_INVALID_ARG
-
-
-@pytest.mark.parametrize("name", ["llama3_8b_down_4096x14336x4096_o1792", "llama3_70b_gateup_8192x8192x57344_o512",
-                                  "sweep_M8192_o1/16"])
-def test_mx_full_size_sampled(name):
-    """The remaining full-size configurations with the MX low path, every quantizer row, sampled GEMM rows."""
-    w = workloads.CONFIGS[name]
-    O, X, W = workloads.make(w)
-    check_layer_mx(O.numpy(), X, W, rows=sampled_rows(w.M, 8))

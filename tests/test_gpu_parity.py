@@ -248,20 +248,8 @@ def sampled_rows(M, n=64, seed=123):
     return np.sort(np.concatenate([rows, [0, M - 1]]).astype(np.int64))
 
 
-@pytest.mark.parametrize("name", [workloads.LLAMA8B_QKV.name, workloads.LLAMA8B_DOWN.name,
-                                  workloads.LLAMA70B_GATEUP.name])
-def test_full_size_configs_sampled(name):
-    w = workloads.CONFIGS[name]
-    O, X, W = workloads.make(w)
-    rows = sampled_rows(w.M, 32 if w.N > 10000 else 64)
-    check_layer(O.numpy(), X, W, rows=rows)
-
-
-@pytest.mark.parametrize("name", ["sweep_M16_o1/2", "sweep_M16_o0", "sweep_M512_o1/16", "sweep_M8192_o1/4"])
-def test_sweep_points_sampled(name):
-    w = workloads.CONFIGS[name]
-    O, X, W = workloads.make(w)
-    check_layer(O.numpy(), X, W, rows=sampled_rows(w.M, 48))
+# The full-size configurations and every sweep point are checked through
+# sq_linear in test_gpu_linear.py.
 
 
 # ----------------------------------------------------------------- failure detection
