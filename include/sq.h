@@ -23,8 +23,11 @@
  * a row whose normal channels are all zero gets s = 0 and zero codes.
  *
  * Conventions for every call
- *   - Memory: every buffer is allocated by the caller.  The library keeps
- *     only a per-device error word; it never allocates device memory.
+ *   - Memory: every buffer is allocated by the caller; no call allocates
+ *     device memory.  The library's own device state is a per-device error
+ *     word and the fixed SQ_NOALLOC_WS_BYTES scratch array of
+ *     sq_linear_noalloc (below), both module variables that every device
+ *     holds from the moment it loads the library.
  *   - Pointers named "dev" are device pointers, "host" host pointers.  All
  *     device pointers must be 16-byte aligned (SQ_ERR_MISALIGNED otherwise).
  *   - Matrices are row-major.  bf16 buffers are passed as void* holding IEEE
@@ -166,7 +169,8 @@ sq_status sq_linear(const void *X, int64_t M, int64_t K, int64_t ldx,
  *     larger requests return SQ_ERR_UNSUPPORTED before anything is enqueued.
  *   - Every device that loads the library holds this 16 MiB until the process
  *     exits.
- *   - The first call on a device looks up the array's device address once;
+ *   - The first call on a device looks up the array's device address once
+ *     (again only after a device reset has replaced the device's context);
  *     make that first call before any stream capture begins.
  *   - All calls share the one array and it keeps the previous call's
  *     contents.  Nothing in it has to start at zero (the quantize-and-gather

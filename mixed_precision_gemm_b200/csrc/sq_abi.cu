@@ -83,15 +83,40 @@ sq_status device_info(DevInfo &out)
     return SQ_OK;
 }
 
+// ---------------------------------------------------------------- current context
+// Settings made on a device (a kernel's shared-memory opt-in, the address of
+// a module variable) belong to the device's current context; a device reset
+// (cudaDeviceReset) ends it and the next call runs in a new one.  The caches
+// below are therefore keyed by the context handle, read from the driver.
+typedef CUresult (*PFN_ctx_get_current)(CUcontext *);
+PFN_ctx_get_current g_ctx_get = nullptr;
+std::once_flag g_ctx_once;
+
+sq_status current_context(CUcontext &ctx)
+{
+    std::call_once(g_ctx_once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 4000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_get = reinterpret_cast<PFN_ctx_get_current>(p);
+    });
+    if (!g_ctx_get) return fail(SQ_ERR_CUDA, "cuCtxGetCurrent is not available from the driver");
+    ctx = nullptr;
+    if (g_ctx_get(&ctx) != CUDA_SUCCESS) return fail(SQ_ERR_CUDA, "cuCtxGetCurrent failed");
+    return SQ_OK;   // NULL when the runtime has not made a context current on this thread yet
+}
+
 // ---------------------------------------------------------------- per-kernel launch set-up
 // The dynamic shared-memory opt-in of each kernel (a per-function limit:
 // only ever raised, to the largest size launched so far) and its occupancy
-// per launch shape are set and queried once per device; later calls
-// (including calls made while a stream is captured into a CUDA graph) only
-// look them up.
+// per launch shape are set and queried once per device and context; later
+// calls (including calls made while a stream is captured into a CUDA graph)
+// only look them up.
 struct KernelLimit {
     const void *fn;
     int dev;
+    CUcontext ctx;
     size_t smem_max;
 };
 struct KernelSetup {
@@ -110,12 +135,16 @@ sq_status kernel_setup(const void *fn, int threads, size_t smem, int &per_sm, co
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    CUcontext ctx;
+    const sq_status cst = current_context(ctx);
+    if (cst != SQ_OK) return cst;
     std::lock_guard<std::mutex> lk(g_setup_mu);
     KernelLimit *lim = nullptr;
     for (KernelLimit &l : g_limits)
         if (l.fn == fn && l.dev == dev) lim = &l;
+    if (lim && ctx && lim->ctx != ctx) *lim = {fn, dev, ctx, 48 * 1024};   // a new context: the opt-in is gone
     if (!lim) {
-        g_limits.push_back({fn, dev, 48 * 1024});
+        g_limits.push_back({fn, dev, ctx, 48 * 1024});
         lim = &g_limits.back();
     }
     if (smem > lim->smem_max) {
@@ -1298,22 +1327,29 @@ static __device__ __align__(256) uint8_t g_sq_noalloc_ws[SQ_NOALLOC_WS_BYTES];
 namespace {
 
 void *g_noalloc_addr[kMaxDevices];
+CUcontext g_noalloc_ctx[kMaxDevices];
 std::mutex g_noalloc_mu;
 
-// Device address of the scratch array on the current device (looked up on the
-// first call for each device, with that device current).
+// Device address of the scratch array on the current device, looked up on the
+// first call for each device (with that device current) and again only if
+// the device's context has changed since (after a device reset the module,
+// and with it the array, is loaded anew).
 sq_status noalloc_scratch(void **out)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
     if (dev < 0 || dev >= kMaxDevices) return fail(SQ_ERR_UNSUPPORTED, "device index %d", dev);
+    CUcontext ctx;
+    SQ_TRY(current_context(ctx));
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_addr[dev]) {
+    if (!g_noalloc_addr[dev] || (ctx && g_noalloc_ctx[dev] != ctx)) {
         void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_sq_noalloc_ws);
+        e = cudaGetSymbolAddress(&p, g_sq_noalloc_ws);   // makes the device's context current if needed
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        SQ_TRY(current_context(ctx));
         g_noalloc_addr[dev] = p;
+        g_noalloc_ctx[dev] = ctx;
     }
     *out = g_noalloc_addr[dev];
     return SQ_OK;
