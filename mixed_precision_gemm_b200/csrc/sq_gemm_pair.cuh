@@ -72,7 +72,8 @@ struct CfgPair {
     static constexpr int OFF_STG = OFF_SF + OPS * SF_BYTES;
     static constexpr int OFF_BAR = OFF_STG + STG * STG_BYTES;
     // barriers: op_full[OPS] op_empty[OPS] stg_full[STG] stg_empty[STG] acc_full acc_empty drain
-    static constexpr int NBAR = 2 * OPS + 2 * STG + 3;
+    // low_full conv_done
+    static constexpr int NBAR = 2 * OPS + 2 * STG + 5;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SW = (OFF_MISC + 16 + 15) / 16 * 16;   // per epilogue warp: its 128 s_w values
     // Per epilogue warp: YB boxes of 32 x 16 bf16, the source of bulk tensor
@@ -130,6 +131,8 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
     const uint32_t acc_full = bar0 + 8u * (2 * OPS + 2 * STG);
     const uint32_t acc_empty = acc_full + 8u;
     const uint32_t drain = acc_full + 16u;
+    const uint32_t low_full = acc_full + 24u;   // (not MX) a tile's low-path sums are complete
+    const uint32_t conv_done = acc_full + 32u;  // (not MX) both CTAs' epilogue warps have folded them
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC + 4);
     auto op_a = [&](int e) { return sbase + C::OFF_OP + e * C::OP_BYTES; };
@@ -147,6 +150,8 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         sqd::mbar_init(acc_full, 1);                        // multicast commit
         sqd::mbar_init(acc_empty, 2 * PAIR_EPI_WARPS);      // epilogue warps of both CTAs (first CTA's copy)
         sqd::mbar_init(drain, 1);
+        sqd::mbar_init(low_full, 1);                        // multicast commit
+        sqd::mbar_init(conv_done, 2 * PAIR_EPI_WARPS);      // epilogue warps of both CTAs (first CTA's copy)
         *abort_flag = 0u;
         sqd::fence_barrier_init();
         sqd::fence_proxy_async_smem();
@@ -214,28 +219,73 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             constexpr uint32_t idesc_f8 = sqd::make_idesc_e4m3(PAIR_BM, PAIR_BN);
             constexpr uint32_t idesc_mx = sqd::make_idesc_mxf4(PAIR_BM, PAIR_BN);
             bool ok = true;
-            for (int lt = 0; lt < my_tiles && ok; ++lt) {
-                if (!sqd::mbar_wait(acc_empty, (lt & 1) ^ 1u, abort_flag, SITE_MMA_ACC)) { ok = false; break; }
-                sqd::tc_fence_after();
-                for (int i = 0; i < per_tile; ++i) {
-                    const int u = lt * per_tile + i;
-                    const int e = u % OPS;
-                    if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_MMA_FULL)) { ok = false; break; }
+            if constexpr (!MX) {
+                // Per tile: the low-path blocks into acc_i (columns [0, 256)); the epilogue
+                // warps fold acc_i * s_x * s_w into columns [256, 512) (conv_done), which
+                // frees acc_i for the next tile at once; the bf16 blocks then accumulate
+                // on top of the folded values, and the epilogue only rounds and stores
+                // them while the next tile's low blocks run.
+                for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                    for (int i = 0; i < nkb_i; ++i) {
+                        const int u = lt * per_tile + i;
+                        const int e = u % OPS;
+                        if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_MMA_FULL)) { ok = false; break; }
+                        sqd::tc_fence_after();
+                        const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
+                        const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t acc = (i == 0 && k == 0) ? 0u : 1u;
+                            if constexpr (FP8) sqd::mma_f8_pair(tmem, adesc + 2 * k, bdesc + 2 * k, idesc_f8, acc);
+                            else sqd::mma_s8_pair(tmem, adesc + 2 * k, bdesc + 2 * k, idesc_i8, acc);
+                        }
+                        sqd::mma_commit_pair_multicast(op_empty(e), 0x3);
+                    }
+                    if (!ok) break;
+                    if (nkb_i > 0) sqd::mma_commit_pair_multicast(low_full, 0x3);
+                    // The folded values are in place (and the previous tile's stores have read
+                    // columns [256, 512)) once every epilogue warp of both CTAs has arrived.
+                    if (!sqd::mbar_wait(conv_done, lt & 1, abort_flag, SITE_MMA_ACC)) { ok = false; break; }
                     sqd::tc_fence_after();
-                    const bool is_bf = i < nkb_o;
-                    const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
-                    const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
-                    // MX: one accumulator for both paths; otherwise the low path has its own.
-                    const uint32_t d = tmem + ((is_bf || MX) ? 0u : static_cast<uint32_t>(PAIR_BN));
-                    const bool first = MX ? (i == 0) : ((i == 0) || (i == nkb_o));
-                    if constexpr (MX) {
+                    for (int i = nkb_i; i < per_tile; ++i) {
+                        const int u = lt * per_tile + i;
+                        const int e = u % OPS;
+                        if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_MMA_FULL)) { ok = false; break; }
+                        sqd::tc_fence_after();
+                        const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
+                        const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            // without a low part nothing was folded in: the first MMA clears
+                            const uint32_t acc = (nkb_i == 0 && i == 0 && k == 0) ? 0u : 1u;
+                            sqd::mma_bf16_pair(tmem + static_cast<uint32_t>(PAIR_BN), adesc + 2 * k, bdesc + 2 * k,
+                                               idesc_bf, acc);
+                        }
+                        sqd::mma_commit_pair_multicast(op_empty(e), 0x3);
+                    }
+                    if (ok) sqd::mma_commit_pair_multicast(acc_full, 0x3);
+                }
+            } else {
+                // MX: the block-scaled products and the 16-bit branch share one fp32
+                // accumulator (columns [0, 256)); the bf16 blocks come first.
+                for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                    if (!sqd::mbar_wait(acc_empty, (lt & 1) ^ 1u, abort_flag, SITE_MMA_ACC)) { ok = false; break; }
+                    sqd::tc_fence_after();
+                    for (int i = 0; i < per_tile; ++i) {
+                        const int u = lt * per_tile + i;
+                        const int e = u % OPS;
+                        if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_MMA_FULL)) { ok = false; break; }
+                        sqd::tc_fence_after();
+                        const bool is_bf = i < nkb_o;
+                        const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
+                        const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
+                        // Two TMEM scale buffers alternate by K-block, so the copies of one
+                        // block need not wait for the MMAs that read the previous one.
+                        const uint32_t sb = tmem + MX_SF_BUF * static_cast<uint32_t>((i - nkb_o) & 1);
                         if (!is_bf) {
                             // Scales of this K-block: X-row tiles (K-tiles 0, 1) at sf, sf + 512; W-row
                             // tiles of rows 0-127 at sf + 1024 (+512 for K-tile 1), rows 128-255 at sf + 2048.
-                            // Two TMEM scale buffers alternate by K-block, so the copies of one
-                            // block need not wait for the MMAs that read the previous one.
                             const uint32_t sf = sbase + C::OFF_SF + e * C::SF_BYTES;
-                            const uint32_t sb = tmem + MX_SF_BUF * static_cast<uint32_t>((i - nkb_o) & 1);
                             sqd::sf_copy_pair(sb + MX_SFA_COL, sqd::make_sf_desc(sf));
                             sqd::sf_copy_pair(sb + MX_SFA_COL + 4, sqd::make_sf_desc(sf + 512));
                             sqd::sf_copy_pair(sb + MX_SFB_COL, sqd::make_sf_desc(sf + 1024));
@@ -243,25 +293,24 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                             sqd::sf_copy_pair(sb + MX_SFB_COL + 8, sqd::make_sf_desc(sf + 1536));
                             sqd::sf_copy_pair(sb + MX_SFB_COL + 12, sqd::make_sf_desc(sf + 2560));
                         }
-                    }
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const uint32_t acc = (first && k == 0) ? 0u : 1u;
-                        if (is_bf) sqd::mma_bf16_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_bf, acc);
-                        else if constexpr (MX) {
-                            // MMA k covers scale blocks 2k, 2k+1: K-tile k / 2, bytes 2 (k % 2) and up.
-                            const uint32_t id = 2u * static_cast<uint32_t>(k & 1);
-                            const uint32_t sb = tmem + MX_SF_BUF * static_cast<uint32_t>((i - nkb_o) & 1);
-                            const uint32_t sfa = (sb + MX_SFA_COL + 4 * (k >> 1)) | (id << 30);
-                            const uint32_t sfb = (sb + MX_SFB_COL + 8 * (k >> 1)) | (id << 30);
-                            sqd::mma_mxf4_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_mx | (id << 29) | (id << 4), acc,
-                                               sfa, sfb);
-                        } else if constexpr (FP8) sqd::mma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_f8, acc);
-                        else sqd::mma_s8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_i8, acc);
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t acc = (i == 0 && k == 0) ? 0u : 1u;
+                            if (is_bf) {
+                                sqd::mma_bf16_pair(tmem, adesc + 2 * k, bdesc + 2 * k, idesc_bf, acc);
+                            } else {
+                                // MMA k covers scale blocks 2k, 2k+1: K-tile k / 2, bytes 2 (k % 2) and up.
+                                const uint32_t id = 2u * static_cast<uint32_t>(k & 1);
+                                const uint32_t sfa = (sb + MX_SFA_COL + 4 * (k >> 1)) | (id << 30);
+                                const uint32_t sfb = (sb + MX_SFB_COL + 8 * (k >> 1)) | (id << 30);
+                                sqd::mma_mxf4_pair(tmem, adesc + 2 * k, bdesc + 2 * k, idesc_mx | (id << 29) | (id << 4),
+                                                   acc, sfa, sfb);
+                            }
+                        }
+                        sqd::mma_commit_pair_multicast(op_empty(e), 0x3);
                     }
-                    sqd::mma_commit_pair_multicast(op_empty(e), 0x3);
+                    if (ok) sqd::mma_commit_pair_multicast(acc_full, 0x3);
                 }
-                if (ok) sqd::mma_commit_pair_multicast(acc_full, 0x3);
             }
             if (!ok) {
                 sqd::mma_commit_pair(drain);
@@ -282,7 +331,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
           } else {
             const int lt = f / nkb_i;
             const int kb = f - lt * nkb_i;
-            const int u = lt * per_tile + nkb_o + kb;
+            const int u = lt * per_tile + kb;   // low blocks open the tile (not MX)
             const int e = u % OPS;
             const int si = f % STG;
             if (!sqd::mbar_wait(stg_full(si), (f / STG) & 1, abort_flag, SITE_EXP_OP)) return false;
@@ -374,17 +423,24 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             }
         };
 
-        // Ring uses of this group, in order: u = gi, gi + NG, ...  bf16 blocks
-        // first, then the low-path blocks (E4M3 or E2M1 by TMA, or INT4 expanded).
+        // Ring uses of this group, in order: u = gi, gi + NG, ...  Per tile the
+        // low-path blocks (E4M3 by TMA, or INT4 expanded), then the bf16 blocks;
+        // MX: the bf16 blocks, then the E2M1 blocks.
         bool ok = true;
         const int total = my_tiles * per_tile;
         for (int u = gi; u < total && ok; u += C::NG) {
             const int lt = u / per_tile;
             const int i = u - lt * per_tile;
-            if (i < nkb_o) ok = produce_tma(lt, u, &tm_xo, &tm_wo, i * KB_BF);
-            else if constexpr (FP8) ok = produce_tma(lt, u, &tm_xn, &tm_wn, (i - nkb_o) * KB_I8);
-            else if constexpr (MX) ok = produce_mx(lt, u, i - nkb_o);
-            else ok = store(lt * nkb_i + (i - nkb_o));
+            if constexpr (MX) {
+                if (i < nkb_o) ok = produce_tma(lt, u, &tm_xo, &tm_wo, i * KB_BF);
+                else ok = produce_mx(lt, u, i - nkb_o);
+            } else if (i >= nkb_i) {
+                ok = produce_tma(lt, u, &tm_xo, &tm_wo, (i - nkb_i) * KB_BF);
+            } else if constexpr (FP8) {
+                ok = produce_tma(lt, u, &tm_xn, &tm_wn, i * KB_I8);
+            } else {
+                ok = store(lt * nkb_i + i);
+            }
         }
         if (!ok && tma_thread && last_armed >= 0 && leader) {
             // Let the last copies that were issued land before the CTA exits.
@@ -392,19 +448,35 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         }
     } else if (warp >= PAIR_EPI_WARP0 && warp < PAIR_EPI_WARP0 + PAIR_EPI_WARPS) {
         // ------------------------------------------------------------ epilogue (each CTA: its 128 rows)
-        // Warp w reads TMEM lane quarter w % 4 and half (w - 2) / 4 of the 256
-        // columns, 16 columns at a time; the load of the next 16 columns is in
-        // flight while the current ones are scaled, fused and stored.
+        // Warp w serves TMEM lane quarter w % 4 and half (w - 2) / 4 of the 256
+        // columns, 16 columns at a time, the load of the next 16 columns in
+        // flight while the current ones are processed.
+        //
+        // Not MX, per tile: (1) fold -- once the low-path sums are complete, each
+        // value y0 = ((float)acc_i * s_x) * s_w (+ the SQ-format high part) is
+        // written into the columns of the 16-bit branch, [256, 512), which frees
+        // acc_i for the next tile's MMAs (conv_done); the bf16 MMAs then
+        // accumulate the branch on top of y0 in the same fp32 accumulator.
+        // (2) store -- once the tile is complete, the columns are rounded to
+        // bf16 and written to Y while the next tile's low blocks run.
+        // With debug outputs the fold writes zeros instead, so the branch sum
+        // stays separate, and the store adds y0 (from the exact sums just
+        // written to dbg_i) the same way.
+        // MX: one pass over the single accumulator after the tile.
         const int sub = warp & 3;
         const int half = (warp - PAIR_EPI_WARP0) >> 2;
         const uint32_t tl = tmem + (static_cast<uint32_t>(sub * 32) << 16);
         const bool has_i = nkb_i > 0, has_o = nkb_o > 0;
         const uint32_t empty_leader = sqd::map_to_cta(acc_empty, 0);
+        const uint32_t conv_leader = sqd::map_to_cta(conv_done, 0);
         constexpr int CW = 16;                   // columns per TMEM load
         constexpr int NCH = (PAIR_BN / 2) / CW;  // 8 loads per accumulator per warp
         static_assert(CW == 16, "one staging box is 16 columns");
         const bool y_tma = C::YB > 0 && args.y_tma != 0;
+        const bool split = DBG && args.dbg_i != nullptr;   // keep the branch sum apart (debug outputs)
         const uint32_t yst = sbase + C::OFF_YST + (warp - PAIR_EPI_WARP0) * C::YB * 1024;
+        const uint32_t sw_smem = sbase + C::OFF_SW + (warp - PAIR_EPI_WARP0) * 512;
+        const uint32_t acc_col = MX ? 0u : static_cast<uint32_t>(PAIR_BN);   // what the store pass reads
         int last_box = -1;  // staging box of this warp's latest bulk store
         for (int lt = 0; lt < my_tiles; ++lt) {
             int tmi, tni;
@@ -419,28 +491,90 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
             const float sx = (!MX && row_ok) ? args.s_x[m] : 0.0f;
             uint16_t *yrow = args.Y + static_cast<long long>(row_ok ? m : 0) * args.ldy;
+            const int m0 = tmi * PAIR_BM + static_cast<int>(rank) * 128 + sub * 32;  // this warp's first row
+
+            if constexpr (!MX) {
+                // ---------------------------------------------------- (1) fold
+                if (has_i) {
+                    if (!sqd::mbar_wait(low_full, lt & 1, abort_flag, SITE_EPI)) break;
+                    sqd::tc_fence_after();
+                    sqd::sts128(sw_smem + 16 * lane, __float_as_uint(swp.x), __float_as_uint(swp.y),
+                                __float_as_uint(swp.z), __float_as_uint(swp.w));
+                    __syncwarp();
+                    uint32_t va[2][CW];
+                    sqd::tmem_ld_32x32b_x16(tl + c_base, va[0]);
+                    sqd::tmem_wait_ld_dep1(va[0]);
+#pragma unroll
+                    for (int ch = 0; ch < NCH; ++ch) {
+                        const int b = ch & 1;
+                        if (ch + 1 < NCH) sqd::tmem_ld_32x32b_x16(tl + c_base + (ch + 1) * CW, va[b ^ 1]);
+                        const int n0 = tni * PAIR_BN + c_base + ch * CW;
+                        uint32_t y0[CW];
+#pragma unroll
+                        for (int g = 0; g < CW / 8; ++g) {
+                            const int n = n0 + 8 * g;
+                            const bool ok8 = row_ok && n < args.N;  // N is a multiple of 8
+                            const uint4 sw0 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g));
+                            const uint4 sw1 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g + 4));
+                            const float swv[8] = {__uint_as_float(sw0.x), __uint_as_float(sw0.y), __uint_as_float(sw0.z),
+                                                  __uint_as_float(sw0.w), __uint_as_float(sw1.x), __uint_as_float(sw1.y),
+                                                  __uint_as_float(sw1.z), __uint_as_float(sw1.w)};
+                            float adv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                            if constexpr (SQF) {
+                                // the precomputed high part of these 8 outputs
+                                if (ok8 && !split) {
+                                    const float4 *ap = reinterpret_cast<const float4 *>(args.addend + static_cast<long long>(m) * args.N + n);
+                                    const float4 a0 = ap[0], a1 = ap[1];
+                                    adv[0] = a0.x; adv[1] = a0.y; adv[2] = a0.z; adv[3] = a0.w;
+                                    adv[4] = a1.x; adv[5] = a1.y; adv[6] = a1.z; adv[7] = a1.w;
+                                }
+                            }
+#pragma unroll
+                            for (int q = 0; q < 8; ++q) {
+                                const int t = 8 * g + q;
+                                // exact int32 sum (x256) for INT4, fp32 sum for E4M3
+                                float al;
+                                int32_t dbg_lo;
+                                if constexpr (FP8) {
+                                    al = __uint_as_float(va[b][t]);
+                                    dbg_lo = __float_as_int(al);
+                                } else {
+                                    const int ai = static_cast<int>(va[b][t]) >> 8;
+                                    al = static_cast<float>(ai);
+                                    dbg_lo = ai;
+                                }
+                                const float v = __fadd_rn(__fmul_rn(__fmul_rn(al, sx), swv[q]), adv[q]);
+                                y0[t] = split ? 0u : __float_as_uint(v);
+                                if constexpr (DBG) {
+                                    if (ok8 && args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + q] = dbg_lo;
+                                }
+                            }
+                        }
+                        sqd::tmem_st_32x32b_x16(tl + PAIR_BN + c_base + ch * CW, y0);
+                        if (ch + 1 < NCH) sqd::tmem_wait_ld_dep1(va[b ^ 1]);
+                    }
+                    sqd::tmem_wait_st();
+                }
+                // acc_i has been read and [256, 512) holds y0 (and this warp's stores of
+                // the previous tile have read those columns): the MMAs may go on.
+                sqd::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) sqd::mbar_arrive_cluster(conv_leader);
+            }
+
+            // -------------------------------------------------------- (2) store
             if (!sqd::mbar_wait(acc_full, lt & 1, abort_flag, SITE_EPI)) break;
             sqd::tc_fence_after();
-            const uint32_t sw_smem = sbase + C::OFF_SW + (warp - PAIR_EPI_WARP0) * 512;
-            sqd::sts128(sw_smem + 16 * lane, __float_as_uint(swp.x), __float_as_uint(swp.y), __float_as_uint(swp.z),
-                        __float_as_uint(swp.w));
-            __syncwarp();
-            uint32_t vi[2][CW] = {}, vf[2][CW] = {};
-            auto issue = [&](int ch, int b) {
-                if constexpr (MX) {
-                    sqd::tmem_ld_32x32b_x16(tl + c_base + ch * CW, vf[b]);  // the one accumulator
-                } else {
-                    if (has_i) sqd::tmem_ld_32x32b_x16(tl + PAIR_BN + c_base + ch * CW, vi[b]);
-                    if (has_o) sqd::tmem_ld_32x32b_x16(tl + c_base + ch * CW, vf[b]);
-                }
-            };
-            issue(0, 0);
-            sqd::tmem_wait_ld_dep(vi[0], vf[0]);
-            const int m0 = tmi * PAIR_BM + static_cast<int>(rank) * 128 + sub * 32;  // this warp's first row
+            const bool has_acc = MX || has_i || has_o;
+            uint32_t vf[2][CW] = {};
+            if (has_acc) {
+                sqd::tmem_ld_32x32b_x16(tl + acc_col + c_base, vf[0]);
+                sqd::tmem_wait_ld_dep1(vf[0]);
+            }
 #pragma unroll
             for (int ch = 0; ch < NCH; ++ch) {
                 const int b = ch & 1;
-                if (ch + 1 < NCH) issue(ch + 1, b ^ 1);
+                if (has_acc && ch + 1 < NCH) sqd::tmem_ld_32x32b_x16(tl + acc_col + c_base + (ch + 1) * CW, vf[b ^ 1]);
                 const int n0 = tni * PAIR_BN + c_base + ch * CW;
                 // Bulk-store form: all 32 lanes fill the 32 x 16 box (the store
                 // drops rows past M and columns past N); otherwise each lane
@@ -461,21 +595,6 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                     for (int g = 0; g < CW / 8; ++g) {
                         const int n = n0 + 8 * g;
                         const bool ok8 = row_ok && n < args.N;  // N is a multiple of 8
-                        const uint4 sw0 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g));
-                        const uint4 sw1 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g + 4));
-                        // SQF: the precomputed high part of these 8 outputs
-                        float4 ad0 = make_float4(0.f, 0.f, 0.f, 0.f), ad1 = ad0;
-                        if constexpr (SQF) {
-                            if (ok8) {
-                                const float4 *ap = reinterpret_cast<const float4 *>(args.addend + static_cast<long long>(m) * args.N + n);
-                                ad0 = ap[0];
-                                ad1 = ap[1];
-                            }
-                        }
-                        const float adv[8] = {ad0.x, ad0.y, ad0.z, ad0.w, ad1.x, ad1.y, ad1.z, ad1.w};
-                        const float swv[8] = {__uint_as_float(sw0.x), __uint_as_float(sw0.y), __uint_as_float(sw0.z),
-                                              __uint_as_float(sw0.w), __uint_as_float(sw1.x), __uint_as_float(sw1.y),
-                                              __uint_as_float(sw1.z), __uint_as_float(sw1.w)};
                         uint32_t out[4];
 #pragma unroll
                         for (int h = 0; h < 4; ++h) {
@@ -483,27 +602,22 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
 #pragma unroll
                             for (int u = 0; u < 2; ++u) {
                                 const int t = 8 * g + 2 * h + u;
-                                // low path: exact int32 sum (x256) for INT4, fp32 sum for E4M3;
-                                // MX: the accumulator already holds the whole sum
-                                float al;
-                                int32_t dbg_lo;
-                                if constexpr (MX) {
-                                    al = 0.0f;
-                                    dbg_lo = 0;
-                                } else if constexpr (FP8) {
-                                    al = has_i ? __uint_as_float(vi[b][t]) : 0.0f;
-                                    dbg_lo = __float_as_int(al);
-                                } else {
-                                    const int ai = has_i ? (static_cast<int>(vi[b][t]) >> 8) : 0;
-                                    al = static_cast<float>(ai);
-                                    dbg_lo = ai;
-                                }
-                                const float af = SQF ? adv[2 * h + u] : (MX || has_o) ? __uint_as_float(vf[b][t]) : 0.0f;
-                                y2[u] = MX ? af : __fadd_rn(__fmul_rn(__fmul_rn(al, sx), swv[2 * h + u]), af);
+                                const float acc = __uint_as_float(vf[b][t]);
+                                y2[u] = acc;
                                 if constexpr (DBG) {
-                                    if (ok8) {
-                                        if (args.dbg_i) args.dbg_i[static_cast<long long>(m) * args.N + n + 2 * h + u] = dbg_lo;
-                                        if (args.dbg_f) args.dbg_f[static_cast<long long>(m) * args.N + n + 2 * h + u] = af;
+                                    const long long o = static_cast<long long>(m) * args.N + n + 2 * h + u;
+                                    if (MX && ok8 && args.dbg_f) args.dbg_f[o] = acc;
+                                    if (!MX && !has_i && ok8 && args.dbg_i) args.dbg_i[o] = 0;  // no low part
+                                    if (!MX && split && ok8) {
+                                        // y0 from the exact low-path sum written by the fold pass
+                                        float al = 0.0f, swq = 0.0f;
+                                        if (has_i) {
+                                            al = FP8 ? __int_as_float(args.dbg_i[o]) : static_cast<float>(args.dbg_i[o]);
+                                            swq = __uint_as_float(sqd::lds32(sw_smem + 4 * (ch * CW + 8 * g + 2 * h + u)));
+                                        }
+                                        const float af = SQF ? args.addend[o] : acc;
+                                        y2[u] = __fadd_rn(__fmul_rn(__fmul_rn(al, sx), swq), af);
+                                        if (args.dbg_f) args.dbg_f[o] = af;
                                     }
                                 }
                             }
@@ -523,10 +637,10 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                         last_box = bb;
                     }
                 }
-                if (ch + 1 < NCH) {
-                    sqd::tmem_wait_ld_dep(vi[b ^ 1], vf[b ^ 1]);
-                    if (ch + 2 == NCH) {
-                        // Last load of this warp landed: the accumulators may be reused.
+                if (has_acc && ch + 1 < NCH) {
+                    sqd::tmem_wait_ld_dep1(vf[b ^ 1]);
+                    if (MX && ch + 2 == NCH) {
+                        // Last load of this warp landed: the accumulator may be reused.
                         sqd::tc_fence_before();
                         __syncwarp();
                         if (lane == 0) sqd::mbar_arrive_cluster(empty_leader);

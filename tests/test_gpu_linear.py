@@ -8,10 +8,11 @@ workspace, in the launch configuration the benchmark times, and then checks:
   * the quantize-and-gather outputs that sq_linear left in its workspace
     (codes, scales, compact outlier channels), bit-exact on every token row;
   * Y on a seeded sample of rows, within |dY| <= 1e-2 * max(|Y_ref|, rms(Y_ref));
+  * the GEMM alone on that same workspace gives sq_linear's Y bit for bit;
   * the GEMM's accumulators on the same rows, from a debug run of the GEMM on
-    that same workspace, whose Y must equal sq_linear's bit for bit: the int32
-    sums exactly, the fp32 sums within the fp32 summation bound of the
-    oracle's exact fp64 sums;
+    that workspace: the int32 sums exactly, the fp32 sums within the fp32
+    summation bound of the oracle's exact fp64 sums, and its Y (which adds
+    the two sums outside the tensor core) within the Y tolerance too;
   * nothing written outside Y (a guard row and guard columns).
 """
 from __future__ import annotations
@@ -123,12 +124,15 @@ def test_linear_matches_oracle(name, low):
     chk(O, W, pw.W_N, pw.s_w, pw.W_O, K)
     chk(O, X, X_N, s_x, X_O, K)
 
-    # the GEMM alone on that workspace, with its accumulators exposed: same Y, bit for bit
+    # the GEMM alone on that workspace: same Y, bit for bit; then with its accumulators exposed
     g2, Y2 = guarded_y(M, N, dev)
-    _, dbg_a, dbg_b = sq.gemm(X_N, s_x, X_O, pw, Y=Y2, debug=True)
+    sq.gemm(X_N, s_x, X_O, pw, Y=Y2)
+    g3, Y3 = guarded_y(M, N, dev)
+    _, dbg_a, dbg_b = sq.gemm(X_N, s_x, X_O, pw, Y=Y3, debug=True)
     torch.cuda.synchronize()
     sq.sq_check()
     check_guard(g2, M, N)
+    check_guard(g3, M, N)
     assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16)), "sq_linear and the GEMM on its workspace differ"
 
     sel = sample(M, 16 if N > 10000 else 24)
@@ -157,6 +161,7 @@ def test_linear_matches_oracle(name, low):
         else:
             assert np.all(rows_of(dbg_b, sel) == 0)
     check_y(rows_of(Y, sel), ref["y"])
+    check_y(rows_of(Y3, sel), ref["y"])
 
 
 @pytest.mark.parametrize("name", SQF_CASES)
@@ -195,10 +200,13 @@ def test_linear_sqf_matches_oracle(name):
     assert np.array_equal(s_x8.cpu().numpy().view(np.uint32), sx8.view(np.uint32)), "s_x8 differs"
 
     g2, Y2 = guarded_y(M, N, dev)
-    _, acc_lo, P = sq.gemm_sqf(X_N, s_x4, X_8, s_x8, pw, Y=Y2, debug=True)
+    sq.gemm_sqf(X_N, s_x4, X_8, s_x8, pw, Y=Y2)
+    g3, Y3 = guarded_y(M, N, dev)
+    _, acc_lo, P = sq.gemm_sqf(X_N, s_x4, X_8, s_x8, pw, Y=Y3, debug=True)
     torch.cuda.synchronize()
     sq.sq_check()
     check_guard(g2, M, N)
+    check_guard(g3, M, N)
     assert torch.equal(Y.view(torch.int16), Y2.view(torch.int16)), "sq_linear_sqf and the GEMM differ"
 
     sel = sample(M, 8 if N > 10000 else 16)
@@ -213,3 +221,4 @@ def test_linear_sqf_matches_oracle(name):
     bound = ACC_8_REL * (dx @ dw.T).astype(np.float64) * scale + 2.0 ** -20 * np.abs(p_ref) + 1e-30
     assert np.all(np.abs(rows_of(P, sel) - p_ref) <= bound), "high part off"
     check_y(rows_of(Y, sel), ref["y"])
+    check_y(rows_of(Y3, sel), ref["y"])
