@@ -219,7 +219,36 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             constexpr uint32_t idesc_f8 = sqd::make_idesc_e4m3(PAIR_BM, PAIR_BN);
             constexpr uint32_t idesc_mx = sqd::make_idesc_mxf4(PAIR_BM, PAIR_BN);
             bool ok = true;
-            if constexpr (!MX) {
+            if (!MX && nkb_o == 0) {
+                // No 16-bit branch: two acc_i buffers, columns [0, 256) for even tiles and
+                // [256, 512) for odd ones, so tile t+1's MMAs run under tile t's epilogue.
+                // Buffer r: full = acc_full / low_full, free = acc_empty / conv_done.
+                for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                    const int r = lt & 1;
+                    if (lt >= 2) {
+                        if (!sqd::mbar_wait(r ? conv_done : acc_empty, static_cast<uint32_t>(((lt >> 1) - 1) & 1),
+                                            abort_flag, SITE_MMA_ACC)) { ok = false; break; }
+                        sqd::tc_fence_after();
+                    }
+                    const uint32_t d = tmem + static_cast<uint32_t>(r * PAIR_BN);
+                    for (int i = 0; i < nkb_i; ++i) {
+                        const int u = lt * per_tile + i;
+                        const int e = u % OPS;
+                        if (!sqd::mbar_wait(op_full(e), (u / OPS) & 1, abort_flag, SITE_MMA_FULL)) { ok = false; break; }
+                        sqd::tc_fence_after();
+                        const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
+                        const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint32_t acc = (i == 0 && k == 0) ? 0u : 1u;
+                            if constexpr (FP8) sqd::mma_f8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_f8, acc);
+                            else if constexpr (!MX) sqd::mma_s8_pair(d, adesc + 2 * k, bdesc + 2 * k, idesc_i8, acc);
+                        }
+                        sqd::mma_commit_pair_multicast(op_empty(e), 0x3);
+                    }
+                    if (ok) sqd::mma_commit_pair_multicast(r ? low_full : acc_full, 0x3);
+                }
+            } else if constexpr (!MX) {
                 // Per tile: the low-path blocks into acc_i (columns [0, 256)); the epilogue
                 // warps fold acc_i * s_x * s_w into columns [256, 512) (conv_done), which
                 // frees acc_i for the next tile at once; the bf16 blocks then accumulate
@@ -477,6 +506,12 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         const uint32_t yst = sbase + C::OFF_YST + (warp - PAIR_EPI_WARP0) * C::YB * 1024;
         const uint32_t sw_smem = sbase + C::OFF_SW + (warp - PAIR_EPI_WARP0) * 512;
         const uint32_t acc_col = MX ? 0u : static_cast<uint32_t>(PAIR_BN);   // what the store pass reads
+        // Y is written once: its lines go first when L2 needs room, so the X band
+        // and the W tiles that later tiles reuse stay resident.
+        const uint64_t y_policy = sqd::l2_evict_first();
+        // Not MX and no 16-bit branch: two acc_i buffers, no fold; the store pass
+        // applies the scales itself.
+        const bool dbuf = !MX && !has_o;
         int last_box = -1;  // staging box of this warp's latest bulk store
         for (int lt = 0; lt < my_tiles; ++lt) {
             int tmi, tni;
@@ -493,7 +528,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             uint16_t *yrow = args.Y + static_cast<long long>(row_ok ? m : 0) * args.ldy;
             const int m0 = tmi * PAIR_BM + static_cast<int>(rank) * 128 + sub * 32;  // this warp's first row
 
-            if constexpr (!MX) {
+            if (!MX && !dbuf) {
                 // ---------------------------------------------------- (1) fold
                 if (has_i) {
                     if (!sqd::mbar_wait(low_full, lt & 1, abort_flag, SITE_EPI)) break;
@@ -563,18 +598,27 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             }
 
             // -------------------------------------------------------- (2) store
-            if (!sqd::mbar_wait(acc_full, lt & 1, abort_flag, SITE_EPI)) break;
+            const int rb = dbuf ? (lt & 1) : 0;   // accumulator buffer of this tile (double-buffer mode)
+            if (!sqd::mbar_wait(rb ? low_full : acc_full, static_cast<uint32_t>(dbuf ? ((lt >> 1) & 1) : (lt & 1)),
+                                abort_flag, SITE_EPI))
+                break;
             sqd::tc_fence_after();
+            if (dbuf) {
+                sqd::sts128(sw_smem + 16 * lane, __float_as_uint(swp.x), __float_as_uint(swp.y), __float_as_uint(swp.z),
+                            __float_as_uint(swp.w));
+                __syncwarp();
+            }
+            const uint32_t col = dbuf ? static_cast<uint32_t>(rb * PAIR_BN) : acc_col;
             const bool has_acc = MX || has_i || has_o;
             uint32_t vf[2][CW] = {};
             if (has_acc) {
-                sqd::tmem_ld_32x32b_x16(tl + acc_col + c_base, vf[0]);
+                sqd::tmem_ld_32x32b_x16(tl + col + c_base, vf[0]);
                 sqd::tmem_wait_ld_dep1(vf[0]);
             }
 #pragma unroll
             for (int ch = 0; ch < NCH; ++ch) {
                 const int b = ch & 1;
-                if (has_acc && ch + 1 < NCH) sqd::tmem_ld_32x32b_x16(tl + acc_col + c_base + (ch + 1) * CW, vf[b ^ 1]);
+                if (has_acc && ch + 1 < NCH) sqd::tmem_ld_32x32b_x16(tl + col + c_base + (ch + 1) * CW, vf[b ^ 1]);
                 const int n0 = tni * PAIR_BN + c_base + ch * CW;
                 // Bulk-store form: all 32 lanes fill the 32 x 16 box (the store
                 // drops rows past M and columns past N); otherwise each lane
@@ -595,6 +639,25 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                     for (int g = 0; g < CW / 8; ++g) {
                         const int n = n0 + 8 * g;
                         const bool ok8 = row_ok && n < args.N;  // N is a multiple of 8
+                        float swv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        float adv[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                        if (dbuf) {
+                            const uint4 sw0 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g));
+                            const uint4 sw1 = sqd::lds128(sw_smem + 4 * (ch * CW + 8 * g + 4));
+                            swv[0] = __uint_as_float(sw0.x); swv[1] = __uint_as_float(sw0.y);
+                            swv[2] = __uint_as_float(sw0.z); swv[3] = __uint_as_float(sw0.w);
+                            swv[4] = __uint_as_float(sw1.x); swv[5] = __uint_as_float(sw1.y);
+                            swv[6] = __uint_as_float(sw1.z); swv[7] = __uint_as_float(sw1.w);
+                            if constexpr (SQF) {
+                                // the precomputed high part of these 8 outputs
+                                if (ok8) {
+                                    const float4 *ap = reinterpret_cast<const float4 *>(args.addend + static_cast<long long>(m) * args.N + n);
+                                    const float4 a0 = ap[0], a1 = ap[1];
+                                    adv[0] = a0.x; adv[1] = a0.y; adv[2] = a0.z; adv[3] = a0.w;
+                                    adv[4] = a1.x; adv[5] = a1.y; adv[6] = a1.z; adv[7] = a1.w;
+                                }
+                            }
+                        }
                         uint32_t out[4];
 #pragma unroll
                         for (int h = 0; h < 4; ++h) {
@@ -604,6 +667,26 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                                 const int t = 8 * g + 2 * h + u;
                                 const float acc = __uint_as_float(vf[b][t]);
                                 y2[u] = acc;
+                                if (dbuf) {
+                                    // exact int32 sum (x256) for INT4, fp32 sum for E4M3, scaled here
+                                    float al;
+                                    int32_t dbg_lo;
+                                    if constexpr (FP8) {
+                                        al = has_i ? acc : 0.0f;
+                                        dbg_lo = __float_as_int(al);
+                                    } else {
+                                        const int ai = has_i ? (static_cast<int>(vf[b][t]) >> 8) : 0;
+                                        al = static_cast<float>(ai);
+                                        dbg_lo = ai;
+                                    }
+                                    y2[u] = __fadd_rn(__fmul_rn(__fmul_rn(al, sx), swv[2 * h + u]), adv[2 * h + u]);
+                                    if constexpr (DBG) {
+                                        const long long o = static_cast<long long>(m) * args.N + n + 2 * h + u;
+                                        if (ok8 && args.dbg_i) args.dbg_i[o] = dbg_lo;
+                                        if (ok8 && args.dbg_f) args.dbg_f[o] = adv[2 * h + u];
+                                    }
+                                    continue;
+                                }
                                 if constexpr (DBG) {
                                     const long long o = static_cast<long long>(m) * args.N + n + 2 * h + u;
                                     if (MX && ok8 && args.dbg_f) args.dbg_f[o] = acc;
@@ -625,13 +708,13 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                             out[h] = *reinterpret_cast<const uint32_t *>(&b2);
                         }
                         if (y_tma) sqd::sts128(box + 32 * lane + 16 * g, out[0], out[1], out[2], out[3]);
-                        else if (n < args.N) *reinterpret_cast<uint4 *>(yrow + n) = make_uint4(out[0], out[1], out[2], out[3]);
+                        else if (n < args.N) sqd::stg128_hint(yrow + n, make_uint4(out[0], out[1], out[2], out[3]), y_policy);
                     }
                     if (y_tma) {
                         sqd::fence_proxy_async_smem();
                         __syncwarp();
                         if (lane == 0) {
-                            sqd::tma_store_2d(&tm_y, box, n0, m0);
+                            sqd::tma_store_2d_hint(&tm_y, box, n0, m0, y_policy);
                             sqd::bulk_commit();
                         }
                         last_box = bb;
@@ -639,11 +722,11 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                 }
                 if (has_acc && ch + 1 < NCH) {
                     sqd::tmem_wait_ld_dep1(vf[b ^ 1]);
-                    if (MX && ch + 2 == NCH) {
-                        // Last load of this warp landed: the accumulator may be reused.
+                    if ((MX || dbuf) && ch + 2 == NCH) {
+                        // Last load of this warp landed: the accumulator (buffer) may be reused.
                         sqd::tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) sqd::mbar_arrive_cluster(empty_leader);
+                        if (lane == 0) sqd::mbar_arrive_cluster(rb ? conv_leader : empty_leader);
                     }
                 }
             }
