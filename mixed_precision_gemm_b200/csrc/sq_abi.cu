@@ -277,9 +277,15 @@ sq_status launch_rowquant_stream(const DevInfo &di, const uint16_t *src, int64_t
                                  uint16_t *dout, cudaStream_t stream)
 {
     constexpr int kSmemLimit = 232448 - 1024;
-    int ngrp = sqq::stream_max_groups(G);
-    while (ngrp > 1 && sqq::StreamLayout(K, kn_pad, no_pad, ngrp, FP8).bytes > kSmemLimit) --ngrp;
-    const size_t smem = static_cast<size_t>(sqq::StreamLayout(K, kn_pad, no_pad, ngrp, FP8).bytes);
+    // Three row slots per group (two rows in flight while one is read) when that
+    // still leaves at least three groups; otherwise two.
+    int ngrp = 0, spg = 3;
+    for (; spg >= 2; --spg) {
+        ngrp = sqq::stream_max_groups(G);
+        while (ngrp > 1 && sqq::StreamLayout(K, kn_pad, no_pad, ngrp, spg, FP8).bytes > kSmemLimit) --ngrp;
+        if (ngrp >= 3 || spg == 2) break;
+    }
+    const size_t smem = static_cast<size_t>(sqq::StreamLayout(K, kn_pad, no_pad, ngrp, spg, FP8).bytes);
     if (smem > static_cast<size_t>(kSmemLimit))
         return fail(SQ_ERR_UNSUPPORTED, "quantize-gather: K=%d, nO=%d do not fit in shared memory", K, nO);
     auto kern = sqq::rowquant_stream_kernel<G, FP8>;
@@ -289,7 +295,7 @@ sq_status launch_rowquant_stream(const DevInfo &di, const uint16_t *src, int64_t
     if (st != SQ_OK) return st;
     const int64_t grid = std::min<int64_t>(rows, static_cast<int64_t>(per_sm) * di.sms);
     cudaError_t e = launch_k(kern, dim3(static_cast<unsigned>(grid)), dim3(threads), smem, stream, 0u, src, rows, K, ld,
-                             tab, nO, kn_pad, no_pad, dn, ds, dout, ngrp);
+                             tab, nO, kn_pad, no_pad, dn, ds, dout, ngrp, spg);
     if (e != cudaSuccess) return cuda_fail(e, "rowquant stream launch");
     return SQ_OK;
 }

@@ -6,17 +6,18 @@
 // thread of warp 0 copies whole rows (2K bytes, one bulk asynchronous copy
 // each) into a ring of shared-memory slots, completion counted on an
 // mbarrier per slot; NGRP groups of G consumer warps take the CTA's rows in
-// turn (row i of the CTA goes to group i % NGRP), two slots per group, so a
-// group's next row is in flight while it works on the current one.  The ring
-// holds 2 * NGRP rows, which keeps enough bytes in flight per SM to stream
-// HBM without spending registers on them.
+// turn (row i of the CTA goes to group i % NGRP), SPG slots per group, so a
+// group's next rows are in flight while it works on the current one.
 //
-// A group works on a row in two passes over the slot: (1) absolute maximum
-// over the normal channels (outlier halves cleared with the keep masks),
-// group-wide maximum (shuffles; a named barrier when G > 1), scale; (2) codes
-// of every chunk, packed and OR-ed into the group's packed row (as in
-// rowquant_kernel), and the compact outlier row gathered from the slot.  The
-// slot is then released and the packed row written out.
+// A group works on a row in this order: (0) the compact outlier row is
+// gathered from the slot and the outlier channels are set to zero there;
+// (1) each thread loads its chunks of the row into registers and takes their
+// absolute maximum (zeros cannot raise it, so no masking is needed), the
+// group-wide maximum follows (shuffles; a named barrier when G > 1) -- the
+// slot is handed back at this point, as the row now lives in registers;
+// (2) scale, then the codes of every chunk, the normal channels' codes packed
+// and OR-ed into the group's packed row (as in rowquant_kernel); the packed
+// row is then written out.
 //
 // Every wait is bounded; after a timeout the abort flag makes the remaining
 // waits return at once, and every group still walks through the same rows
@@ -33,22 +34,25 @@ constexpr int kStreamChunks = 8;  // most 8-channel chunks per thread and row: K
 enum : unsigned { SITE_RQ_PROD = 0x601, SITE_RQ_CONS = 0x602 };
 
 // Shared-memory layout, computed identically on the host and the device.
+// The table is the packing half of QuantTables (pack[256][4]).
 struct StreamLayout {
     int row_bytes;   // 2K, rounded up to 128
     int pk_alloc;    // code bytes per row (kn_pad / 2 INT4, kn_pad E4M3) + 16
+    int nslot;       // ring slots (spg per group)
     int off_pl, off_olist, off_pbuf, off_bar, off_misc, off_ring, bytes;
 
-    __host__ __device__ StreamLayout(int K, int kn_pad, int no_pad, int ngrp, bool fp8)
+    __host__ __device__ StreamLayout(int K, int kn_pad, int no_pad, int ngrp, int spg, bool fp8)
     {
         row_bytes = (2 * K + 127) & ~127;
         pk_alloc = (fp8 ? kn_pad : kn_pad / 2) + 16;
-        off_pl = static_cast<int>(sizeof(QuantTables));
+        nslot = spg * ngrp;
+        off_pl = static_cast<int>(sizeof(QuantTables::pack));
         off_olist = off_pl + ((4 * (K / 8) + 15) & ~15);
         off_pbuf = off_olist + ((2 * no_pad + 15) & ~15);
         off_bar = off_pbuf + ngrp * ((pk_alloc + 15) & ~15);
-        off_misc = off_bar + 2 * (2 * ngrp) * 8;
+        off_misc = off_bar + 2 * nslot * 8;
         off_ring = (off_misc + 16 + 8 * ngrp * 4 + 127) & ~127;   // + per-group reduction words
-        bytes = off_ring + 2 * ngrp * row_bytes;
+        bytes = off_ring + nslot * row_bytes;
     }
 };
 
@@ -57,10 +61,10 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Most consumer groups per CTA for G warps per row (shared memory holds
-// two row slots per group; more warps per row raise the warps per SM
-// without more shared memory).
-__host__ __device__ constexpr int stream_max_groups(int G) { return G <= 2 ? 10 : G == 4 ? 7 : 3; }
+// Most consumer groups per CTA for G warps per row (more warps per row
+// raise the warps per SM without more shared memory; every thread holds its
+// chunks of the row in registers).
+__host__ __device__ constexpr int stream_max_groups(int G) { return G <= 2 ? 8 : G == 4 ? 5 : 3; }
 
 // FP8: E4M3 codes (one byte per normal channel, scale absmax / 448) in place
 // of INT4 codes (OSC's FP8 fallback for the inputs of W2).
@@ -68,15 +72,15 @@ template <int G, bool FP8>
 __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowquant_stream_kernel(
     const uint16_t *__restrict__ src, int64_t rows, int K, int64_t ld,
     const uint32_t *__restrict__ chan_tab, int nO, int kn_pad, int no_pad,
-    uint8_t *__restrict__ dst_n, float *__restrict__ dst_s, uint16_t *__restrict__ dst_o, int ngrp)
+    uint8_t *__restrict__ dst_n, float *__restrict__ dst_s, uint16_t *__restrict__ dst_o, int ngrp, int spg)
 {
     extern __shared__ __align__(128) uint8_t rs_smem[];
-    const StreamLayout L(K, kn_pad, no_pad, ngrp, FP8);
-    QuantTables *tabs = reinterpret_cast<QuantTables *>(rs_smem);
+    const StreamLayout L(K, kn_pad, no_pad, ngrp, spg, FP8);
+    uint32_t (*pack_tab)[4] = reinterpret_cast<uint32_t (*)[4]>(rs_smem);
     uint32_t *pl_tab = reinterpret_cast<uint32_t *>(rs_smem + L.off_pl);
     uint16_t *olist = reinterpret_cast<uint16_t *>(rs_smem + L.off_olist);
     const uint32_t sbase = sqd::smem_u32(rs_smem);
-    const int nslot = 2 * ngrp;
+    const int nslot = L.nslot;
     auto full = [&](int s) { return sbase + L.off_bar + 8u * s; };
     auto empty = [&](int s) { return sbase + L.off_bar + 8u * (nslot + s); };
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(rs_smem + L.off_misc);
@@ -97,8 +101,8 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
         *abort_flag = 0u;
         sqd::fence_barrier_init();
     }
-    for (int i = tid; i < static_cast<int>(sizeof(QuantTables) / 16); i += nthr)
-        reinterpret_cast<uint4 *>(tabs)[i] = __ldg(reinterpret_cast<const uint4 *>(&g_qtab) + i);
+    for (int i = tid; i < static_cast<int>(sizeof(QuantTables::pack) / 16); i += nthr)
+        reinterpret_cast<uint4 *>(rs_smem)[i] = __ldg(reinterpret_cast<const uint4 *>(&g_qtab.pack[0][0]) + i);
     for (int i = tid; i < ngrp * ((L.pk_alloc + 15) / 16); i += nthr)
         reinterpret_cast<uint4 *>(rs_smem + L.off_pbuf)[i] = make_uint4(0, 0, 0, 0);
     for (int j = nO + tid; j < no_pad; j += nthr) olist[j] = kNoChannel;
@@ -147,6 +151,10 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
     const int gt = tid - 32 - gi * 32 * G;  // thread index inside the group
     const int GT = 32 * G;
     const int bar_id = 1 + gi;
+    auto group_sync = [&] {
+        if constexpr (G > 1) named_bar_sync(bar_id, GT);
+        else __syncwarp();
+    };
     uint32_t *pbuf = reinterpret_cast<uint32_t *>(rs_smem + L.off_pbuf + gi * L.pk_alloc);
     const uint32_t *ol2 = reinterpret_cast<const uint32_t *>(olist);
     const int pk_bytes = FP8 ? kn_pad : (kn_pad >> 1);
@@ -158,6 +166,8 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
         r.up2 = f2_pack(__float_as_uint(kUpScale), __float_as_uint(kUpScale));
         return r;
     }();
+    // Packing of a chunk without outliers: codes 0, 2, 4, 6 / 1, 3, 5, 7, all 8 kept.
+    const uint4 pk_plain = make_uint4(pack_tab[0][0], pack_tab[0][1], pack_tab[0][2], pack_tab[0][3]);
 
     for (int64_t i = gi;; i += ngrp) {
         const int64_t r = blockIdx.x + i * gridDim.x;
@@ -166,18 +176,39 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
         // A timed-out wait only raises the abort flag: the group goes on with
         // whatever the slot holds, so that every barrier below is still met.
         sqd::mbar_wait(full(s), static_cast<uint32_t>((i / nslot) & 1), abort_flag, SITE_RQ_CONS);
+        uint16_t *xrow = reinterpret_cast<uint16_t *>(rs_smem + L.off_ring + s * L.row_bytes);
 
-        // 1. absolute maximum over the normal channels
+        // 0. compact outlier row X_O[r, j] = X[r, O[j]], then the outlier channels set to zero
+        if (nO > 0) {
+            uint32_t *out_o = reinterpret_cast<uint32_t *>(dst_o + r * static_cast<int64_t>(no_pad));
+#pragma unroll 4
+            for (int jp = gt; jp < (no_pad >> 1); jp += GT) {
+                const uint32_t e2 = ol2[jp];
+                const uint32_t e0 = e2 & 0xFFFFu, e1 = e2 >> 16;
+                const uint32_t x0 = e0 != kNoChannel ? xrow[e0] : 0u;
+                const uint32_t x1 = e1 != kNoChannel ? xrow[e1] : 0u;
+                out_o[jp] = x0 | (x1 << 16);
+                if (e0 != kNoChannel) xrow[e0] = 0;
+                if (e1 != kNoChannel) xrow[e1] = 0;
+            }
+            group_sync();   // the zeros are in place for every warp of the group
+        }
+
+        // 1. the row's chunks into registers; absolute maximum (outliers are zero now)
+        uint4 v[kStreamChunks];
         uint32_t am = 0u;
 #pragma unroll
         for (int k = 0; k < kStreamChunks; ++k) {
             const int c = gt + k * GT;
-            if (c >= nchunk) break;
-            const uint4 v = *reinterpret_cast<const uint4 *>(rs_smem + L.off_ring + s * L.row_bytes + 16 * c);
-            const uint4 kp = *reinterpret_cast<const uint4 *>(tabs->keep[chunk_mask(pl_tab[c])]);
-            am = maxabs_bf16x2(am, maxabs_bf16x2(maxabs_bf16x2(v.x & kp.x, v.y & kp.y),
-                                                 maxabs_bf16x2(v.z & kp.z, v.w & kp.w)));
+            v[k] = c < nchunk ? *reinterpret_cast<const uint4 *>(rs_smem + L.off_ring + s * L.row_bytes + 16 * c)
+                              : make_uint4(0u, 0u, 0u, 0u);
+            am = maxabs_bf16x2(am, maxabs_bf16x2(maxabs_bf16x2(v[k].x, v[k].y), maxabs_bf16x2(v[k].z, v[k].w)));
         }
+        // The slot has been read by this warp: hand it back (after the zeros it
+        // wrote, which the next bulk copy into the slot must not overtake).
+        if (nO > 0) sqd::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) sqd::mbar_arrive(empty(s));
         uint32_t amax = max(am & 0x7FFFu, (am >> 16) & 0x7FFFu);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) amax = max(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, off));
@@ -205,13 +236,13 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
         for (int k = 0; k < kStreamChunks; ++k) {
             const int c = gt + k * GT;
             if (c >= nchunk) break;
-            const uint4 v = *reinterpret_cast<const uint4 *>(rs_smem + L.off_ring + s * L.row_bytes + 16 * c);
             const uint32_t pl = pl_tab[c];
             uint32_t lo, hi;
-            const uint4 pk = *reinterpret_cast<const uint4 *>(tabs->pack[chunk_mask(pl)]);
+            uint4 pk = pk_plain;
+            if (chunk_mask(pl)) pk = *reinterpret_cast<const uint4 *>(pack_tab[chunk_mask(pl)]);
             if constexpr (!FP8) {
-                if (!up) quant8_pairs<false>(v, rs, lo, hi);
-                else quant8_pairs<true>(v, rs, lo, hi);
+                if (!up) quant8_pairs<false>(v[k], rs, lo, hi);
+                else quant8_pairs<true>(v[k], rs, lo, hi);
                 const uint32_t ev = __byte_perm(lo, hi, pk.x);  // normal codes 0, 2, 4, 6
                 const uint32_t od = __byte_perm(lo, hi, pk.y);  // normal codes 1, 3, 5, 7
                 const uint32_t V = ((ev & 0x0F0F0F0Fu) | ((od << 4) & 0xF0F0F0F0u)) & pk.z;
@@ -223,9 +254,9 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
                 if (zero) {
                     lo = hi = 0u;  // a zero row has all-zero codes
                 } else if (!up) {
-                    quant8_fp8_pairs<false>(v, rs, lo, hi);
+                    quant8_fp8_pairs<false>(v[k], rs, lo, hi);
                 } else {
-                    quant8_fp8_pairs<true>(v, rs, lo, hi);
+                    quant8_fp8_pairs<true>(v[k], rs, lo, hi);
                 }
                 // normal codes in channel order: A = codes 0..3, B = 4..7, the
                 // bytes past the n normal channels cleared
@@ -242,33 +273,17 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
                 if (sh) atomicOr(dst + 2, __funnelshift_l(B, 0u, sh));
             }
         }
+        group_sync();   // the packed row is complete
 
-        // 4. compact outlier row X_O[r, j] = X[r, O[j]], read from the slot
-        if (nO > 0) {
-            const uint16_t *xrow = reinterpret_cast<const uint16_t *>(rs_smem + L.off_ring + s * L.row_bytes);
-            uint32_t *out_o = reinterpret_cast<uint32_t *>(dst_o + r * static_cast<int64_t>(no_pad));
-#pragma unroll 4
-            for (int jp = gt; jp < (no_pad >> 1); jp += GT) {
-                const uint32_t e2 = ol2[jp];
-                const uint32_t e0 = e2 & 0xFFFFu, e1 = e2 >> 16;
-                const uint32_t x0 = e0 != kNoChannel ? xrow[e0] : 0u;
-                const uint32_t x1 = e1 != kNoChannel ? xrow[e1] : 0u;
-                out_o[jp] = x0 | (x1 << 16);
-            }
-        }
-        // The slot has been read by this warp: hand it back.
-        __syncwarp();
-        if (lane == 0) sqd::mbar_arrive(empty(s));
-        if constexpr (G > 1) named_bar_sync(bar_id, GT);
-        else __syncwarp();
-
-        // 5. packed row out, cleared for the group's next row
+        // 4. packed row out, cleared for the group's next row
         uint4 *pk16 = reinterpret_cast<uint4 *>(pbuf);
         uint4 *out_n = reinterpret_cast<uint4 *>(dst_n + r * static_cast<int64_t>(pk_bytes));
         for (int j = gt; j < (L.pk_alloc >> 4); j += GT) {
             if (j < (pk_bytes >> 4)) out_n[j] = pk16[j];
             pk16[j] = make_uint4(0, 0, 0, 0);
         }
+        // Cleared before the group's next row ORs into it: with G > 1 the next
+        // row's named barriers order it; a single warp only needs its own lanes.
         if constexpr (G == 1) __syncwarp();
     }
 }
