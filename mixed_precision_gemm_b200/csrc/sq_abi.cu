@@ -277,14 +277,12 @@ sq_status launch_rowquant_stream(const DevInfo &di, const uint16_t *src, int64_t
                                  uint16_t *dout, cudaStream_t stream)
 {
     constexpr int kSmemLimit = 232448 - 1024;
-    // Three row slots per group (two rows in flight while one is read) when that
-    // still leaves at least three groups; otherwise two.
-    int ngrp = 0, spg = 3;
-    for (; spg >= 2; --spg) {
-        ngrp = sqq::stream_max_groups(G);
-        while (ngrp > 1 && sqq::StreamLayout(K, kn_pad, no_pad, ngrp, spg, FP8).bytes > kSmemLimit) --ngrp;
-        if (ngrp >= 3 || spg == 2) break;
-    }
+    // Two row slots per group (the next row in flight while one is read) and as
+    // many groups as fit: more groups measured faster than deeper slots, the
+    // kernel being bound by instruction issue rather than by memory latency.
+    const int spg = 2;
+    int ngrp = sqq::stream_max_groups(G);
+    while (ngrp > 1 && sqq::StreamLayout(K, kn_pad, no_pad, ngrp, spg, FP8).bytes > kSmemLimit) --ngrp;
     const size_t smem = static_cast<size_t>(sqq::StreamLayout(K, kn_pad, no_pad, ngrp, spg, FP8).bytes);
     if (smem > static_cast<size_t>(kSmemLimit))
         return fail(SQ_ERR_UNSUPPORTED, "quantize-gather: K=%d, nO=%d do not fit in shared memory", K, nO);

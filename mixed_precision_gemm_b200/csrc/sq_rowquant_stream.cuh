@@ -64,7 +64,7 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads)
 // Most consumer groups per CTA for G warps per row (more warps per row
 // raise the warps per SM without more shared memory; every thread holds its
 // chunks of the row in registers).
-__host__ __device__ constexpr int stream_max_groups(int G) { return G <= 2 ? 8 : G == 4 ? 5 : 3; }
+__host__ __device__ constexpr int stream_max_groups(int G) { return G <= 2 ? 8 : G == 4 ? 6 : 3; }
 
 // FP8: E4M3 codes (one byte per normal channel, scale absmax / 448) in place
 // of INT4 codes (OSC's FP8 fallback for the inputs of W2).
