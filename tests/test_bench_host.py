@@ -39,3 +39,15 @@ def test_algorithmic_bytes():
     assert g == N * KN // 2 + 2 * N * nO + 4 * N + M * KN // 2 + 2 * M * nO + 4 * M + 2 * M * N
     # E4M3 codes are one byte each, MX codes half a byte plus one scale byte per 32
     assert bench.gemm_bytes(M, N, K, nO, cb=1.0) - g == (N + M) * KN // 2
+
+
+def test_both_arms_describe_the_same_config():
+    """The GPU arm and the reference arm print the same `config` dict for a run."""
+    import argparse
+    import workloads
+    args = argparse.Namespace(low="int4", bank=16, high=1)
+    w = workloads.LLAMA70B_GATEUP
+    c = bench.run_config(w, args, 1)
+    assert c["workload"] == w.name and c["M"] == 8192 and c["N"] == 57344 and c["nO"] == 512
+    assert c["parallelism"] == "single" and bench.run_config(w, args, 2)["parallelism"] == "dp2"
+    assert bench.DEFAULT_WORKLOAD == w.name
