@@ -867,7 +867,7 @@ sq_status linear_mx_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const
 // ---------------------------------------------------------------- element-level SQ-format
 using CfgHigh32 = sqf::CfgHigh<32, 6>;
 using CfgHigh128 = sqf::CfgHigh<128, 4>;
-using CfgHighPair = sqf::CfgHighPair<4>;
+using CfgHighPair = sqf::CfgHighPair<4, 8>;
 
 bool sqf_bank_ok(int bank, int h) { return (bank == 4 || bank == 8 || bank == 16) && (h == 1 || h == 2); }
 
@@ -977,15 +977,19 @@ sq_status gemm_sqf_impl(const void *X_N, const float *s_x4, const void *X_8, con
     ha.M = static_cast<int>(M);
     ha.N = static_cast<int>(N);
     ha.K = static_cast<int>(K);
+    // bands of M-tiles whose E4M3 token rows (K bytes each) stay in L2 while the W tiles stream
+    ha.group_m = raster_group(static_cast<int>((M + 255) / 256), 256, 2 * K, 0);
     cudaError_t e;
     if (pair) {
+        // persistent: one cluster per SM pair, tiles handed out in the band order
         auto kern = sqf::sqf_high_pair_kernel<CfgHighPair>;
-        const int64_t pairs = ((N + 255) / 256) * ((M + 255) / 256);
+        const int64_t tiles = ((N + 255) / 256) * ((M + 255) / 256);
+        const int64_t clusters = std::min<int64_t>(tiles, di.sms / 2);
         int per_sm = 0;
-        SQ_TRY(kernel_setup(reinterpret_cast<const void *>(kern), sqf::kHiThreads, CfgHighPair::SMEM_BYTES, per_sm,
-                            "SQ-format high part set-up"));
-        e = launch_k(kern, dim3(static_cast<unsigned>(2 * pairs)), dim3(sqf::kHiThreads), CfgHighPair::SMEM_BYTES, s,
-                     0u, m_wh, m_we, m_x8, ha);
+        SQ_TRY(kernel_setup(reinterpret_cast<const void *>(kern), CfgHighPair::THREADS, CfgHighPair::SMEM_BYTES,
+                            per_sm, "SQ-format high part set-up"));
+        e = launch_k(kern, dim3(static_cast<unsigned>(2 * clusters)), dim3(CfgHighPair::THREADS),
+                     CfgHighPair::SMEM_BYTES, s, 0u, m_wh, m_we, m_x8, ha);
     } else {
         const dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((M + mt - 1) / mt));
         auto kern = small ? sqf::sqf_high_kernel<CfgHigh32> : sqf::sqf_high_kernel<CfgHigh128>;

@@ -194,7 +194,11 @@ struct CfgHigh {
     static constexpr int STAGE = A_BYTES + 2 * B_BYTES + 2 * E_BYTES;
     static constexpr int OFF_BAR = NST * STAGE;
     static constexpr int SMEM_BYTES = OFF_BAR + (2 * NST + 2) * 8 + 16 + 1024;
-    static constexpr int TMEM_COLS = MT + 8 <= 32 ? 32 : MT + 8 <= 64 ? 64 : MT + 8 <= 128 ? 128 : 256;
+    // MT accumulator columns, then 8 metadata columns per stage (a stage's copy never waits
+    // for the MMAs of the one before it)
+    static constexpr int TMEM_USED = MT + 8 * NST;
+    static constexpr int TMEM_COLS = TMEM_USED <= 32 ? 32 : TMEM_USED <= 64 ? 64 : TMEM_USED <= 128 ? 128 : 256;
+    static_assert(TMEM_USED <= 256, "tensor memory columns");
     static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -204,6 +208,7 @@ struct HighArgs {
     const float *s_hi;
     float *P;
     int M, N, K;
+    int group_m;   // pair kernel: tiles are handed out M-fastest in bands of group_m M-tiles
 };
 
 template <class C>
@@ -279,12 +284,12 @@ sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant
             // kind::f8f6f4, E4M3 x E4M3, fp32 D, sparse A (bit 2), M = 128, N = MT
             constexpr uint32_t idesc = (1u << 2) | (1u << 4) | (static_cast<uint32_t>(MT >> 3) << 17) |
                                        (static_cast<uint32_t>(128 >> 4) << 24);
-            const uint32_t ecol = tmem + MT;
             bool ok = true;
             for (int t = 0; t < nst_k && ok; ++t) {
                 const int s = t % NST;
                 if (!sqd::mbar_wait(full(s), (t / NST) & 1, abort_flag, SITE_HI_MMA)) { ok = false; break; }
                 sqd::tc_fence_after();
+                const uint32_t ecol = tmem + MT + 8 * s;
                 const uint32_t st = stage(s);
                 const uint32_t e0 = st + C::A_BYTES + 2 * C::B_BYTES;
                 asm volatile("tcgen05.cp.cta_group::1.128x128b [%0], %1;" ::"r"(ecol), "l"(sqd::make_sf_desc(e0))
@@ -351,22 +356,37 @@ sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant
 // 52 KB as the single-CTA kernel for twice the products, which halves the L2
 // traffic per product.  The metadata copy of a pair moves each CTA's own
 // shared memory into its own tensor memory.
-template <int NST_>
+//
+// Persistent: one cluster per SM pair takes tiles t = pair, pair + pairs, ...
+// (M-fastest in bands of group_m M-tiles, so the token band stays in L2 while
+// the W tiles stream).  The staging ring runs on across tiles, so the next
+// tile's operands load while the current one's epilogue writes P; the MMAs of
+// the next tile wait for the epilogue to have read the accumulator.
+template <int NST_, int EPI_WARPS_>
 struct CfgHighPair {
     static constexpr int NST = NST_;
+    // epilogue warps: 4 (one per TMEM lane quarter, all 256 columns, streamed through two
+    // 16-column buffers) or 8 (two per quarter, 128 columns each, held in registers so the
+    // accumulator goes back to the next tile's MMAs before P is stored)
+    static constexpr int EPI_WARPS = EPI_WARPS_;
+    static constexpr int THREADS = 32 * (2 + EPI_WARPS);
+    static_assert(EPI_WARPS == 4 || EPI_WARPS == 8, "epilogue warps");
     static constexpr int A_BYTES = 128 * 128;   // this CTA's 128 W rows, 256 channels (2:4)
     static constexpr int B_BYTES = 128 * 128;   // this CTA's 128 tokens, one 128-channel box
     static constexpr int E_BYTES = 128 * 16;    // metadata of this CTA's W rows, 128 channels
     static constexpr int STAGE = A_BYTES + 2 * B_BYTES + 2 * E_BYTES;
     static constexpr int OFF_BAR = NST * STAGE;
-    static constexpr int SMEM_BYTES = OFF_BAR + (2 * NST + 2) * 8 + 16 + 1024;
-    static constexpr int TMEM_COLS = 512;       // 256 accumulator columns + 8 metadata columns
+    // barriers: full[NST] empty[NST] acc_full acc_empty drain; then the TMEM slot and the abort flag
+    static constexpr int NBAR = 2 * NST + 3;
+    static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 + 1024;
+    static constexpr int TMEM_COLS = 512;       // 256 accumulator columns + 8 metadata columns per stage
+    static_assert(256 + 8 * NST <= TMEM_COLS, "tensor memory columns");
     static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 template <class C>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kHiThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
 sqf_high_pair_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant__ CUtensorMap tm_we,
                      const __grid_constant__ CUtensorMap tm_x8, const HighArgs args)
 {
@@ -378,17 +398,30 @@ sqf_high_pair_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_con
     const uint32_t rank = sqd::cluster_ctarank();
     const bool leader = rank == 0;
     const int tiles_n = (args.N + 255) / 256;
+    const int tiles_m = (args.M + 255) / 256;
+    const int num_tiles = tiles_n * tiles_m;
     const int pair = static_cast<int>(blockIdx.x >> 1);
-    const int n0 = (pair % tiles_n) * 256 + static_cast<int>(rank) * 128;   // this CTA's W rows
-    const int m0 = (pair / tiles_n) * 256;                                   // the pair's tokens
+    const int num_pairs = static_cast<int>(gridDim.x >> 1);
+    const int my_tiles = (num_tiles - pair + num_pairs - 1) / num_pairs;
+    // tile t -> (M-tile, N-tile): bands of group_m M-tiles, M-fastest inside a band
+    auto coords = [&](int t, int &mi, int &ni) {
+        const int gsz = args.group_m * tiles_n;
+        const int g = t / gsz;
+        const int first_m = g * args.group_m;
+        const int gm = min(tiles_m - first_m, args.group_m);
+        const int idx = t - g * gsz;
+        mi = first_m + idx % gm;
+        ni = idx / gm;
+    };
     sqd::pdl_launch_dependents();
 
     const uint32_t bar0 = sbase + C::OFF_BAR;
     auto full = [&](int s) { return bar0 + 8u * s; };
     auto empty = [&](int s) { return bar0 + 8u * (NST + s); };
     const uint32_t acc_full = bar0 + 8u * (2 * NST);
-    const uint32_t drain = acc_full + 8u;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + (2 * NST + 2) * 8);
+    const uint32_t acc_empty = acc_full + 8u;
+    const uint32_t drain = acc_full + 16u;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + C::NBAR * 8);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(tmem_slot + 1);
     auto stage = [&](int s) { return sbase + s * C::STAGE; };
     const int nst_k = args.K / 256;
@@ -399,6 +432,7 @@ sqf_high_pair_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_con
             sqd::mbar_init(empty(s), 1);   // multicast commit
         }
         sqd::mbar_init(acc_full, 1);       // multicast commit
+        sqd::mbar_init(acc_empty, 2 * C::EPI_WARPS);   // the epilogue warps of both CTAs (the first CTA's copy)
         sqd::mbar_init(drain, 1);
         *abort_flag = 0u;
         sqd::fence_barrier_init();
@@ -423,19 +457,25 @@ sqf_high_pair_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_con
         if (lane == 0) {
             int last = -1;
             bool ok = true;
-            for (int t = 0; t < nst_k; ++t) {
-                const int s = t % NST;
-                if (!sqd::mbar_wait(empty(s), ((t / NST) & 1) ^ 1u, abort_flag, SITE_HI_STG)) { ok = false; break; }
-                const uint32_t st = stage(s);
-                const uint32_t fl = sqd::map_to_cta(full(s), 0);
-                const int mt = m0 + static_cast<int>(rank) * 128;
-                sqd::mbar_arrive_expect_tx_cluster(fl, C::STAGE);
-                sqd::tma_load_2d_pair(st, &tm_wh, fl, t * 128, n0);
-                sqd::tma_load_2d_pair(st + C::A_BYTES, &tm_x8, fl, t * 256, mt);
-                sqd::tma_load_2d_pair(st + C::A_BYTES + C::B_BYTES, &tm_x8, fl, t * 256 + 128, mt);
-                sqd::tma_load_2d_pair(st + C::A_BYTES + 2 * C::B_BYTES, &tm_we, fl, t * 32, n0);
-                sqd::tma_load_2d_pair(st + C::A_BYTES + 2 * C::B_BYTES + C::E_BYTES, &tm_we, fl, t * 32 + 16, n0);
-                last = t;
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                int mi, ni;
+                coords(pair + lt * num_pairs, mi, ni);
+                const int n0 = ni * 256 + static_cast<int>(rank) * 128;   // this CTA's W rows
+                const int mt = mi * 256 + static_cast<int>(rank) * 128;   // this CTA's tokens
+                for (int t = 0; t < nst_k; ++t) {
+                    const int u = lt * nst_k + t;
+                    const int s = u % NST;
+                    if (!sqd::mbar_wait(empty(s), ((u / NST) & 1) ^ 1u, abort_flag, SITE_HI_STG)) { ok = false; break; }
+                    const uint32_t st = stage(s);
+                    const uint32_t fl = sqd::map_to_cta(full(s), 0);
+                    sqd::mbar_arrive_expect_tx_cluster(fl, C::STAGE);
+                    sqd::tma_load_2d_pair(st, &tm_wh, fl, t * 128, n0);
+                    sqd::tma_load_2d_pair(st + C::A_BYTES, &tm_x8, fl, t * 256, mt);
+                    sqd::tma_load_2d_pair(st + C::A_BYTES + C::B_BYTES, &tm_x8, fl, t * 256 + 128, mt);
+                    sqd::tma_load_2d_pair(st + C::A_BYTES + 2 * C::B_BYTES, &tm_we, fl, t * 32, n0);
+                    sqd::tma_load_2d_pair(st + C::A_BYTES + 2 * C::B_BYTES + C::E_BYTES, &tm_we, fl, t * 32 + 16, n0);
+                    last = u;
+                }
             }
             if (!ok && last >= 0 && leader) sqd::mbar_drain(full(last % NST), (last / NST) & 1);
         }
@@ -444,58 +484,104 @@ sqf_high_pair_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_con
             // kind::f8f6f4, E4M3 x E4M3, fp32 D, sparse A (bit 2), M = 256 (pair), N = 256
             constexpr uint32_t idesc = (1u << 2) | (1u << 4) | (static_cast<uint32_t>(256 >> 3) << 17) |
                                        (static_cast<uint32_t>(256 >> 4) << 24);
-            const uint32_t ecol = tmem + 256;
             bool ok = true;
-            for (int t = 0; t < nst_k && ok; ++t) {
-                const int s = t % NST;
-                if (!sqd::mbar_wait(full(s), (t / NST) & 1, abort_flag, SITE_HI_MMA)) { ok = false; break; }
+            for (int lt = 0; lt < my_tiles && ok; ++lt) {
+                // the accumulator of the previous tile has been read
+                if (!sqd::mbar_wait(acc_empty, (lt & 1) ^ 1u, abort_flag, SITE_HI_MMA)) { ok = false; break; }
                 sqd::tc_fence_after();
-                const uint32_t st = stage(s);
-                const uint32_t e0 = st + C::A_BYTES + 2 * C::B_BYTES;
-                asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(ecol), "l"(sqd::make_sf_desc(e0))
-                             : "memory");
-                asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(ecol + 4),
-                             "l"(sqd::make_sf_desc(e0 + C::E_BYTES))
-                             : "memory");
-                const uint64_t adesc = sqd::make_sw128_desc(st);
+                for (int t = 0; t < nst_k; ++t) {
+                    const int u = lt * nst_k + t;
+                    const int s = u % NST;
+                    if (!sqd::mbar_wait(full(s), (u / NST) & 1, abort_flag, SITE_HI_MMA)) { ok = false; break; }
+                    sqd::tc_fence_after();
+                    const uint32_t ecol = tmem + 256 + 8 * s;   // this stage's metadata columns
+                    const uint32_t st = stage(s);
+                    const uint32_t e0 = st + C::A_BYTES + 2 * C::B_BYTES;
+                    asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(ecol), "l"(sqd::make_sf_desc(e0))
+                                 : "memory");
+                    asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(ecol + 4),
+                                 "l"(sqd::make_sf_desc(e0 + C::E_BYTES))
+                                 : "memory");
+                    const uint64_t adesc = sqd::make_sw128_desc(st);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint64_t bdesc = sqd::make_sw128_desc(st + C::A_BYTES + (j >> 1) * C::B_BYTES) + 4 * (j & 1);
-                    asm volatile(
-                        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-                        "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %1, %2, [%5], %3, p;\n\t}\n" ::"r"(tmem),
-                        "l"(adesc + 2 * j), "l"(bdesc), "r"(idesc), "r"((t == 0 && j == 0) ? 0u : 1u),
-                        "r"(ecol + 2 * j)
-                        : "memory");
+                    for (int j = 0; j < 4; ++j) {
+                        const uint64_t bdesc = sqd::make_sw128_desc(st + C::A_BYTES + (j >> 1) * C::B_BYTES) + 4 * (j & 1);
+                        asm volatile(
+                            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                            "tcgen05.mma.sp.cta_group::2.kind::f8f6f4 [%0], %1, %2, [%5], %3, p;\n\t}\n" ::"r"(tmem),
+                            "l"(adesc + 2 * j), "l"(bdesc), "r"(idesc), "r"((t == 0 && j == 0) ? 0u : 1u),
+                            "r"(ecol + 2 * j)
+                            : "memory");
+                    }
+                    sqd::mma_commit_pair_multicast(empty(s), 0x3);
                 }
-                sqd::mma_commit_pair_multicast(empty(s), 0x3);
+                if (ok) sqd::mma_commit_pair_multicast(acc_full, 0x3);
             }
-            if (ok) {
-                sqd::mma_commit_pair_multicast(acc_full, 0x3);
-            } else {
+            if (!ok) {
                 sqd::mma_commit_pair(drain);
                 sqd::mbar_drain(drain, 0);
             }
         }
     } else {
-        // epilogue (each CTA): TMEM lane quarter warp % 4 = W rows n0 + 32 (warp % 4) + lane
+        // epilogue (each CTA): TMEM lane quarter warp % 4 = W rows n0 + 32 (warp % 4) + lane;
+        // with 8 warps the second four take the upper 128 columns
         const int q = warp & 3;
-        const int n = n0 + 32 * q + lane;
-        const bool n_ok = n < args.N;
-        const float sh = n_ok ? args.s_hi[n] : 0.0f;
-        if (sqd::mbar_wait(acc_full, 0, abort_flag, SITE_HI_EPI)) {
+        constexpr int NCOL = 256 / (C::EPI_WARPS / 4);
+        const int c_lo = ((warp - 2) >> 2) * NCOL;
+        const uint32_t empty_leader = sqd::map_to_cta(acc_empty, 0);
+        const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
+        for (int lt = 0; lt < my_tiles; ++lt) {
+            int mi, ni;
+            coords(pair + lt * num_pairs, mi, ni);
+            const int n = ni * 256 + static_cast<int>(rank) * 128 + 32 * q + lane;
+            const int m0 = mi * 256;
+            const bool n_ok = n < args.N;
+            const float sh = n_ok ? args.s_hi[n] : 0.0f;
+            if (!sqd::mbar_wait(acc_full, lt & 1, abort_flag, SITE_HI_EPI)) break;
             sqd::tc_fence_after();
-            const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
-            for (int c = 0; c < 256; c += 16) {
-                uint32_t v[16];
-                sqd::tmem_ld_32x32b_x16(tl + c, v);
-                sqd::tmem_wait_ld();
+            const int64_t row0 = static_cast<int64_t>(m0) * args.N + n;
+            auto put = [&](const uint32_t (&v)[16], int c) {
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int m = m0 + c + i;
                     if (n_ok && m < args.M)
-                        args.P[static_cast<int64_t>(m) * args.N + n] =
+                        args.P[row0 + static_cast<int64_t>(c + i) * args.N] =
                             __fmul_rn(__fmul_rn(__uint_as_float(v[i]), args.s_x8[m]), sh);
+                }
+            };
+            if constexpr (NCOL == 128) {
+                // all 128 columns into registers, hand the accumulator back, then store: the
+                // next tile's MMAs run while P is written
+                uint32_t v[8][16];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) sqd::tmem_ld_32x32b_x16(tl + c_lo + 16 * j, v[j]);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) sqd::tmem_wait_ld_dep1(v[j]);
+                sqd::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) sqd::mbar_arrive_cluster(empty_leader);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) put(v[j], c_lo + 16 * j);
+            } else {
+                // two 16-column buffers: the next chunk loads while this one is stored
+                uint32_t va[16], vb[16];
+                sqd::tmem_ld_32x32b_x16(tl + c_lo, va);
+                sqd::tmem_wait_ld_dep1(va);
+#pragma unroll 1
+                for (int c = c_lo; c < c_lo + NCOL; c += 32) {
+                    sqd::tmem_ld_32x32b_x16(tl + c + 16, vb);
+                    put(va, c);
+                    sqd::tmem_wait_ld_dep1(vb);
+                    if (c + 32 < c_lo + NCOL) {
+                        sqd::tmem_ld_32x32b_x16(tl + c + 32, va);
+                    } else {
+                        // every accumulator column this warp reads has been read
+                        sqd::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) sqd::mbar_arrive_cluster(empty_leader);
+                    }
+                    put(vb, c + 16);
+                    if (c + 32 < c_lo + NCOL) sqd::tmem_wait_ld_dep1(va);
                 }
             }
         }
