@@ -59,7 +59,7 @@ constexpr int KB_MX = 256;        // E2M1 K elements per block (128 packed bytes
 constexpr int MX_SF_BYTES = 3072; // scale bytes per ring slot: 2 tiles of X rows, 4 of W rows
 constexpr int MX_SFA_COL = 256;   // TMEM columns of the X-row scales (2 K-tiles x 4)
 constexpr int MX_SFB_COL = 264;   // TMEM columns of the W-row scales (2 K-tiles x 8)
-constexpr int MX_SF_BUF = 24;     // second scale buffer of the pair kernel: columns 280..303
+constexpr int MX_SF_SLOT = 24;    // pair kernel: ring slot e keeps its scales at the columns above + 24 e
 
 // Site codes stored in the device error word by a bounded wait that ran out.
 enum : unsigned {

@@ -35,9 +35,15 @@
 //
 // MX low path (kLowMx): the packed E2M1 tiles travel by TMA straight into
 // the operand ring, together with their E8M0 scales (tiles of 128 rows x 4
-// blocks, see sq_mxquant.cuh); the MMA thread copies the scales into tensor
-// memory (tcgen05.cp, columns MX_SFA_COL / MX_SFB_COL) just before the
-// K-block's four kind::mxf4 MMAs.  The block-scaled products and the 16-bit
+// blocks, see sq_mxquant.cuh).  The scales land on a barrier of their own CTA
+// (sf_full); the four warps of the producer group that owns the ring slot,
+// one per TMEM lane quarter, write them into the slot's scale columns
+// (MX_SFA_COL / MX_SFB_COL + MX_SF_SLOT * slot, tcgen05.st) and only then
+// arrive on op_full, so the MMA thread issues nothing but the K-block's four
+// kind::mxf4 MMAs and the scale writes of later slots run beside them.  (A
+// tcgen05.cp per scale tile from the MMA thread, six per K-block, shared the
+// in-order MMA pipe and cost about a quarter of the MMA time.)  The
+// block-scaled products and the 16-bit
 // branch accumulate into the one fp32 accumulator in columns [0, 256), and
 // the epilogue only rounds it to bf16.
 #pragma once
@@ -72,8 +78,8 @@ struct CfgPair {
     static constexpr int OFF_STG = OFF_SF + OPS * SF_BYTES;
     static constexpr int OFF_BAR = OFF_STG + STG * STG_BYTES;
     // barriers: op_full[OPS] op_empty[OPS] stg_full[STG] stg_empty[STG] acc_full acc_empty drain
-    // low_full conv_done
-    static constexpr int NBAR = 2 * OPS + 2 * STG + 5;
+    // low_full conv_done sf_full[OPS] (MX scales)
+    static constexpr int NBAR = 2 * OPS + 2 * STG + 5 + (SF_ > 0 ? OPS : 0);
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int OFF_SW = (OFF_MISC + 16 + 15) / 16 * 16;   // per epilogue warp: its 128 s_w values
     // Per epilogue warp: YB boxes of 32 x 16 bf16, the source of bulk tensor
@@ -112,6 +118,8 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
     constexpr bool SQF = LOW == kLowSqf;
     constexpr bool EXPAND = LOW == kLowInt4 || SQF;
     constexpr int OPS = C::OPS, EC = C::EXP_CHUNKS;
+    static_assert(!MX || (C::GW == 4 && MX_SFA_COL + MX_SF_SLOT * OPS <= C::TMEM_COLS),
+                  "MX: one producer warp per TMEM lane quarter, every slot's scale columns inside TMEM");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = sqd::smem_u32(smem);
@@ -133,6 +141,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
     const uint32_t drain = acc_full + 16u;
     const uint32_t low_full = acc_full + 24u;   // (not MX) a tile's low-path sums are complete
     const uint32_t conv_done = acc_full + 32u;  // (not MX) both CTAs' epilogue warps have folded them
+    auto sf_full = [&](int e) { return acc_full + 40u + 8u * e; };   // (MX) this CTA's scales of slot e landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_MISC);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC + 4);
     auto op_a = [&](int e) { return sbase + C::OFF_OP + e * C::OP_BYTES; };
@@ -140,8 +149,11 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
 
     if (threadIdx.x == 0) {
         for (int e = 0; e < OPS; ++e) {
-            sqd::mbar_init(op_full(e), 2 * C::GW);          // the owning group's warps in both CTAs (first CTA's copy)
+            // the owning group's warps in both CTAs (first CTA's copy); MX: plus the
+            // byte-count arrival of each CTA's TMA thread
+            sqd::mbar_init(op_full(e), 2 * (C::GW + (MX ? 1 : 0)));
             sqd::mbar_init(op_empty(e), 1);                 // multicast commit
+            if constexpr (MX) sqd::mbar_init(sf_full(e), 1);   // this CTA's TMA thread (expect-tx)
         }
         for (int i = 0; i < STG; ++i) {
             sqd::mbar_init(stg_full(i), 1);                 // this CTA's staging TMA (expect-tx)
@@ -308,20 +320,8 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                         const bool is_bf = i < nkb_o;
                         const uint64_t adesc = sqd::make_sw128_desc(op_a(e));
                         const uint64_t bdesc = sqd::make_sw128_desc(op_a(e) + C::A_BYTES);
-                        // Two TMEM scale buffers alternate by K-block, so the copies of one
-                        // block need not wait for the MMAs that read the previous one.
-                        const uint32_t sb = tmem + MX_SF_BUF * static_cast<uint32_t>((i - nkb_o) & 1);
-                        if (!is_bf) {
-                            // Scales of this K-block: X-row tiles (K-tiles 0, 1) at sf, sf + 512; W-row
-                            // tiles of rows 0-127 at sf + 1024 (+512 for K-tile 1), rows 128-255 at sf + 2048.
-                            const uint32_t sf = sbase + C::OFF_SF + e * C::SF_BYTES;
-                            sqd::sf_copy_pair(sb + MX_SFA_COL, sqd::make_sf_desc(sf));
-                            sqd::sf_copy_pair(sb + MX_SFA_COL + 4, sqd::make_sf_desc(sf + 512));
-                            sqd::sf_copy_pair(sb + MX_SFB_COL, sqd::make_sf_desc(sf + 1024));
-                            sqd::sf_copy_pair(sb + MX_SFB_COL + 4, sqd::make_sf_desc(sf + 2048));
-                            sqd::sf_copy_pair(sb + MX_SFB_COL + 8, sqd::make_sf_desc(sf + 1536));
-                            sqd::sf_copy_pair(sb + MX_SFB_COL + 12, sqd::make_sf_desc(sf + 2560));
-                        }
+                        // the producer group wrote this slot's scales before arriving on op_full
+                        const uint32_t sb = tmem + MX_SF_SLOT * static_cast<uint32_t>(e);
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const uint32_t acc = (i == 0 && k == 0) ? 0u : 1u;
@@ -414,6 +414,12 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                 sqd::tma_load_2d_pair(op_a(e), mx, full_leader, x, tmi * PAIR_BM + static_cast<int>(r0));
                 sqd::tma_load_2d_pair(op_a(e) + C::A_BYTES, mw, full_leader, x, tni * PAIR_BN + static_cast<int>(r0));
                 last_armed = u;
+                if constexpr (MX) {
+                    // no scales in this block: the first warp's own arrival, and the slot's
+                    // sf_full phase passes too, so its parity keeps counting the slot's uses
+                    sqd::mbar_arrive_cluster(full_leader);
+                    sqd::mbar_arrive(sf_full(e));
+                }
             } else if (lane == 0) {
                 sqd::mbar_arrive_cluster(full_leader);
             }
@@ -423,29 +429,52 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         // MX ring use u (tile lt, low K-block kb): the packed E2M1 tiles plus
         // the block scales of this CTA's 128 X rows (one box: K-tiles 2kb,
         // 2kb+1) and of all 256 W rows of the tile (two boxes, one per
-        // 128-row band).  Both CTAs of the pair need every W-row scale.
+        // 128-row band).  Both CTAs of the pair need every W-row scale.  The
+        // scales land on this CTA's sf_full; then each warp of the group writes
+        // them into its lane quarter of the slot's TMEM scale columns: a tile's
+        // byte 16 r + 4 c + j goes to byte j of column c of lane r in every
+        // quarter (the layout the block-scaled MMA reads).
+        int last_sf = -1;
         auto produce_mx = [&](int lt, int u, int kb) -> bool {
             if constexpr (MX) {
                 int tmi, tni;
                 tile_coords(args, pair + lt * num_pairs, tmi, tni);
                 const int e = u % OPS;
                 if (!sqd::mbar_wait(op_empty(e), ((u / OPS) & 1) ^ 1u, abort_flag, SITE_EXP_OP)) return false;
+                sqd::tc_fence_after();   // the MMAs that read slot e's scale columns are done
                 const uint32_t full_leader = sqd::map_to_cta(op_full(e), 0);
+                const uint32_t sf = sbase + C::OFF_SF + e * C::SF_BYTES;
                 if (tma_thread) {
                     const int na = 2 * nkb_i;  // scale tiles per 128-row band
-                    const uint32_t sf = sbase + C::OFF_SF + e * C::SF_BYTES;
-                    sqd::mbar_arrive_expect_tx_cluster(full_leader, C::OP_BYTES + C::SF_BYTES);
+                    sqd::mbar_arrive_expect_tx_cluster(full_leader, C::OP_BYTES);
                     sqd::tma_load_2d_pair(op_a(e), &tm_xn, full_leader, kb * (KB_MX / 2),
                                           tmi * PAIR_BM + static_cast<int>(r0));
                     sqd::tma_load_2d_pair(op_a(e) + C::A_BYTES, &tm_wn, full_leader, kb * (KB_MX / 2),
                                           tni * PAIR_BN + static_cast<int>(r0));
-                    sqd::tma_load_2d_pair(sf, &tm_sx, full_leader, 0, ((2 * tmi + static_cast<int>(rank)) * na + 2 * kb) * 4);
-                    sqd::tma_load_2d_pair(sf + 1024, &tm_sw, full_leader, 0, ((2 * tni) * na + 2 * kb) * 4);
-                    sqd::tma_load_2d_pair(sf + 2048, &tm_sw, full_leader, 0, ((2 * tni + 1) * na + 2 * kb) * 4);
+                    sqd::mbar_arrive_expect_tx(sf_full(e), C::SF_BYTES);
+                    sqd::tma_load_2d(sf, &tm_sx, sf_full(e), 0, ((2 * tmi + static_cast<int>(rank)) * na + 2 * kb) * 4);
+                    sqd::tma_load_2d(sf + 1024, &tm_sw, sf_full(e), 0, ((2 * tni) * na + 2 * kb) * 4);
+                    sqd::tma_load_2d(sf + 2048, &tm_sw, sf_full(e), 0, ((2 * tni + 1) * na + 2 * kb) * 4);
                     last_armed = u;
-                } else if (lane == 0) {
-                    sqd::mbar_arrive_cluster(full_leader);
+                    last_sf = u;
                 }
+                if (!sqd::mbar_wait(sf_full(e), (u / OPS) & 1, abort_flag, SITE_EXP_OP)) return false;
+                // columns +0..7: X rows, K-tiles 0 and 1; +8..23: W rows 0-127 and 128-255 of
+                // K-tile 0, then of K-tile 1
+                const uint4 x0 = sqd::lds128(sf + 16 * lane), x1 = sqd::lds128(sf + 512 + 16 * lane);
+                const uint4 w00 = sqd::lds128(sf + 1024 + 16 * lane), w10 = sqd::lds128(sf + 2048 + 16 * lane);
+                const uint4 w01 = sqd::lds128(sf + 1536 + 16 * lane), w11 = sqd::lds128(sf + 2560 + 16 * lane);
+                const uint32_t va[16] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w,
+                                         w00.x, w00.y, w00.z, w00.w, w10.x, w10.y, w10.z, w10.w};
+                const uint32_t vb[8] = {w01.x, w01.y, w01.z, w01.w, w11.x, w11.y, w11.z, w11.w};
+                const uint32_t tq = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) +
+                                    static_cast<uint32_t>(MX_SFA_COL + MX_SF_SLOT * e);
+                sqd::tmem_st_32x32b_x16(tq, va);
+                sqd::tmem_st_32x32b_x8(tq + 16, vb);
+                sqd::tmem_wait_st();
+                sqd::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) sqd::mbar_arrive_cluster(full_leader);
                 return true;
             } else {
                 return false;
@@ -475,6 +504,7 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
             // Let the last copies that were issued land before the CTA exits.
             sqd::mbar_drain(op_full(last_armed % OPS), (last_armed / OPS) & 1);
         }
+        if (MX && !ok && tma_thread && last_sf >= 0) sqd::mbar_drain(sf_full(last_sf % OPS), (last_sf / OPS) & 1);
     } else if (warp >= PAIR_EPI_WARP0 && warp < PAIR_EPI_WARP0 + PAIR_EPI_WARPS) {
         // ------------------------------------------------------------ epilogue (each CTA: its 128 rows)
         // Warp w serves TMEM lane quarter w % 4 and half (w - 2) / 4 of the 256
