@@ -627,6 +627,57 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
                 if (lane == 0) sqd::mbar_arrive_cluster(conv_leader);
             }
 
+            if constexpr (MX && !DBG) {
+                // MX: the warp's 128 columns are rounded to bf16 into registers as they are
+                // read, the accumulator goes back to the next tile's MMAs, and only then are
+                // the rows stored (the stores overlap the next tile's MMAs).
+                if (!sqd::mbar_wait(acc_full, lt & 1, abort_flag, SITE_EPI)) break;
+                sqd::tc_fence_after();
+                uint32_t pk[NCH][CW / 2];
+#pragma unroll
+                for (int ch = 0; ch < NCH; ++ch) {
+                    uint32_t v[CW];
+                    sqd::tmem_ld_32x32b_x16(tl + c_base + ch * CW, v);
+                    sqd::tmem_wait_ld_dep1(v);
+#pragma unroll
+                    for (int h = 0; h < CW / 2; ++h) {
+                        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * h]), __uint_as_float(v[2 * h + 1]));
+                        pk[ch][h] = *reinterpret_cast<const uint32_t *>(&b2);
+                    }
+                }
+                sqd::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) sqd::mbar_arrive_cluster(empty_leader);
+#pragma unroll
+                for (int ch = 0; ch < NCH; ++ch) {
+                    const int n0 = tni * PAIR_BN + c_base + ch * CW;
+                    if (!(y_tma ? (m0 < args.M && n0 < args.N) : (row_ok && n0 < args.N))) continue;
+                    if (y_tma) {
+                        // the one staging box of this warp: its previous bulk store has read it
+                        if (lane == 0) sqd::bulk_wait_read<0>();
+                        __syncwarp();
+                        const uint32_t box = yst;
+                        sqd::sts128(box + 32 * lane, pk[ch][0], pk[ch][1], pk[ch][2], pk[ch][3]);
+                        sqd::sts128(box + 32 * lane + 16, pk[ch][4], pk[ch][5], pk[ch][6], pk[ch][7]);
+                        sqd::fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            sqd::tma_store_2d_hint(&tm_y, box, n0, m0, y_policy);
+                            sqd::bulk_commit();
+                        }
+                    } else {
+#pragma unroll
+                        for (int g = 0; g < CW / 8; ++g) {
+                            const int n = n0 + 8 * g;
+                            if (n < args.N)
+                                sqd::stg128_hint(yrow + n, make_uint4(pk[ch][4 * g], pk[ch][4 * g + 1], pk[ch][4 * g + 2],
+                                                                      pk[ch][4 * g + 3]), y_policy);
+                        }
+                    }
+                }
+                continue;
+            }
+
             // -------------------------------------------------------- (2) store
             const int rb = dbuf ? (lt & 1) : 0;   // accumulator buffer of this tile (double-buffer mode)
             if (!sqd::mbar_wait(rb ? low_full : acc_full, static_cast<uint32_t>(dbuf ? ((lt >> 1) & 1) : (lt & 1)),
