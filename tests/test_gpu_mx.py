@@ -116,6 +116,9 @@ SHAPES = [
     (64, 8192, 256, 512),
     (1, 1024, 64, 8),
     (33, 2048, 1032, 0),
+    # 632 pair tiles on 74 clusters (several tiles per cluster: the accumulator handed back before
+    # Y is stored, the scale slots reused across tiles), ragged last M and N tiles
+    (1800, 1024, 20000, 64),
 ]
 
 

@@ -123,6 +123,18 @@ def test_sqf_qkv_sampled():
     check_sqf(X, W, 16, 1, rows=rows)
 
 
+def test_sqf_many_tiles_per_cluster():
+    """632 high-part pair tiles on 74 clusters (the persistent kernel walks several tiles per
+    cluster, its staging ring and accumulator hand-back running across them), ragged last M and
+    N tiles; sampled rows, including the last."""
+    M, K, N = 1800, 1024, 20000
+    X = workloads.activations(M, K, workloads.outlier_channels(K, 0), seed=91)
+    W = workloads.weights(N, K, seed=92)
+    rng = np.random.default_rng(9)
+    rows = np.unique(np.concatenate([rng.choice(M, 10, replace=False), [0, 255, 256, 1791, M - 1]]))
+    check_sqf(X, W, 16, 1, rows=rows)
+
+
 def test_sqf_linear_matches_calls():
     M, K, N = 257, 1024, 392
     X = workloads.activations(M, K, workloads.outlier_channels(K, 0), seed=81).to("cuda")
