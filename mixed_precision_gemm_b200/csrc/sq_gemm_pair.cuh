@@ -521,7 +521,8 @@ dual_gemm_pair_kernel(const __grid_constant__ CUtensorMap tm_xo, const __grid_co
         // With debug outputs the fold writes zeros instead, so the branch sum
         // stays separate, and the store adds y0 (from the exact sums just
         // written to dbg_i) the same way.
-        // MX: one pass over the single accumulator after the tile.
+        // MX: the single accumulator is rounded into registers after the tile and handed
+        // back before the stores (debug builds: one pass that also writes the fp32 sums).
         const int sub = warp & 3;
         const int half = (warp - PAIR_EPI_WARP0) >> 2;
         const uint32_t tl = tmem + (static_cast<uint32_t>(sub * 32) << 16);
