@@ -169,13 +169,18 @@ __global__ void __launch_bounds__(32 * (1 + stream_max_groups(G) * G), 1) rowqua
     // Packing of a chunk without outliers: codes 0, 2, 4, 6 / 1, 3, 5, 7, all 8 kept.
     const uint4 pk_plain = make_uint4(pack_tab[0][0], pack_tab[0][1], pack_tab[0][2], pack_tab[0][3]);
 
-    for (int64_t i = gi;; i += ngrp) {
-        const int64_t r = blockIdx.x + i * gridDim.x;
-        if (r >= rows) break;
-        const int s = static_cast<int>(i % nslot);
+    // Row i = gi + j ngrp of the CTA (the group's j-th row) sits in slot i % nslot =
+    // gi + ngrp (j % spg) with phase parity (i / nslot) & 1 = (j / spg) & 1; both are
+    // kept as counters (no 64-bit division per row).
+    int sj = 0;
+    uint32_t ph = 0u;
+    const int64_t rstep = static_cast<int64_t>(ngrp) * gridDim.x;
+    for (int64_t r = blockIdx.x + static_cast<int64_t>(gi) * gridDim.x; r < rows; r += rstep) {
+        const int s = gi + ngrp * sj;
         // A timed-out wait only raises the abort flag: the group goes on with
         // whatever the slot holds, so that every barrier below is still met.
-        sqd::mbar_wait(full(s), static_cast<uint32_t>((i / nslot) & 1), abort_flag, SITE_RQ_CONS);
+        sqd::mbar_wait(full(s), ph, abort_flag, SITE_RQ_CONS);
+        if (++sj == spg) { sj = 0; ph ^= 1u; }
         uint16_t *xrow = reinterpret_cast<uint16_t *>(rs_smem + L.off_ring + s * L.row_bytes);
 
         // 0. compact outlier row X_O[r, j] = X[r, O[j]], then the outlier channels set to zero
