@@ -867,6 +867,8 @@ sq_status linear_mx_impl(const void *X, int64_t M, int64_t K, int64_t ldx, const
 // ---------------------------------------------------------------- element-level SQ-format
 using CfgHigh32 = sqf::CfgHigh<32, 6>;
 using CfgHigh128 = sqf::CfgHigh<128, 4>;
+using CfgHigh32x2 = sqf::CfgHigh<32, 6, 2>;     // K stages split over a cluster of two CTAs
+using CfgHigh128x2 = sqf::CfgHigh<128, 4, 2>;
 using CfgHighPair = sqf::CfgHighPair<4, 8>;
 
 bool sqf_bank_ok(int bank, int h) { return (bank == 4 || bank == 8 || bank == 16) && (h == 1 || h == 2); }
@@ -991,13 +993,18 @@ sq_status gemm_sqf_impl(const void *X_N, const float *s_x4, const void *X_8, con
         e = launch_k(kern, dim3(static_cast<unsigned>(2 * clusters)), dim3(CfgHighPair::THREADS),
                      CfgHighPair::SMEM_BYTES, s, 0u, m_wh, m_we, m_x8, ha);
     } else {
-        const dim3 grid(static_cast<unsigned>((N + 127) / 128), static_cast<unsigned>((M + mt - 1) / mt));
-        auto kern = small ? sqf::sqf_high_kernel<CfgHigh32> : sqf::sqf_high_kernel<CfgHigh128>;
+        // One CTA per 128 W rows x mt tokens; when that fills at most half of the SMs and there
+        // are two or more K stages, a cluster of two CTAs splits each tile's K stages.
+        const int64_t tiles = ((N + 127) / 128) * ((M + mt - 1) / mt);
+        const bool split = K / 256 >= 2 && 2 * tiles <= di.sms;
+        const dim3 grid(static_cast<unsigned>((N + 127) / 128 * (split ? 2 : 1)), static_cast<unsigned>((M + mt - 1) / mt));
+        auto kern = split ? (small ? sqf::sqf_high_kernel<CfgHigh32x2> : sqf::sqf_high_kernel<CfgHigh128x2>)
+                          : (small ? sqf::sqf_high_kernel<CfgHigh32> : sqf::sqf_high_kernel<CfgHigh128>);
         const size_t smem = small ? CfgHigh32::SMEM_BYTES : CfgHigh128::SMEM_BYTES;
         int per_sm = 0;
         SQ_TRY(kernel_setup(reinterpret_cast<const void *>(kern), sqf::kHiThreads, smem, per_sm,
                             "SQ-format high part set-up"));
-        e = launch_k(kern, grid, dim3(sqf::kHiThreads), smem, s, 0u, m_wh, m_we, m_x8, ha);
+        e = launch_k(kern, grid, dim3(sqf::kHiThreads), smem, s, split ? 2u : 0u, m_wh, m_we, m_x8, ha);
     }
     if (e != cudaSuccess) return cuda_fail(e, "SQ-format high part launch");
     // 2. low part (INT4, mask code cleared) with P added before the bf16 rounding

@@ -184,10 +184,16 @@ constexpr int kHiWarps = 6;                 // 0 TMA, 1 MMA, 2..5 epilogue
 constexpr int kHiThreads = 32 * kHiWarps;
 enum : unsigned { SITE_HI_STG = 0x601, SITE_HI_MMA = 0x602, SITE_HI_EPI = 0x603 };
 
-template <int MT_, int NST_>
+// KS = 2: the K stages of a tile are split over a cluster of two CTAs; the
+// second adds its fp32 accumulator into the first's through distributed shared
+// memory (one fixed order, so P is deterministic).  Used when one CTA per tile
+// would leave more than half of the SMs idle.
+template <int MT_, int NST_, int KS_ = 1>
 struct CfgHigh {
     static constexpr int MT = MT_;
     static constexpr int NST = NST_;
+    static constexpr int KS = KS_;
+    static_assert(KS == 1 || KS == 2, "K split");
     static constexpr int A_BYTES = 128 * 128;
     static constexpr int B_BYTES = MT * 128;          // one 128-channel box of tokens
     static constexpr int E_BYTES = 128 * 16;          // one 128-channel metadata box
@@ -201,6 +207,7 @@ struct CfgHigh {
     static_assert(TMEM_USED <= 256, "tensor memory columns");
     static_assert(STAGE % 1024 == 0, "stages stay 1024-byte aligned");
     static_assert(SMEM_BYTES <= 232448, "shared memory");
+    static_assert(KS == 1 || MT * 128 * 4 <= NST * STAGE, "the partial accumulator fits in the staging ring");
 };
 
 struct HighArgs {
@@ -216,12 +223,14 @@ __global__ void __launch_bounds__(kHiThreads, 1)
 sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant__ CUtensorMap tm_we,
                 const __grid_constant__ CUtensorMap tm_x8, const HighArgs args)
 {
-    constexpr int MT = C::MT, NST = C::NST;
+    constexpr int MT = C::MT, NST = C::NST, KS = C::KS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = sqd::smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n0 = static_cast<int>(blockIdx.x) * 128;
+    // KS = 2: CTAs 2j and 2j + 1 (one cluster) take the first and second half of tile j's stages
+    const int kz = KS == 2 ? static_cast<int>(sqd::cluster_ctarank()) : 0;
+    const int n0 = static_cast<int>(KS == 2 ? (blockIdx.x >> 1) : blockIdx.x) * 128;
     const int m0 = static_cast<int>(blockIdx.y) * MT;
     sqd::pdl_launch_dependents();
 
@@ -233,7 +242,9 @@ sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::OFF_BAR + (2 * NST + 2) * 8);
     volatile uint32_t *abort_flag = reinterpret_cast<volatile uint32_t *>(tmem_slot + 1);
     auto stage = [&](int s) { return sbase + s * C::STAGE; };
-    const int nst_k = args.K / 256;   // stages
+    const int nst_all = args.K / 256;   // stages of the whole K range
+    const int t_first = kz * nst_all / KS;   // this CTA's stages: [t_first, t_first + nst_k), nst_k >= 1
+    const int nst_k = (kz + 1) * nst_all / KS - t_first;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
@@ -265,9 +276,10 @@ sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant
         if (lane == 0) {
             int last = -1;
             bool ok = true;
-            for (int t = 0; t < nst_k; ++t) {
-                const int s = t % NST;
-                if (!sqd::mbar_wait(empty(s), ((t / NST) & 1) ^ 1u, abort_flag, SITE_HI_STG)) { ok = false; break; }
+            for (int u = 0; u < nst_k; ++u) {
+                const int t = t_first + u;   // K stage
+                const int s = u % NST;
+                if (!sqd::mbar_wait(empty(s), ((u / NST) & 1) ^ 1u, abort_flag, SITE_HI_STG)) { ok = false; break; }
                 const uint32_t st = stage(s);
                 sqd::mbar_arrive_expect_tx(full(s), C::STAGE);
                 sqd::tma_load_2d(st, &tm_wh, full(s), t * 128, n0);
@@ -275,9 +287,14 @@ sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant
                 sqd::tma_load_2d(st + C::A_BYTES + C::B_BYTES, &tm_x8, full(s), t * 256 + 128, m0);
                 sqd::tma_load_2d(st + C::A_BYTES + 2 * C::B_BYTES, &tm_we, full(s), t * 32, n0);
                 sqd::tma_load_2d(st + C::A_BYTES + 2 * C::B_BYTES + C::E_BYTES, &tm_we, full(s), t * 32 + 16, n0);
-                last = t;
+                last = u;
             }
             if (!ok && last >= 0) sqd::mbar_drain(full(last % NST), (last / NST) & 1);
+        }
+        if constexpr (KS == 2) {
+            __syncwarp();
+            sqd::cluster_sync();   // the epilogue's two cluster barriers
+            sqd::cluster_sync();
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -285,9 +302,9 @@ sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant
             constexpr uint32_t idesc = (1u << 2) | (1u << 4) | (static_cast<uint32_t>(MT >> 3) << 17) |
                                        (static_cast<uint32_t>(128 >> 4) << 24);
             bool ok = true;
-            for (int t = 0; t < nst_k && ok; ++t) {
-                const int s = t % NST;
-                if (!sqd::mbar_wait(full(s), (t / NST) & 1, abort_flag, SITE_HI_MMA)) { ok = false; break; }
+            for (int u = 0; u < nst_k && ok; ++u) {
+                const int s = u % NST;
+                if (!sqd::mbar_wait(full(s), (u / NST) & 1, abort_flag, SITE_HI_MMA)) { ok = false; break; }
                 sqd::tc_fence_after();
                 const uint32_t ecol = tmem + MT + 8 * s;
                 const uint32_t st = stage(s);
@@ -304,7 +321,7 @@ sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant
                     asm volatile(
                         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
                         "tcgen05.mma.sp.cta_group::1.kind::f8f6f4 [%0], %1, %2, [%5], %3, p;\n\t}\n" ::"r"(tmem),
-                        "l"(adesc + 2 * j), "l"(bdesc), "r"(idesc), "r"((t == 0 && j == 0) ? 0u : 1u),
+                        "l"(adesc + 2 * j), "l"(bdesc), "r"(idesc), "r"((u == 0 && j == 0) ? 0u : 1u),
                         "r"(ecol + 2 * j)
                         : "memory");
                 }
@@ -315,6 +332,53 @@ sqf_high_kernel(const __grid_constant__ CUtensorMap tm_wh, const __grid_constant
             } else {
                 sqd::mma_commit(drain);
                 sqd::mbar_drain(drain, 0);
+            }
+        }
+        if constexpr (KS == 2) {
+            __syncwarp();
+            sqd::cluster_sync();   // the epilogue's two cluster barriers
+            sqd::cluster_sync();
+        }
+    } else if constexpr (KS == 2) {
+        // epilogue of a split tile.  The second CTA's accumulator goes into the first's staging
+        // ring (free once the first CTA's MMAs are done: first barrier), column-major
+        // ([MT][128 rows], conflict-free); after the second barrier the first CTA adds it.
+        const int q = warp & 3;
+        const int row = 32 * q + lane;   // TMEM lane = W row n0 + row
+        const int n = n0 + row;
+        const bool n_ok = n < args.N;
+        const float sh = n_ok ? args.s_hi[n] : 0.0f;
+        const uint32_t tl = tmem + (static_cast<uint32_t>(32 * q) << 16);
+        const bool have = sqd::mbar_wait(acc_full, 0, abort_flag, SITE_HI_EPI);
+        if (have) sqd::tc_fence_after();
+        __syncwarp();
+        sqd::cluster_sync();
+        if (kz == 1 && have) {
+            const uint32_t buf0 = sqd::map_to_cta(sbase, 0);
+            for (int c = 0; c < MT; c += 16) {
+                uint32_t v[16];
+                sqd::tmem_ld_32x32b_x16(tl + c, v);
+                sqd::tmem_wait_ld_dep1(v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    sqd::st_cluster_f32(buf0 + 4u * static_cast<uint32_t>((c + i) * 128 + row), __uint_as_float(v[i]));
+            }
+        }
+        __syncwarp();
+        sqd::cluster_sync();
+        if (kz == 0 && have) {
+            const float *part = reinterpret_cast<const float *>(smem);
+            for (int c = 0; c < MT; c += 16) {
+                uint32_t v[16];
+                sqd::tmem_ld_32x32b_x16(tl + c, v);
+                sqd::tmem_wait_ld_dep1(v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int m = m0 + c + i;
+                    const float acc = __fadd_rn(__uint_as_float(v[i]), part[(c + i) * 128 + row]);
+                    if (n_ok && m < args.M)
+                        args.P[static_cast<int64_t>(m) * args.N + n] = __fmul_rn(__fmul_rn(acc, args.s_x8[m]), sh);
+                }
             }
         }
     } else {

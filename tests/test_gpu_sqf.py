@@ -80,7 +80,9 @@ def check_sqf(X, W, bank, h, rows=None, ldy_extra=0):
 
 
 SHAPES = [
-    # (M, K, N, bank, h): the pair kernel (M > 128) and every split-K token class, both high-part tile sizes
+    # (M, K, N, bank, h): the pair kernel (M > 128) and every split-K token class, both high-part tile
+    # sizes; for M <= 128 the high part splits each tile's K stages over two CTAs unless the tiles
+    # already fill half of the SMs
     (300, 1024, 520, 8, 2),
     (1000, 2048, 1288, 16, 1),
     (130, 512, 264, 8, 1),
@@ -89,6 +91,9 @@ SHAPES = [
     (40, 2048, 384, 16, 2),
     (100, 3072, 1152, 4, 2),
     (128, 1024, 512, 16, 1),
+    # more W tiles than half the SMs: one CTA per tile (no K split), both token tile sizes
+    (16, 1024, 10240, 16, 1),
+    (100, 1024, 9728, 8, 2),
 ]
 
 
